@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Benchmark of the layer-routed hybrid attention hot path on B200.
+
+One step = one pass of the whole hot path over one batch of the workload:
+  * the CSR of the block pattern (fa_blocksparse_index),
+  * two routed layers (fa_hybrid_layer: router pool -> MLP -> argmax on the
+    device, then the attention kernel reading the mode): the router head bias
+    sends one layer to FULL and one to SPARSE, as in a half-sparse stack,
+  * one decode token per layer in that layer's mode (fa_attn_decode).
+value = algorithmic FLOPs of the step / time: full layer 4*D*Hq*B*S(S+1)/2,
+sparse layer 4*D*Hq*B*(exact attended pairs), decode 4*D*Hq*B*(keys read).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--workload NAME]
+Multi-GPU (torchrun): every rank runs an independent replica of the step on
+its own GPU (the path has no exchange step); value = all ranks' FLOPs / the
+slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill attn TFLOP/s & % bf16 peak; decode HBM GB/s; hybrid vs full at 256K"
+DEFAULT_WORKLOAD = "qwen3-4b-layer-s8192"
+N_INPUT_SETS = 4           # rotated so each step reads inputs not resident in L2
+KERNEL_SRC = os.path.join(ROOT, "block_sparse_attention_layerrouter_b200", "csrc",
+                          "fa_prefill.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "prefill_full_dram_traffic.txt")
+
+
+# ------------------------------------------------------------ accounting
+def flops_full(wl) -> float:
+    return 4.0 * 128 * wl.Hq * wl.B * (wl.S * (wl.S + 1) / 2)
+
+
+def flops_sparse_exact(wl) -> float:
+    import oracle  # pair counting only (host arithmetic of the pattern)
+    return 4.0 * 128 * wl.Hq * wl.B * oracle.attended_pairs_sparse(wl.S, 64, wl.sink, wl.window)
+
+
+def csr_nnz(S, sink, window) -> int:
+    nb = -(-S // 64)
+    sb, wb = sink // 64, window // 64
+    n = 0
+    for i in range(nb):
+        a = min(sb, i + 1)
+        lo = max(a, i - wb + 1)
+        n += a + (i - lo + 1)
+    return n
+
+
+def decode_keys(L, mode, sink, window) -> int:
+    if mode == 0:
+        return L
+    last = (L - 1) // 64
+    a = min(sink // 64, last + 1)
+    lo = max(a, last - window // 64 + 1)
+    keys = a * 64
+    for blk in range(lo, last + 1):
+        keys += min(L, (blk + 1) * 64) - blk * 64
+    return keys
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read only)."""
+
+    def __init__(self, device: torch.device, period_s: float = 0.1):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(device)
+            bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nvml = None
+            self.error = str(e)
+
+    _NAMES = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+              0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+              0x100: "display_clocks", 0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self._NAMES.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self._period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def report(self):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples),
+                "note": "sampled during warm-up and the timed region"}
+
+
+# ----------------------------------------------------------------- helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_traffic():
+    """DRAM bytes per full-prefill launch from the committed ncu summary, only
+    if it was taken on the current kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, None
+    kv = {}
+    for line in open(TRAFFIC_FILE):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    src_sha = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+    if kv.get("kernel_src_sha256_16") != src_sha:
+        return None, kv.get("workload")
+    try:
+        return float(kv["dram_bytes_per_full_launch"]), kv.get("workload")
+    except (KeyError, ValueError):
+        return None, kv.get("workload")
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# -------------------------------------------------------------- our arm
+class Step:
+    """Device buffers of one input set and the launches of one step."""
+
+    def __init__(self, wl, seed, dev, capi, inputs, pinned=False):
+        self.wl, self.dev = wl, dev
+        B, S, Hq, Hkv = wl.B, wl.S, wl.Hq, wl.Hkv
+        self.layers = []
+        for li, bias in enumerate(((0.1, 0.0), (0.0, 0.1))):   # FULL, SPARSE
+            q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, seed + 7919 * li, device=dev)
+            w1, b1, w2, b2 = inputs.router_weights(Hq * 128, wl.hidden, seed, li, b2=bias)
+            qd = inputs.randn_bf16((B, Hq, 128), seed + 31 * li + 5, device=dev)
+            self.layers.append(dict(q=q, k=k, v=v, w1=w1.to(dev), b1=b1.to(dev), w2=w2.to(dev),
+                                    b2=b2.to(dev), o=torch.empty_like(q), qd=qd,
+                                    od=torch.empty_like(qd),
+                                    logits=torch.empty(B, 2, device=dev),
+                                    mode=torch.empty(B, dtype=torch.int32, device=dev)))
+        self.c = capi.cfg(64, wl.sink, wl.window)
+        rows, nnz = capi.blocksparse_index_size(S, self.c)
+        self.row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+        self.col_idx = torch.empty(max(1, nnz), dtype=torch.int32, device=dev)
+        self.ws = torch.empty(capi.hybrid_workspace_size(B, Hq, 128, wl.hidden),
+                              dtype=torch.uint8, device=dev)
+        self.dws = torch.empty(capi.decode_workspace_size(B, Hq, Hkv, S), dtype=torch.uint8,
+                               device=dev)
+        self.seqlens = torch.full((B,), S, dtype=torch.int32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.capi = capi
+
+    def run(self, ev=None):
+        """Enqueue one step.  ev: optional (start, end) events around the
+        FULL layer's attention launch."""
+        capi, c = self.capi, self.c
+        L = capi.lib()
+        st = capi._stream(self.dev)
+        rc = L.fa_blocksparse_index(self.wl.S, c, capi._ptr(self.row_ptr), capi._ptr(self.col_idx),
+                                    st)
+        capi._check("fa_blocksparse_index", rc)
+        for li, lay in enumerate(self.layers):
+            if ev is not None and li == 0:
+                ev[0].record()
+            capi.hybrid_layer(lay["q"], lay["k"], lay["v"], lay["w1"], lay["b1"], lay["w2"],
+                              lay["b2"], self.row_ptr, self.col_idx, c, o=lay["o"],
+                              logits=lay["logits"], mode=lay["mode"], workspace=self.ws,
+                              status=self.status)
+            if ev is not None and li == 0:
+                ev[1].record()
+            capi.attn_decode(lay["qd"], lay["k"], lay["v"], self.seqlens, mode_dev=lay["mode"],
+                             c=c, o=lay["od"], workspace=self.dws, status=self.status)
+
+    LAUNCHES_PER_STEP = 1 + 2 * (3 + 1) + 2 * 2   # index, 2x(router 3 + attn), 2x decode
+
+
+def time_kernel_alone(fn, reps=5):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fn()
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(reps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / reps
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    """The oracle as it stands, on the host cores, on a bounded sample of the
+    workload: seeded query rows of the full and the sparse layer; scaled to
+    TFLOP/s by the algorithmic FLOPs of the rows computed."""
+    import oracle
+    from block_sparse_attention_layerrouter_b200 import inputs
+    B, S, Hq, Hkv = wl.B, wl.S, wl.Hq, wl.Hkv
+    q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, wl.seed, device="cpu")
+    qb, kb, vb = inputs.bits(q), inputs.bits(k), inputs.bits(v)
+    mask = oracle.rows_to_dense_mask(oracle.blocksparse_rows(S, 64, wl.sink, wl.window))
+    rng = np.random.default_rng(wl.seed)
+    flops, elapsed, nrows = 0.0, 0.0, 0
+    chunk = 64
+    oracle.attention_rows(qb, kb, vb, 0.1, np.array([[0, 0, 0]]))   # load + warm
+    while elapsed < budget_s:
+        ts = rng.integers(0, S, size=chunk)
+        hs = rng.integers(0, Hq, size=chunk)
+        rows = np.stack([np.zeros(chunk, np.int64), hs, ts], axis=1)
+        t0 = time.perf_counter()
+        oracle.attention_rows(qb, kb, vb, 1 / math.sqrt(128), rows)           # full layer rows
+        oracle.attention_rows(qb, kb, vb, 1 / math.sqrt(128), rows, mask)     # sparse layer rows
+        elapsed += time.perf_counter() - t0
+        full_pairs = float(np.sum(ts + 1))
+        kept = mask[ts // 64]                                                 # [chunk, nkb]
+        sparse_pairs = 0.0
+        for t, krow in zip(ts, kept):
+            blocks = np.nonzero(krow)[0]
+            sparse_pairs += float(np.sum(np.minimum(blocks * 64 + 64, t + 1) - blocks * 64))
+        flops += 4.0 * 128 * (full_pairs + sparse_pairs)
+        nrows += 2 * chunk
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d query rows (random head and position; each row once in the full and "
+                      "once in the sparse layer) of %s, %.1f s" % (nrows, wl.name, elapsed)}
+
+
+def run_ours(args, wl):
+    from block_sparse_attention_layerrouter_b200 import build, capi, inputs
+    ws, rank, local = dist_env()
+    if ws > 1 and not torch.distributed.is_initialized():
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build.build()
+    if ws > 1:
+        torch.distributed.barrier()
+    capi.lib()
+
+    sets = [Step(wl, wl.seed + 101 * i, dev, capi, inputs) for i in range(N_INPUT_SETS)]
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for i in range(args.warmup):
+        sets[i % N_INPUT_SETS].run()
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev_full = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        sets[i % N_INPUT_SETS].run(ev_full[i])
+    t1.record()
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.stop()
+    ms = t0.elapsed_time(t1)
+    ms_full = [s.elapsed_time(e) for s, e in ev_full]
+    status = max(int(s.status.item()) for s in sets)
+    modes = [int(l["mode"][0].item()) for l in sets[0].layers]
+    if ws > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, wl, dev, capi, inputs, ws)
+
+    # ---- components, each timed alone (for the breakdown; not the headline)
+    s0 = sets[0]
+    lay0, lay1 = s0.layers
+    comp = {}
+    comp["prefill_full_ms"] = time_kernel_alone(
+        lambda: capi.attn_prefill_full(lay0["q"], lay0["k"], lay0["v"], o=lay0["o"]))
+    comp["prefill_sparse_ms"] = time_kernel_alone(
+        lambda: capi.attn_prefill_blocksparse(lay1["q"], lay1["k"], lay1["v"], s0.row_ptr,
+                                              s0.col_idx, o=lay1["o"]))
+    comp["router_ms"] = time_kernel_alone(
+        lambda: capi.router_decide(lay0["q"], lay0["w1"], lay0["b1"], lay0["w2"], lay0["b2"],
+                                   logits=lay0["logits"], mode=lay0["mode"], workspace=s0.ws))
+    for name, md in (("decode_full_ms", 0), ("decode_sparse_ms", 1)):
+        comp[name] = time_kernel_alone(
+            lambda md=md: capi.attn_decode(lay0["qd"], lay0["k"], lay0["v"], s0.seqlens, md,
+                                           s0.c, o=lay0["od"], workspace=s0.dws))
+    torch.cuda.synchronize()
+
+    if rank != 0:
+        return None
+    hbm, peak_burst, peak_sust, peak_kind = measured_peaks()
+    f_full = flops_full(wl)
+    f_sparse = flops_sparse_exact(wl)
+    f_sparse_exec = 4.0 * 128 * wl.Hq * wl.B * csr_nnz(wl.S, wl.sink, wl.window) * 64 * 64
+    keys_dec = decode_keys(wl.S, 0, wl.sink, wl.window) + decode_keys(wl.S, 1, wl.sink, wl.window)
+    f_dec = 4.0 * 128 * wl.Hq * wl.B * keys_dec
+    step_flops = f_full + f_sparse + f_dec
+    value = ws * step_flops / (ms / args.steps * 1e-3) / 1e12
+    avg_full_ms = statistics.mean(ms_full)
+    achieved = f_full / (avg_full_ms * 1e-3) / 1e12
+    traffic, traffic_wl = kernel_traffic()
+    dec_bytes_full = 2 * wl.B * wl.Hkv * 128 * 2 * wl.S
+    comp.update({
+        "prefill_full_tflops": f_full / (comp["prefill_full_ms"] * 1e-3) / 1e12,
+        "prefill_sparse_exec_tflops": f_sparse_exec / (comp["prefill_sparse_ms"] * 1e-3) / 1e12,
+        "prefill_sparse_exact_tflops": f_sparse / (comp["prefill_sparse_ms"] * 1e-3) / 1e12,
+        "decode_full_gbs": dec_bytes_full / (comp["decode_full_ms"] * 1e-3) / 1e9,
+        "routed_modes": modes,
+        "device_status": status,
+    })
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q/K/V; "
+        "router weights N(0,0.02)); stands in for LongBench-E/RULER prompts of this shape",
+        "config": {"workload": wl.name, "B": wl.B, "S": wl.S, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                   "D": 128, "block": 64, "sink": wl.sink, "window": wl.window,
+                   "router": "%d->%d->2" % (wl.Hq * 128, wl.hidden),
+                   "step": "index + 2 routed layers (1 FULL, 1 SPARSE) + 1 decode token each",
+                   "parallelism": "replicas" if ws > 1 else "single GPU",
+                   "l2": "inputs larger than L2: %d rotated input sets, %.2f GB" % (
+                       N_INPUT_SETS, N_INPUT_SETS * sum(
+                           t.numel() * t.element_size() for t in
+                           (sets[0].layers[0]["q"], sets[0].layers[0]["k"],
+                            sets[0].layers[0]["v"], sets[0].layers[0]["o"])) * 2 / 1e9)},
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel (FULL layer)",
+                     "achieved": round(achieved, 2), "peak": peak_sust, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_sust, 4),
+                     "peak_kind": "%s bf16 sustained" % peak_kind,
+                     "frac_of_burst_peak": round(achieved / peak_burst, 4),
+                     "traffic": traffic, "traffic_workload": traffic_wl,
+                     "algorithmic_flops_per_launch": f_full,
+                     "avg_launch_ms": round(avg_full_ms, 4)},
+        "e2e": e2e,
+        "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
+        "clocks": sampler.report(),
+        "components": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in comp.items()},
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    return line
+
+
+def run_e2e(args, wl, dev, capi, inputs, ws):
+    """Same step through the public API with host buffers: per step, copy
+    the two layers' Q/K/V and decode queries from pinned host memory, run,
+    and read both layers' outputs back."""
+    host = []
+    for li in range(2):
+        q, k, v = inputs.qkv(wl.B, wl.S, wl.Hq, wl.Hkv, 128, wl.seed + 7919 * li)
+        qd = inputs.randn_bf16((wl.B, wl.Hq, 128), wl.seed + 31 * li + 5)
+        host.append([t.pin_memory() for t in (q, k, v, qd)])
+    step = Step(wl, wl.seed, dev, capi, inputs)
+    outs = [(torch.empty_like(step.layers[i]["o"], device="cpu").pin_memory(),
+             torch.empty_like(step.layers[i]["od"], device="cpu").pin_memory()) for i in range(2)]
+    h2d = sum(t.numel() * t.element_size() for hs in host for t in hs)
+    d2h = sum(t.numel() * t.element_size() for o in outs for t in o)
+
+    def one():
+        for li, lay in enumerate(step.layers):
+            for name, t in zip(("q", "k", "v", "qd"), host[li]):
+                lay[name].copy_(t, non_blocking=True)
+        step.run()
+        for li, lay in enumerate(step.layers):
+            outs[li][0].copy_(lay["o"], non_blocking=True)
+            outs[li][1].copy_(lay["od"], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        one()
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    if ws > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    keys_dec = decode_keys(wl.S, 0, wl.sink, wl.window) + decode_keys(wl.S, 1, wl.sink, wl.window)
+    step_flops = flops_full(wl) + flops_sparse_exact(wl) + 4.0 * 128 * wl.Hq * wl.B * keys_dec
+    return {"value": round(ws * step_flops / (ms / args.steps * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / args.steps, 4)}
+
+
+# --------------------------------------------------------- reference arm
+def run_reference(args, wl):
+    """The oracle as it stands on the host cores, same metric and unit; each
+    step a bounded sample of the workload (see cpu_baseline)."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    budget = float(os.environ.get("FA_REF_STEP_S", "4"))
+    vals, t_total = [], 0.0
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        r = cpu_baseline(wl, budget_s=budget)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            t_total += time.perf_counter() - t0
+    value = statistics.mean(vals)
+    r["value"] = value
+    return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "impl": "reference",
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * t_total / max(1, args.steps), 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "S": wl.S, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                       "D": 128, "block": 64, "sink": wl.sink, "window": wl.window},
+            "cpu_baseline": r,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from block_sparse_attention_layerrouter_b200.inputs import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if wl.decode_len:
+        ap.error("the decode workload is measured by bench_decode in this file's sibling flags")
+    line = run_reference(args, wl) if args.impl == "reference" else run_ours(args, wl)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

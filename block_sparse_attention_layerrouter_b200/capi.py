@@ -1,0 +1,259 @@
+"""ctypes binding of libfa_hybrid.so, one function per C-ABI entry point.
+
+Argument marshalling only: every function checks dtypes, devices and
+contiguity, takes ``data_ptr()`` and the current CUDA stream, calls the C entry
+point of the same name and raises :class:`FaError` on a non-zero status.
+Every step of the computation runs in the library's CUDA kernels; there is no
+fallback.  Outputs and workspaces are allocated with torch when the caller
+does not pass them (torch is the memory and stream plumbing only).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa_hybrid.so")
+
+FA_OK = 0
+FA_MODE_FULL = 0
+FA_MODE_SPARSE = 1
+FA_DEV_TIMEOUT = 1
+FA_DEV_BAD_INDEX = 2
+
+
+class FaError(RuntimeError):
+    def __init__(self, name: str, status: int, text: str):
+        super().__init__("%s failed: %s (status %d)" % (name, text, status))
+        self.status = status
+
+
+class SparseCfg(ctypes.Structure):
+    """fa_sparse_cfg: block, sink and window in tokens."""
+    _fields_ = [("block", ctypes.c_int32), ("sink", ctypes.c_int32), ("window", ctypes.c_int32)]
+
+
+_lib = None
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_SIGNATURES = {
+    "fa_status_string": (ctypes.c_char_p, [_I]),
+    "fa_version": (_I, []),
+    "fa_router_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "fa_router_decide": (_I, [_VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _I, _VP, _VP, _VP, _VP,
+                              _VP, _SZ, _VP]),
+    "fa_blocksparse_index_size": (_I, [_I, SparseCfg, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
+    "fa_blocksparse_index": (_I, [_I, SparseCfg, _VP, _VP, _VP]),
+    "fa_attn_prefill_full": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP]),
+    "fa_attn_prefill_blocksparse": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP,
+                                         _VP, _I, _VP, _VP]),
+    "fa_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_attn_decode": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, SparseCfg, _VP,
+                            _VP, _VP, _SZ, _VP, _VP]),
+    "fa_hybrid_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "fa_hybrid_layer": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
+                             _VP, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
+}
+EXPORTED = tuple(_SIGNATURES)
+
+
+def lib():
+    """Load the library (once).  Raises if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libfa_hybrid.so not found at %s: build it with "
+                "`python -m block_sparse_attention_layerrouter_b200.build`" % LIB_PATH)
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def _check(name: str, rc: int):
+    if rc != FA_OK:
+        raise FaError(name, rc, status_string(rc))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, dim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (no CPU path exists)" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if t.dim() != dim:
+        raise ValueError("%s must have %d dims, got %d" % (name, dim, t.dim()))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def cfg(block: int = 64, sink: int = 128, window: int = 128) -> SparseCfg:
+    return SparseCfg(block, sink, window)
+
+
+# ------------------------------------------------------------------ router
+def router_workspace_size(B, Hq, D, hidden) -> int:
+    return int(lib().fa_router_workspace_size(B, Hq, D, hidden))
+
+
+def router_decide(q, w1, b1, w2, b2, n_head=100, n_tail=100, logits=None, mode=None,
+                  workspace=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """fa_router_decide.  q bf16 [B,S,Hq,D]; fp32 weights on q's device."""
+    _need(q, "q", torch.bfloat16, 4)
+    B, S, Hq, D = q.shape
+    hidden = w1.shape[0]
+    for t, n in ((w1, "w1"), (w2, "w2")):
+        _need(t, n, torch.float32, 2)
+    for t, n in ((b1, "b1"), (b2, "b2")):
+        if t is not None:
+            _need(t, n, torch.float32, 1)
+    dev = q.device
+    logits = torch.empty(B, 2, device=dev, dtype=torch.float32) if logits is None else logits
+    mode = torch.empty(B, device=dev, dtype=torch.int32) if mode is None else mode
+    ws_bytes = router_workspace_size(B, Hq, D, hidden)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    rc = lib().fa_router_decide(_ptr(q), B, S, Hq, D, n_head, n_tail, _ptr(w1), _ptr(b1), hidden,
+                                _ptr(w2), _ptr(b2), _ptr(logits), _ptr(mode), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(dev))
+    _check("fa_router_decide", rc)
+    return logits, mode
+
+
+# ------------------------------------------------------------------- index
+def blocksparse_index_size(S: int, c: SparseCfg) -> Tuple[int, int]:
+    rows, nnz = ctypes.c_int(0), ctypes.c_int(0)
+    _check("fa_blocksparse_index_size",
+           lib().fa_blocksparse_index_size(S, c, ctypes.byref(rows), ctypes.byref(nnz)))
+    return rows.value, nnz.value
+
+
+def blocksparse_index(S: int, c: SparseCfg, device="cuda"):
+    """fa_blocksparse_index -> (row_ptr int32 [n+1], col_idx int32 [nnz]) on device."""
+    rows, nnz = blocksparse_index_size(S, c)
+    dev = torch.device(device)
+    row_ptr = torch.empty(rows + 1, device=dev, dtype=torch.int32)
+    col_idx = torch.empty(max(nnz, 1), device=dev, dtype=torch.int32)
+    _check("fa_blocksparse_index",
+           lib().fa_blocksparse_index(S, c, _ptr(row_ptr), _ptr(col_idx), _stream(dev)))
+    return row_ptr, col_idx[:nnz]
+
+
+# ----------------------------------------------------------------- prefill
+def _prefill_common(q, k, v, o, lse):
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, S, Hkv, D) or v.shape != k.shape:
+        raise ValueError("k/v must be [B, S, Hkv, D] matching q")
+    o = torch.empty_like(q) if o is None else o
+    _need(o, "o", torch.bfloat16, 4)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+    return B, S, Hq, Hkv, D, o
+
+
+def attn_prefill_full(q, k, v, scale=None, o=None, lse=None, status=None) -> torch.Tensor:
+    B, S, Hq, Hkv, D, o = _prefill_common(q, k, v, o, lse)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rc = lib().fa_attn_prefill_full(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, S, Hq, Hkv,
+                                    D, scale, _ptr(status), _stream(q.device))
+    _check("fa_attn_prefill_full", rc)
+    return o
+
+
+def attn_prefill_blocksparse(q, k, v, row_ptr, col_idx, block=64, scale=None, o=None, lse=None,
+                             status=None) -> torch.Tensor:
+    B, S, Hq, Hkv, D, o = _prefill_common(q, k, v, o, lse)
+    _need(row_ptr, "row_ptr", torch.int32, 1)
+    _need(col_idx, "col_idx", torch.int32, 1)
+    if row_ptr.numel() != -(-S // block) + 1:
+        raise ValueError("row_ptr must have ceil(S/block)+1 entries")
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rc = lib().fa_attn_prefill_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, S,
+                                           Hq, Hkv, D, scale, _ptr(row_ptr), _ptr(col_idx), block,
+                                           _ptr(status), _stream(q.device))
+    _check("fa_attn_prefill_blocksparse", rc)
+    return o
+
+
+# ------------------------------------------------------------------ decode
+def decode_workspace_size(B, Hq, Hkv, Lmax, D=128) -> int:
+    return int(lib().fa_decode_workspace_size(B, Hq, Hkv, Lmax, D))
+
+
+def attn_decode(q, kcache, vcache, seqlens, mode=FA_MODE_FULL, c: Optional[SparseCfg] = None,
+                scale=None, mode_dev=None, o=None, lse=None, workspace=None,
+                status=None) -> torch.Tensor:
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, D = q.shape
+    Lmax, Hkv = kcache.shape[1], kcache.shape[2]
+    if vcache.shape != kcache.shape or kcache.shape[0] != B or kcache.shape[3] != D:
+        raise ValueError("caches must be [B, Lmax, Hkv, D] matching q")
+    c = cfg() if c is None else c
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    o = torch.empty_like(q) if o is None else o
+    ws_bytes = decode_workspace_size(B, Hq, Hkv, Lmax, D)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), device=q.device, dtype=torch.uint8)
+    rc = lib().fa_attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), B, Lmax, Hq,
+                              Hkv, D, scale, int(mode), _ptr(mode_dev), c, _ptr(o), _ptr(lse),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _ptr(status), _stream(q.device))
+    _check("fa_attn_decode", rc)
+    return o
+
+
+# ------------------------------------------------------------------ hybrid
+def hybrid_workspace_size(B, Hq, D, hidden) -> int:
+    return int(lib().fa_hybrid_workspace_size(B, Hq, D, hidden))
+
+
+def hybrid_layer(q, k, v, w1, b1, w2, b2, row_ptr, col_idx, c: SparseCfg, scale=None, o=None,
+                 lse=None, logits=None, mode=None, workspace=None, status=None):
+    """fa_hybrid_layer -> (o, logits, mode)."""
+    B, S, Hq, Hkv, D, o = _prefill_common(q, k, v, o, lse)
+    hidden = w1.shape[0]
+    dev = q.device
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    logits = torch.empty(B, 2, device=dev, dtype=torch.float32) if logits is None else logits
+    mode = torch.empty(B, device=dev, dtype=torch.int32) if mode is None else mode
+    ws_bytes = hybrid_workspace_size(B, Hq, D, hidden)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    rc = lib().fa_hybrid_layer(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, S, Hq, Hkv, D,
+                               scale, _ptr(w1), _ptr(b1), hidden, _ptr(w2), _ptr(b2), c,
+                               _ptr(row_ptr), _ptr(col_idx), _ptr(logits), _ptr(mode),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _ptr(status), _stream(dev))
+    _check("fa_hybrid_layer", rc)
+    return o, logits, mode

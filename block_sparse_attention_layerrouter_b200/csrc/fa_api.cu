@@ -1,0 +1,225 @@
+// fa_api.cu -- the extern "C" entry points declared in include/fa_hybrid.h:
+// argument checks, TMA descriptor setup and kernel launches.  No allocation,
+// no synchronisation, no state beyond one-time driver entry-point lookup.
+#include "fa_common.cuh"
+#include "fa_internal.h"
+
+#include <mutex>
+
+namespace fa {
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols,
+                   int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return -1;
+  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {128 * 2, static_cast<cuuint64_t>(H) * 256,
+                                 static_cast<cuuint64_t>(S) * H * 256};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols), 1,
+                             static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+namespace {
+
+constexpr int kHeadDim = 128;
+
+int check_heads(int Hq, int Hkv, int D) {
+  if (Hq <= 0 || Hkv <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (D != kHeadDim) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+int check_cfg(fa_sparse_cfg c) {
+  if (c.block != 64) return c.block <= 0 ? FA_ERR_INVALID_ARG : FA_ERR_UNSUPPORTED;
+  if (c.sink < 0 || c.window < c.block) return FA_ERR_INVALID_ARG;
+  if (c.sink % c.block || c.window % c.block) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+int check_prefill(const void *q, const void *k, const void *v, void *o, int B, int S, int Hq,
+                  int Hkv, int D) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || S <= 0) return FA_ERR_INVALID_ARG;
+  if (int rc = check_heads(Hq, Hkv, D)) return rc;
+  // TMA global dims and the flattened grid must fit.
+  if (static_cast<long long>(S) * Hq * kHeadDim * 2 > (1ll << 40)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+int check_router(const void *q, int B, int S, int Hq, int D, int n_head, int n_tail,
+                 const float *w1, int hidden, const float *w2) {
+  if (!q || !w1 || !w2) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(w1)) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || n_head < 0 || n_tail < 0 || n_head + n_tail < 1)
+    return FA_ERR_INVALID_ARG;
+  if (S < n_head + n_tail) return FA_ERR_UNSUPPORTED;
+  if (D != kHeadDim) return FA_ERR_UNSUPPORTED;
+  if (hidden < 1 || hidden > 65536) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+FA_API const char *fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: shape or option not supported";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA launch or driver call failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: wait timed out";
+    default: return "unknown fa_status";
+  }
+}
+
+FA_API int fa_version(void) { return 100; }
+
+FA_API size_t fa_router_workspace_size(int B, int Hq, int D, int hidden) {
+  if (B <= 0 || Hq <= 0 || D <= 0 || hidden <= 0) return 0;
+  return router_workspace_bytes(B, Hq, D, hidden);
+}
+
+FA_API int fa_router_decide(const void *q, int B, int S, int Hq, int D, int n_head_tok, int n_tail_tok,
+                     const float *w1, const float *b1, int hidden, const float *w2,
+                     const float *b2, float *logits_out, int32_t *mode_out, void *workspace,
+                     size_t ws_bytes, void *stream) {
+  if (int rc = check_router(q, B, S, Hq, D, n_head_tok, n_tail_tok, w1, hidden, w2)) return rc;
+  if (!logits_out && !mode_out) return FA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < router_workspace_bytes(B, Hq, D, hidden)) return FA_ERR_WORKSPACE;
+  RouterLaunch a{q, B, S, Hq, n_head_tok, n_tail_tok, w1, b1, w2, b2, hidden, logits_out,
+                 mode_out, workspace};
+  return launch_router(a, static_cast<cudaStream_t>(stream));
+}
+
+FA_API int fa_blocksparse_index_size(int S, fa_sparse_cfg cfg, int *n_rows, int *nnz) {
+  if (S <= 0 || !n_rows || !nnz) return FA_ERR_INVALID_ARG;
+  if (int rc = check_cfg(cfg)) return rc;
+  const int rows = (S + cfg.block - 1) / cfg.block;
+  const long long n = index_nnz(rows, cfg.sink / cfg.block, cfg.window / cfg.block);
+  if (n > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  *n_rows = rows;
+  *nnz = static_cast<int>(n);
+  return FA_OK;
+}
+
+FA_API int fa_blocksparse_index(int S, fa_sparse_cfg cfg, int32_t *row_ptr, int32_t *col_idx,
+                         void *stream) {
+  int rows = 0, nnz = 0;
+  if (int rc = fa_blocksparse_index_size(S, cfg, &rows, &nnz)) return rc;
+  if (!row_ptr || !col_idx) return FA_ERR_INVALID_ARG;
+  return launch_index(rows, cfg.sink / cfg.block, cfg.window / cfg.block, row_ptr, col_idx,
+                      static_cast<cudaStream_t>(stream));
+}
+
+FA_API int fa_attn_prefill_full(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                         int S, int Hq, int Hkv, int D, float scale, int32_t *dev_status,
+                         void *stream) {
+  if (int rc = check_prefill(q, k, v, o, B, S, Hq, Hkv, D)) return rc;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  PrefillLaunch a{q, k, v, o, lse, B, S, Hq, Hkv, scale, nullptr, nullptr, nullptr,
+                  FA_MODE_FULL, dev_status};
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+FA_API int fa_attn_prefill_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
+                                int B, int S, int Hq, int Hkv, int D, float scale,
+                                const int32_t *row_ptr, const int32_t *col_idx, int block,
+                                int32_t *dev_status, void *stream) {
+  if (int rc = check_prefill(q, k, v, o, B, S, Hq, Hkv, D)) return rc;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (!row_ptr || !col_idx) return FA_ERR_INVALID_ARG;
+  if (block != 64) return block <= 0 ? FA_ERR_INVALID_ARG : FA_ERR_UNSUPPORTED;
+  PrefillLaunch a{q, k, v, o, lse, B, S, Hq, Hkv, scale, row_ptr, col_idx, nullptr,
+                  FA_MODE_SPARSE, dev_status};
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+FA_API size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || D != kHeadDim || Hq % Hkv) return 0;
+  return decode_workspace_bytes(B, Hq, Hkv, Lmax);
+}
+
+FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                   int B, int Lmax, int Hq, int Hkv, int D, float scale, int mode,
+                   const int32_t *mode_dev, fa_sparse_cfg cfg, void *o, float *lse,
+                   void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!q || !kcache || !vcache || !seqlens || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Lmax <= 0) return FA_ERR_INVALID_ARG;
+  if (int rc = check_heads(Hq, Hkv, D)) return rc;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
+  if (mode != FA_MODE_FULL && mode != FA_MODE_SPARSE) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (int rc = check_cfg(cfg)) return rc;
+  if (!workspace || !aligned16(workspace) || ws_bytes < decode_workspace_bytes(B, Hq, Hkv, Lmax))
+    return FA_ERR_WORKSPACE;
+  DecodeLaunch a{q, kcache, vcache, seqlens, B, Lmax, Hq, Hkv, scale, mode, mode_dev,
+                 cfg.sink, cfg.window, o, lse, workspace, dev_status};
+  return launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+FA_API size_t fa_hybrid_workspace_size(int B, int Hq, int D, int hidden) {
+  return fa_router_workspace_size(B, Hq, D, hidden);
+}
+
+FA_API int fa_hybrid_layer(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                    int S, int Hq, int Hkv, int D, float scale, const float *w1, const float *b1,
+                    int hidden, const float *w2, const float *b2, fa_sparse_cfg cfg,
+                    const int32_t *row_ptr, const int32_t *col_idx, float *logits_out,
+                    int32_t *mode_out, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                    void *stream) {
+  if (int rc = check_prefill(q, k, v, o, B, S, Hq, Hkv, D)) return rc;
+  if (int rc = check_router(q, B, S, Hq, D, 100, 100, w1, hidden, w2)) return rc;
+  if (int rc = check_cfg(cfg)) return rc;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (!row_ptr || !col_idx || !mode_out) return FA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < router_workspace_bytes(B, Hq, D, hidden)) return FA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RouterLaunch r{q, B, S, Hq, 100, 100, w1, b1, w2, b2, hidden, logits_out, mode_out, workspace};
+  if (int rc = launch_router(r, st)) return rc;
+  PrefillLaunch a{q, k, v, o, lse, B, S, Hq, Hkv, scale, row_ptr, col_idx, mode_out,
+                  FA_MODE_FULL, dev_status};
+  return launch_prefill(a, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,374 @@
+// fa_decode.cu -- single-token decode attention over a bf16 KV cache, sm_100a.
+//
+// o = softmax(scale * q K^T) V for the query at position L-1 of each sequence.
+// FULL attends keys 0..L-1; SPARSE attends the sink blocks and the local
+// window of the prefill block rule for row L-1 and never loads any other KV
+// block ("Flux Attention": a sparse layer bypasses the KV cache outside its
+// pattern).  Memory-bound: every byte of K and V it needs is read once.
+//
+// Grid (split, kv head, batch).  A CTA owns one KV head (all G query heads
+// of its group share each K/V tile) and a contiguous share of the sequence's
+// 64-key tiles.  Thread 0 streams the tiles with 4-D TMA loads (128-byte
+// swizzle, 4 boxes of 64 keys x 64 dims per tile) into a 3-stage ring; all
+// threads compute from shared memory:
+//   QK^T   thread = (key, 1/PARTS of the head dim), dot products for the G
+//          heads, reduced across the PARTS lanes with shuffles;
+//   softmax one warp per query head: running max / sum in log2 units;
+//   PV     thread = (8 output dims, one of 16 key streams), G accumulators.
+// Each CTA writes its partial (max, sum, unnormalised output) per head; the
+// combine kernel merges the splits by log-sum-exp.
+#include "fa_common.cuh"
+#include "fa_internal.h"
+
+#include <math.h>
+
+namespace fa {
+namespace decode {
+
+constexpr int KT = 64;                         // keys per tile = one block
+constexpr int HD = 128;
+constexpr int NSTAGE = 3;
+constexpr int BOX_BYTES = KT * 64 * 2;         // 64 keys x 64 dims bf16
+constexpr int STAGE_BYTES = 4 * BOX_BYTES;     // K (2 boxes) + V (2 boxes)
+constexpr int NT = 256;
+constexpr int SMEM_BYTES = 1024 + NSTAGE * STAGE_BYTES + 8 * NSTAGE + 16 +
+                           /* scores */ 8 * KT * 4 + /* probs */ KT * 8 * 4 + 8 * 4;
+
+struct Params {
+  const __nv_bfloat16 *q;
+  float *o_part;    // [B, Hq, nsplit, HD]
+  float *ml_part;   // [B, Hq, nsplit, 2] (max, sum) in log2 units
+  const int32_t *seqlens;
+  const int32_t *mode;
+  int32_t *status;
+  int B, Lmax, Hq, Hkv, nsplit;
+  int mode_default, sink_blocks, win_blocks;
+  float scale_log2;
+};
+
+// Tiles (64-key blocks) a sequence of length L attends, as a virtual list:
+// positions [0, a) are blocks [0, a); positions [a, count) are blocks
+// lo .. last.  FULL: a = last + 1, count = a.
+struct TileList {
+  int a, lo, count, L;
+  FA_DEV void init(int L_, bool sparse, int sink_blocks, int win_blocks) {
+    L = L_;
+    const int last = (L - 1) / KT;
+    if (!sparse) {
+      a = last + 1;
+      lo = a;
+      count = a;
+    } else {
+      a = min(sink_blocks, last + 1);
+      lo = max(a, last - win_blocks + 1);
+      count = a + (last - lo + 1);
+    }
+  }
+  FA_DEV int block(int pos) const { return pos < a ? pos : lo + (pos - a); }
+};
+
+template <int G>
+struct Cfg {
+  static constexpr int PARTS = (G <= 4) ? 8 : 16;       // threads per key in QK^T
+  static constexpr int DPT = HD / PARTS;                 // dims per thread
+  static constexpr int KPP = NT / PARTS;                 // keys per pass
+  static constexpr int PASSES = KT / KPP;
+  static constexpr int MIN_BLOCKS = (G <= 4) ? 2 : 1;
+};
+
+FA_DEV void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Byte offset of the 16-byte chunk holding dims [8*chunk16, 8*chunk16+8) of
+// `key` inside one K or V tile written by TMA with the 128-byte swizzle.
+FA_DEV uint32_t tile_offset(int key, int chunk16) {
+  const int box = chunk16 >> 3;
+  const int phys = (chunk16 & 7) ^ (key & 7);
+  return static_cast<uint32_t>(box * BOX_BYTES + key * 128 + phys * 16);
+}
+
+template <int G>
+__global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
+    decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const Params p) {
+  using C = Cfg<G>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *stages = base;
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + NSTAGE * STAGE_BYTES);
+  volatile int *abort = reinterpret_cast<volatile int *>(full + NSTAGE);
+  float *s_sm = reinterpret_cast<float *>(base + NSTAGE * STAGE_BYTES + 8 * NSTAGE + 16);
+  float *p_sm = s_sm + 8 * KT;          // [KT][G]
+  float *alpha_sm = p_sm + KT * 8;      // [G]
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int L_raw = p.seqlens[b];
+  const int L = max(1, min(L_raw, p.Lmax));   // out-of-range lengths are clamped
+  if (L != L_raw && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(p.status, FA_DEV_BAD_INDEX);
+  const int mode = p.mode ? p.mode[b] : p.mode_default;
+  TileList tl;
+  tl.init(L, mode == FA_MODE_SPARSE, p.sink_blocks, p.win_blocks);
+  const int per = (tl.count + p.nsplit - 1) / p.nsplit;
+  const int pos0 = min(tl.count, split * per);
+  const int pos1 = min(tl.count, pos0 + per);
+  const int ntiles = pos1 - pos0;
+
+  if (tid == 0) {
+    for (int i = 0; i < NSTAGE; ++i) mbar_init(&full[i], 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  int issued = 0;            // tiles whose copies thread 0 has started
+  auto issue = [&](int i) {  // tile i of this CTA into stage i % NSTAGE
+    const int st = i % NSTAGE;
+    const int key0 = tl.block(pos0 + i) * KT;
+    uint8_t *dst = stages + st * STAGE_BYTES;
+    mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
+    tma_load_4d(dst, &tmK, &full[st], 0, kvh, key0, b);
+    tma_load_4d(dst + BOX_BYTES, &tmK, &full[st], 64, kvh, key0, b);
+    tma_load_4d(dst + 2 * BOX_BYTES, &tmV, &full[st], 0, kvh, key0, b);
+    tma_load_4d(dst + 3 * BOX_BYTES, &tmV, &full[st], 64, kvh, key0, b);
+    issued = i + 1;
+  };
+  if (tid == 0) {
+    for (int i = 0; i < NSTAGE && i < ntiles; ++i) issue(i);
+  }
+
+  // Query slice of this thread for QK^T, pre-scaled by scale*log2(e).
+  const int part = tid % C::PARTS;
+  float qr[G][C::DPT];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const __nv_bfloat16 *qrow = p.q + (static_cast<size_t>(b) * p.Hq + kvh * G + g) * HD + part * C::DPT;
+#pragma unroll
+    for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
+      float f[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + c8 * 8), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qr[g][c8 * 8 + e] = f[e] * p.scale_log2;
+    }
+  }
+  const int dc = tid & 15;     // PV: output dims [8*dc, 8*dc+8)
+  const int ks = tid >> 4;     // PV: key stream
+  float acc[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;  // meaningful in warp g < G
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i % NSTAGE;
+    const bool ok = mbar_wait(&full[st], static_cast<uint32_t>(i / NSTAGE) & 1u, abort, p.status);
+    if (__syncthreads_or(!ok)) break;
+    const uint8_t *sK = stages + st * STAGE_BYTES;
+    const uint8_t *sV = sK + 2 * BOX_BYTES;
+    const int key_base = tl.block(pos0 + i) * KT;
+
+    // ---- scores
+#pragma unroll
+    for (int pass = 0; pass < C::PASSES; ++pass) {
+      const int key = pass * C::KPP + tid / C::PARTS;
+      float d[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) d[g] = 0.f;
+#pragma unroll
+      for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
+        float kf[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(sK + tile_offset(key, part * (C::DPT / 8) + c8)), kf);
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) d[g] = fmaf(qr[g][c8 * 8 + e], kf[e], d[g]);
+      }
+#pragma unroll
+      for (int off = 1; off < C::PARTS; off <<= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g) d[g] += __shfl_xor_sync(0xffffffffu, d[g], off);
+      if (part == 0) {
+        const bool valid = key_base + key < L;
+#pragma unroll
+        for (int g = 0; g < G; ++g) s_sm[g * KT + key] = valid ? d[g] : -INFINITY;
+      }
+    }
+    __syncthreads();
+
+    // ---- online softmax, one warp per query head
+    if (warp < G) {
+      const float v0 = s_sm[warp * KT + lane], v1 = s_sm[warp * KT + lane + 32];
+      float mt = fmaxf(v0, v1);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+      const float m_new = fmaxf(m_run, mt);
+      const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float p0 = ex2(v0 - m_use), p1 = ex2(v1 - m_use);
+      float ps = p0 + p1;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      l_run = l_run * alpha + ps;
+      m_run = m_new;
+      p_sm[lane * G + warp] = p0;
+      p_sm[(lane + 32) * G + warp] = p1;
+      if (lane == 0) alpha_sm[warp] = alpha;
+    }
+    __syncthreads();
+
+    // ---- O += P V
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float a = alpha_sm[g];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[g][e] *= a;
+    }
+#pragma unroll
+    for (int kk = 0; kk < KT / 16; ++kk) {
+      const int key = ks + 16 * kk;
+      float vf[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(sV + tile_offset(key, dc)), vf);
+      float pg[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) pg[g] = p_sm[key * G + g];
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg[g], vf[e], acc[g][e]);
+    }
+    __syncthreads();
+    if (tid == 0 && i + NSTAGE < ntiles) issue(i + NSTAGE);
+  }
+
+  if (*abort) {  // let the copies still in flight land, then leave
+    if (tid == 0) {
+      for (int x = (issued > NSTAGE ? issued - NSTAGE : 0); x < issued; ++x)
+        mbar_wait_drain(&full[x % NSTAGE], static_cast<uint32_t>(x / NSTAGE) & 1u, 200000000ull);
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---- reduce the 16 key streams through shared memory (stage buffers free)
+  float *red = reinterpret_cast<float *>(stages);   // [16][G][HD]
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[(ks * G + g) * HD + dc * 8 + e] = acc[g][e];
+  __syncthreads();
+  const size_t row0 = (static_cast<size_t>(b) * p.Hq + kvh * G) * p.nsplit + split;
+  for (int idx = tid; idx < G * HD; idx += NT) {
+    const int g = idx / HD, dd = idx % HD;
+    float sum = 0.f;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) sum += red[(s * G + g) * HD + dd];
+    p.o_part[(row0 + static_cast<size_t>(g) * p.nsplit) * HD + dd] = sum;
+  }
+  if (warp < G && lane == 0) {
+    float *ml = p.ml_part + (row0 + static_cast<size_t>(warp) * p.nsplit) * 2;
+    ml[0] = m_run;
+    ml[1] = l_run;
+  }
+}
+
+// Merge the splits of one (batch, head): M = max m_s, w_s = 2^(m_s - M),
+// o = sum w_s o_s / sum w_s l_s.
+__global__ void __launch_bounds__(128) combine_kernel(const float *o_part, const float *ml_part,
+                                                      __nv_bfloat16 *o, float *lse, int Hq,
+                                                      int nsplit) {
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const size_t row = (static_cast<size_t>(b) * Hq + h);
+  const float *ml = ml_part + row * nsplit * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, ml[2 * s]);
+  float num = 0.f, den = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < nsplit; ++s) {
+      const float m = ml[2 * s];
+      if (m == -INFINITY) continue;
+      const float w = ex2(m - M);
+      den = fmaf(w, ml[2 * s + 1], den);
+      num = fmaf(w, o_part[(row * nsplit + s) * HD + d], num);
+    }
+  }
+  const float out = den > 0.f ? num / den : 0.f;
+  o[row * HD + d] = __float2bfloat16_rn(out);
+  if (lse && d == 0)
+    lse[row] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace decode
+
+int decode_num_splits(int B, int Hkv, int Lmax) {
+  const int tiles = (Lmax + decode::KT - 1) / decode::KT;
+  const int target_ctas = 148 * 2 * 4;
+  int ns = (target_ctas + B * Hkv - 1) / (B * Hkv);
+  ns = ns < 1 ? 1 : ns;
+  ns = ns > tiles ? tiles : ns;
+  ns = ns > 256 ? 256 : ns;
+  return ns;
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax) {
+  const size_t ns = static_cast<size_t>(decode_num_splits(B, Hkv, Lmax));
+  return static_cast<size_t>(B) * Hq * ns * (decode::HD + 2) * sizeof(float) + 256;
+}
+
+int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
+  using namespace decode;
+  CUtensorMap tmK, tmV;
+  if (make_tmap_bhsd(&tmK, a.kcache, a.B, a.Lmax, a.Hkv, 64, KT) != 0) return FA_ERR_CUDA;
+  if (make_tmap_bhsd(&tmV, a.vcache, a.B, a.Lmax, a.Hkv, 64, KT) != 0) return FA_ERR_CUDA;
+  const int G = a.Hq / a.Hkv;
+  // Splits: sized for FULL unless every sequence is known to be SPARSE.
+  int ns = decode_num_splits(a.B, a.Hkv, a.Lmax);
+  if (a.mode_dev == nullptr && a.mode == FA_MODE_SPARSE) {
+    const int sparse_tiles = a.sink / KT + a.window / KT;
+    ns = ns > sparse_tiles ? sparse_tiles : ns;
+    if (ns < 1) ns = 1;
+  }
+  Params p;
+  p.q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+  float *ws = reinterpret_cast<float *>(a.workspace);
+  p.o_part = ws;
+  p.ml_part = ws + static_cast<size_t>(a.B) * a.Hq * ns * HD;
+  p.seqlens = a.seqlens;
+  p.mode = a.mode_dev;
+  p.status = a.status;
+  p.B = a.B;
+  p.Lmax = a.Lmax;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.nsplit = ns;
+  p.mode_default = a.mode;
+  p.sink_blocks = a.sink / KT;
+  p.win_blocks = a.window / KT;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  const dim3 grid(ns, a.Hkv, a.B);
+  void (*kern)(const CUtensorMap, const CUtensorMap, const Params) = nullptr;
+  switch (G) {
+    case 1: kern = decode_kernel<1>; break;
+    case 2: kern = decode_kernel<2>; break;
+    case 4: kern = decode_kernel<4>; break;
+    case 8: kern = decode_kernel<8>; break;
+    default: return FA_ERR_UNSUPPORTED;
+  }
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  kern<<<grid, NT, SMEM_BYTES, stream>>>(tmK, tmV, p);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  combine_kernel<<<dim3(a.Hq, a.B), 128, 0, stream>>>(
+      p.o_part, p.ml_part, reinterpret_cast<__nv_bfloat16 *>(a.o), a.lse, a.Hq, ns);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace fa

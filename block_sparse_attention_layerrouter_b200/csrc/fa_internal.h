@@ -1,0 +1,63 @@
+// fa_internal.h -- launch descriptors shared by the C-ABI layer and the
+// kernel files.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fa {
+
+// 4-D TMA map over a bf16 tensor [B, S, H, 128] (row-major), boxes of
+// box_cols x 1 x box_rows x 1 with the 128-byte swizzle.  Returns 0 on success.
+int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols,
+                   int box_rows);
+
+struct PrefillLaunch {
+  const void *q, *k, *v;
+  void *o;
+  float *lse;
+  int B, S, Hq, Hkv;
+  float scale;
+  const int32_t *row_ptr, *col_idx;  // nullptr: FULL only
+  const int32_t *mode_dev;           // nullptr: use mode_default
+  int mode_default;
+  int32_t *status;
+};
+int launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
+
+struct DecodeLaunch {
+  const void *q, *kcache, *vcache;
+  const int32_t *seqlens;
+  int B, Lmax, Hq, Hkv;
+  float scale;
+  int mode;
+  const int32_t *mode_dev;
+  int sink, window;  // tokens, multiples of 64
+  void *o;
+  float *lse;
+  void *workspace;
+  int32_t *status;
+};
+int decode_num_splits(int B, int Hkv, int Lmax);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax);
+int launch_decode(const DecodeLaunch &a, cudaStream_t stream);
+
+struct RouterLaunch {
+  const void *q;
+  int B, S, Hq, n_head, n_tail;
+  const float *w1, *b1, *w2, *b2;
+  int hidden;
+  float *logits;
+  int32_t *mode;
+  void *workspace;
+};
+size_t router_workspace_bytes(int B, int Hq, int D, int hidden);
+int launch_router(const RouterLaunch &a, cudaStream_t stream);
+
+long long index_nnz(int nrows, int sb, int wb);
+int launch_index(int nrows, int sb, int wb, int32_t *row_ptr, int32_t *col_idx,
+                 cudaStream_t stream);
+
+}  // namespace fa

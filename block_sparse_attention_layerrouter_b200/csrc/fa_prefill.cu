@@ -1,0 +1,512 @@
+// fa_prefill.cu -- causal full and block-sparse attention prefill for sm_100a.
+//
+// What it computes (see include/fa_hybrid.h): O = softmax(scale * Q K^T
+// + mask) V per (batch, query head), with the causal mask, and for the sparse
+// mode the 64-token block pattern of a CSR row list ("Flux Attention",
+// implementation paragraph: 64-token block sparsity, 128 sink tokens).  The
+// softmax is the online form of the FlashAttention newsletter (section
+// "어려움을 극복하기 위한 Online Softmax"): a running maximum and sum per row,
+// with earlier partial results rescaled by exp(m_old - m_new).
+//
+// Design (one CTA = one 128-row query tile of one (batch, head)):
+//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys into a
+//               ring of 32 KB slots, in exactly the order the MMAs use them.
+//   warp 1      MMA issuer (one thread) and TMEM owner: S_j = Q K_j^T into one
+//               of two TMEM score buffers, O += P_j V_j with P read from TMEM.
+//   warps 4-7   softmax warpgroup, one thread per query row: reads S_j from
+//               TMEM, masks, updates the running max/sum, writes P_j (bf16) to
+//               TMEM, rescales O in TMEM only when the running max grew by
+//               more than 2^8 (exact: the final division uses the same max),
+//               and finally normalises O and stores it.
+// TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
+// All operands are bf16; accumulation and softmax are fp32.
+#include "fa_common.cuh"
+#include "fa_internal.h"
+
+#include <math.h>
+
+namespace fa {
+namespace prefill {
+
+constexpr int BM = 128;                       // query rows per CTA (MMA M)
+constexpr int BN = 128;                       // keys per KV tile
+constexpr int HD = 128;                       // head dim
+constexpr int NSLOT = 5;                      // K/V ring depth
+constexpr int TILE_BYTES = BN * HD * 2;       // one K or V tile, 32 KB
+constexpr int HALF_BYTES = TILE_BYTES / 2;    // one 64-column TMA box, 16 KB
+constexpr int NUM_THREADS = 256;
+constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 2 + 1;
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + TILE_BYTES /*Q*/ + NSLOT * TILE_BYTES +
+                           NUM_BARS * 8 + 16;
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P0 = 384, TM_P1 = 448;
+constexpr uint32_t TMEM_COLS = 512;
+// Rescale O only when the running max (log2 units) grew by more than this.
+constexpr float kRescaleThreshold = 8.0f;
+constexpr uint64_t kDrainNs = 200000000ull;  // 0.2 s bound on the abort path
+
+struct Params {
+  __nv_bfloat16 *o;
+  float *lse;
+  const int32_t *row_ptr;  // sparse CSR (nullptr: full mode only)
+  const int32_t *col_idx;
+  const int32_t *mode;     // per-batch mode on device, or nullptr
+  int32_t *status;
+  int B, S, Hq, G;
+  int n_qtiles, nqb;
+  int mode_default;
+  float scale_log2;        // scale * log2(e)
+};
+
+// Walks the 128-key tiles a 128-row query tile (query blocks 2qt, 2qt+1)
+// attends, ascending, each with a 4-bit block mask: bit 2*qs + ks is set iff
+// query block 2qt+qs may attend key block 2n+ks.  FULL mode: tiles 0..qt with
+// every bit set.  SPARSE mode: the union of the two CSR rows; an entry outside
+// [0, own block] or not ascending is skipped and reported.
+struct TileIter {
+  const int32_t *col;
+  int32_t *status;
+  int p0, e0, p1, e1, last0, last1, qb0;
+  int n, n_end;
+  bool full;
+
+  FA_DEV void init(const Params &p, int qt, bool sparse) {
+    status = p.status;
+    full = !sparse;
+    n = 0;
+    n_end = qt + 1;
+    qb0 = 2 * qt;
+    col = p.col_idx;
+    last0 = last1 = -1;
+    p0 = e0 = p1 = e1 = 0;
+    if (sparse) {
+      p0 = p.row_ptr[qb0];
+      e0 = p.row_ptr[qb0 + 1];
+      if (qb0 + 1 < p.nqb) {
+        p1 = e0;
+        e1 = p.row_ptr[qb0 + 2];
+      }
+    }
+  }
+  FA_DEV int peek(int &pp, int e, int last, int own) {
+    while (pp < e) {
+      const int c = __ldg(col + pp);
+      if (c >= 0 && c <= own && c > last) return c;
+      report(status, FA_DEV_BAD_INDEX);
+      ++pp;
+    }
+    return 0x7fffffff;
+  }
+  FA_DEV bool next(int &tile, uint32_t &bits) {
+    if (full) {
+      if (n >= n_end) return false;
+      tile = n++;
+      bits = 0xFu;
+      return true;
+    }
+    int c0 = peek(p0, e0, last0, qb0);
+    int c1 = peek(p1, e1, last1, qb0 + 1);
+    const int t = min(c0 >> 1, c1 >> 1);
+    if (t >= (0x7fffffff >> 1)) return false;
+    bits = 0;
+    while (c0 >> 1 == t) {
+      bits |= 1u << (c0 & 1);
+      last0 = c0;
+      ++p0;
+      c0 = peek(p0, e0, last0, qb0);
+    }
+    while (c1 >> 1 == t) {
+      bits |= 1u << (2 + (c1 & 1));
+      last1 = c1;
+      ++p1;
+      c1 = peek(p1, e1, last1, qb0 + 1);
+    }
+    tile = t;
+    return true;
+  }
+};
+
+struct Shared {
+  uint8_t *q;
+  uint8_t *ring;
+  uint64_t *q_full, *full, *empty, *s_full, *p_full, *pv_done, *drain;
+  uint32_t *tmem_slot;
+  volatile int *abort;
+};
+
+FA_DEV Shared carve(uint8_t *raw) {
+  Shared s;
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  s.q = base;
+  s.ring = base + TILE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + TILE_BYTES + NSLOT * TILE_BYTES);
+  s.q_full = bars;
+  s.full = bars + 1;
+  s.empty = s.full + NSLOT;
+  s.s_full = s.empty + NSLOT;
+  s.p_full = s.s_full + 2;
+  s.pv_done = s.p_full + 2;
+  s.drain = s.pv_done + 2;
+  s.tmem_slot = reinterpret_cast<uint32_t *>(s.drain + 1);
+  s.abort = reinterpret_cast<volatile int *>(s.tmem_slot + 1);
+  return s;
+}
+
+// ------------------------------------------------------------- producer ---
+FA_DEV void run_producer(const Shared &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                         const CUtensorMap *tmV, const Params &p, int qt, int b, int h,
+                         int kvh, bool sparse) {
+  mbar_arrive_expect_tx(sh.q_full, TILE_BYTES);
+  tma_load_4d(sh.q, tmQ, sh.q_full, 0, h, qt * BM, b);
+  tma_load_4d(sh.q + HALF_BYTES, tmQ, sh.q_full, 64, h, qt * BM, b);
+
+  TileIter it;
+  it.init(p, qt, sparse);
+  int li = 0;  // loads issued, in consumption order
+  auto load = [&](const CUtensorMap *map, int n) -> bool {
+    const int slot = li % NSLOT;
+    const uint32_t round = static_cast<uint32_t>(li / NSLOT);
+    if (!mbar_wait(&sh.empty[slot], (round & 1u) ^ 1u, sh.abort, p.status)) return false;
+    uint8_t *dst = sh.ring + slot * TILE_BYTES;
+    mbar_arrive_expect_tx(&sh.full[slot], TILE_BYTES);
+    tma_load_4d(dst, map, &sh.full[slot], 0, kvh, n * BN, b);
+    tma_load_4d(dst + HALF_BYTES, map, &sh.full[slot], 64, kvh, n * BN, b);
+    ++li;
+    return true;
+  };
+  int n_cur = 0;
+  uint32_t bits;
+  bool has = it.next(n_cur, bits);
+  bool ok = !has || load(tmK, n_cur);
+  while (ok && has) {
+    int n_next = 0;
+    const bool has_next = it.next(n_next, bits);
+    if (has_next && !load(tmK, n_next)) break;
+    if (!load(tmV, n_cur)) break;
+    n_cur = n_next;
+    has = has_next;
+  }
+  if (*sh.abort) {  // let every copy this thread issued land before exit
+    mbar_wait_drain(sh.q_full, 0, kDrainNs);
+    for (int x = (li > NSLOT ? li - NSLOT : 0); x < li; ++x)
+      mbar_wait_drain(&sh.full[x % NSLOT], static_cast<uint32_t>(x / NSLOT) & 1u, kDrainNs);
+  }
+}
+
+// ------------------------------------------------------------------ MMA ---
+FA_DEV void run_mma(const Shared &sh, uint32_t tmem, const Params &p, int qt, bool sparse) {
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);  // B = K tile, K-major
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);   // B = V tile, MN-major
+  bool ok = mbar_wait(sh.q_full, 0, sh.abort, p.status);
+  tc_fence_after_sync();
+  const uint32_t q_addr = smem_u32(sh.q);
+  int ci = 0;  // ring slots consumed
+  auto qk = [&](int j) -> bool {
+    const int slot = ci % NSLOT;
+    const uint32_t round = static_cast<uint32_t>(ci / NSLOT);
+    ++ci;
+    if (!mbar_wait(&sh.full[slot], round & 1u, sh.abort, p.status)) return false;
+    tc_fence_after_sync();
+    const uint32_t k_addr = smem_u32(sh.ring + slot * TILE_BYTES);
+    const uint32_t d = tmem + ((j & 1) ? TM_S1 : TM_S0);
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+      // 16 bf16 = 32 bytes per K step inside a 128-byte swizzled row; the
+      // second 64 columns live in the second TMA box.
+      const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+      mma_bf16_ss(d, smem_desc_sw128(q_addr + off, 16, 1024),
+                  smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+    }
+    tc_commit(&sh.empty[slot]);
+    tc_commit(&sh.s_full[j & 1]);
+    return true;
+  };
+  auto pv = [&](int j) -> bool {
+    if (!mbar_wait(&sh.p_full[j & 1], static_cast<uint32_t>(j >> 1) & 1u, sh.abort, p.status))
+      return false;
+    const int slot = ci % NSLOT;
+    const uint32_t round = static_cast<uint32_t>(ci / NSLOT);
+    ++ci;
+    if (!mbar_wait(&sh.full[slot], round & 1u, sh.abort, p.status)) return false;
+    tc_fence_after_sync();
+    const uint32_t v_addr = smem_u32(sh.ring + slot * TILE_BYTES);
+    const uint32_t a = tmem + ((j & 1) ? TM_P1 : TM_P0);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk) {
+      // V tile [key][dim]: dims are the MN (N) mode, keys the K mode.  One K
+      // step = 16 keys = two 8-row atoms (2048 bytes); the two 64-dim halves
+      // are one TMA box (16 KB) apart (leading byte offset).
+      mma_bf16_ts(tmem + TM_O, a + kk * 8, smem_desc_sw128(v_addr + kk * 2048, HALF_BYTES, 1024),
+                  kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+    }
+    tc_commit(&sh.empty[slot]);
+    tc_commit(&sh.pv_done[j & 1]);
+    return true;
+  };
+
+  TileIter it;
+  it.init(p, qt, sparse);
+  int n_cur = 0;
+  uint32_t bits;
+  bool has = ok && it.next(n_cur, bits);
+  if (has) ok = qk(0);
+  for (int j = 0; ok && has; ++j) {
+    int n_next = 0;
+    const bool has_next = it.next(n_next, bits);
+    if (has_next && !(ok = qk(j + 1))) break;
+    if (!(ok = pv(j))) break;
+    has = has_next;
+  }
+  if (*sh.abort) {  // let every MMA this thread issued finish before exit
+    tc_commit(sh.drain);
+    mbar_wait_drain(sh.drain, 0, kDrainNs);
+  }
+}
+
+// -------------------------------------------------------------- softmax ---
+// A wait whose result is the same for every lane of the warp (the TMEM
+// loads and stores it guards are warp-collective).
+FA_DEV bool warp_wait(uint64_t *bar, uint32_t parity, const Shared &sh, const Params &p) {
+  const bool done = mbar_wait(bar, parity, sh.abort, p.status);
+  return __all_sync(0xffffffffu, done);
+}
+
+FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt, int b, int h,
+                        bool sparse) {
+  const int r = threadIdx.x - 128;                  // row within the tile
+  const uint32_t quad = (threadIdx.x >> 5) & 3u;     // TMEM lanes 32*quad..
+  const uint32_t lane_base = tmem + ((quad * 32u) << 16);
+  const float c = p.scale_log2;
+  float m_run = -INFINITY, l_run = 0.f;
+
+  TileIter it;
+  it.init(p, qt, sparse);
+  int j = 0, n = 0;
+  uint32_t bits = 0;
+  bool ok = true;
+  while (it.next(n, bits)) {
+    if (!warp_wait(&sh.s_full[j & 1], static_cast<uint32_t>(j >> 1) & 1u, sh, p)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after_sync();
+    float s[BN];
+    {
+      const uint32_t sa = lane_base + ((j & 1) ? TM_S1 : TM_S0);
+#pragma unroll
+      for (int q4 = 0; q4 < BN / 32; ++q4) {
+        uint32_t raw[32];
+        tmem_ld32(sa + q4 * 32, raw);
+        tmem_ld_wait(raw);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(raw[i]);
+      }
+    }
+    const bool diag = (n == qt);
+    if (diag || bits != 0xFu) {
+      const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
+#pragma unroll
+      for (int i = 0; i < BN; ++i) {
+        const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
+        s[i] = keep ? s[i] : -INFINITY;
+      }
+    }
+    float mx8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+    for (int i = 8; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+    float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+    const float m_tile = mx * c;
+    const float m_new = fmaxf(m_run, m_tile);
+    const bool need = m_new > m_run + kRescaleThreshold;
+    if (j > 0 && __any_sync(0xffffffffu, need)) {
+      // O holds sum_{k<j} exp2(s*c - m_run) V; bring it to the new max.  The
+      // previous PV must have landed first.
+      if (!warp_wait(&sh.pv_done[(j - 1) & 1], static_cast<uint32_t>((j - 1) >> 1) & 1u, sh, p)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const float alpha = need ? ex2(m_run - m_new) : 1.0f;
+#pragma unroll
+      for (int q4 = 0; q4 < HD / 32; ++q4) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + TM_O + q4 * 32, o);
+        tmem_ld_wait(o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        tmem_st32(lane_base + TM_O + q4 * 32, o);
+      }
+      tmem_st_wait();
+    }
+    if (need) {
+      l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
+      m_run = m_new;
+    }
+    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+    float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < BN; ++i) {
+      s[i] = ex2(fmaf(s[i], c, -m_use));
+      sum4[i & 3] += s[i];
+    }
+    l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+    // P buffer j&1 was last read by PV(j-2).
+    if (j >= 2 && !warp_wait(&sh.pv_done[j & 1], static_cast<uint32_t>((j - 2) >> 1) & 1u, sh, p)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after_sync();
+    {
+      const uint32_t pa = lane_base + ((j & 1) ? TM_P1 : TM_P0);
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[q2 * 64 + 2 * i], s[q2 * 64 + 2 * i + 1]);
+        tmem_st32(pa + q2 * 32, pk);
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before_sync();
+    mbar_arrive(&sh.p_full[j & 1]);
+    ++j;
+  }
+
+  // Epilogue: O / l -> bf16, one row per thread.
+  const bool have_o =
+      ok && j > 0 &&
+      warp_wait(&sh.pv_done[(j - 1) & 1], static_cast<uint32_t>((j - 1) >> 1) & 1u, sh, p);
+  tc_fence_after_sync();
+  const int t = qt * BM + r;
+  const bool store = (t < p.S) && !*sh.abort;
+  const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+  __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.S + t) * p.Hq + h) * HD;
+#pragma unroll
+  for (int q4 = 0; q4 < HD / 32; ++q4) {
+    uint32_t o[32];
+    if (have_o) {
+      tmem_ld32(lane_base + TM_O + q4 * 32, o);
+      tmem_ld_wait(o);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = 0u;
+    }
+    if (store) {
+      uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+        w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+        w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+        w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+        dst[v] = w;
+      }
+    }
+  }
+  if (store && p.lse) {
+    const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + t] = lse;
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const Shared sh = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // CTA -> (query tile, batch, head): longest causal rows first; the query
+  // heads of one KV group run side by side so K/V tiles are shared in L2.
+  const int bh = p.B * p.Hq;
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / bh;
+  const int rem = static_cast<int>(blockIdx.x) % bh;
+  const int b = rem / p.Hq, h = rem % p.Hq, kvh = h / p.G;
+  const int mode = p.mode ? p.mode[b] : p.mode_default;
+  const bool sparse = (mode == FA_MODE_SPARSE) && p.row_ptr != nullptr;
+
+  if (threadIdx.x == 0) {
+    mbar_init(sh.q_full, 1);
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.s_full[i], 1);
+      mbar_init(&sh.p_full[i], 128);
+      mbar_init(&sh.pv_done[i], 1);
+    }
+    mbar_init(sh.drain, 1);
+    *sh.abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(sh.tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *sh.tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) run_producer(sh, &tmQ, &tmK, &tmV, p, qt, b, h, kvh, sparse);
+  } else if (warp == 1) {
+    if (lane == 0) run_mma(sh, tmem, p, qt, sparse);
+    __syncwarp();
+  } else if (warp >= 4) {
+    run_softmax(sh, tmem, p, qt, b, h, sparse);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace prefill
+
+// ----------------------------------------------------------------- host ---
+int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
+  using namespace prefill;
+  CUtensorMap tmQ, tmK, tmV;
+  if (make_tmap_bhsd(&tmQ, a.q, a.B, a.S, a.Hq, 64, BM) != 0) return FA_ERR_CUDA;
+  if (make_tmap_bhsd(&tmK, a.k, a.B, a.S, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
+  if (make_tmap_bhsd(&tmV, a.v, a.B, a.S, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return FA_ERR_CUDA;
+    attr_done = true;
+  }
+  Params p;
+  p.o = reinterpret_cast<__nv_bfloat16 *>(a.o);
+  p.lse = a.lse;
+  p.row_ptr = a.row_ptr;
+  p.col_idx = a.col_idx;
+  p.mode = a.mode_dev;
+  p.status = a.status;
+  p.B = a.B;
+  p.S = a.S;
+  p.Hq = a.Hq;
+  p.G = a.Hq / a.Hkv;
+  p.n_qtiles = (a.S + BM - 1) / BM;
+  p.nqb = (a.S + 63) / 64;
+  p.mode_default = a.mode_default;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  const long long grid = static_cast<long long>(p.n_qtiles) * a.B * a.Hq;
+  if (grid <= 0 || grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  prefill_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace fa

@@ -1,0 +1,171 @@
+/*
+ * fa_hybrid.h -- C ABI of the layer-routed hybrid attention library
+ * (libfa_hybrid.so, hand-written CUDA kernels for B200 / sm_100a).
+ *
+ * The method ("Flux Attention: 효율적인 LLM 추론을 위한 문맥 인식형 하이브리드
+ * 어텐션", router and implementation paragraphs): a layer router mean-pools the
+ * first and last 100 query tokens of a layer, an MLP context encoder and a
+ * router head give two logits pi_FA and pi_SA, the argmax picks the layer's
+ * mode, and the layer then runs either exact causal attention or block-sparse
+ * attention over 64-token blocks (sink blocks plus a local window).  A sparse
+ * layer never loads the KV blocks outside its pattern.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensor pointers are DEVICE memory owned by the caller.  The library
+ *    allocates nothing, keeps no state between calls and never synchronises.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call only enqueues work on it.
+ *  - The return value reports host-side argument checks and launch errors
+ *    (fa_status).  On any non-zero return nothing was launched, except
+ *    FA_ERR_CUDA, which reports a failed launch.
+ *  - Device-side failures (a bounded wait that ran out, an index outside the
+ *    query's causal range) are OR-ed into the caller's int32 `dev_status`
+ *    (nullable) as FA_DEV_* bits; the caller zeroes it, synchronises, reads it.
+ *  - bf16 tensors are row-major with these layouts:
+ *      prefill Q, O [B, S, Hq, D];  K, V [B, S, Hkv, D];  LSE fp32 [B, Hq, S]
+ *      decode  q, o [B, Hq, D];     K/V caches [B, Lmax, Hkv, D]
+ *    Every pointer must be 16-byte aligned.  D must be 128.  Hq % Hkv == 0
+ *    and the query head h reads KV head h / (Hq / Hkv).
+ *  - Scores are scale * (q . k); the usual scale is 1/sqrt(D) ("Self-Attention
+ *    이후", section "셀프 어텐션이 비싼 이유": Q K^T divided by sqrt(d_k)).
+ */
+#ifndef FA_HYBRID_H
+#define FA_HYBRID_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = -1,   /* null pointer, bad size, misaligned pointer */
+    FA_ERR_UNSUPPORTED = -2,   /* valid but not built: D != 128, G > 8, ... */
+    FA_ERR_WORKSPACE = -3,     /* workspace missing or smaller than required */
+    FA_ERR_CUDA = -4,          /* a CUDA launch or driver call failed */
+    FA_ERR_TIMEOUT = -5        /* reserved for host-side waits (none today) */
+} fa_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define FA_DEV_TIMEOUT   1     /* a bounded wait ran out; outputs invalid */
+#define FA_DEV_BAD_INDEX 2     /* a block index outside [0, query block] or
+                                  out of order was skipped */
+
+typedef enum { FA_MODE_FULL = 0, FA_MODE_SPARSE = 1 } fa_mode;
+
+/* Sparse pattern, in tokens: block = 64 ("Flux Attention", implementation
+ * paragraph: 64-token blocks), sink = 128 sink tokens, window = local window
+ * counted in whole blocks and including the query's own block.  sink and
+ * window must be multiples of block; window >= block. */
+typedef struct {
+    int32_t block;
+    int32_t sink;
+    int32_t window;
+} fa_sparse_cfg;
+
+/* Human-readable name of a fa_status value; never NULL. */
+FA_API const char *fa_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+FA_API int fa_version(void);
+
+/* ------------------------------------------------------------ router ---
+ * "Flux Attention", router paragraphs: pool tokens [0, n_head) and
+ * [S - n_tail, S) of Q (mean, fp32), flatten head-major to x[h*D + d],
+ * hidden = ReLU(W1 x + b1), [pi_FA, pi_SA] = W2 hidden + b2, and
+ * mode = FA_MODE_SPARSE iff pi_SA > pi_FA (a tie routes to FULL).
+ *   q        bf16 [B, S, Hq, D], device
+ *   w1       fp32 [hidden, Hq*D], b1 fp32 [hidden], w2 fp32 [2, hidden],
+ *            b2 fp32 [2]; device; b1/b2 may be NULL (zero bias)
+ *   logits_out fp32 [B, 2] (pi_FA, pi_SA); mode_out int32 [B]; device
+ *   workspace  >= fa_router_workspace_size(B, Hq, D, hidden) bytes, device
+ * Requires S >= n_head + n_tail, n_head + n_tail >= 1, 1 <= hidden <= 65536. */
+FA_API size_t fa_router_workspace_size(int B, int Hq, int D, int hidden);
+FA_API int fa_router_decide(const void *q, int B, int S, int Hq, int D,
+                     int n_head_tok, int n_tail_tok,
+                     const float *w1, const float *b1, int hidden,
+                     const float *w2, const float *b2,
+                     float *logits_out, int32_t *mode_out,
+                     void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------- index ---
+ * CSR of the key blocks each query block keeps ("Flux Attention",
+ * implementation paragraph): row i (query block i, nqb = ceil(S/block) rows)
+ * lists, ascending, the sink blocks j < sink/block (j <= i) and the window
+ * blocks i - window/block + 1 .. i, each once.
+ * fa_blocksparse_index_size is host arithmetic only (no device access). */
+FA_API int fa_blocksparse_index_size(int S, fa_sparse_cfg cfg, int *n_rows, int *nnz);
+/*   row_ptr int32 [n_rows + 1], col_idx int32 [nnz]; device. */
+FA_API int fa_blocksparse_index(int S, fa_sparse_cfg cfg, int32_t *row_ptr,
+                         int32_t *col_idx, void *stream);
+
+/* ----------------------------------------------------------- prefill ---
+ * Exact causal attention, FlashAttention-style: tiles of QK^T on the tensor
+ * cores, online softmax with a running max and sum rescaled by
+ * exp(m_old - m_new) (newsletter on Softmax/FlashAttention, section on
+ * Online Softmax), then PV; the S x S matrix never reaches memory.
+ *   o   bf16 [B, S, Hq, D]; lse fp32 [B, Hq, S] or NULL (natural log of the
+ *       softmax denominator of scale*q.k, -inf for a row with no key).
+ *   Any S >= 1.  dev_status: see conventions. */
+FA_API int fa_attn_prefill_full(const void *q, const void *k, const void *v, void *o,
+                         float *lse, int B, int S, int Hq, int Hkv, int D,
+                         float scale, int32_t *dev_status, void *stream);
+
+/* Block-sparse attention: query block i attends only the key blocks of CSR
+ * row i (row_ptr int32 [ceil(S/block) + 1], col_idx ascending per row, every
+ * entry in [0, i]); causal masking inside the diagonal block.  KV blocks
+ * outside the list are never loaded.  block must be 64.  An all-ones lower
+ * triangle reproduces fa_attn_prefill_full. */
+FA_API int fa_attn_prefill_blocksparse(const void *q, const void *k, const void *v,
+                                void *o, float *lse, int B, int S, int Hq,
+                                int Hkv, int D, float scale,
+                                const int32_t *row_ptr, const int32_t *col_idx,
+                                int block, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------ decode ---
+ * One query token per sequence at position L-1, L = seqlens[b] (device int32
+ * [B], 1 <= L <= Lmax; the cache holds L tokens including the current one).
+ * FULL attends keys 0..L-1; SPARSE attends the keys the prefill block rule
+ * keeps for row L-1 and loads no other KV block ("Flux Attention": a sparse
+ * layer bypasses the KV cache outside its pattern).
+ *   mode_dev: NULL to use `mode` for every sequence, else device int32 [B]
+ *   (e.g. the router's mode_out) read on the device.
+ *   o bf16 [B, Hq, D]; lse fp32 [B, Hq] or NULL.
+ *   workspace >= fa_decode_workspace_size(B, Hq, Hkv, Lmax, D) bytes, device.
+ * Split-KV: partial (max, sum, output) per split, merged by log-sum-exp. */
+FA_API size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
+FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
+                   const int32_t *seqlens, int B, int Lmax, int Hq, int Hkv,
+                   int D, float scale, int mode, const int32_t *mode_dev,
+                   fa_sparse_cfg cfg, void *o, float *lse, void *workspace,
+                   size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------ hybrid ---
+ * One routed layer: fa_router_decide on this layer's Q, then one attention
+ * launch that reads the mode from device memory per sequence (no host sync)
+ * and runs exact causal attention (FULL) or block-sparse attention over the
+ * caller's CSR (SPARSE; build it once with fa_blocksparse_index for this S and
+ * cfg).  Arguments as for the calls above; n_head/n_tail are 100/100.
+ *   workspace >= fa_hybrid_workspace_size(B, Hq, D, hidden) bytes. */
+FA_API size_t fa_hybrid_workspace_size(int B, int Hq, int D, int hidden);
+FA_API int fa_hybrid_layer(const void *q, const void *k, const void *v, void *o,
+                    float *lse, int B, int S, int Hq, int Hkv, int D,
+                    float scale, const float *w1, const float *b1, int hidden,
+                    const float *w2, const float *b2, fa_sparse_cfg cfg,
+                    const int32_t *row_ptr, const int32_t *col_idx,
+                    float *logits_out, int32_t *mode_out, void *workspace,
+                    size_t ws_bytes, int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_HYBRID_H */
