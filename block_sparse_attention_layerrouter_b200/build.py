@@ -11,7 +11,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa_hybrid.so")
-SOURCES = ["fa_api.cu", "fa_router.cu", "fa_index.cu", "fa_prefill.cu", "fa_decode.cu"]
+SOURCES = ["fa_api.cu", "fa_router.cu", "fa_index.cu", "fa_prefill.cu", "fa_decode.cu",
+           "fa_noalloc.cu"]
 HEADERS = ["fa_common.cuh", "fa_internal.h", os.path.join("..", "..", "include", "fa_hybrid.h")]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

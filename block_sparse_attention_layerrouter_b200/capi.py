@@ -57,6 +57,9 @@ _SIGNATURES = {
     "fa_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_attn_decode": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, SparseCfg, _VP,
                             _VP, _VP, _SZ, _VP, _VP]),
+    "fa_noalloc_scratch_bytes": (_SZ, []),
+    "fa_attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP,
+                                    SparseCfg, _VP, _VP, _VP, _VP]),
     "fa_hybrid_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_hybrid_layer": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
                              _VP, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
@@ -230,6 +233,33 @@ def attn_decode(q, kcache, vcache, seqlens, mode=FA_MODE_FULL, c: Optional[Spars
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _ptr(status), _stream(q.device))
     _check("fa_attn_decode", rc)
+    return o
+
+
+def attn_decode_noalloc(q, kcache, vcache, seqlens, mode=FA_MODE_FULL,
+                        c: Optional[SparseCfg] = None, scale=None, mode_dev=None, o=None,
+                        lse=None, status=None) -> torch.Tensor:
+    """fa_attn_decode_noalloc: decode with the library's static scratch (for
+    callers that cannot allocate a workspace).  Raises ValueError when the
+    shape needs more scratch than the library holds."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, D = q.shape
+    Lmax, Hkv = kcache.shape[1], kcache.shape[2]
+    need = decode_workspace_size(B, Hq, Hkv, Lmax, D)
+    cap = int(lib().fa_noalloc_scratch_bytes())
+    if need > cap:
+        raise ValueError("decode needs %d bytes of scratch; the static scratch holds %d"
+                         % (need, cap))
+    c = cfg() if c is None else c
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    o = torch.empty_like(q) if o is None else o
+    rc = lib().fa_attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), B,
+                                      Lmax, Hq, Hkv, D, scale, int(mode), _ptr(mode_dev), c,
+                                      _ptr(o), _ptr(lse), _ptr(status), _stream(q.device))
+    _check("fa_attn_decode_noalloc", rc)
     return o
 
 

@@ -148,6 +148,30 @@ FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
                    fa_sparse_cfg cfg, void *o, float *lse, void *workspace,
                    size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/* ------------------------------------------- decode without allocation ---
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory where they run decode (a plugin behind
+ * a fixed operator interface with no workspace argument, an engine whose
+ * memory is all reserved up front, a real-time loop where cudaMalloc is not
+ * allowed).  Same arguments and results as fa_attn_decode without the
+ * workspace: the split-KV scratch lives in one static device array of
+ * fa_noalloc_scratch_bytes() (8 MiB) that every GPU loading this library
+ * holds until exit.  The call allocates nothing.
+ *  - Returns FA_ERR_UNSUPPORTED when the shape needs more scratch than that
+ *    (fa_decode_workspace_size(B, Hq, Hkv, Lmax, D) > 8 MiB).
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address once; make it before any stream capture.
+ *  - All calls share the array (nothing in it needs to start at zero): calls
+ *    whose kernels overlap on the GPU race and must be serialised. */
+FA_API size_t fa_noalloc_scratch_bytes(void);
+FA_API int fa_attn_decode_noalloc(const void *q, const void *kcache,
+                                  const void *vcache, const int32_t *seqlens,
+                                  int B, int Lmax, int Hq, int Hkv, int D,
+                                  float scale, int mode,
+                                  const int32_t *mode_dev, fa_sparse_cfg cfg,
+                                  void *o, float *lse, int32_t *dev_status,
+                                  void *stream);
+
 /* ------------------------------------------------------------ hybrid ---
  * One routed layer: fa_router_decide on this layer's Q, then one attention
  * launch that reads the mode from device memory per sequence (no host sync)
