@@ -169,22 +169,37 @@ def dist_env():
 
 
 # -------------------------------------------------------------- our arm
+def stack_plan(wl):
+    """(number of layers, set of SPARSE layers, decode token per layer?,
+    rotated input sets) of one step of a prefill workload."""
+    if wl.layers > 1:     # routed stack: a seeded half of the layers biased to SPARSE
+        rng = np.random.default_rng(wl.seed)
+        sparse = set(rng.choice(wl.layers, size=wl.layers // 2, replace=False).tolist())
+        return wl.layers, sparse, False, 1
+    if wl.S >= 65536:     # one layer per mode at long context
+        return 2, {1}, False, 1
+    return 2, {1}, True, N_INPUT_SETS
+
+
 class Step:
     """Device buffers of one input set and the launches of one step."""
 
-    def __init__(self, wl, seed, dev, capi, inputs, pinned=False):
-        self.wl, self.dev = wl, dev
+    def __init__(self, wl, seed, dev, capi, inputs, n_layers=2, sparse_layers=(1,),
+                 with_decode=True):
+        self.wl, self.dev, self.with_decode = wl, dev, with_decode
         B, S, Hq, Hkv = wl.B, wl.S, wl.Hq, wl.Hkv
         self.layers = []
-        for li, bias in enumerate(((0.1, 0.0), (0.0, 0.1))):   # FULL, SPARSE
+        for li in range(n_layers):
+            bias = (0.0, 0.1) if li in sparse_layers else (0.1, 0.0)
             q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, seed + 7919 * li, device=dev)
             w1, b1, w2, b2 = inputs.router_weights(Hq * 128, wl.hidden, seed, li, b2=bias)
-            qd = inputs.randn_bf16((B, Hq, 128), seed + 31 * li + 5, device=dev)
-            self.layers.append(dict(q=q, k=k, v=v, w1=w1.to(dev), b1=b1.to(dev), w2=w2.to(dev),
-                                    b2=b2.to(dev), o=torch.empty_like(q), qd=qd,
-                                    od=torch.empty_like(qd),
-                                    logits=torch.empty(B, 2, device=dev),
-                                    mode=torch.empty(B, dtype=torch.int32, device=dev)))
+            lay = dict(q=q, k=k, v=v, w1=w1.to(dev), b1=b1.to(dev), w2=w2.to(dev), b2=b2.to(dev),
+                       o=torch.empty_like(q), logits=torch.empty(B, 2, device=dev),
+                       mode=torch.empty(B, dtype=torch.int32, device=dev), sparse=li in sparse_layers)
+            if with_decode:
+                lay["qd"] = inputs.randn_bf16((B, Hq, 128), seed + 31 * li + 5, device=dev)
+                lay["od"] = torch.empty_like(lay["qd"])
+            self.layers.append(lay)
         self.c = capi.cfg(64, wl.sink, wl.window)
         rows, nnz = capi.blocksparse_index_size(S, self.c)
         self.row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
@@ -196,29 +211,41 @@ class Step:
         self.seqlens = torch.full((B,), S, dtype=torch.int32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.capi = capi
+        self.launches = 1 + 4 * n_layers + (2 * n_layers if with_decode else 0)
 
     def run(self, ev=None):
-        """Enqueue one step.  ev: optional (start, end) events around the
-        FULL layer's attention launch."""
+        """Enqueue one step.  ev: optional {layer: (start, end)} events
+        recorded around that layer's routed attention call."""
         capi, c = self.capi, self.c
         L = capi.lib()
-        st = capi._stream(self.dev)
-        rc = L.fa_blocksparse_index(self.wl.S, c, capi._ptr(self.row_ptr), capi._ptr(self.col_idx),
-                                    st)
+        rc = L.fa_blocksparse_index(self.wl.S, c, capi._ptr(self.row_ptr),
+                                    capi._ptr(self.col_idx), capi._stream(self.dev))
         capi._check("fa_blocksparse_index", rc)
         for li, lay in enumerate(self.layers):
-            if ev is not None and li == 0:
-                ev[0].record()
+            e = ev.get(li) if ev else None
+            if e is not None:
+                e[0].record()
             capi.hybrid_layer(lay["q"], lay["k"], lay["v"], lay["w1"], lay["b1"], lay["w2"],
                               lay["b2"], self.row_ptr, self.col_idx, c, o=lay["o"],
                               logits=lay["logits"], mode=lay["mode"], workspace=self.ws,
                               status=self.status)
-            if ev is not None and li == 0:
-                ev[1].record()
-            capi.attn_decode(lay["qd"], lay["k"], lay["v"], self.seqlens, mode_dev=lay["mode"],
-                             c=c, o=lay["od"], workspace=self.dws, status=self.status)
+            if e is not None:
+                e[1].record()
+            if self.with_decode:
+                capi.attn_decode(lay["qd"], lay["k"], lay["v"], self.seqlens,
+                                 mode_dev=lay["mode"], c=c, o=lay["od"], workspace=self.dws,
+                                 status=self.status)
 
-    LAUNCHES_PER_STEP = 1 + 2 * (3 + 1) + 2 * 2   # index, 2x(router 3 + attn), 2x decode
+    def flops(self):
+        wl = self.wl
+        nf = sum(1 for l in self.layers if not l["sparse"])
+        ns = len(self.layers) - nf
+        f = nf * flops_full(wl) + ns * flops_sparse_exact(wl)
+        if self.with_decode:
+            keys = nf * decode_keys(wl.S, 0, wl.sink, wl.window) + \
+                ns * decode_keys(wl.S, 1, wl.sink, wl.window)
+            f += 4.0 * 128 * wl.Hq * wl.B * keys
+        return f
 
 
 def time_kernel_alone(fn, reps=5):
@@ -242,10 +269,11 @@ def cpu_baseline(wl, budget_s=15.0):
     B, S, Hq, Hkv = wl.B, wl.S, wl.Hq, wl.Hkv
     q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, wl.seed, device="cpu")
     qb, kb, vb = inputs.bits(q), inputs.bits(k), inputs.bits(v)
+    del q, k, v
     mask = oracle.rows_to_dense_mask(oracle.blocksparse_rows(S, 64, wl.sink, wl.window))
     rng = np.random.default_rng(wl.seed)
     flops, elapsed, nrows = 0.0, 0.0, 0
-    chunk = 64
+    chunk = 64 if S <= 32768 else 16
     oracle.attention_rows(qb, kb, vb, 0.1, np.array([[0, 0, 0]]))   # load + warm
     while elapsed < budget_s:
         ts = rng.integers(0, S, size=chunk)
@@ -256,10 +284,9 @@ def cpu_baseline(wl, budget_s=15.0):
         oracle.attention_rows(qb, kb, vb, 1 / math.sqrt(128), rows, mask)     # sparse layer rows
         elapsed += time.perf_counter() - t0
         full_pairs = float(np.sum(ts + 1))
-        kept = mask[ts // 64]                                                 # [chunk, nkb]
         sparse_pairs = 0.0
-        for t, krow in zip(ts, kept):
-            blocks = np.nonzero(krow)[0]
+        for t in ts:
+            blocks = np.nonzero(mask[t // 64])[0]
             sparse_pairs += float(np.sum(np.minimum(blocks * 64 + 64, t + 1) - blocks * 64))
         flops += 4.0 * 128 * (full_pairs + sparse_pairs)
         nrows += 2 * chunk
@@ -269,8 +296,8 @@ def cpu_baseline(wl, budget_s=15.0):
                       "once in the sparse layer) of %s, %.1f s" % (nrows, wl.name, elapsed)}
 
 
-def run_ours(args, wl):
-    from block_sparse_attention_layerrouter_b200 import build, capi, inputs
+def setup_device(args):
+    from block_sparse_attention_layerrouter_b200 import build, capi
     ws, rank, local = dist_env()
     if ws > 1 and not torch.distributed.is_initialized():
         from datetime import timedelta
@@ -282,110 +309,126 @@ def run_ours(args, wl):
     if ws > 1:
         torch.distributed.barrier()
     capi.lib()
+    return ws, rank, dev
 
-    sets = [Step(wl, wl.seed + 101 * i, dev, capi, inputs) for i in range(N_INPUT_SETS)]
-    torch.cuda.synchronize()
-    sampler = ClockSampler(dev)
-    sampler.start()
-    for i in range(args.warmup):
-        sets[i % N_INPUT_SETS].run()
+
+def sync_all(ws):
     torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    ev_full = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for i in range(args.steps):
-        sets[i % N_INPUT_SETS].run(ev_full[i])
-    t1.record()
-    torch.cuda.synchronize()
-    if ws > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    sampler.stop()
-    ms = t0.elapsed_time(t1)
-    ms_full = [s.elapsed_time(e) for s, e in ev_full]
-    status = max(int(s.status.item()) for s in sets)
-    modes = [int(l["mode"][0].item()) for l in sets[0].layers]
+
+
+def max_over_ranks(ms, ws, dev):
     if ws > 1:
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
+    return ms
 
-    # ---- end to end through the public API with host buffers
-    e2e = run_e2e(args, wl, dev, capi, inputs, ws)
 
-    # ---- components, each timed alone (for the breakdown; not the headline)
+def base_line(args, wl, ws, ms, unit, value):
+    return {"metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 Q/K/V; router weights N(0,0.02)); stands in "
+                    "for LongBench-E/RULER prompts of this shape"}
+
+
+def run_ours(args, wl):
+    from block_sparse_attention_layerrouter_b200 import capi, inputs
+    ws, rank, dev = setup_device(args)
+    n_layers, sparse_layers, with_decode, n_sets = stack_plan(wl)
+    sets = [Step(wl, wl.seed + 101 * i, dev, capi, inputs, n_layers, sparse_layers, with_decode)
+            for i in range(n_sets)]
+    full_layer = min(li for li in range(n_layers) if li not in sparse_layers)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for i in range(args.warmup):
+        sets[i % n_sets].run()
+    sync_all(ws)
+    ev_full = [{full_layer: (torch.cuda.Event(enable_timing=True),
+                             torch.cuda.Event(enable_timing=True))} for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        sets[i % n_sets].run(ev_full[i])
+    t1.record()
+    sync_all(ws)
+    sampler.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
+    ms_full = [e[full_layer][0].elapsed_time(e[full_layer][1]) for e in ev_full]
+    status = max(int(s.status.item()) for s in sets)
+    modes = [int(l["mode"][0].item()) for l in sets[0].layers]
+    want = [1 if li in sparse_layers else 0 for li in range(n_layers)]
+
+    e2e = run_e2e(args, wl, dev, capi, inputs, ws) if with_decode else None
+
+    # ---- components, each timed alone (breakdown only, not the headline)
     s0 = sets[0]
-    lay0, lay1 = s0.layers
+    lay_f = s0.layers[full_layer]
+    lay_s = s0.layers[min(sparse_layers)]
     comp = {}
     comp["prefill_full_ms"] = time_kernel_alone(
-        lambda: capi.attn_prefill_full(lay0["q"], lay0["k"], lay0["v"], o=lay0["o"]))
+        lambda: capi.attn_prefill_full(lay_f["q"], lay_f["k"], lay_f["v"], o=lay_f["o"]))
     comp["prefill_sparse_ms"] = time_kernel_alone(
-        lambda: capi.attn_prefill_blocksparse(lay1["q"], lay1["k"], lay1["v"], s0.row_ptr,
-                                              s0.col_idx, o=lay1["o"]))
+        lambda: capi.attn_prefill_blocksparse(lay_s["q"], lay_s["k"], lay_s["v"], s0.row_ptr,
+                                              s0.col_idx, o=lay_s["o"]))
     comp["router_ms"] = time_kernel_alone(
-        lambda: capi.router_decide(lay0["q"], lay0["w1"], lay0["b1"], lay0["w2"], lay0["b2"],
-                                   logits=lay0["logits"], mode=lay0["mode"], workspace=s0.ws))
-    for name, md in (("decode_full_ms", 0), ("decode_sparse_ms", 1)):
-        comp[name] = time_kernel_alone(
-            lambda md=md: capi.attn_decode(lay0["qd"], lay0["k"], lay0["v"], s0.seqlens, md,
-                                           s0.c, o=lay0["od"], workspace=s0.dws))
+        lambda: capi.router_decide(lay_f["q"], lay_f["w1"], lay_f["b1"], lay_f["w2"],
+                                   lay_f["b2"], logits=lay_f["logits"], mode=lay_f["mode"],
+                                   workspace=s0.ws))
     torch.cuda.synchronize()
-
     if rank != 0:
         return None
     hbm, peak_burst, peak_sust, peak_kind = measured_peaks()
     f_full = flops_full(wl)
     f_sparse = flops_sparse_exact(wl)
     f_sparse_exec = 4.0 * 128 * wl.Hq * wl.B * csr_nnz(wl.S, wl.sink, wl.window) * 64 * 64
-    keys_dec = decode_keys(wl.S, 0, wl.sink, wl.window) + decode_keys(wl.S, 1, wl.sink, wl.window)
-    f_dec = 4.0 * 128 * wl.Hq * wl.B * keys_dec
-    step_flops = f_full + f_sparse + f_dec
-    value = ws * step_flops / (ms / args.steps * 1e-3) / 1e12
+    value = ws * s0.flops() / (ms / args.steps * 1e-3) / 1e12
     avg_full_ms = statistics.mean(ms_full)
     achieved = f_full / (avg_full_ms * 1e-3) / 1e12
     traffic, traffic_wl = kernel_traffic()
-    dec_bytes_full = 2 * wl.B * wl.Hkv * 128 * 2 * wl.S
     comp.update({
         "prefill_full_tflops": f_full / (comp["prefill_full_ms"] * 1e-3) / 1e12,
         "prefill_sparse_exec_tflops": f_sparse_exec / (comp["prefill_sparse_ms"] * 1e-3) / 1e12,
+        "prefill_sparse_exec_frac_of_burst": f_sparse_exec / (comp["prefill_sparse_ms"] * 1e-3)
+        / 1e12 / peak_burst,
         "prefill_sparse_exact_tflops": f_sparse / (comp["prefill_sparse_ms"] * 1e-3) / 1e12,
-        "decode_full_gbs": dec_bytes_full / (comp["decode_full_ms"] * 1e-3) / 1e9,
-        "routed_modes": modes,
+        "routed_modes_match_plan": modes == want,
         "device_status": status,
     })
-    line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q/K/V; "
-        "router weights N(0,0.02)); stands in for LongBench-E/RULER prompts of this shape",
-        "config": {"workload": wl.name, "B": wl.B, "S": wl.S, "Hq": wl.Hq, "Hkv": wl.Hkv,
-                   "D": 128, "block": 64, "sink": wl.sink, "window": wl.window,
-                   "router": "%d->%d->2" % (wl.Hq * 128, wl.hidden),
-                   "step": "index + 2 routed layers (1 FULL, 1 SPARSE) + 1 decode token each",
-                   "parallelism": "replicas" if ws > 1 else "single GPU",
-                   "l2": "inputs larger than L2: %d rotated input sets, %.2f GB" % (
-                       N_INPUT_SETS, N_INPUT_SETS * sum(
-                           t.numel() * t.element_size() for t in
-                           (sets[0].layers[0]["q"], sets[0].layers[0]["k"],
-                            sets[0].layers[0]["v"], sets[0].layers[0]["o"])) * 2 / 1e9)},
-        "roofline": {"bound": "tensor", "kernel": "prefill_kernel (FULL layer)",
-                     "achieved": round(achieved, 2), "peak": peak_sust, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak_sust, 4),
-                     "peak_kind": "%s bf16 sustained" % peak_kind,
-                     "frac_of_burst_peak": round(achieved / peak_burst, 4),
-                     "traffic": traffic, "traffic_workload": traffic_wl,
-                     "algorithmic_flops_per_launch": f_full,
-                     "avg_launch_ms": round(avg_full_ms, 4)},
-        "e2e": e2e,
-        "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
-        "clocks": sampler.report(),
-        "components": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in comp.items()},
-    }
+    if wl.S >= 65536 or n_layers > 2:
+        tf, tsp = comp["prefill_full_ms"], comp["prefill_sparse_ms"]
+        nl = 36 if wl.S >= 65536 else n_layers
+        comp["hybrid_vs_full"] = {
+            "layers": nl, "split": "50/50", "t_full_layer_ms": tf, "t_sparse_layer_ms": tsp,
+            "hybrid_ms": nl / 2 * (tf + tsp), "all_full_ms": nl * tf,
+            "speedup": (nl * tf) / (nl / 2 * (tf + tsp))}
+    line = base_line(args, wl, ws, ms, "TFLOP/s", value)
+    line["config"] = {
+        "workload": wl.name, "B": wl.B, "S": wl.S, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": 128,
+        "block": 64, "sink": wl.sink, "window": wl.window,
+        "router": "%d->%d->2" % (wl.Hq * 128, wl.hidden),
+        "step": "index + %d routed layers (%d FULL, %d SPARSE)%s" % (
+            n_layers, n_layers - len(sparse_layers), len(sparse_layers),
+            " + 1 decode token each" if with_decode else ""),
+        "parallelism": "replicas" if ws > 1 else "single GPU",
+        "l2": "inputs larger than L2: %d input set(s) of %.2f GB" % (
+            n_sets, sum(t.numel() * t.element_size() for l in s0.layers
+                        for t in (l["q"], l["k"], l["v"], l["o"])) / 1e9)}
+    line["roofline"] = {
+        "bound": "tensor", "kernel": "prefill_kernel (a FULL layer of the step)",
+        "achieved": round(achieved, 2), "peak": peak_sust, "unit": "TFLOP/s",
+        "frac": round(achieved / peak_sust, 4), "peak_kind": "%s bf16 sustained" % peak_kind,
+        "frac_of_burst_peak": round(achieved / peak_burst, 4), "traffic": traffic,
+        "traffic_workload": traffic_wl, "algorithmic_flops_per_launch": f_full,
+        "avg_launch_ms": round(avg_full_ms, 4)}
+    line["e2e"] = e2e
+    line["gpu_launches"] = s0.launches * args.steps
+    line["clocks"] = sampler.report()
+    line["components"] = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in comp.items()}
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     return line
@@ -395,14 +438,13 @@ def run_e2e(args, wl, dev, capi, inputs, ws):
     """Same step through the public API with host buffers: per step, copy
     the two layers' Q/K/V and decode queries from pinned host memory, run,
     and read both layers' outputs back."""
-    host = []
-    for li in range(2):
-        q, k, v = inputs.qkv(wl.B, wl.S, wl.Hq, wl.Hkv, 128, wl.seed + 7919 * li)
-        qd = inputs.randn_bf16((wl.B, wl.Hq, 128), wl.seed + 31 * li + 5)
-        host.append([t.pin_memory() for t in (q, k, v, qd)])
     step = Step(wl, wl.seed, dev, capi, inputs)
-    outs = [(torch.empty_like(step.layers[i]["o"], device="cpu").pin_memory(),
-             torch.empty_like(step.layers[i]["od"], device="cpu").pin_memory()) for i in range(2)]
+    host = []
+    for lay in step.layers:
+        host.append([lay[n].cpu().pin_memory() for n in ("q", "k", "v", "qd")])
+    outs = [(torch.empty(lay["o"].shape, dtype=lay["o"].dtype).pin_memory(),
+             torch.empty(lay["od"].shape, dtype=lay["od"].dtype).pin_memory())
+            for lay in step.layers]
     h2d = sum(t.numel() * t.element_size() for hs in host for t in hs)
     d2h = sum(t.numel() * t.element_size() for o in outs for t in o)
 
@@ -417,25 +459,180 @@ def run_e2e(args, wl, dev, capi, inputs, ws):
 
     for _ in range(max(1, args.warmup)):
         one()
-    torch.cuda.synchronize()
-    if ws > 1:
-        torch.distributed.barrier()
+    sync_all(ws)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for _ in range(args.steps):
         one()
     e.record()
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e)
-    if ws > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    keys_dec = decode_keys(wl.S, 0, wl.sink, wl.window) + decode_keys(wl.S, 1, wl.sink, wl.window)
-    step_flops = flops_full(wl) + flops_sparse_exact(wl) + 4.0 * 128 * wl.Hq * wl.B * keys_dec
-    return {"value": round(ws * step_flops / (ms / args.steps * 1e-3) / 1e12, 3),
+    ms = max_over_ranks(s.elapsed_time(e), ws, dev)
+    return {"value": round(ws * step.flops() / (ms / args.steps * 1e-3) / 1e12, 3),
             "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / args.steps, 4)}
+
+
+# ------------------------------------------------------------ decode stack
+DECODE_CACHE_SETS = 8
+
+
+def run_decode(args, wl):
+    """Decode step of a 32-layer model: one token per sequence per layer,
+    layers alternating FULL / SPARSE (16 + 16, fixed by the router at
+    prefill).  Each layer reads its own KV cache; 8 distinct cache sets (4 GiB
+    each) are rotated over the 32 layers, so consecutive reads of one set are
+    8 layers (>= 16 GiB of other traffic) apart and come from HBM."""
+    from block_sparse_attention_layerrouter_b200 import capi, inputs
+    ws, rank, dev = setup_device(args)
+    B, L, Hq, Hkv = wl.B, wl.decode_len, wl.Hq, wl.Hkv
+    caches = []
+    for i in range(DECODE_CACHE_SETS):
+        _, kc, vc = inputs.decode_inputs(B, L, Hq, Hkv, 128, wl.seed + 17 * i, device=dev)
+        caches.append((kc, vc))
+    qs = [inputs.randn_bf16((B, Hq, 128), wl.seed + 1000 + li, device=dev)
+          for li in range(wl.layers)]
+    outs = [torch.empty_like(q) for q in qs]
+    sl = torch.full((B,), L, dtype=torch.int32, device=dev)
+    c = capi.cfg(64, wl.sink, wl.window)
+    wsb = torch.empty(capi.decode_workspace_size(B, Hq, Hkv, L), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    modes = [li % 2 for li in range(wl.layers)]      # 0 FULL, 1 SPARSE
+
+    def step(ev=None):
+        for li in range(wl.layers):
+            kc, vc = caches[li % DECODE_CACHE_SETS]
+            if ev is not None and li == 0:
+                ev[0].record()
+            capi.attn_decode(qs[li], kc, vc, sl, modes[li], c, o=outs[li], workspace=wsb,
+                             status=status)
+            if ev is not None and li == 0:
+                ev[1].record()
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    sync_all(ws)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record()
+    sync_all(ws)
+    sampler.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
+    full_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    sparse_ms = time_kernel_alone(lambda: capi.attn_decode(qs[1], *caches[1], sl, 1, c, o=outs[1],
+                                                           workspace=wsb))
+    # e2e: the caches are device-resident state; per step the 32 layers'
+    # query tokens go up from pinned host memory and their outputs come back.
+    hq = [q.cpu().pin_memory() for q in qs]
+    ho = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+
+    def step_e2e():
+        for li in range(wl.layers):
+            qs[li].copy_(hq[li], non_blocking=True)
+        step()
+        for li in range(wl.layers):
+            ho[li].copy_(outs[li], non_blocking=True)
+
+    for _ in range(2):
+        step_e2e()
+    sync_all(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step_e2e()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), ws, dev)
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    if rank != 0:
+        return None
+    hbm, _, _, peak_kind = measured_peaks()
+    kv_row = 2 * Hkv * 128 * 2                               # K and V bytes per token
+    qo = 2 * B * Hq * 128 * 2
+    full_bytes = B * kv_row * decode_keys(L, 0, wl.sink, wl.window) + qo
+    sparse_bytes = B * kv_row * decode_keys(L, 1, wl.sink, wl.window) + qo
+    step_bytes = sum(full_bytes if m == 0 else sparse_bytes for m in modes)
+    value = ws * step_bytes / (ms / args.steps * 1e-3) / 1e9
+    line = base_line(args, wl, ws, ms, "GB/s", value)
+    line["config"] = {"workload": wl.name, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv, "D": 128,
+                      "layers": wl.layers, "split": "16 FULL + 16 SPARSE (alternating)",
+                      "sink": wl.sink, "window": wl.window,
+                      "l2": "inputs larger than L2: %d cache sets of %.2f GB rotated" % (
+                          DECODE_CACHE_SETS, 2 * caches[0][0].numel() * 2 / 1e9)}
+    achieved = full_bytes / (full_ms * 1e-3) / 1e9
+    line["roofline"] = {"bound": "hbm", "kernel": "decode_kernel + combine (a FULL layer)",
+                        "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                        "frac": round(achieved / hbm, 4), "peak_kind": "%s HBM copy" % peak_kind,
+                        "traffic": None, "algorithmic_bytes_per_launch": full_bytes,
+                        "avg_launch_ms": round(full_ms, 4)}
+    line["e2e"] = {"value": round(ws * step_bytes / (ms_e2e / args.steps * 1e-3) / 1e9, 1),
+                   "unit": "GB/s", "h2d_bytes_per_step": sum(t.numel() * 2 for t in hq),
+                   "d2h_bytes_per_step": sum(t.numel() * 2 for t in ho),
+                   "note": "KV caches are device-resident decode state"}
+    line["gpu_launches"] = 2 * wl.layers * args.steps
+    line["clocks"] = sampler.report()
+    line["components"] = {
+        "decode_full_layer_ms": round(full_ms, 4), "decode_sparse_layer_ms": round(sparse_ms, 4),
+        "decode_sparse_gbs": round(sparse_bytes / (sparse_ms * 1e-3) / 1e9, 1),
+        "all_full_step_ms_est": round(wl.layers * full_ms, 3),
+        "hybrid_vs_all_full": round(wl.layers * full_ms / (ms / args.steps), 3)}
+    return line
+
+
+# ------------------------------------------------------- one kernel alone
+def run_only(args, wl):
+    """Runs a single kernel of the path `warmup + steps` times on the
+    workload's shapes (used for ncu captures and quick timing)."""
+    from block_sparse_attention_layerrouter_b200 import capi, inputs
+    ws, rank, dev = setup_device(args)
+    B, Hq, Hkv = wl.B, wl.Hq, wl.Hkv
+    S = wl.decode_len or wl.S
+    c = capi.cfg(64, wl.sink, wl.window)
+    if args.only.startswith("decode"):
+        q, kc, vc = inputs.decode_inputs(B, S, Hq, Hkv, 128, wl.seed, device=dev)
+        sl = torch.full((B,), S, dtype=torch.int32, device=dev)
+        wsb = torch.empty(capi.decode_workspace_size(B, Hq, Hkv, S), dtype=torch.uint8,
+                          device=dev)
+        md = 0 if args.only == "decode_full" else 1
+        o = torch.empty_like(q)
+        fn = lambda: capi.attn_decode(q, kc, vc, sl, md, c, o=o, workspace=wsb)  # noqa: E731
+        work = B * 2 * Hkv * 128 * 2 * decode_keys(S, md, wl.sink, wl.window) / 1e9
+        unit = "GB/s"
+    else:
+        q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, wl.seed, device=dev)
+        o = torch.empty_like(q)
+        rp, ci = capi.blocksparse_index(S, c, device=dev)
+        w1, b1, w2, b2 = [t.to(dev) for t in inputs.router_weights(Hq * 128, wl.hidden, wl.seed)]
+        unit = "TFLOP/s"
+        if args.only == "prefill_full":
+            fn = lambda: capi.attn_prefill_full(q, k, v, o=o)  # noqa: E731
+            work = flops_full(wl) / 1e12
+        elif args.only == "prefill_sparse":
+            fn = lambda: capi.attn_prefill_blocksparse(q, k, v, rp, ci, o=o)  # noqa: E731
+            work = 4.0 * 128 * Hq * B * csr_nnz(S, wl.sink, wl.window) * 4096 / 1e12
+        elif args.only == "router":
+            fn = lambda: capi.router_decide(q, w1, b1, w2, b2)  # noqa: E731
+            work = (B * 200 * Hq * 128 * 2 + w1.numel() * 4) / 1e9
+            unit = "GB/s"
+        else:
+            raise SystemExit("unknown --only " + args.only)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / args.steps
+    return {"only": args.only, "workload": wl.name, "ms": round(ms, 4),
+            "value": round(work / (ms * 1e-3), 2), "unit": unit, "steps": args.steps}
 
 
 # --------------------------------------------------------- reference arm
@@ -474,14 +671,21 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None,
+                    help="prefill_full | prefill_sparse | decode_full | decode_sparse | router")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from block_sparse_attention_layerrouter_b200.inputs import WORKLOADS
     wl = WORKLOADS[args.workload]
-    if wl.decode_len:
-        ap.error("the decode workload is measured by bench_decode in this file's sibling flags")
-    line = run_reference(args, wl) if args.impl == "reference" else run_ours(args, wl)
+    if args.impl == "reference":
+        line = run_reference(args, wl)
+    elif args.only:
+        line = run_only(args, wl)
+    elif wl.decode_len:
+        line = run_decode(args, wl)
+    else:
+        line = run_ours(args, wl)
     if line is not None:
         print(json.dumps(line), flush=True)
     if torch.distributed.is_available() and torch.distributed.is_initialized():

@@ -58,6 +58,11 @@ WORKLOADS = {
                                       layers=32, window=2048, hidden=256,
                                       decode_len=131072, seed=1004,
                                       notes="decode, 16 full + 16 sparse layers"),
+    # Profiling shape: the decode workload at a quarter of the context
+    # (1 GiB of K/V, still far above the 126 MB L2).
+    "decode-b8-l32768": Workload("decode-b8-l32768", B=8, S=1, Hq=32, Hkv=8, layers=2,
+                                 window=2048, hidden=256, decode_len=32768, seed=1005,
+                                 notes="decode profiling shape"),
 }
 
 
