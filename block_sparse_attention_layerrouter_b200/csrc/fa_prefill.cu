@@ -474,6 +474,387 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 }  // namespace prefill
 
+// =====================================================================
+// Two query tiles per CTA: the same 128-row tile of two query heads of one
+// GQA group (G even).  Both heads attend the same K/V tiles under the same
+// mask, so each K and V tile is loaded once for 256 query rows.
+//   warps 0-3   softmax warpgroup of tile 0, warps 4-7 of tile 1
+//   warp 8      TMA producer, warp 9 MMA issuer + TMEM owner
+// TMEM: tile t uses S at columns 256t..256t+127 and O at 256t+128..256t+255;
+// P_t (bf16) overwrites the first 64 columns of S_t.  The MMA issue order
+//   QK_0(0) QK_1(0) | PV_0(j) QK_0(j+1) PV_1(j) QK_1(j+1) | ...
+// makes the tensor core work on one tile while the other tile's softmax
+// runs.  MMAs complete in issue order, so "S_t(j) ready" (a commit after
+// QK_t(j)) also means PV_t(j-1) has finished: the softmax may rescale O_t
+// and overwrite S_t with P_t without any further wait.
+// A quarter of the exp2 evaluations (every fourth key) run on the FMA pipe
+// as a polynomial so the special-function unit is not the bottleneck.
+// =====================================================================
+namespace prefill2 {
+
+using prefill::Params;
+using prefill::TileIter;
+constexpr int BM = 128, BN = 128, HD = 128, NQ = 2;
+constexpr int NSLOT = 5;
+constexpr int TILE_BYTES = BN * HD * 2;
+constexpr int HALF_BYTES = TILE_BYTES / 2;
+constexpr int NUM_THREADS = 320;
+constexpr int WARP_PRODUCER = 8, WARP_MMA = 9;
+constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 * NQ + NQ + 1;
+constexpr int SMEM_BYTES = 1024 + NQ * TILE_BYTES + NSLOT * TILE_BYTES + NUM_BARS * 8 + 16;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr uint64_t kDrainNs = 200000000ull;
+
+// 2^x on the FMA pipe: round-to-nearest range reduction with the 1.5*2^23
+// shifter (x = n + f, f in [-1/2, 1/2]), a degree-3 polynomial for 2^f
+// (coefficients fitted here by minimax linear programming on [-1/2, 1/2];
+// max relative error 1.0e-4, below bf16 rounding of P), and n added to the
+// exponent field.  Inputs below -127 give 0.
+constexpr float kExp2C1 = 0.693282962f;
+constexpr float kExp2C2 = 0.242210999f;
+constexpr float kExp2C3 = 0.0550087839f;
+FA_DEV float ex2_poly(float x) {
+  x = fmaxf(x, -127.0f);
+  const float t = x + 12582912.0f;          // 1.5 * 2^23: low mantissa bits = round(x)
+  const float n = t - 12582912.0f;
+  const float f = x - n;
+  float p = fmaf(kExp2C3, f, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+struct Shared {
+  uint8_t *q[NQ];
+  uint8_t *ring;
+  uint64_t *q_full, *full, *empty, *s_full, *p_full, *o_done, *drain;
+  uint32_t *tmem_slot;
+  volatile int *abort;
+};
+
+FA_DEV Shared carve(uint8_t *raw) {
+  Shared s;
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  s.q[0] = base;
+  s.q[1] = base + TILE_BYTES;
+  s.ring = base + NQ * TILE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(s.ring + NSLOT * TILE_BYTES);
+  s.q_full = bars;
+  s.full = bars + 1;
+  s.empty = s.full + NSLOT;
+  s.s_full = s.empty + NSLOT;
+  s.p_full = s.s_full + NQ;
+  s.o_done = s.p_full + NQ;
+  s.drain = s.o_done + NQ;
+  s.tmem_slot = reinterpret_cast<uint32_t *>(s.drain + 1);
+  s.abort = reinterpret_cast<volatile int *>(s.tmem_slot + 1);
+  return s;
+}
+
+FA_DEV void run_producer(const Shared &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                         const CUtensorMap *tmV, const Params &p, int qt, int b, int h0, int kvh,
+                         bool sparse) {
+  mbar_arrive_expect_tx(sh.q_full, NQ * TILE_BYTES);
+#pragma unroll
+  for (int t = 0; t < NQ; ++t) {
+    tma_load_4d(sh.q[t], tmQ, sh.q_full, 0, h0 + t, qt * BM, b);
+    tma_load_4d(sh.q[t] + HALF_BYTES, tmQ, sh.q_full, 64, h0 + t, qt * BM, b);
+  }
+  TileIter it;
+  it.init(p, qt, sparse);
+  int li = 0;
+  auto load = [&](const CUtensorMap *map, int n) -> bool {
+    const int slot = li % NSLOT;
+    const uint32_t round = static_cast<uint32_t>(li / NSLOT);
+    if (!mbar_wait(&sh.empty[slot], (round & 1u) ^ 1u, sh.abort, p.status)) return false;
+    uint8_t *dst = sh.ring + slot * TILE_BYTES;
+    mbar_arrive_expect_tx(&sh.full[slot], TILE_BYTES);
+    tma_load_4d(dst, map, &sh.full[slot], 0, kvh, n * BN, b);
+    tma_load_4d(dst + HALF_BYTES, map, &sh.full[slot], 64, kvh, n * BN, b);
+    ++li;
+    return true;
+  };
+  int n = 0;
+  uint32_t bits;
+  while (it.next(n, bits)) {
+    if (!load(tmK, n) || !load(tmV, n)) break;
+  }
+  if (*sh.abort) {
+    mbar_wait_drain(sh.q_full, 0, kDrainNs);
+    for (int x = (li > NSLOT ? li - NSLOT : 0); x < li; ++x)
+      mbar_wait_drain(&sh.full[x % NSLOT], static_cast<uint32_t>(x / NSLOT) & 1u, kDrainNs);
+  }
+}
+
+FA_DEV void run_mma(const Shared &sh, uint32_t tmem, const Params &p, int qt, bool sparse) {
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
+  bool ok = mbar_wait(sh.q_full, 0, sh.abort, p.status);
+  tc_fence_after_sync();
+  int ci = 0;
+  auto take = [&](int &slot) -> bool {
+    slot = ci % NSLOT;
+    const uint32_t round = static_cast<uint32_t>(ci / NSLOT);
+    ++ci;
+    if (!mbar_wait(&sh.full[slot], round & 1u, sh.abort, p.status)) return false;
+    tc_fence_after_sync();
+    return true;
+  };
+  auto qk = [&](int t, int slot) {
+    const uint32_t q_addr = smem_u32(sh.q[t]);
+    const uint32_t k_addr = smem_u32(sh.ring + slot * TILE_BYTES);
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+      mma_bf16_ss(tmem + 256u * t, smem_desc_sw128(q_addr + off, 16, 1024),
+                  smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+    }
+    tc_commit(&sh.s_full[t]);
+  };
+  auto pv = [&](int t, int j, int slot) -> bool {
+    if (!mbar_wait(&sh.p_full[t], static_cast<uint32_t>(j) & 1u, sh.abort, p.status))
+      return false;
+    tc_fence_after_sync();
+    const uint32_t v_addr = smem_u32(sh.ring + slot * TILE_BYTES);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk) {
+      mma_bf16_ts(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
+                  smem_desc_sw128(v_addr + kk * 2048, HALF_BYTES, 1024), kIdescPV,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+    }
+    return true;
+  };
+
+  TileIter it;
+  it.init(p, qt, sparse);
+  int n = 0;
+  uint32_t bits;
+  bool has = ok && it.next(n, bits);
+  int k_slot = 0, v_slot = 0;
+  if (has) {
+    ok = take(k_slot);
+    if (ok) {
+      qk(0, k_slot);
+      qk(1, k_slot);
+      tc_commit(&sh.empty[k_slot]);
+    }
+  }
+  for (int j = 0; ok && has; ++j) {
+    const bool has_next = it.next(n, bits);
+    if (!(ok = take(v_slot))) break;
+    if (!(ok = pv(0, j, v_slot))) break;
+    if (has_next) {
+      if (!(ok = take(k_slot))) break;
+      qk(0, k_slot);
+    } else {
+      tc_commit(&sh.o_done[0]);
+    }
+    if (!(ok = pv(1, j, v_slot))) break;
+    tc_commit(&sh.empty[v_slot]);
+    if (has_next) {
+      qk(1, k_slot);
+      tc_commit(&sh.empty[k_slot]);
+    } else {
+      tc_commit(&sh.o_done[1]);
+    }
+    has = has_next;
+  }
+  if (*sh.abort) {
+    tc_commit(sh.drain);
+    mbar_wait_drain(sh.drain, 0, kDrainNs);
+  }
+}
+
+FA_DEV bool warp_wait(uint64_t *bar, uint32_t parity, const Shared &sh, const Params &p) {
+  const bool done = mbar_wait(bar, parity, sh.abort, p.status);
+  return __all_sync(0xffffffffu, done);
+}
+
+FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt, int b, int h,
+                        int t, bool sparse) {
+  const int r = threadIdx.x - 128 * t;                 // row within the tile
+  const uint32_t quad = (threadIdx.x >> 5) & 3u;
+  const uint32_t s_base = tmem + ((quad * 32u) << 16) + 256u * t;
+  const uint32_t o_base = s_base + 128u;
+  const float c = p.scale_log2;
+  float m_run = -INFINITY, l_run = 0.f;
+
+  TileIter it;
+  it.init(p, qt, sparse);
+  int j = 0, n = 0;
+  uint32_t bits = 0;
+  bool ok = true;
+  while (it.next(n, bits)) {
+    if (!warp_wait(&sh.s_full[t], static_cast<uint32_t>(j) & 1u, sh, p)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after_sync();
+    float s[BN];
+#pragma unroll
+    for (int q4 = 0; q4 < BN / 32; ++q4) {
+      uint32_t raw[32];
+      tmem_ld32(s_base + q4 * 32, raw);
+      tmem_ld_wait(raw);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(raw[i]);
+    }
+    const bool diag = (n == qt);
+    if (diag || bits != 0xFu) {
+      const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
+#pragma unroll
+      for (int i = 0; i < BN; ++i) {
+        const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
+        s[i] = keep ? s[i] : -INFINITY;
+      }
+    }
+    float mx8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+    for (int i = 8; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+    const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+    const float m_new = fmaxf(m_run, mx * c);
+    const bool need = m_new > m_run + kRescaleThreshold;
+    const float m_next = need ? m_new : m_run;
+    const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
+    float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q2 = 0; q2 < 2; ++q2) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int k0 = q2 * 64 + 2 * i;
+        const float x0 = fmaf(s[k0], c, -m_use), x1 = fmaf(s[k0 + 1], c, -m_use);
+        const float p0 = ex2(x0);
+        const float p1 = ((k0 + 1) & 3) == 3 ? ex2_poly(x1) : ex2(x1);
+        sum4[(2 * i) & 3] += p0;
+        sum4[(2 * i + 1) & 3] += p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(s_base + q2 * 32, pk);
+    }
+    if (j > 0 && __any_sync(0xffffffffu, need)) {
+      const float alpha = need ? ex2(m_run - m_new) : 1.0f;
+#pragma unroll
+      for (int q4 = 0; q4 < HD / 32; ++q4) {
+        uint32_t o[32];
+        tmem_ld32(o_base + q4 * 32, o);
+        tmem_ld_wait(o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        tmem_st32(o_base + q4 * 32, o);
+      }
+    }
+    if (need) l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
+    m_run = m_next;
+    l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+    tmem_st_wait();
+    tc_fence_before_sync();
+    mbar_arrive(&sh.p_full[t]);
+    ++j;
+  }
+
+  const bool have_o = ok && j > 0 && warp_wait(&sh.o_done[t], 0u, sh, p);
+  tc_fence_after_sync();
+  const int tok = qt * BM + r;
+  const bool store = (tok < p.S) && !*sh.abort;
+  const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+  __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.S + tok) * p.Hq + h) * HD;
+#pragma unroll
+  for (int q4 = 0; q4 < HD / 32; ++q4) {
+    uint32_t o[32];
+    if (have_o) {
+      tmem_ld32(o_base + q4 * 32, o);
+      tmem_ld_wait(o);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = 0u;
+    }
+    if (store) {
+      uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+        w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+        w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+        w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+        dst[v] = w;
+      }
+    }
+  }
+  if (store && p.lse) {
+    const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + tok] = lse;
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const Shared sh = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA -> (query tile, batch, head pair): longest causal rows first; the
+  // head pairs of one KV group are adjacent.
+  const int hp_count = p.Hq / NQ;
+  const int bh = p.B * hp_count;
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / bh;
+  const int rem = static_cast<int>(blockIdx.x) % bh;
+  const int b = rem / hp_count, h0 = (rem % hp_count) * NQ, kvh = h0 / p.G;
+  const int mode = p.mode ? p.mode[b] : p.mode_default;
+  const bool sparse = (mode == FA_MODE_SPARSE) && p.row_ptr != nullptr;
+
+  if (threadIdx.x == 0) {
+    mbar_init(sh.q_full, 1);
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.empty[i], 1);
+    }
+    for (int t = 0; t < NQ; ++t) {
+      mbar_init(&sh.s_full[t], 1);
+      mbar_init(&sh.p_full[t], 128);
+      mbar_init(&sh.o_done[t], 1);
+    }
+    mbar_init(sh.drain, 1);
+    *sh.abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(sh.tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *sh.tmem_slot;
+
+  if (warp == WARP_PRODUCER) {
+    if (lane == 0) run_producer(sh, &tmQ, &tmK, &tmV, p, qt, b, h0, kvh, sparse);
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) run_mma(sh, tmem, p, qt, sparse);
+    __syncwarp();
+  } else {
+    const int t = warp >> 2;
+    run_softmax(sh, tmem, p, qt, b, h0 + t, t, sparse);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace prefill2
+
 // ----------------------------------------------------------------- host ---
 int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   using namespace prefill;
@@ -481,13 +862,14 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   if (make_tmap_bhsd(&tmQ, a.q, a.B, a.S, a.Hq, 64, BM) != 0) return FA_ERR_CUDA;
   if (make_tmap_bhsd(&tmK, a.k, a.B, a.S, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
   if (make_tmap_bhsd(&tmV, a.v, a.B, a.S, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return FA_ERR_CUDA;
-    attr_done = true;
-  }
+  const int G = a.Hq / a.Hkv;
+  const bool two_tiles = (G % 2) == 0;
+  if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SMEM_BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(prefill2::prefill2_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           prefill2::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
   Params p;
   p.o = reinterpret_cast<__nv_bfloat16 *>(a.o);
   p.lse = a.lse;
@@ -498,14 +880,20 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   p.B = a.B;
   p.S = a.S;
   p.Hq = a.Hq;
-  p.G = a.Hq / a.Hkv;
+  p.G = G;
   p.n_qtiles = (a.S + BM - 1) / BM;
   p.nqb = (a.S + 63) / 64;
   p.mode_default = a.mode_default;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  const long long grid = static_cast<long long>(p.n_qtiles) * a.B * a.Hq;
+  const long long grid =
+      static_cast<long long>(p.n_qtiles) * a.B * (two_tiles ? a.Hq / 2 : a.Hq);
   if (grid <= 0 || grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  prefill_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  if (two_tiles)
+    prefill2::prefill2_kernel<<<static_cast<unsigned>(grid), prefill2::NUM_THREADS,
+                                prefill2::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  else
+    prefill_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmK,
+                                                                                    tmV, p);
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
