@@ -226,6 +226,32 @@ FA_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
 }
 FA_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ------------------------------------------------- packed fp32x2 arithmetic
+// sm_100 executes these as one instruction for two fp32 lanes.
+FA_DEV uint64_t f2_make(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+FA_DEV void f2_split(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+FA_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {  // a*b + c, round to nearest
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+FA_DEV uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+FA_DEV float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // -------------------------------------------------------------------- math
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32).
 FA_DEV float ex2(float x) {

@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // GQA group (G even).  Both heads attend the same K/V tiles under the same
 // mask, so each K and V tile is loaded once for 256 query rows.
 //   warps 0-3   softmax warpgroup of tile 0, warps 4-7 of tile 1
-//   warp 8      TMA producer, warp 9 MMA issuer + TMEM owner
+//   warp 8      TMA producer, warp 9 MMA issuer + TMEM owner (10-11 idle)
 // TMEM: tile t uses S at columns 256t..256t+127 and O at 256t+128..256t+255;
 // P_t (bf16) overwrites the first 64 columns of S_t.  The MMA issue order
 //   QK_0(0) QK_1(0) | PV_0(j) QK_0(j+1) PV_1(j) QK_1(j+1) | ...
@@ -487,8 +487,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // runs.  MMAs complete in issue order, so "S_t(j) ready" (a commit after
 // QK_t(j)) also means PV_t(j-1) has finished: the softmax may rescale O_t
 // and overwrite S_t with P_t without any further wait.
-// A quarter of the exp2 evaluations (every fourth key) run on the FMA pipe
-// as a polynomial so the special-function unit is not the bottleneck.
+// A share of the exp2 evaluations (kPolyPer8 keys of every 8) run on the FMA
+// pipe as a polynomial so the special-function unit is not the bottleneck.
 // =====================================================================
 namespace prefill2 {
 
@@ -498,8 +498,13 @@ constexpr int BM = 128, BN = 128, HD = 128, NQ = 2;
 constexpr int NSLOT = 5;
 constexpr int TILE_BYTES = BN * HD * 2;
 constexpr int HALF_BYTES = TILE_BYTES / 2;
-constexpr int NUM_THREADS = 320;
-constexpr int WARP_PRODUCER = 8, WARP_MMA = 9;
+constexpr int NUM_THREADS = 384;                 // 3 warpgroups
+constexpr int WARP_PRODUCER = 8, WARP_MMA = 9;   // warps 10-11 idle
+// Register split (setmaxnreg): the two softmax warpgroups grow to
+// kSoftmaxRegs, the producer/MMA warpgroup shrinks to kOtherRegs.  The sum
+// must not exceed what the block was launched with (384 x the compiled
+// count); the launcher checks it before every launch.
+constexpr int kSoftmaxRegs = 208, kOtherRegs = 88;
 constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 * NQ + NQ + 1;
 constexpr int SMEM_BYTES = 1024 + NQ * TILE_BYTES + NSLOT * TILE_BYTES + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
@@ -511,6 +516,11 @@ constexpr uint64_t kDrainNs = 200000000ull;
 // (coefficients fitted here by minimax linear programming on [-1/2, 1/2];
 // max relative error 1.0e-4, below bf16 rounding of P), and n added to the
 // exponent field.  Inputs below -127 give 0.
+#ifndef FA_POLY_PER_8
+#define FA_POLY_PER_8 2
+#endif
+// Keys k with (k mod 8) >= 8 - kPolyPer8 take the polynomial; the rest use ex2.approx.
+constexpr int kPolyPer8 = FA_POLY_PER_8;
 constexpr float kExp2C1 = 0.693282962f;
 constexpr float kExp2C2 = 0.242210999f;
 constexpr float kExp2C3 = 0.0550087839f;
@@ -523,6 +533,23 @@ FA_DEV float ex2_poly(float x) {
   p = fmaf(p, f, kExp2C1);
   p = fmaf(p, f, 1.0f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+// The same for two lanes at once with the packed fp32x2 instructions.
+FA_DEV void ex2_poly2(uint64_t x2, float &r0, float &r1) {
+  float a, b;
+  f2_split(x2, a, b);
+  const uint64_t x = f2_make(fmaxf(a, -127.0f), fmaxf(b, -127.0f));
+  const uint64_t t = f2_add(x, f2_make(12582912.0f, 12582912.0f));
+  const uint64_t n = f2_add(t, f2_make(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(n, f2_make(-1.0f, -1.0f), x);
+  uint64_t p = f2_fma(f2_make(kExp2C3, kExp2C3), f, f2_make(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_make(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_make(1.0f, 1.0f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 struct Shared {
@@ -710,29 +737,41 @@ FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt
         s[i] = keep ? s[i] : -INFINITY;
       }
     }
+    // Row max: 3-input max over pairs, 8 independent chains.
     float mx8[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+    for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(s[2 * k], s[2 * k + 1]);
 #pragma unroll
-    for (int i = 8; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
-    const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+    for (int i = 16; i < BN; i += 16)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[i + 2 * k], s[i + 2 * k + 1]);
+    const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                           fmaxf(mx8[6], mx8[7]));
     const float m_new = fmaxf(m_run, mx * c);
     const bool need = m_new > m_run + kRescaleThreshold;
     const float m_next = need ? m_new : m_run;
     const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
-    float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+    // p = 2^(s*c - m), two lanes per instruction; every fourth pair of keys
+    // on the FMA pipe, the rest on ex2.approx.
+    const uint64_t c2 = f2_make(c, c), negm2 = f2_make(-m_use, -m_use);
+    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int q2 = 0; q2 < 2; ++q2) {
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const int k0 = q2 * 64 + 2 * i;
-        const float x0 = fmaf(s[k0], c, -m_use), x1 = fmaf(s[k0 + 1], c, -m_use);
-        const float p0 = ex2(x0);
-        const float p1 = ((k0 + 1) & 3) == 3 ? ex2_poly(x1) : ex2(x1);
-        sum4[(2 * i) & 3] += p0;
-        sum4[(2 * i + 1) & 3] += p1;
+        const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
+        float p0, p1;
+        if ((k0 & 7) >= 8 - kPolyPer8) {
+          ex2_poly2(x, p0, p1);
+        } else {
+          float x0, x1;
+          f2_split(x, x0, x1);
+          p0 = ex2(x0);
+          p1 = ex2(x1);
+        }
+        acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
         pk[i] = pack_bf16x2(p0, p1);
       }
       tmem_st32(s_base + q2 * 32, pk);
@@ -751,7 +790,13 @@ FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt
     }
     if (need) l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
     m_run = m_next;
-    l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+    {
+      float a0, a1, b0, b1;
+      f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+      l_run += a0 + a1;
+      (void)b0;
+      (void)b1;
+    }
     tmem_st_wait();
     tc_fence_before_sync();
     mbar_arrive(&sh.p_full[t]);
@@ -836,12 +881,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *sh.tmem_slot;
 
-  if (warp == WARP_PRODUCER) {
-    if (lane == 0) run_producer(sh, &tmQ, &tmK, &tmV, p, qt, b, h0, kvh, sparse);
-  } else if (warp == WARP_MMA) {
-    if (lane == 0) run_mma(sh, tmem, p, qt, sparse);
-    __syncwarp();
+  if (warp >= WARP_PRODUCER) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
+    if (warp == WARP_PRODUCER) {
+      if (lane == 0) run_producer(sh, &tmQ, &tmK, &tmV, p, qt, b, h0, kvh, sparse);
+    } else if (warp == WARP_MMA) {
+      if (lane == 0) run_mma(sh, tmem, p, qt, sparse);
+      __syncwarp();
+    }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
     const int t = warp >> 2;
     run_softmax(sh, tmem, p, qt, b, h0 + t, t, sparse);
   }
@@ -864,6 +913,15 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   if (make_tmap_bhsd(&tmV, a.v, a.B, a.S, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
   const int G = a.Hq / a.Hkv;
   const bool two_tiles = (G % 2) == 0;
+  if (two_tiles) {
+    // setmaxnreg only redistributes what the block was launched with.
+    cudaFuncAttributes fattr;
+    if (cudaFuncGetAttributes(&fattr, prefill2::prefill2_kernel) != cudaSuccess)
+      return FA_ERR_CUDA;
+    if (2 * 128 * prefill2::kSoftmaxRegs + 128 * prefill2::kOtherRegs >
+        prefill2::NUM_THREADS * fattr.numRegs)
+      return FA_ERR_UNSUPPORTED;
+  }
   if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SMEM_BYTES) != cudaSuccess ||
       cudaFuncSetAttribute(prefill2::prefill2_kernel,
