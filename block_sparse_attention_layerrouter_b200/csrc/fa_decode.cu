@@ -85,6 +85,14 @@ FA_DEV void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
   }
 }
 
+// Eight bf16 (one 16-byte chunk) -> four packed fp32 pairs (element 2i in
+// the low lane of pair i).
+FA_DEV void bf16x8_to_f2(const uint4 &v, uint64_t (&f)[4]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) f[i] = f2_make(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+
 // Byte offset of the 16-byte chunk holding dims [8*chunk16, 8*chunk16+8) of
 // `key` inside one K or V tile written by TMA with the 128-byte swizzle.
 FA_DEV uint32_t tile_offset(int key, int chunk16) {
@@ -146,7 +154,7 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 
   // Query slice of this thread for QK^T, pre-scaled by scale*log2(e).
   const int part = tid % C::PARTS;
-  float qr[G][C::DPT];
+  uint64_t qr[G][C::DPT / 2];   // packed pairs of dims
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const __nv_bfloat16 *qrow = p.q + (static_cast<size_t>(b) * p.Hq + kvh * G + g) * HD + part * C::DPT;
@@ -155,16 +163,17 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
       float f[8];
       bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + c8 * 8), f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qr[g][c8 * 8 + e] = f[e] * p.scale_log2;
+      for (int e = 0; e < 4; ++e)
+        qr[g][c8 * 4 + e] = f2_make(f[2 * e] * p.scale_log2, f[2 * e + 1] * p.scale_log2);
     }
   }
   const int dc = tid & 15;     // PV: output dims [8*dc, 8*dc+8)
   const int ks = tid >> 4;     // PV: key stream
-  float acc[G][8];
+  uint64_t acc[G][4];           // packed pairs of output dims
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[g][e] = 0ull;
   float m_run = -INFINITY, l_run = 0.f;  // meaningful in warp g < G
 
   for (int i = 0; i < ntiles; ++i) {
@@ -179,17 +188,24 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 #pragma unroll
     for (int pass = 0; pass < C::PASSES; ++pass) {
       const int key = pass * C::KPP + tid / C::PARTS;
-      float d[G];
+      uint64_t d2[G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) d[g] = 0.f;
+      for (int g = 0; g < G; ++g) d2[g] = 0ull;
 #pragma unroll
       for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
-        float kf[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(sK + tile_offset(key, part * (C::DPT / 8) + c8)), kf);
+        uint64_t k2[4];
+        bf16x8_to_f2(*reinterpret_cast<const uint4 *>(sK + tile_offset(key, part * (C::DPT / 8) + c8)), k2);
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) d[g] = fmaf(qr[g][c8 * 8 + e], kf[e], d[g]);
+          for (int e = 0; e < 4; ++e) d2[g] = f2_fma(qr[g][c8 * 4 + e], k2[e], d2[g]);
+      }
+      float d[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float lo, hi;
+        f2_split(d2[g], lo, hi);
+        d[g] = lo + hi;
       }
 #pragma unroll
       for (int off = 1; off < C::PARTS; off <<= 1)
@@ -227,22 +243,22 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     // ---- O += P V
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float a = alpha_sm[g];
+      const uint64_t a2 = f2_make(alpha_sm[g], alpha_sm[g]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] *= a;
+      for (int e = 0; e < 4; ++e) acc[g][e] = f2_mul(acc[g][e], a2);
     }
 #pragma unroll
     for (int kk = 0; kk < KT / 16; ++kk) {
       const int key = ks + 16 * kk;
-      float vf[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(sV + tile_offset(key, dc)), vf);
-      float pg[G];
+      uint64_t v2[4];
+      bf16x8_to_f2(*reinterpret_cast<const uint4 *>(sV + tile_offset(key, dc)), v2);
 #pragma unroll
-      for (int g = 0; g < G; ++g) pg[g] = p_sm[key * G + g];
+      for (int g = 0; g < G; ++g) {
+        const float pg = p_sm[key * G + g];
+        const uint64_t p2 = f2_make(pg, pg);
 #pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg[g], vf[e], acc[g][e]);
+        for (int e = 0; e < 4; ++e) acc[g][e] = f2_fma(p2, v2[e], acc[g][e]);
+      }
     }
     __syncthreads();
     if (tid == 0 && i + NSTAGE < ntiles) issue(i + NSTAGE);
@@ -262,7 +278,12 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red[(ks * G + g) * HD + dc * 8 + e] = acc[g][e];
+    for (int e = 0; e < 4; ++e) {
+      float lo, hi;
+      f2_split(acc[g][e], lo, hi);
+      red[(ks * G + g) * HD + dc * 8 + 2 * e] = lo;
+      red[(ks * G + g) * HD + dc * 8 + 2 * e + 1] = hi;
+    }
   __syncthreads();
   const size_t row0 = (static_cast<size_t>(b) * p.Hq + kvh * G) * p.nsplit + split;
   for (int idx = tid; idx < G * HD; idx += NT) {
@@ -280,41 +301,78 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 }
 
 // Merge the splits of one (batch, head): M = max m_s, w_s = 2^(m_s - M),
-// o = sum w_s o_s / sum w_s l_s.
+// o = sum w_s o_s / sum w_s l_s.  The weights are computed once into shared
+// memory; then thread d walks the splits for output dim d (coalesced rows).
+constexpr int kMaxSplits = 256;
 __global__ void __launch_bounds__(128) combine_kernel(const float *o_part, const float *ml_part,
                                                       __nv_bfloat16 *o, float *lse, int Hq,
                                                       int nsplit) {
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  __shared__ float w_sm[kMaxSplits];
+  __shared__ float red[4];
+  __shared__ float M_sm, den_sm;
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x, lane = d & 31, warp = d >> 5;
   const size_t row = (static_cast<size_t>(b) * Hq + h);
   const float *ml = ml_part + row * nsplit * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, ml[2 * s]);
-  float num = 0.f, den = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float m = ml[2 * s];
-      if (m == -INFINITY) continue;
-      const float w = ex2(m - M);
-      den = fmaf(w, ml[2 * s + 1], den);
-      num = fmaf(w, o_part[(row * nsplit + s) * HD + d], num);
-    }
+  float mx = -INFINITY;
+  for (int s = d; s < nsplit; s += 128) mx = fmaxf(mx, ml[2 * s]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  if (d == 0) M_sm = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  const float M = M_sm;
+  float den = 0.f;
+  for (int s = d; s < nsplit; s += 128) {
+    const float m = ml[2 * s];
+    const float w = (m == -INFINITY) ? 0.f : ex2(m - M);
+    w_sm[s] = w;
+    den = fmaf(w, ml[2 * s + 1], den);
   }
-  const float out = den > 0.f ? num / den : 0.f;
-  o[row * HD + d] = __float2bfloat16_rn(out);
-  if (lse && d == 0)
-    lse[row] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994531f : -INFINITY;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+  __syncthreads();
+  if (lane == 0) red[warp] = den;
+  __syncthreads();
+  if (d == 0) den_sm = (red[0] + red[1]) + (red[2] + red[3]);
+  __syncthreads();
+  den = den_sm;
+  float num = 0.f;
+  const float *op = o_part + row * nsplit * HD + d;
+  for (int s = 0; s < nsplit; ++s) num = fmaf(w_sm[s], op[static_cast<size_t>(s) * HD], num);
+  const bool any = (M != -INFINITY) && den > 0.f;
+  o[row * HD + d] = __float2bfloat16_rn(any ? num / den : 0.f);
+  if (lse && d == 0) lse[row] = any ? (M + __log2f(den)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace decode
 
+// Splits per (batch, KV head) for a sequence of `tiles` 64-key tiles.  The
+// CTA count B*Hkv*splits is chosen to fill whole waves of 2 CTAs on each of
+// 148 SMs (a partial last wave leaves SMs idle), with at least 4 tiles per
+// CTA and at most kMaxSplits splits; small problems take the most splits.
+int decode_splits_for_tiles(int B, int Hkv, int tiles) {
+  constexpr int kSlots = 148 * 2;
+  const int base = B * Hkv;
+  int ns_max = tiles / 4;
+  ns_max = ns_max < 1 ? 1 : (ns_max > decode::kMaxSplits ? decode::kMaxSplits : ns_max);
+  if (static_cast<long long>(base) * ns_max <= 2 * kSlots) return ns_max;
+  const int ns_min = (2 * kSlots + base - 1) / base;
+  int best = ns_max;
+  double best_eff = -1.0;
+  for (int ns = ns_min; ns <= ns_max; ++ns) {
+    const double waves = static_cast<double>(base) * ns / kSlots;
+    const double eff = waves / static_cast<double>(static_cast<long long>(waves + 0.999999));
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = ns;
+    }
+  }
+  return best;
+}
+
 int decode_num_splits(int B, int Hkv, int Lmax) {
-  const int tiles = (Lmax + decode::KT - 1) / decode::KT;
-  const int target_ctas = 148 * 2 * 4;
-  int ns = (target_ctas + B * Hkv - 1) / (B * Hkv);
-  ns = ns < 1 ? 1 : ns;
-  ns = ns > tiles ? tiles : ns;
-  ns = ns > 256 ? 256 : ns;
-  return ns;
+  return decode_splits_for_tiles(B, Hkv, (Lmax + decode::KT - 1) / decode::KT);
 }
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax) {
@@ -332,8 +390,8 @@ int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
   int ns = decode_num_splits(a.B, a.Hkv, a.Lmax);
   if (a.mode_dev == nullptr && a.mode == FA_MODE_SPARSE) {
     const int sparse_tiles = a.sink / KT + a.window / KT;
-    ns = ns > sparse_tiles ? sparse_tiles : ns;
-    if (ns < 1) ns = 1;
+    const int ns_sparse = decode_splits_for_tiles(a.B, a.Hkv, sparse_tiles);
+    ns = ns_sparse < ns ? ns_sparse : ns;   // the workspace is sized for the FULL count
   }
   Params p;
   p.q = reinterpret_cast<const __nv_bfloat16 *>(a.q);

@@ -41,6 +41,7 @@ struct DecodeLaunch {
   int32_t *status;
 };
 int decode_num_splits(int B, int Hkv, int Lmax);
+int decode_splits_for_tiles(int B, int Hkv, int tiles);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax);
 int launch_decode(const DecodeLaunch &a, cudaStream_t stream);
 
