@@ -93,6 +93,59 @@ FA_DEV bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
   return true;
 }
 
+// The same operations on 32-bit shared-window addresses (no generic pointer
+// kept live: kernels that carve one buffer use base + constant offsets).
+FA_DEV bool mbar_try_wait_a(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+FA_DEV int ld_shared_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+FA_DEV void st_shared_s32(uint32_t addr, int v) {
+  asm volatile("st.volatile.shared.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Bounded wait; `abort_flag` is the shared address of the CTA's abort word.
+FA_DEV bool mbar_wait_a(uint32_t bar, uint32_t parity, uint32_t abort_flag, int32_t *status) {
+  if (mbar_try_wait_a(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait_a(bar, parity)) return true;
+    if (ld_shared_s32(abort_flag)) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      st_shared_s32(abort_flag, 1);
+      report(status, FA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+FA_DEV bool mbar_wait_drain_a(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait_a(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+FA_DEV void mbar_init_a(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+FA_DEV void mbar_arrive_a(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+FA_DEV void mbar_arrive_expect_tx_a(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
 // ---------------------------------------------------------------------- TMA
 FA_DEV void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -108,6 +161,15 @@ FA_DEV void tma_load_4d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, i
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
       "r"(smem_u32(bar))
+      : "memory");
+}
+
+FA_DEV void tma_load_4d_a(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1,
+                          int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
       : "memory");
 }
 
@@ -136,6 +198,17 @@ FA_DEV void tc_fence_after_sync() {
 FA_DEV void tc_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
+               : "memory");
+}
+
+FA_DEV void tc_commit_a(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+FA_DEV void tmem_alloc_a(uint32_t dst, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+               "r"(ncols)
                : "memory");
 }
 

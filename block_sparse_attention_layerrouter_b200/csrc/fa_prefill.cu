@@ -475,8 +475,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }  // namespace prefill
 
 // =====================================================================
-// Two query tiles per CTA: the same 128-row tile of two query heads of one
-// GQA group (G even).  Both heads attend the same K/V tiles under the same
+// Two query tiles per work item: the same 128-row tile of two query heads of
+// one GQA group (G even).  The kernel is persistent: one CTA per SM walks its
+// share of the items, and the next item's Q/K/V loads and first QK^T overlap
+// the current item's epilogue.  Both heads attend the same K/V tiles under the same
 // mask, so each K and V tile is loaded once for 256 query rows.
 //   warps 0-3   softmax warpgroup of tile 0, warps 4-7 of tile 1
 //   warp 8      TMA producer, warp 9 MMA issuer + TMEM owner (10-11 idle)
@@ -504,8 +506,8 @@ constexpr int WARP_PRODUCER = 8, WARP_MMA = 9;   // warps 10-11 idle
 // kSoftmaxRegs, the producer/MMA warpgroup shrinks to kOtherRegs.  The sum
 // must not exceed what the block was launched with (384 x the compiled
 // count); the launcher checks it before every launch.
-constexpr int kSoftmaxRegs = 208, kOtherRegs = 88;
-constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 * NQ + NQ + 1;
+constexpr int kSoftmaxRegs = 184, kOtherRegs = 136;
+constexpr int NUM_BARS = 2 + 2 * NSLOT + 4 * NQ + 1;
 constexpr int SMEM_BYTES = 1024 + NQ * TILE_BYTES + NSLOT * TILE_BYTES + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;
@@ -552,347 +554,406 @@ FA_DEV void ex2_poly2(uint64_t x2, float &r0, float &r1) {
   r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-struct Shared {
-  uint8_t *q[NQ];
-  uint8_t *ring;
-  uint64_t *q_full, *full, *empty, *s_full, *p_full, *o_done, *drain;
-  uint32_t *tmem_slot;
-  volatile int *abort;
+// Shared-memory layout, as offsets from one 1024-byte aligned base:
+// Q tiles | K/V ring | mbarriers | TMEM address | abort word.
+struct Smem {
+  uint32_t base;
+  static constexpr uint32_t kRing = NQ * TILE_BYTES;
+  static constexpr uint32_t kBars = kRing + NSLOT * TILE_BYTES;
+  enum : uint32_t {
+    Q_FULL = 0, Q_EMPTY = 1, FULL0 = 2, EMPTY0 = FULL0 + NSLOT, S_FULL0 = EMPTY0 + NSLOT,
+    P_FULL0 = S_FULL0 + NQ, O_DONE0 = P_FULL0 + NQ, O_FREE0 = O_DONE0 + NQ, DRAIN = O_FREE0 + NQ,
+    NBARS = DRAIN + 1
+  };
+  FA_DEV uint32_t q(int t) const { return base + t * TILE_BYTES; }
+  FA_DEV uint32_t ring(int slot) const { return base + kRing + slot * TILE_BYTES; }
+  FA_DEV uint32_t bar(uint32_t i) const { return base + kBars + 8u * i; }
+  FA_DEV uint32_t tmem_slot() const { return base + kBars + 8u * NBARS; }
+  FA_DEV uint32_t abort_flag() const { return tmem_slot() + 4u; }
 };
 
-FA_DEV Shared carve(uint8_t *raw) {
-  Shared s;
-  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
-  s.q[0] = base;
-  s.q[1] = base + TILE_BYTES;
-  s.ring = base + NQ * TILE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(s.ring + NSLOT * TILE_BYTES);
-  s.q_full = bars;
-  s.full = bars + 1;
-  s.empty = s.full + NSLOT;
-  s.s_full = s.empty + NSLOT;
-  s.p_full = s.s_full + NQ;
-  s.o_done = s.p_full + NQ;
-  s.drain = s.o_done + NQ;
-  s.tmem_slot = reinterpret_cast<uint32_t *>(s.drain + 1);
-  s.abort = reinterpret_cast<volatile int *>(s.tmem_slot + 1);
+FA_DEV Smem carve(uint8_t *raw) {
+  Smem s;
+  s.base = (smem_u32(raw) + 1023u) & ~1023u;
   return s;
 }
 
-FA_DEV void run_producer(const Shared &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
-                         const CUtensorMap *tmV, const Params &p, int qt, int b, int h0, int kvh,
-                         bool sparse) {
-  mbar_arrive_expect_tx(sh.q_full, NQ * TILE_BYTES);
+// Work item -> (query tile, batch, first head of the pair).  Items are
+// numbered longest causal rows first; the head pairs of one KV group are
+// adjacent so K/V tiles are shared through L2.
+struct Item {
+  int qt, b, h0, kvh;
+  bool sparse;
+};
+FA_DEV Item item_of(const Params &p, int w) {
+  const int hp_count = p.Hq / NQ;
+  const int bh = p.B * hp_count;
+  Item it;
+  it.qt = p.n_qtiles - 1 - w / bh;
+  const int rem = w % bh;
+  it.b = rem / hp_count;
+  it.h0 = (rem % hp_count) * NQ;
+  it.kvh = it.h0 / p.G;
+  const int mode = p.mode ? p.mode[it.b] : p.mode_default;
+  it.sparse = (mode == FA_MODE_SPARSE) && p.row_ptr != nullptr;
+  return it;
+}
+// The k-th item of this CTA: rounds of gridDim.x items, walked forwards in
+// even rounds and backwards in odd ones, so a CTA that drew one of the
+// longest items in a round draws one of the shortest in the next.
+FA_DEV int item_index(int k, int total) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const int w = k * G + ((k & 1) ? (G - 1 - c) : c);
+  return w < total ? w : -1;
+}
+
+FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                         const CUtensorMap *tmV, const Params &p, int total) {
+  int li = 0;       // ring loads issued (continues across items)
+  int nq = 0;       // Q loads issued
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = item_index(k, total);
+    if (w < 0) break;
+    const Item im = item_of(p, w);
+    if (k > 0 && !mbar_wait_a(sh.bar(Smem::Q_EMPTY), static_cast<uint32_t>(k - 1) & 1u, sh.abort_flag(), p.status))
+      break;
+    mbar_arrive_expect_tx_a(sh.bar(Smem::Q_FULL), NQ * TILE_BYTES);
 #pragma unroll
-  for (int t = 0; t < NQ; ++t) {
-    tma_load_4d(sh.q[t], tmQ, sh.q_full, 0, h0 + t, qt * BM, b);
-    tma_load_4d(sh.q[t] + HALF_BYTES, tmQ, sh.q_full, 64, h0 + t, qt * BM, b);
+    for (int t = 0; t < NQ; ++t) {
+      tma_load_4d_a(sh.q(t), tmQ, sh.bar(Smem::Q_FULL), 0, im.h0 + t, im.qt * BM, im.b);
+      tma_load_4d_a(sh.q(t) + HALF_BYTES, tmQ, sh.bar(Smem::Q_FULL), 64, im.h0 + t, im.qt * BM, im.b);
+    }
+    ++nq;
+    TileIter it;
+    it.init(p, im.qt, im.sparse);
+    auto load = [&](const CUtensorMap *map, int n) -> bool {
+      const int slot = li % NSLOT;
+      const uint32_t round = static_cast<uint32_t>(li / NSLOT);
+      if (!mbar_wait_a(sh.bar(Smem::EMPTY0 + slot), (round & 1u) ^ 1u, sh.abort_flag(), p.status)) return false;
+      const uint32_t dst = sh.ring(slot);
+      mbar_arrive_expect_tx_a(sh.bar(Smem::FULL0 + slot), TILE_BYTES);
+      tma_load_4d_a(dst, map, sh.bar(Smem::FULL0 + slot), 0, im.kvh, n * BN, im.b);
+      tma_load_4d_a(dst + HALF_BYTES, map, sh.bar(Smem::FULL0 + slot), 64, im.kvh, n * BN, im.b);
+      ++li;
+      return true;
+    };
+    int n = 0;
+    uint32_t bits;
+    while (it.next(n, bits)) {
+      if (!load(tmK, n) || !load(tmV, n)) {
+        ok = false;
+        break;
+      }
+    }
   }
-  TileIter it;
-  it.init(p, qt, sparse);
-  int li = 0;
-  auto load = [&](const CUtensorMap *map, int n) -> bool {
-    const int slot = li % NSLOT;
-    const uint32_t round = static_cast<uint32_t>(li / NSLOT);
-    if (!mbar_wait(&sh.empty[slot], (round & 1u) ^ 1u, sh.abort, p.status)) return false;
-    uint8_t *dst = sh.ring + slot * TILE_BYTES;
-    mbar_arrive_expect_tx(&sh.full[slot], TILE_BYTES);
-    tma_load_4d(dst, map, &sh.full[slot], 0, kvh, n * BN, b);
-    tma_load_4d(dst + HALF_BYTES, map, &sh.full[slot], 64, kvh, n * BN, b);
-    ++li;
-    return true;
-  };
-  int n = 0;
-  uint32_t bits;
-  while (it.next(n, bits)) {
-    if (!load(tmK, n) || !load(tmV, n)) break;
-  }
-  if (*sh.abort) {
-    mbar_wait_drain(sh.q_full, 0, kDrainNs);
+  if (ld_shared_s32(sh.abort_flag())) {  // let every copy this thread issued land before exit
+    if (nq > 0) mbar_wait_drain_a(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(nq - 1) & 1u, kDrainNs);
     for (int x = (li > NSLOT ? li - NSLOT : 0); x < li; ++x)
-      mbar_wait_drain(&sh.full[x % NSLOT], static_cast<uint32_t>(x / NSLOT) & 1u, kDrainNs);
+      mbar_wait_drain_a(sh.bar(Smem::FULL0 + x % NSLOT), static_cast<uint32_t>(x / NSLOT) & 1u, kDrainNs);
   }
 }
 
-FA_DEV void run_mma(const Shared &sh, uint32_t tmem, const Params &p, int qt, bool sparse) {
+FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
-  bool ok = mbar_wait(sh.q_full, 0, sh.abort, p.status);
-  tc_fence_after_sync();
-  int ci = 0;
+  int ci = 0;         // ring slots consumed
+  int jp = 0;         // P tiles consumed (per tile index, both advance together)
+  int done_items = 0; // items that produced an output (o_done / o_free phases)
+  bool ok = true;
   auto take = [&](int &slot) -> bool {
     slot = ci % NSLOT;
     const uint32_t round = static_cast<uint32_t>(ci / NSLOT);
     ++ci;
-    if (!mbar_wait(&sh.full[slot], round & 1u, sh.abort, p.status)) return false;
+    if (!mbar_wait_a(sh.bar(Smem::FULL0 + slot), round & 1u, sh.abort_flag(), p.status)) return false;
     tc_fence_after_sync();
     return true;
   };
   auto qk = [&](int t, int slot) {
-    const uint32_t q_addr = smem_u32(sh.q[t]);
-    const uint32_t k_addr = smem_u32(sh.ring + slot * TILE_BYTES);
+    const uint32_t q_addr = sh.q(t);
+    const uint32_t k_addr = sh.ring(slot);
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
       const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
       mma_bf16_ss(tmem + 256u * t, smem_desc_sw128(q_addr + off, 16, 1024),
                   smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
     }
-    tc_commit(&sh.s_full[t]);
+    tc_commit_a(sh.bar(Smem::S_FULL0 + t));
   };
-  auto pv = [&](int t, int j, int slot) -> bool {
-    if (!mbar_wait(&sh.p_full[t], static_cast<uint32_t>(j) & 1u, sh.abort, p.status))
+  auto pv = [&](int t, bool first, int slot) -> bool {
+    if (!mbar_wait_a(sh.bar(Smem::P_FULL0 + t), static_cast<uint32_t>(jp) & 1u, sh.abort_flag(), p.status))
+      return false;
+    if (first && done_items > 0 &&
+        !mbar_wait_a(sh.bar(Smem::O_FREE0 + t), static_cast<uint32_t>(done_items - 1) & 1u, sh.abort_flag(), p.status))
       return false;
     tc_fence_after_sync();
-    const uint32_t v_addr = smem_u32(sh.ring + slot * TILE_BYTES);
+    const uint32_t v_addr = sh.ring(slot);
 #pragma unroll
     for (int kk = 0; kk < BN / 16; ++kk) {
       mma_bf16_ts(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
                   smem_desc_sw128(v_addr + kk * 2048, HALF_BYTES, 1024), kIdescPV,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+                  (!first || kk > 0) ? 1u : 0u);
     }
     return true;
   };
 
-  TileIter it;
-  it.init(p, qt, sparse);
-  int n = 0;
-  uint32_t bits;
-  bool has = ok && it.next(n, bits);
-  int k_slot = 0, v_slot = 0;
-  if (has) {
-    ok = take(k_slot);
-    if (ok) {
-      qk(0, k_slot);
+  for (int k = 0; ok; ++k) {
+    const int w = item_index(k, total);
+    if (w < 0) break;
+    const Item im = item_of(p, w);
+    if (!(ok = mbar_wait_a(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(k) & 1u, sh.abort_flag(), p.status))) break;
+    tc_fence_after_sync();
+    TileIter it;
+    it.init(p, im.qt, im.sparse);
+    int n = 0;
+    uint32_t bits;
+    if (!it.next(n, bits)) {          // no KV tile: Q is free again at once
+      tc_commit_a(sh.bar(Smem::Q_EMPTY));
+      continue;
+    }
+    int k_slot = 0, v_slot = 0;
+    if (!(ok = take(k_slot))) break;
+    qk(0, k_slot);
+    qk(1, k_slot);
+    tc_commit_a(sh.bar(Smem::EMPTY0 + k_slot));
+    bool has_next = it.next(n, bits);
+    if (!has_next) tc_commit_a(sh.bar(Smem::Q_EMPTY));     // the last QK of this item is issued
+    for (int j = 0;; ++j) {
+      if (!(ok = take(v_slot))) break;
+      if (!(ok = pv(0, j == 0, v_slot))) break;
+      if (has_next) {
+        if (!(ok = take(k_slot))) break;
+        qk(0, k_slot);
+      } else {
+        tc_commit_a(sh.bar(Smem::O_DONE0));
+      }
+      if (!(ok = pv(1, j == 0, v_slot))) break;
+      ++jp;
+      tc_commit_a(sh.bar(Smem::EMPTY0 + v_slot));
+      if (!has_next) {
+        tc_commit_a(sh.bar(Smem::O_DONE0 + 1));
+        break;
+      }
       qk(1, k_slot);
-      tc_commit(&sh.empty[k_slot]);
+      tc_commit_a(sh.bar(Smem::EMPTY0 + k_slot));
+      has_next = it.next(n, bits);
+      if (!has_next) tc_commit_a(sh.bar(Smem::Q_EMPTY));
     }
+    ++done_items;
   }
-  for (int j = 0; ok && has; ++j) {
-    const bool has_next = it.next(n, bits);
-    if (!(ok = take(v_slot))) break;
-    if (!(ok = pv(0, j, v_slot))) break;
-    if (has_next) {
-      if (!(ok = take(k_slot))) break;
-      qk(0, k_slot);
-    } else {
-      tc_commit(&sh.o_done[0]);
-    }
-    if (!(ok = pv(1, j, v_slot))) break;
-    tc_commit(&sh.empty[v_slot]);
-    if (has_next) {
-      qk(1, k_slot);
-      tc_commit(&sh.empty[k_slot]);
-    } else {
-      tc_commit(&sh.o_done[1]);
-    }
-    has = has_next;
-  }
-  if (*sh.abort) {
-    tc_commit(sh.drain);
-    mbar_wait_drain(sh.drain, 0, kDrainNs);
+  if (ld_shared_s32(sh.abort_flag())) {  // let every MMA this thread issued finish before exit
+    tc_commit_a(sh.bar(Smem::DRAIN));
+    mbar_wait_drain_a(sh.bar(Smem::DRAIN), 0, kDrainNs);
   }
 }
 
-FA_DEV bool warp_wait(uint64_t *bar, uint32_t parity, const Shared &sh, const Params &p) {
-  const bool done = mbar_wait(bar, parity, sh.abort, p.status);
+FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Params &p) {
+  const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
   return __all_sync(0xffffffffu, done);
 }
 
-FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt, int b, int h,
-                        int t, bool sparse) {
+FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int total, int t) {
   const int r = threadIdx.x - 128 * t;                 // row within the tile
   const uint32_t quad = (threadIdx.x >> 5) & 3u;
   const uint32_t s_base = tmem + ((quad * 32u) << 16) + 256u * t;
   const uint32_t o_base = s_base + 128u;
   const float c = p.scale_log2;
-  float m_run = -INFINITY, l_run = 0.f;
-
-  TileIter it;
-  it.init(p, qt, sparse);
-  int j = 0, n = 0;
-  uint32_t bits = 0;
+  int js = 0;           // S tiles consumed (continues across items)
+  int done_items = 0;   // items whose O this warpgroup has read
   bool ok = true;
-  while (it.next(n, bits)) {
-    if (!warp_wait(&sh.s_full[t], static_cast<uint32_t>(j) & 1u, sh, p)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after_sync();
-    float s[BN];
-#pragma unroll
-    for (int q4 = 0; q4 < BN / 32; ++q4) {
-      uint32_t raw[32];
-      tmem_ld32(s_base + q4 * 32, raw);
-      tmem_ld_wait(raw);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(raw[i]);
-    }
-    const bool diag = (n == qt);
-    if (diag || bits != 0xFu) {
-      const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
-#pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
-        s[i] = keep ? s[i] : -INFINITY;
+  for (int k = 0; ok; ++k) {
+    const int w = item_index(k, total);
+    if (w < 0) break;
+    const Item im = item_of(p, w);
+    const int h = im.h0 + t;
+    float m_run = -INFINITY, l_run = 0.f;
+    TileIter it;
+    it.init(p, im.qt, im.sparse);
+    int j = 0, n = 0;
+    uint32_t bits = 0;
+    while (it.next(n, bits)) {
+      if (!warp_wait(sh.bar(Smem::S_FULL0 + t), static_cast<uint32_t>(js) & 1u, sh, p)) {
+        ok = false;
+        break;
       }
-    }
-    // Row max: 3-input max over pairs, 8 independent chains.
-    float mx8[8];
+      tc_fence_after_sync();
+      float s[BN];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+      for (int q4 = 0; q4 < BN / 32; ++q4) {
+        uint32_t raw[32];
+        tmem_ld32(s_base + q4 * 32, raw);
+        tmem_ld_wait(raw);
 #pragma unroll
-    for (int i = 16; i < BN; i += 16)
+        for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(raw[i]);
+      }
+      const bool diag = (n == im.qt);
+      if (diag || bits != 0xFu) {
+        const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[i + 2 * k], s[i + 2 * k + 1]);
-    const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                           fmaxf(mx8[6], mx8[7]));
-    const float m_new = fmaxf(m_run, mx * c);
-    const bool need = m_new > m_run + kRescaleThreshold;
-    const float m_next = need ? m_new : m_run;
-    const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
-    // p = 2^(s*c - m), two lanes per instruction; every fourth pair of keys
-    // on the FMA pipe, the rest on ex2.approx.
-    const uint64_t c2 = f2_make(c, c), negm2 = f2_make(-m_use, -m_use);
-    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-    for (int q2 = 0; q2 < 2; ++q2) {
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int k0 = q2 * 64 + 2 * i;
-        const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
-        float p0, p1;
-        if ((k0 & 7) >= 8 - kPolyPer8) {
-          ex2_poly2(x, p0, p1);
-        } else {
-          float x0, x1;
-          f2_split(x, x0, x1);
-          p0 = ex2(x0);
-          p1 = ex2(x1);
+        for (int i = 0; i < BN; ++i) {
+          const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
+          s[i] = keep ? s[i] : -INFINITY;
         }
-        acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
-        pk[i] = pack_bf16x2(p0, p1);
       }
-      tmem_st32(s_base + q2 * 32, pk);
-    }
-    if (j > 0 && __any_sync(0xffffffffu, need)) {
-      const float alpha = need ? ex2(m_run - m_new) : 1.0f;
+      // Row max: 3-input max over pairs, 8 independent chains.
+      float mx8[8];
 #pragma unroll
-      for (int q4 = 0; q4 < HD / 32; ++q4) {
-        uint32_t o[32];
+      for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmaxf(s[2 * kk], s[2 * kk + 1]);
+#pragma unroll
+      for (int i = 16; i < BN; i += 16)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmax3(mx8[kk], s[i + 2 * kk], s[i + 2 * kk + 1]);
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
+      const float m_new = fmaxf(m_run, mx * c);
+      const bool need = m_new > m_run + kRescaleThreshold;
+      const float m_next = need ? m_new : m_run;
+      const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
+      // p = 2^(s*c - m), two lanes per instruction; every fourth pair of
+      // keys on the FMA pipe, the rest on ex2.approx.
+      const uint64_t c2 = f2_make(c, c), negm2 = f2_make(-m_use, -m_use);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int k0 = q2 * 64 + 2 * i;
+          const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
+          float p0, p1;
+          if ((k0 & 7) >= 8 - kPolyPer8) {
+            ex2_poly2(x, p0, p1);
+          } else {
+            float x0, x1;
+            f2_split(x, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_base + q2 * 32, pk);
+      }
+      // S_t(j) ready implies PV_t(j-1) is done (MMAs complete in order), so
+      // O_t may be rescaled here before P_t(j) is released.
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2(m_run - m_new) : 1.0f;
+#pragma unroll
+        for (int q4 = 0; q4 < HD / 32; ++q4) {
+          uint32_t o[32];
+          tmem_ld32(o_base + q4 * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(o_base + q4 * 32, o);
+        }
+      }
+      if (need) l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
+      m_run = m_next;
+      {
+        float a0, a1;
+        f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+        l_run += a0 + a1;
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      mbar_arrive_a(sh.bar(Smem::P_FULL0 + t));
+      ++j;
+      ++js;
+    }
+    if (!ok) break;
+
+    // Epilogue: O / l -> bf16, one row per thread; then hand O back.
+    const bool have_o =
+        j > 0 && warp_wait(sh.bar(Smem::O_DONE0 + t), static_cast<uint32_t>(done_items) & 1u, sh, p);
+    if (j > 0 && !have_o) break;
+    tc_fence_after_sync();
+    const int tok = im.qt * BM + r;
+    const bool store = (tok < p.S) && !ld_shared_s32(sh.abort_flag());
+    const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+    __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(im.b) * p.S + tok) * p.Hq + h) * HD;
+#pragma unroll
+    for (int q4 = 0; q4 < HD / 32; ++q4) {
+      uint32_t o[32];
+      if (have_o) {
         tmem_ld32(o_base + q4 * 32, o);
         tmem_ld_wait(o);
+      } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-        tmem_st32(o_base + q4 * 32, o);
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (store) {
+        uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 wv;
+          wv.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+          wv.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+          wv.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+          wv.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+          dst[v] = wv;
+        }
       }
     }
-    if (need) l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
-    m_run = m_next;
-    {
-      float a0, a1, b0, b1;
-      f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
-      l_run += a0 + a1;
-      (void)b0;
-      (void)b1;
-    }
-    tmem_st_wait();
-    tc_fence_before_sync();
-    mbar_arrive(&sh.p_full[t]);
-    ++j;
-  }
-
-  const bool have_o = ok && j > 0 && warp_wait(&sh.o_done[t], 0u, sh, p);
-  tc_fence_after_sync();
-  const int tok = qt * BM + r;
-  const bool store = (tok < p.S) && !*sh.abort;
-  const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
-  __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(b) * p.S + tok) * p.Hq + h) * HD;
-#pragma unroll
-  for (int q4 = 0; q4 < HD / 32; ++q4) {
-    uint32_t o[32];
     if (have_o) {
-      tmem_ld32(o_base + q4 * 32, o);
-      tmem_ld_wait(o);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] = 0u;
+      tc_fence_before_sync();
+      mbar_arrive_a(sh.bar(Smem::O_FREE0 + t));
+      ++done_items;
     }
-    if (store) {
-      uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-        w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-        w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-        w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-        dst[v] = w;
-      }
+    if (store && p.lse) {
+      const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      p.lse[(static_cast<size_t>(im.b) * p.Hq + h) * p.S + tok] = lse;
     }
-  }
-  if (store && p.lse) {
-    const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-    p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + tok] = lse;
   }
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const Params p) {
+                    const __grid_constant__ CUtensorMap tmV, const Params p, int total_items) {
   extern __shared__ uint8_t smem_raw[];
-  const Shared sh = carve(smem_raw);
+  const Smem sh = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // CTA -> (query tile, batch, head pair): longest causal rows first; the
-  // head pairs of one KV group are adjacent.
-  const int hp_count = p.Hq / NQ;
-  const int bh = p.B * hp_count;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / bh;
-  const int rem = static_cast<int>(blockIdx.x) % bh;
-  const int b = rem / hp_count, h0 = (rem % hp_count) * NQ, kvh = h0 / p.G;
-  const int mode = p.mode ? p.mode[b] : p.mode_default;
-  const bool sparse = (mode == FA_MODE_SPARSE) && p.row_ptr != nullptr;
 
   if (threadIdx.x == 0) {
-    mbar_init(sh.q_full, 1);
+    mbar_init_a(sh.bar(Smem::Q_FULL), 1);
+    mbar_init_a(sh.bar(Smem::Q_EMPTY), 1);
     for (int i = 0; i < NSLOT; ++i) {
-      mbar_init(&sh.full[i], 1);
-      mbar_init(&sh.empty[i], 1);
+      mbar_init_a(sh.bar(Smem::FULL0 + i), 1);
+      mbar_init_a(sh.bar(Smem::EMPTY0 + i), 1);
     }
     for (int t = 0; t < NQ; ++t) {
-      mbar_init(&sh.s_full[t], 1);
-      mbar_init(&sh.p_full[t], 128);
-      mbar_init(&sh.o_done[t], 1);
+      mbar_init_a(sh.bar(Smem::S_FULL0 + t), 1);
+      mbar_init_a(sh.bar(Smem::P_FULL0 + t), 128);
+      mbar_init_a(sh.bar(Smem::O_DONE0 + t), 1);
+      mbar_init_a(sh.bar(Smem::O_FREE0 + t), 128);
     }
-    mbar_init(sh.drain, 1);
-    *sh.abort = 0;
+    mbar_init_a(sh.bar(Smem::DRAIN), 1);
+    st_shared_s32(sh.abort_flag(), 0);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
   if (warp == WARP_MMA) {
-    tmem_alloc(sh.tmem_slot, TMEM_COLS);
+    tmem_alloc_a(sh.tmem_slot(), TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem = *sh.tmem_slot;
+  const uint32_t tmem = static_cast<uint32_t>(ld_shared_s32(sh.tmem_slot()));
 
   if (warp >= WARP_PRODUCER) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
     if (warp == WARP_PRODUCER) {
-      if (lane == 0) run_producer(sh, &tmQ, &tmK, &tmV, p, qt, b, h0, kvh, sparse);
+      if (lane == 0) run_producer(sh, &tmQ, &tmK, &tmV, p, total_items);
     } else if (warp == WARP_MMA) {
-      if (lane == 0) run_mma(sh, tmem, p, qt, sparse);
+      if (lane == 0) run_mma(sh, tmem, p, total_items);
       __syncwarp();
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
-    const int t = warp >> 2;
-    run_softmax(sh, tmem, p, qt, b, h0 + t, t, sparse);
+    run_softmax(sh, tmem, p, total_items, warp >> 2);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -946,9 +1007,20 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   const long long grid =
       static_cast<long long>(p.n_qtiles) * a.B * (two_tiles ? a.Hq / 2 : a.Hq);
   if (grid <= 0 || grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  if (two_tiles)
-    prefill2::prefill2_kernel<<<static_cast<unsigned>(grid), prefill2::NUM_THREADS,
-                                prefill2::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  if (two_tiles) {
+    // Persistent: one CTA per SM walks the work items.
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+#ifndef FA_PREFILL_PERSISTENT
+#define FA_PREFILL_PERSISTENT 1
+#endif
+    const long long cap = FA_PREFILL_PERSISTENT ? sms : grid;
+    const int ctas = static_cast<int>(grid < cap ? grid : cap);
+    prefill2::prefill2_kernel<<<ctas, prefill2::NUM_THREADS, prefill2::SMEM_BYTES, stream>>>(
+        tmQ, tmK, tmV, p, static_cast<int>(grid));
+  }
   else
     prefill_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmK,
                                                                                     tmV, p);
