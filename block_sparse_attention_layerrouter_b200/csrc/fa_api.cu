@@ -88,6 +88,7 @@ int check_router(const void *q, int B, int S, int Hq, int D, int n_head, int n_t
   if (S < n_head + n_tail) return FA_ERR_UNSUPPORTED;
   if (D != kHeadDim) return FA_ERR_UNSUPPORTED;
   if (hidden < 1 || hidden > 65536) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(Hq) * kHeadDim * 4 > 200 * 1024) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 

@@ -778,13 +778,11 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
       }
       tc_fence_after_sync();
       float s[BN];
+      {
+        uint32_t raw[BN];
+        tmem_ld128_wait(s_base, raw);
 #pragma unroll
-      for (int q4 = 0; q4 < BN / 32; ++q4) {
-        uint32_t raw[32];
-        tmem_ld32(s_base + q4 * 32, raw);
-        tmem_ld_wait(raw);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(raw[i]);
+        for (int i = 0; i < BN; ++i) s[i] = __uint_as_float(raw[i]);
       }
       const bool diag = (n == im.qt);
       if (diag || bits != 0xFu) {

@@ -4,10 +4,9 @@
 // [pi_FA, pi_SA] = W2 h + b2, hard routing by argmax (a tie routes to FULL).
 //
 // Three small launches, all memory/latency bound:
-//   pool_kernel   grid (Hq, B): 16 token groups x 16 chunks of 8 dims, fp32
-//                 sums reduced in shared memory -> x [B, Hq*D]
-//   hidden_kernel grid (ceil(H1/8), B): one warp per hidden unit, coalesced
-//                 float4 reads of the W1 row -> h [B, H1]
+//   pool_kernel   grid (Hq, B, 5 token slices): fp32 partial sums per slice
+//   hidden_kernel grid (H1, B): sums the slices into x (shared memory), then
+//                 one W1 row per CTA with coalesced float4 reads -> h [B, H1]
 //   head_kernel   grid (B): one warp per logit, then the argmax -> mode [B]
 #include "fa_common.cuh"
 #include "fa_internal.h"
@@ -16,15 +15,21 @@ namespace fa {
 namespace router {
 
 constexpr int HD = 128;
+constexpr int kPoolSlices = 5;     // token slices per (head, batch)
 
-__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *q, float *x, int S, int Hq,
-                                                   int n_head, int n_tail) {
+// Partial sums of the selected tokens: slice z of (head h, batch b) adds
+// up its share of the n_head + n_tail selected tokens for all 128 dims.
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *q, float *part, int S,
+                                                   int Hq, int n_head, int n_tail) {
   __shared__ float red[16][HD];
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int h = blockIdx.x, b = blockIdx.y, z = blockIdx.z, B = gridDim.y;
   const int chunk = threadIdx.x & 15, grp = threadIdx.x >> 4;
   const int n_sel = n_head + n_tail;
+  const int per = (n_sel + kPoolSlices - 1) / kPoolSlices;
+  const int i0 = z * per, i1 = min(n_sel, i0 + per);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int i = grp; i < n_sel; i += 16) {
+#pragma unroll 4
+  for (int i = i0 + grp; i < i1; i += 16) {
     const int t = i < n_head ? i : S - n_tail + (i - n_head);
     const uint4 v = *reinterpret_cast<const uint4 *>(
         q + ((static_cast<size_t>(b) * S + t) * Hq + h) * HD + chunk * 8);
@@ -42,35 +47,48 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *q, float
     float s = 0.f;
 #pragma unroll
     for (int g = 0; g < 16; ++g) s += red[g][threadIdx.x];
-    x[static_cast<size_t>(b) * Hq * HD + h * HD + threadIdx.x] = s / static_cast<float>(n_sel);
+    part[(static_cast<size_t>(z) * B + b) * Hq * HD + h * HD + threadIdx.x] = s;
   }
 }
 
-__global__ void __launch_bounds__(256) hidden_kernel(const float *x, const float *w1,
+// One CTA per (hidden unit, batch): x = (sum of the slices) / n_sel into
+// shared memory (head-major x[h*D + d]), then ReLU(W1[u] . x + b1[u]).
+__global__ void __launch_bounds__(256) hidden_kernel(const float *part, const float *w1,
                                                      const float *b1, float *hid, int in_f,
-                                                     int hidden) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u = blockIdx.x * 8 + warp, b = blockIdx.y;
-  if (u >= hidden) return;
+                                                     int hidden, float inv_n) {
+  extern __shared__ float xs[];
+  __shared__ float red[8];
+  const int u = blockIdx.x, b = blockIdx.y, B = gridDim.y, tid = threadIdx.x;
+  for (int i = tid; i < in_f; i += 256) {
+    float v = 0.f;
+#pragma unroll
+    for (int z = 0; z < kPoolSlices; ++z) v += part[(static_cast<size_t>(z) * B + b) * in_f + i];
+    xs[i] = v * inv_n;
+  }
+  __syncthreads();
   const float *wr = w1 + static_cast<size_t>(u) * in_f;
-  const float *xr = x + static_cast<size_t>(b) * in_f;
   float s = 0.f;
   if ((in_f & 3) == 0) {
-    for (int i = lane * 4; i < in_f; i += 128) {
+#pragma unroll 4
+    for (int i = tid * 4; i < in_f; i += 1024) {
       const float4 wv = *reinterpret_cast<const float4 *>(wr + i);
-      const float4 xv = *reinterpret_cast<const float4 *>(xr + i);
-      s = fmaf(wv.x, xv.x, s);
-      s = fmaf(wv.y, xv.y, s);
-      s = fmaf(wv.z, xv.z, s);
-      s = fmaf(wv.w, xv.w, s);
+      s = fmaf(wv.x, xs[i], s);
+      s = fmaf(wv.y, xs[i + 1], s);
+      s = fmaf(wv.z, xs[i + 2], s);
+      s = fmaf(wv.w, xs[i + 3], s);
     }
   } else {
-    for (int i = lane; i < in_f; i += 32) s = fmaf(wr[i], xr[i], s);
+    for (int i = tid; i < in_f; i += 256) s = fmaf(wr[i], xs[i], s);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) {
-    const float v = s + (b1 ? b1[u] : 0.f);
+  if ((tid & 31) == 0) red[tid >> 5] = s;
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w];
+    const float v = t + (b1 ? b1[u] : 0.f);
     hid[static_cast<size_t>(b) * hidden + u] = v > 0.f ? v : 0.f;
   }
 }
@@ -98,22 +116,28 @@ __global__ void __launch_bounds__(64) head_kernel(const float *hid, const float 
 }  // namespace router
 
 size_t router_workspace_bytes(int B, int Hq, int D, int hidden) {
-  const size_t x = static_cast<size_t>(B) * Hq * D * sizeof(float);
+  const size_t x = static_cast<size_t>(router::kPoolSlices) * B * Hq * D * sizeof(float);
   const size_t h = static_cast<size_t>(B) * hidden * sizeof(float);
   return ((x + 255) & ~static_cast<size_t>(255)) + ((h + 255) & ~static_cast<size_t>(255));
 }
 
 int launch_router(const RouterLaunch &a, cudaStream_t stream) {
   using namespace router;
-  const size_t xbytes = static_cast<size_t>(a.B) * a.Hq * HD * sizeof(float);
-  float *x = reinterpret_cast<float *>(a.workspace);
+  const int in_f = a.Hq * HD;
+  const size_t pbytes = static_cast<size_t>(kPoolSlices) * a.B * in_f * sizeof(float);
+  float *part = reinterpret_cast<float *>(a.workspace);
   float *hid = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.workspace) +
-                                         ((xbytes + 255) & ~static_cast<size_t>(255)));
-  pool_kernel<<<dim3(a.Hq, a.B), 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16 *>(a.q),
-                                                   x, a.S, a.Hq, a.n_head, a.n_tail);
+                                         ((pbytes + 255) & ~static_cast<size_t>(255)));
+  const size_t xs_bytes = static_cast<size_t>(in_f) * sizeof(float);
+  if (xs_bytes > 48 * 1024 &&
+      cudaFuncSetAttribute(hidden_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(xs_bytes)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  pool_kernel<<<dim3(a.Hq, a.B, kPoolSlices), 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16 *>(a.q), part, a.S, a.Hq, a.n_head, a.n_tail);
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
-  hidden_kernel<<<dim3((a.hidden + 7) / 8, a.B), 256, 0, stream>>>(x, a.w1, a.b1, hid,
-                                                                   a.Hq * HD, a.hidden);
+  hidden_kernel<<<dim3(a.hidden, a.B), 256, xs_bytes, stream>>>(
+      part, a.w1, a.b1, hid, in_f, a.hidden, 1.0f / static_cast<float>(a.n_head + a.n_tail));
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   head_kernel<<<a.B, 64, 0, stream>>>(hid, a.w2, a.b2, a.logits, a.mode, a.hidden);
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;

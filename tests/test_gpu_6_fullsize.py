@@ -100,3 +100,34 @@ def test_decode_b8_l131072(mode):
                                  1 / math.sqrt(128), mode, 64, wl.sink, wl.window)
     assert_close_attention(to_f64(o[bs]), ref, "decode mode=%d" % mode)
     np.testing.assert_allclose(to_f64(lse[bs]), ref_lse, atol=LSE_ABS_TOL)
+
+
+def test_bench_step_qwen3_4b_routed_layers():
+    """The benchmark's step at full size: CSR, two routed layers (router head
+    bias -> FULL, -> SPARSE) reading the mode on the device, and one decode
+    token per layer with the device-side mode; sampled rows vs the oracle."""
+    wl = W["qwen3-4b-layer-s8192"]
+    B, S, Hq, Hkv = wl.B, wl.S, wl.Hq, wl.Hkv
+    c = capi.cfg(64, wl.sink, wl.window)
+    rp, ci = capi.blocksparse_index(S, c)
+    mask = oracle.rows_to_dense_mask(oracle.blocksparse_rows(S, 64, wl.sink, wl.window))
+    rows = inputs.sample_rows(B, S, Hq, Hkv, seed=wl.seed + 5, n_random=128, n_groups=1)
+    rt = torch.from_numpy(rows).cuda()
+    for li, (bias, want) in enumerate((((0.1, 0.0), 0), ((0.0, 0.1), 1))):
+        q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, wl.seed + 7919 * li, device="cuda")
+        w1, b1, w2, b2 = inputs.router_weights(Hq * 128, wl.hidden, wl.seed, li, b2=bias)
+        status = zero_status()
+        o, logits, mode = capi.hybrid_layer(q, k, v, w1.cuda(), b1.cuda(), w2.cuda(), b2.cuda(),
+                                            rp, ci, c, status=status)
+        qd = inputs.randn_bf16((B, Hq, 128), wl.seed + 31 * li + 5, device="cuda")
+        sl = torch.full((B,), S, dtype=torch.int32, device="cuda")
+        od = capi.attn_decode(qd, k, v, sl, mode_dev=mode, c=c, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0 and int(mode.item()) == want
+        qb, kb, vb = inputs.bits(q), inputs.bits(k), inputs.bits(v)
+        ref, _ = oracle.attention_rows(qb, kb, vb, 1 / math.sqrt(128), rows,
+                                       mask if want == 1 else None)
+        assert_close_attention(to_f64(o[rt[:, 0], rt[:, 2], rt[:, 1]]), ref, "routed layer %d" % li)
+        ref_d, _ = oracle.decode(inputs.bits(qd), kb, vb, np.full(B, S, np.int32),
+                                 1 / math.sqrt(128), want, 64, wl.sink, wl.window)
+        assert_close_attention(to_f64(od), ref_d, "decode layer %d" % li)
