@@ -193,6 +193,23 @@ def router_decide(q_bits, w1, b1, w2, b2, n_head=N_HEAD_TOKENS, n_tail=N_TAIL_TO
     return logits, router_argmax(logits), x
 
 
+def router_soft(logits: np.ndarray, gumbel=None, tau: float = 1.0) -> np.ndarray:
+    """[FLUX] training-time relaxation: r_soft = exp((pi_FA + g_FA)/tau) /
+    sum_i exp((pi_i + g_i)/tau) over i in {FA, SA}, the Gumbel noise g given
+    as an input.  Returns fp64 [B], the weight of the FULL output."""
+    z = np.asarray(logits, np.float64)
+    if gumbel is not None:
+        z = z + np.asarray(gumbel, np.float64)
+    return softmax(z / float(tau))[:, 0]
+
+
+def soft_mix(o_full: np.ndarray, o_sparse: np.ndarray, r: np.ndarray) -> np.ndarray:
+    """[FLUX] training-time output: y = r * O_FA + (1 - r) * O_SA, r per
+    sequence (leading batch axis)."""
+    r = np.asarray(r, np.float64).reshape((-1,) + (1,) * (o_full.ndim - 1))
+    return r * o_full + (1.0 - r) * o_sparse
+
+
 # ---------------------------------------------------------- sparse pattern
 def blocksparse_rows(S: int, block: int = BLOCK, sink: int = SINK_TOKENS,
                      window: int = 2 * BLOCK):
