@@ -60,6 +60,10 @@ _SIGNATURES = {
     "fa_noalloc_scratch_bytes": (_SZ, []),
     "fa_attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP,
                                     SparseCfg, _VP, _VP, _VP, _VP]),
+    "fa_router_soft": (_I, [_VP, _VP, _I, _F, _VP, _VP]),
+    "fa_soft_routed_layer": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
+                                  _VP, _VP, _F, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
+                                  _VP]),
     "fa_hybrid_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_hybrid_layer": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
                              _VP, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
@@ -287,3 +291,41 @@ def hybrid_layer(q, k, v, w1, b1, w2, b2, row_ptr, col_idx, c: SparseCfg, scale=
                                _ptr(status), _stream(dev))
     _check("fa_hybrid_layer", rc)
     return o, logits, mode
+
+
+# ------------------------------------------------------------ soft routing
+def router_soft(logits, gumbel=None, tau=1.0, r=None) -> torch.Tensor:
+    """fa_router_soft: weight of the FULL output per sequence."""
+    _need(logits, "logits", torch.float32, 2)
+    if gumbel is not None:
+        _need(gumbel, "gumbel", torch.float32, 2)
+    B = logits.shape[0]
+    r = torch.empty(B, device=logits.device, dtype=torch.float32) if r is None else r
+    _check("fa_router_soft", lib().fa_router_soft(_ptr(logits), _ptr(gumbel), B, float(tau),
+                                                  _ptr(r), _stream(logits.device)))
+    return r
+
+
+def soft_routed_layer(q, k, v, w1, b1, w2, b2, row_ptr, col_idx, c: SparseCfg, gumbel=None,
+                      tau=1.0, scale=None, o=None, logits=None, r=None, workspace=None,
+                      status=None):
+    """fa_soft_routed_layer -> (y, logits, r)."""
+    B, S, Hq, Hkv, D, o = _prefill_common(q, k, v, o, None)
+    hidden = w1.shape[0]
+    dev = q.device
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    logits = torch.empty(B, 2, device=dev, dtype=torch.float32) if logits is None else logits
+    r = torch.empty(B, device=dev, dtype=torch.float32) if r is None else r
+    if gumbel is not None:
+        _need(gumbel, "gumbel", torch.float32, 2)
+    ws_bytes = hybrid_workspace_size(B, Hq, D, hidden)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    rc = lib().fa_soft_routed_layer(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, S, Hq, Hkv, D, scale,
+                                    _ptr(w1), _ptr(b1), hidden, _ptr(w2), _ptr(b2), _ptr(gumbel),
+                                    float(tau), c, _ptr(row_ptr), _ptr(col_idx), _ptr(logits),
+                                    _ptr(r), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _ptr(status),
+                                    _stream(dev))
+    _check("fa_soft_routed_layer", rc)
+    return o, logits, r

@@ -223,4 +223,37 @@ FA_API int fa_hybrid_layer(const void *q, const void *k, const void *v, void *o,
   return launch_prefill(a, st);
 }
 
+FA_API int fa_router_soft(const float *logits, const float *gumbel, int B, float tau,
+                          float *r_out, void *stream) {
+  if (!logits || !r_out || B <= 0) return FA_ERR_INVALID_ARG;
+  if (!(tau > 0.f)) return FA_ERR_INVALID_ARG;
+  return launch_router_soft(logits, gumbel, B, tau, r_out, static_cast<cudaStream_t>(stream));
+}
+
+FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v, void *o, int B, int S,
+                                int Hq, int Hkv, int D, float scale, const float *w1,
+                                const float *b1, int hidden, const float *w2, const float *b2,
+                                const float *gumbel, float tau, fa_sparse_cfg cfg,
+                                const int32_t *row_ptr, const int32_t *col_idx, float *logits_out,
+                                float *r_out, void *workspace, size_t ws_bytes,
+                                int32_t *dev_status, void *stream) {
+  if (int rc = check_prefill(q, k, v, o, B, S, Hq, Hkv, D)) return rc;
+  if (int rc = check_router(q, B, S, Hq, D, 100, 100, w1, hidden, w2)) return rc;
+  if (int rc = check_cfg(cfg)) return rc;
+  if (!(scale > 0.f) || !(tau > 0.f)) return FA_ERR_INVALID_ARG;
+  if (!row_ptr || !col_idx || !logits_out || !r_out) return FA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < router_workspace_bytes(B, Hq, D, hidden)) return FA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RouterLaunch r{q, B, S, Hq, 100, 100, w1, b1, w2, b2, hidden, logits_out, nullptr, workspace};
+  if (int rc = launch_router(r, st)) return rc;
+  if (int rc = launch_router_soft(logits_out, gumbel, B, tau, r_out, st)) return rc;
+  PrefillLaunch full{q, k, v, o, nullptr, B, S, Hq, Hkv, scale, nullptr, nullptr, nullptr,
+                     FA_MODE_FULL, dev_status};
+  if (int rc = launch_prefill(full, st)) return rc;
+  PrefillLaunch sparse{q, k, v, o, nullptr, B, S, Hq, Hkv, scale, row_ptr, col_idx, nullptr,
+                       FA_MODE_SPARSE, dev_status};
+  sparse.mix_r = r_out;
+  return launch_prefill(sparse, st);
+}
+
 }  // extern "C"

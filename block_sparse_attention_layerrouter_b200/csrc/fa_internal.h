@@ -24,6 +24,7 @@ struct PrefillLaunch {
   const int32_t *mode_dev;           // nullptr: use mode_default
   int mode_default;
   int32_t *status;
+  const float *mix_r = nullptr;      // soft-routing mix weight per batch, or nullptr
 };
 int launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
 
@@ -55,6 +56,8 @@ struct RouterLaunch {
   void *workspace;
 };
 size_t router_workspace_bytes(int B, int Hq, int D, int hidden);
+int launch_router_soft(const float *logits, const float *gumbel, int B, float tau, float *r,
+                       cudaStream_t stream);
 int launch_router(const RouterLaunch &a, cudaStream_t stream);
 
 long long index_nnz(int nrows, int sb, int wb);

@@ -50,12 +50,46 @@ struct Params {
   const int32_t *row_ptr;  // sparse CSR (nullptr: full mode only)
   const int32_t *col_idx;
   const int32_t *mode;     // per-batch mode on device, or nullptr
+  const float *mix_r;      // nullptr, or per-batch weight r: O = r * O_old + (1 - r) * O_new
   int32_t *status;
   int B, S, Hq, G;
   int n_qtiles, nqb;
   int mode_default;
   float scale_log2;        // scale * log2(e)
 };
+
+// Writes 32 output columns of one row: o * inv_l as bf16, or, when mix_r is
+// given, r * (the bf16 already there) + (1 - r) * o * inv_l (the soft-routing
+// mix of the FULL output written by an earlier launch and this SPARSE one).
+FA_DEV void store_row_chunk(uint4 *dst, const uint32_t (&o)[32], float inv_l, const float *mix_r,
+                            int b) {
+  if (mix_r == nullptr) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint4 w;
+      w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+      w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+      w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+      w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+      dst[v] = w;
+    }
+    return;
+  }
+  const float r = mix_r[b], rn = (1.0f - r) * inv_l;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint4 old = dst[v];
+    const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
+    uint32_t nw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a0 = __uint_as_float(ow[k] << 16), a1 = __uint_as_float(ow[k] & 0xffff0000u);
+      nw[k] = pack_bf16x2(fmaf(r, a0, rn * __uint_as_float(o[8 * v + 2 * k])),
+                          fmaf(r, a1, rn * __uint_as_float(o[8 * v + 2 * k + 1])));
+    }
+    dst[v] = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+  }
+}
 
 // Walks the 128-key tiles a 128-row query tile (query blocks 2qt, 2qt+1)
 // attends, ascending, each with a 4-bit block mask: bit 2*qs + ks is set iff
@@ -396,15 +430,7 @@ FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt
     }
     if (store) {
       uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-        w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-        w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-        w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-        dst[v] = w;
-      }
+      store_row_chunk(dst, o, inv_l, p.mix_r, b);
     }
   }
   if (store && p.lse) {
@@ -882,15 +908,7 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
       }
       if (store) {
         uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 wv;
-          wv.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-          wv.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-          wv.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-          wv.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-          dst[v] = wv;
-        }
+        prefill::store_row_chunk(dst, o, inv_l, p.mix_r, im.b);
       }
     }
     if (have_o) {
@@ -993,6 +1011,7 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   p.row_ptr = a.row_ptr;
   p.col_idx = a.col_idx;
   p.mode = a.mode_dev;
+  p.mix_r = a.mix_r;
   p.status = a.status;
   p.B = a.B;
   p.S = a.S;

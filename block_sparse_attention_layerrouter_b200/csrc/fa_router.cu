@@ -113,7 +113,27 @@ __global__ void __launch_bounds__(64) head_kernel(const float *hid, const float 
   if (threadIdx.x == 0 && mode) mode[b] = (lg[1] > lg[0]) ? FA_MODE_SPARSE : FA_MODE_FULL;
 }
 
+// Soft routing (training-time relaxation): r = exp((pi_FA + g_FA)/tau) /
+// sum_i exp((pi_i + g_i)/tau) = 1 / (1 + exp(((pi_SA + g_SA) - (pi_FA + g_FA))/tau)).
+__global__ void soft_kernel(const float *logits, const float *gumbel, float inv_tau, float *r,
+                            int B) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  float zf = logits[2 * b], zs = logits[2 * b + 1];
+  if (gumbel) {
+    zf += gumbel[2 * b];
+    zs += gumbel[2 * b + 1];
+  }
+  r[b] = 1.0f / (1.0f + expf((zs - zf) * inv_tau));
+}
+
 }  // namespace router
+
+int launch_router_soft(const float *logits, const float *gumbel, int B, float tau, float *r,
+                       cudaStream_t stream) {
+  router::soft_kernel<<<(B + 127) / 128, 128, 0, stream>>>(logits, gumbel, 1.0f / tau, r, B);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 size_t router_workspace_bytes(int B, int Hq, int D, int hidden) {
   const size_t x = static_cast<size_t>(router::kPoolSlices) * B * Hq * D * sizeof(float);

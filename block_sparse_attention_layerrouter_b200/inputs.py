@@ -105,6 +105,14 @@ def decode_inputs(B, Lmax, Hq, Hkv, D, seed, device="cpu"):
     return q, kc, vc
 
 
+def gumbel(B: int, seed: int) -> torch.Tensor:
+    """Standard Gumbel samples g = -log(-log(U)), U ~ U(0,1), fp32 [B, 2]
+    (the noise of the soft router, drawn here and passed in as an input)."""
+    g = _gen("cpu", seed)
+    u = torch.rand(B, 2, generator=g, dtype=torch.float64).clamp_(1e-12, 1 - 1e-12)
+    return (-torch.log(-torch.log(u))).float()
+
+
 def bits(t: torch.Tensor) -> np.ndarray:
     """Raw bf16 bit patterns of a tensor as a uint16 numpy array (host copy)."""
     assert t.dtype == torch.bfloat16

@@ -148,6 +148,29 @@ FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
                    fa_sparse_cfg cfg, void *o, float *lse, void *workspace,
                    size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/* ------------------------------------------------------ soft routing ---
+ * "Flux Attention", router paragraph on training: the Gumbel-softmax
+ * relaxation r = exp((pi_FA + g_FA)/tau) / sum_i exp((pi_i + g_i)/tau) and
+ * the mixed output y = r * O_FA + (1 - r) * O_SA.  The Gumbel samples g are
+ * an input (fp32 [B, 2], nullable = no noise); tau > 0.
+ * fa_router_soft: logits fp32 [B, 2] (pi_FA, pi_SA) -> r_out fp32 [B].
+ * fa_soft_routed_layer: router logits, r, one FULL launch writing O_FA into
+ * o, then one SPARSE launch whose epilogue writes r*O_FA + (1-r)*O_SA over
+ * it (O_FA is rounded to bf16 in between).  Forward only; no LSE.
+ *   logits_out fp32 [B, 2], r_out fp32 [B]: device, required.
+ *   workspace >= fa_router_workspace_size(B, Hq, D, hidden). */
+FA_API int fa_router_soft(const float *logits, const float *gumbel, int B,
+                          float tau, float *r_out, void *stream);
+FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v,
+                                void *o, int B, int S, int Hq, int Hkv, int D,
+                                float scale, const float *w1, const float *b1,
+                                int hidden, const float *w2, const float *b2,
+                                const float *gumbel, float tau,
+                                fa_sparse_cfg cfg, const int32_t *row_ptr,
+                                const int32_t *col_idx, float *logits_out,
+                                float *r_out, void *workspace, size_t ws_bytes,
+                                int32_t *dev_status, void *stream);
+
 /* ------------------------------------------- decode without allocation ---
  * The pages have no counterpart to this entry point; it exists for callers
  * that cannot allocate device memory where they run decode (a plugin behind
