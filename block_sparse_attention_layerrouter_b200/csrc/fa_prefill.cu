@@ -633,6 +633,18 @@ FA_DEV int item_index(int k, int total) {
   return w < total ? w : -1;
 }
 
+// A wait whose result is the same for every lane of the warp (warp-collective
+// instructions follow every wait).
+FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Params &p) {
+  const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
+  return __all_sync(0xffffffffu, done);
+}
+FA_DEV bool warp_aborted(const Smem &sh) {
+  return __any_sync(0xffffffffu, ld_shared_s32(sh.abort_flag()) != 0);
+}
+
+// The producer and MMA roles run on all 32 lanes of their warp with
+// warp-uniform state; one elected lane issues each TMA copy, MMA and commit.
 FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
                          const CUtensorMap *tmV, const Params &p, int total) {
   int li = 0;       // ring loads issued (continues across items)
@@ -642,13 +654,14 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
     const int w = item_index(k, total);
     if (w < 0) break;
     const Item im = item_of(p, w);
-    if (k > 0 && !mbar_wait_a(sh.bar(Smem::Q_EMPTY), static_cast<uint32_t>(k - 1) & 1u, sh.abort_flag(), p.status))
+    if (k > 0 && !warp_wait(sh.bar(Smem::Q_EMPTY), static_cast<uint32_t>(k - 1) & 1u, sh, p))
       break;
-    mbar_arrive_expect_tx_a(sh.bar(Smem::Q_FULL), NQ * TILE_BYTES);
+    mbar_arrive_expect_tx_w(sh.bar(Smem::Q_FULL), NQ * TILE_BYTES);
 #pragma unroll
     for (int t = 0; t < NQ; ++t) {
-      tma_load_4d_a(sh.q(t), tmQ, sh.bar(Smem::Q_FULL), 0, im.h0 + t, im.qt * BM, im.b);
-      tma_load_4d_a(sh.q(t) + HALF_BYTES, tmQ, sh.bar(Smem::Q_FULL), 64, im.h0 + t, im.qt * BM, im.b);
+      tma_load_4d_w(sh.q(t), tmQ, sh.bar(Smem::Q_FULL), 0, im.h0 + t, im.qt * BM, im.b);
+      tma_load_4d_w(sh.q(t) + HALF_BYTES, tmQ, sh.bar(Smem::Q_FULL), 64, im.h0 + t, im.qt * BM,
+                    im.b);
     }
     ++nq;
     TileIter it;
@@ -656,11 +669,11 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
     auto load = [&](const CUtensorMap *map, int n) -> bool {
       const int slot = li % NSLOT;
       const uint32_t round = static_cast<uint32_t>(li / NSLOT);
-      if (!mbar_wait_a(sh.bar(Smem::EMPTY0 + slot), (round & 1u) ^ 1u, sh.abort_flag(), p.status)) return false;
-      const uint32_t dst = sh.ring(slot);
-      mbar_arrive_expect_tx_a(sh.bar(Smem::FULL0 + slot), TILE_BYTES);
-      tma_load_4d_a(dst, map, sh.bar(Smem::FULL0 + slot), 0, im.kvh, n * BN, im.b);
-      tma_load_4d_a(dst + HALF_BYTES, map, sh.bar(Smem::FULL0 + slot), 64, im.kvh, n * BN, im.b);
+      if (!warp_wait(sh.bar(Smem::EMPTY0 + slot), (round & 1u) ^ 1u, sh, p)) return false;
+      const uint32_t dst = sh.ring(slot), bar = sh.bar(Smem::FULL0 + slot);
+      mbar_arrive_expect_tx_w(bar, TILE_BYTES);
+      tma_load_4d_w(dst, map, bar, 0, im.kvh, n * BN, im.b);
+      tma_load_4d_w(dst + HALF_BYTES, map, bar, 64, im.kvh, n * BN, im.b);
       ++li;
       return true;
     };
@@ -673,16 +686,24 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
       }
     }
   }
-  if (ld_shared_s32(sh.abort_flag())) {  // let every copy this thread issued land before exit
+  if (warp_aborted(sh)) {  // let every copy this warp issued land before exit
     if (nq > 0) mbar_wait_drain_a(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(nq - 1) & 1u, kDrainNs);
     for (int x = (li > NSLOT ? li - NSLOT : 0); x < li; ++x)
-      mbar_wait_drain_a(sh.bar(Smem::FULL0 + x % NSLOT), static_cast<uint32_t>(x / NSLOT) & 1u, kDrainNs);
+      mbar_wait_drain_a(sh.bar(Smem::FULL0 + x % NSLOT), static_cast<uint32_t>(x / NSLOT) & 1u,
+                        kDrainNs);
   }
 }
 
 FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
+  // Descriptors of the Q tiles (fixed) and of ring slot 0; slot s adds
+  // s * TILE_BYTES / 16 to the start-address field, a K step kk adds the
+  // byte offset / 16 of its 16-column slice.
+  const uint64_t q_desc0 = smem_desc_sw128(sh.q(0), 16, 1024);
+  const uint64_t q_desc1 = smem_desc_sw128(sh.q(1), 16, 1024);
+  const uint64_t k_desc_base = smem_desc_sw128(sh.ring(0), 16, 1024);
+  const uint64_t v_desc_base = smem_desc_sw128(sh.ring(0), HALF_BYTES, 1024);
   int ci = 0;         // ring slots consumed
   int jp = 0;         // P tiles consumed (per tile index, both advance together)
   int done_items = 0; // items that produced an output (o_done / o_free phases)
@@ -691,34 +712,33 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     slot = ci % NSLOT;
     const uint32_t round = static_cast<uint32_t>(ci / NSLOT);
     ++ci;
-    if (!mbar_wait_a(sh.bar(Smem::FULL0 + slot), round & 1u, sh.abort_flag(), p.status)) return false;
+    if (!warp_wait(sh.bar(Smem::FULL0 + slot), round & 1u, sh, p)) return false;
     tc_fence_after_sync();
     return true;
   };
   auto qk = [&](int t, int slot) {
-    const uint32_t q_addr = sh.q(t);
-    const uint32_t k_addr = sh.ring(slot);
+    const uint64_t qd = t ? q_desc1 : q_desc0;
+    const uint64_t kd = k_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
-      const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-      mma_bf16_ss(tmem + 256u * t, smem_desc_sw128(q_addr + off, 16, 1024),
-                  smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+      const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+      mma_bf16_ss_w(tmem + 256u * t, qd + off, kd + off, kIdescQK, kk > 0 ? 1u : 0u);
     }
-    tc_commit_a(sh.bar(Smem::S_FULL0 + t));
+    tc_commit_w(sh.bar(Smem::S_FULL0 + t));
   };
   auto pv = [&](int t, bool first, int slot) -> bool {
-    if (!mbar_wait_a(sh.bar(Smem::P_FULL0 + t), static_cast<uint32_t>(jp) & 1u, sh.abort_flag(), p.status))
+    if (!warp_wait(sh.bar(Smem::P_FULL0 + t), static_cast<uint32_t>(jp) & 1u, sh, p))
       return false;
     if (first && done_items > 0 &&
-        !mbar_wait_a(sh.bar(Smem::O_FREE0 + t), static_cast<uint32_t>(done_items - 1) & 1u, sh.abort_flag(), p.status))
+        !warp_wait(sh.bar(Smem::O_FREE0 + t), static_cast<uint32_t>(done_items - 1) & 1u, sh, p))
       return false;
     tc_fence_after_sync();
-    const uint32_t v_addr = sh.ring(slot);
+    const uint64_t vd = v_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
 #pragma unroll
     for (int kk = 0; kk < BN / 16; ++kk) {
-      mma_bf16_ts(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
-                  smem_desc_sw128(v_addr + kk * 2048, HALF_BYTES, 1024), kIdescPV,
-                  (!first || kk > 0) ? 1u : 0u);
+      mma_bf16_ts_w(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
+                    vd + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                    (!first || kk > 0) ? 1u : 0u);
     }
     return true;
   };
@@ -727,23 +747,23 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     const int w = item_index(k, total);
     if (w < 0) break;
     const Item im = item_of(p, w);
-    if (!(ok = mbar_wait_a(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(k) & 1u, sh.abort_flag(), p.status))) break;
+    if (!(ok = warp_wait(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(k) & 1u, sh, p))) break;
     tc_fence_after_sync();
     TileIter it;
     it.init(p, im.qt, im.sparse);
     int n = 0;
     uint32_t bits;
     if (!it.next(n, bits)) {          // no KV tile: Q is free again at once
-      tc_commit_a(sh.bar(Smem::Q_EMPTY));
+      tc_commit_w(sh.bar(Smem::Q_EMPTY));
       continue;
     }
     int k_slot = 0, v_slot = 0;
     if (!(ok = take(k_slot))) break;
     qk(0, k_slot);
     qk(1, k_slot);
-    tc_commit_a(sh.bar(Smem::EMPTY0 + k_slot));
+    tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
     bool has_next = it.next(n, bits);
-    if (!has_next) tc_commit_a(sh.bar(Smem::Q_EMPTY));     // the last QK of this item is issued
+    if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));     // the last QK of this item is issued
     for (int j = 0;; ++j) {
       if (!(ok = take(v_slot))) break;
       if (!(ok = pv(0, j == 0, v_slot))) break;
@@ -751,32 +771,28 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
         if (!(ok = take(k_slot))) break;
         qk(0, k_slot);
       } else {
-        tc_commit_a(sh.bar(Smem::O_DONE0));
+        tc_commit_w(sh.bar(Smem::O_DONE0));
       }
       if (!(ok = pv(1, j == 0, v_slot))) break;
       ++jp;
-      tc_commit_a(sh.bar(Smem::EMPTY0 + v_slot));
+      tc_commit_w(sh.bar(Smem::EMPTY0 + v_slot));
       if (!has_next) {
-        tc_commit_a(sh.bar(Smem::O_DONE0 + 1));
+        tc_commit_w(sh.bar(Smem::O_DONE0 + 1));
         break;
       }
       qk(1, k_slot);
-      tc_commit_a(sh.bar(Smem::EMPTY0 + k_slot));
+      tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
       has_next = it.next(n, bits);
-      if (!has_next) tc_commit_a(sh.bar(Smem::Q_EMPTY));
+      if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));
     }
     ++done_items;
   }
-  if (ld_shared_s32(sh.abort_flag())) {  // let every MMA this thread issued finish before exit
-    tc_commit_a(sh.bar(Smem::DRAIN));
+  if (warp_aborted(sh)) {  // let every MMA this warp issued finish before exit
+    tc_commit_w(sh.bar(Smem::DRAIN));
     mbar_wait_drain_a(sh.bar(Smem::DRAIN), 0, kDrainNs);
   }
 }
 
-FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Params &p) {
-  const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
-  return __all_sync(0xffffffffu, done);
-}
 
 FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int total, int t) {
   const int r = threadIdx.x - 128 * t;                 // row within the tile
@@ -928,7 +944,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmV, const Params p, int total_items) {
   extern __shared__ uint8_t smem_raw[];
   const Smem sh = carve(smem_raw);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
     mbar_init_a(sh.bar(Smem::Q_FULL), 1);
@@ -962,10 +978,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp >= WARP_PRODUCER) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
     if (warp == WARP_PRODUCER) {
-      if (lane == 0) run_producer(sh, &tmQ, &tmK, &tmV, p, total_items);
+      run_producer(sh, &tmQ, &tmK, &tmV, p, total_items);
     } else if (warp == WARP_MMA) {
-      if (lane == 0) run_mma(sh, tmem, p, total_items);
-      __syncwarp();
+      run_mma(sh, tmem, p, total_items);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
