@@ -60,6 +60,13 @@ _SIGNATURES = {
     "fa_noalloc_scratch_bytes": (_SZ, []),
     "fa_attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP,
                                     SparseCfg, _VP, _VP, _VP, _VP]),
+    "fa_varlen_workspace_size": (_SZ, [_I, _I]),
+    "fa_attn_prefill_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP,
+                                    _VP, _VP, _I, _VP, _SZ, _VP, _VP]),
+    "fa_hybrid_varlen_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_hybrid_layer_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP,
+                                    _VP, _I, _VP, _VP, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ,
+                                    _VP, _VP]),
     "fa_router_soft": (_I, [_VP, _VP, _I, _F, _VP, _VP]),
     "fa_soft_routed_layer": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
                                   _VP, _VP, _F, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
@@ -329,3 +336,61 @@ def soft_routed_layer(q, k, v, w1, b1, w2, b2, row_ptr, col_idx, c: SparseCfg, g
                                     _stream(dev))
     _check("fa_soft_routed_layer", rc)
     return o, logits, r
+
+
+# --------------------------------------------------- variable-length batch
+def _varlen_common(q, k, v, cu_seqlens, o, lse):
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (T, Hkv, D) or v.shape != k.shape:
+        raise ValueError("k/v must be [total_tokens, Hkv, D] matching q")
+    o = torch.empty_like(q) if o is None else o
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    return T, Hq, Hkv, D, cu_seqlens.numel() - 1, o
+
+
+def attn_prefill_varlen(q, k, v, cu_seqlens, max_seqlen, row_ptr=None, col_idx=None,
+                        mode=FA_MODE_FULL, mode_dev=None, scale=None, o=None, lse=None,
+                        workspace=None, status=None) -> torch.Tensor:
+    """fa_attn_prefill_varlen: packed sequences [total_tokens, H, D]."""
+    T, Hq, Hkv, D, B, o = _varlen_common(q, k, v, cu_seqlens, o, lse)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if workspace is None:
+        workspace = torch.empty(int(lib().fa_varlen_workspace_size(B, T)), device=q.device,
+                                dtype=torch.uint8)
+    rc = lib().fa_attn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                      _ptr(cu_seqlens), B, T, int(max_seqlen), Hq, Hkv, D, scale,
+                                      _ptr(row_ptr), _ptr(col_idx), _ptr(mode_dev), int(mode),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _ptr(status), _stream(q.device))
+    _check("fa_attn_prefill_varlen", rc)
+    return o
+
+
+def hybrid_layer_varlen(q, k, v, cu_seqlens, max_seqlen, w1, b1, w2, b2, row_ptr, col_idx,
+                        c: SparseCfg, scale=None, o=None, lse=None, logits=None, mode=None,
+                        workspace=None, status=None):
+    """fa_hybrid_layer_varlen -> (o, logits, mode)."""
+    T, Hq, Hkv, D, B, o = _varlen_common(q, k, v, cu_seqlens, o, lse)
+    hidden = w1.shape[0]
+    dev = q.device
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    logits = torch.empty(B, 2, device=dev, dtype=torch.float32) if logits is None else logits
+    mode = torch.empty(B, device=dev, dtype=torch.int32) if mode is None else mode
+    if workspace is None:
+        workspace = torch.empty(int(lib().fa_hybrid_varlen_workspace_size(B, T, Hq, D, hidden)),
+                                device=dev, dtype=torch.uint8)
+    rc = lib().fa_hybrid_layer_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                      _ptr(cu_seqlens), B, T, int(max_seqlen), Hq, Hkv, D, scale,
+                                      _ptr(w1), _ptr(b1), hidden, _ptr(w2), _ptr(b2), c,
+                                      _ptr(row_ptr), _ptr(col_idx), _ptr(logits), _ptr(mode),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _ptr(status), _stream(dev))
+    _check("fa_hybrid_layer_varlen", rc)
+    return o, logits, mode

@@ -256,4 +256,79 @@ FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v, voi
   return launch_prefill(sparse, st);
 }
 
+FA_API size_t fa_varlen_workspace_size(int B, int total_tokens) {
+  if (B <= 0 || total_tokens <= 0) return 0;
+  return varlen_workspace_bytes(B, total_tokens);
+}
+
+namespace {
+int check_varlen(const void *q, const void *k, const void *v, void *o, const int32_t *cu,
+                 int B, int total, int max_seqlen, int Hq, int Hkv, int D) {
+  if (!cu) return FA_ERR_INVALID_ARG;
+  if (int rc = check_prefill(q, k, v, o, 1, total, Hq, Hkv, D)) return rc;
+  if (B <= 0 || B > 4096 || max_seqlen <= 0 || max_seqlen > total) return FA_ERR_INVALID_ARG;
+  if ((Hq / Hkv) % 2 != 0) return FA_ERR_UNSUPPORTED;   // the two-tile kernel only
+  return FA_OK;
+}
+}  // namespace
+
+FA_API int fa_attn_prefill_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                                  const int32_t *cu_seqlens, int B, int total_tokens,
+                                  int max_seqlen, int Hq, int Hkv, int D, float scale,
+                                  const int32_t *row_ptr, const int32_t *col_idx,
+                                  const int32_t *mode_dev, int mode, void *workspace,
+                                  size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (int rc = check_varlen(q, k, v, o, cu_seqlens, B, total_tokens, max_seqlen, Hq, Hkv, D))
+    return rc;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (mode != FA_MODE_FULL && mode != FA_MODE_SPARSE) return FA_ERR_INVALID_ARG;
+  const bool any_sparse = mode_dev != nullptr || mode == FA_MODE_SPARSE;
+  if (any_sparse && (!row_ptr || !col_idx)) return FA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < varlen_workspace_bytes(B, total_tokens)) return FA_ERR_WORKSPACE;
+  PrefillLaunch a{q, k, v, o, lse, B, max_seqlen, Hq, Hkv, scale, any_sparse ? row_ptr : nullptr,
+                  any_sparse ? col_idx : nullptr, mode_dev, mode, dev_status};
+  a.cu_seqlens = cu_seqlens;
+  a.total_tokens = total_tokens;
+  a.varlen_ws = workspace;
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+FA_API size_t fa_hybrid_varlen_workspace_size(int B, int total_tokens, int Hq, int D,
+                                              int hidden) {
+  const size_t r = fa_router_workspace_size(B, Hq, D, hidden);
+  const size_t v = fa_varlen_workspace_size(B, total_tokens);
+  if (!r || !v) return 0;
+  return ((r + 255) & ~static_cast<size_t>(255)) + v;
+}
+
+FA_API int fa_hybrid_layer_varlen(const void *q, const void *k, const void *v, void *o,
+                                  float *lse, const int32_t *cu_seqlens, int B, int total_tokens,
+                                  int max_seqlen, int Hq, int Hkv, int D, float scale,
+                                  const float *w1, const float *b1, int hidden, const float *w2,
+                                  const float *b2, fa_sparse_cfg cfg, const int32_t *row_ptr,
+                                  const int32_t *col_idx, float *logits_out, int32_t *mode_out,
+                                  void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                  void *stream) {
+  if (int rc = check_varlen(q, k, v, o, cu_seqlens, B, total_tokens, max_seqlen, Hq, Hkv, D))
+    return rc;
+  if (int rc = check_router(q, B, max_seqlen, Hq, D, 100, 100, w1, hidden, w2)) return rc;
+  if (int rc = check_cfg(cfg)) return rc;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (!row_ptr || !col_idx || !mode_out) return FA_ERR_INVALID_ARG;
+  const size_t rws = router_workspace_bytes(B, Hq, D, hidden);
+  const size_t need = ((rws + 255) & ~static_cast<size_t>(255)) + varlen_workspace_bytes(B, total_tokens);
+  if (!workspace || ws_bytes < need) return FA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RouterLaunch r{q, B, max_seqlen, Hq, 100, 100, w1, b1, w2, b2, hidden, logits_out, mode_out,
+                 workspace};
+  r.cu_seqlens = cu_seqlens;
+  if (int rc = launch_router(r, st)) return rc;
+  PrefillLaunch a{q, k, v, o, lse, B, max_seqlen, Hq, Hkv, scale, row_ptr, col_idx, mode_out,
+                  FA_MODE_FULL, dev_status};
+  a.cu_seqlens = cu_seqlens;
+  a.total_tokens = total_tokens;
+  a.varlen_ws = static_cast<uint8_t *>(workspace) + ((rws + 255) & ~static_cast<size_t>(255));
+  return launch_prefill(a, st);
+}
+
 }  // extern "C"

@@ -25,7 +25,13 @@ struct PrefillLaunch {
   int mode_default;
   int32_t *status;
   const float *mix_r = nullptr;      // soft-routing mix weight per batch, or nullptr
+  // Packed variable-length batch: S is then the longest sequence, q/k/v/o
+  // are [total_tokens, H, D], and `varlen_ws` holds the work-item list.
+  const int32_t *cu_seqlens = nullptr;
+  int total_tokens = 0;
+  void *varlen_ws = nullptr;
 };
+size_t varlen_workspace_bytes(int B, int total_tokens);
 int launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
 
 struct DecodeLaunch {
@@ -54,6 +60,7 @@ struct RouterLaunch {
   float *logits;
   int32_t *mode;
   void *workspace;
+  const int32_t *cu_seqlens = nullptr;  // packed sequences (S unused), or nullptr
 };
 size_t router_workspace_bytes(int B, int Hq, int D, int hidden);
 int launch_router_soft(const float *logits, const float *gumbel, int B, float tau, float *r,

@@ -51,6 +51,14 @@ struct Params {
   const int32_t *col_idx;
   const int32_t *mode;     // per-batch mode on device, or nullptr
   const float *mix_r;      // nullptr, or per-batch weight r: O = r * O_old + (1 - r) * O_new
+  // Packed variable-length batch (nullptr: every sequence has length S):
+  // sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]) of [total_tokens, H, D]
+  // tensors; `items` lists its query tiles (qt << 12 | b), longest first,
+  // and *n_items their count (both written on the device).
+  const int32_t *cu_seqlens;
+  const int32_t *items;
+  const int32_t *n_items;
+  int total_tokens;
   int32_t *status;
   int B, S, Hq, G;
   int n_qtiles, nqb;
@@ -103,7 +111,7 @@ struct TileIter {
   int n, n_end;
   bool full;
 
-  FA_DEV void init(const Params &p, int qt, bool sparse) {
+  FA_DEV void init(const Params &p, int qt, bool sparse, int nqb) {
     status = p.status;
     full = !sparse;
     n = 0;
@@ -115,7 +123,7 @@ struct TileIter {
     if (sparse) {
       p0 = p.row_ptr[qb0];
       e0 = p.row_ptr[qb0 + 1];
-      if (qb0 + 1 < p.nqb) {
+      if (qb0 + 1 < nqb) {
         p1 = e0;
         e1 = p.row_ptr[qb0 + 2];
       }
@@ -195,7 +203,7 @@ FA_DEV void run_producer(const Shared &sh, const CUtensorMap *tmQ, const CUtenso
   tma_load_4d(sh.q + HALF_BYTES, tmQ, sh.q_full, 64, h, qt * BM, b);
 
   TileIter it;
-  it.init(p, qt, sparse);
+  it.init(p, qt, sparse, p.nqb);
   int li = 0;  // loads issued, in consumption order
   auto load = [&](const CUtensorMap *map, int n) -> bool {
     const int slot = li % NSLOT;
@@ -279,7 +287,7 @@ FA_DEV void run_mma(const Shared &sh, uint32_t tmem, const Params &p, int qt, bo
   };
 
   TileIter it;
-  it.init(p, qt, sparse);
+  it.init(p, qt, sparse, p.nqb);
   int n_cur = 0;
   uint32_t bits;
   bool has = ok && it.next(n_cur, bits);
@@ -314,7 +322,7 @@ FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt
   float m_run = -INFINITY, l_run = 0.f;
 
   TileIter it;
-  it.init(p, qt, sparse);
+  it.init(p, qt, sparse, p.nqb);
   int j = 0, n = 0;
   uint32_t bits = 0;
   bool ok = true;
@@ -610,20 +618,47 @@ FA_DEV Smem carve(uint8_t *raw) {
 struct Item {
   int qt, b, h0, kvh;
   bool sparse;
+  int L;          // sequence length
+  int row0;       // token row of the sequence's first token in Q/K/V/O
+  int tma_tok0;   // TMA token coordinate of token 0, and TMA batch coordinate
+  int tma_b;
+  long long lse0; // LSE index of (head 0, token 0); head stride lse_hs
+  int lse_hs;
 };
 FA_DEV Item item_of(const Params &p, int w) {
   const int hp_count = p.Hq / NQ;
-  const int bh = p.B * hp_count;
   Item it;
-  it.qt = p.n_qtiles - 1 - w / bh;
-  const int rem = w % bh;
-  it.b = rem / hp_count;
-  it.h0 = (rem % hp_count) * NQ;
+  if (p.cu_seqlens) {
+    const int packed = p.items[w / hp_count];
+    it.qt = packed >> 12;
+    it.b = packed & 4095;
+    it.h0 = (w % hp_count) * NQ;
+    const int t0 = p.cu_seqlens[it.b];
+    it.L = p.cu_seqlens[it.b + 1] - t0;
+    it.row0 = t0;
+    it.tma_tok0 = t0;
+    it.tma_b = 0;
+    it.lse0 = t0;
+    it.lse_hs = p.total_tokens;
+  } else {
+    const int bh = p.B * hp_count;
+    it.qt = p.n_qtiles - 1 - w / bh;
+    const int rem = w % bh;
+    it.b = rem / hp_count;
+    it.h0 = (rem % hp_count) * NQ;
+    it.L = p.S;
+    it.row0 = it.b * p.S;
+    it.tma_tok0 = 0;
+    it.tma_b = it.b;
+    it.lse0 = static_cast<long long>(it.b) * p.Hq * p.S;
+    it.lse_hs = p.S;
+  }
   it.kvh = it.h0 / p.G;
   const int mode = p.mode ? p.mode[it.b] : p.mode_default;
   it.sparse = (mode == FA_MODE_SPARSE) && p.row_ptr != nullptr;
   return it;
 }
+FA_DEV int nqb_of(const Item &im) { return (im.L + 63) / 64; }
 // The k-th item of this CTA: rounds of gridDim.x items, walked forwards in
 // even rounds and backwards in odd ones, so a CTA that drew one of the
 // longest items in a round draws one of the shortest in the next.
@@ -659,21 +694,22 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
     mbar_arrive_expect_tx_w(sh.bar(Smem::Q_FULL), NQ * TILE_BYTES);
 #pragma unroll
     for (int t = 0; t < NQ; ++t) {
-      tma_load_4d_w(sh.q(t), tmQ, sh.bar(Smem::Q_FULL), 0, im.h0 + t, im.qt * BM, im.b);
-      tma_load_4d_w(sh.q(t) + HALF_BYTES, tmQ, sh.bar(Smem::Q_FULL), 64, im.h0 + t, im.qt * BM,
-                    im.b);
+      tma_load_4d_w(sh.q(t), tmQ, sh.bar(Smem::Q_FULL), 0, im.h0 + t,
+                    im.tma_tok0 + im.qt * BM, im.tma_b);
+      tma_load_4d_w(sh.q(t) + HALF_BYTES, tmQ, sh.bar(Smem::Q_FULL), 64, im.h0 + t,
+                    im.tma_tok0 + im.qt * BM, im.tma_b);
     }
     ++nq;
     TileIter it;
-    it.init(p, im.qt, im.sparse);
+    it.init(p, im.qt, im.sparse, nqb_of(im));
     auto load = [&](const CUtensorMap *map, int n) -> bool {
       const int slot = li % NSLOT;
       const uint32_t round = static_cast<uint32_t>(li / NSLOT);
       if (!warp_wait(sh.bar(Smem::EMPTY0 + slot), (round & 1u) ^ 1u, sh, p)) return false;
       const uint32_t dst = sh.ring(slot), bar = sh.bar(Smem::FULL0 + slot);
       mbar_arrive_expect_tx_w(bar, TILE_BYTES);
-      tma_load_4d_w(dst, map, bar, 0, im.kvh, n * BN, im.b);
-      tma_load_4d_w(dst + HALF_BYTES, map, bar, 64, im.kvh, n * BN, im.b);
+      tma_load_4d_w(dst, map, bar, 0, im.kvh, im.tma_tok0 + n * BN, im.tma_b);
+      tma_load_4d_w(dst + HALF_BYTES, map, bar, 64, im.kvh, im.tma_tok0 + n * BN, im.tma_b);
       ++li;
       return true;
     };
@@ -750,7 +786,7 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     if (!(ok = warp_wait(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(k) & 1u, sh, p))) break;
     tc_fence_after_sync();
     TileIter it;
-    it.init(p, im.qt, im.sparse);
+    it.init(p, im.qt, im.sparse, nqb_of(im));
     int n = 0;
     uint32_t bits;
     if (!it.next(n, bits)) {          // no KV tile: Q is free again at once
@@ -810,7 +846,7 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
     const int h = im.h0 + t;
     float m_run = -INFINITY, l_run = 0.f;
     TileIter it;
-    it.init(p, im.qt, im.sparse);
+    it.init(p, im.qt, im.sparse, nqb_of(im));
     int j = 0, n = 0;
     uint32_t bits = 0;
     while (it.next(n, bits)) {
@@ -909,9 +945,9 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
     if (j > 0 && !have_o) break;
     tc_fence_after_sync();
     const int tok = im.qt * BM + r;
-    const bool store = (tok < p.S) && !ld_shared_s32(sh.abort_flag());
+    const bool store = (tok < im.L) && !ld_shared_s32(sh.abort_flag());
     const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
-    __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(im.b) * p.S + tok) * p.Hq + h) * HD;
+    __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(im.row0) + tok) * p.Hq + h) * HD;
 #pragma unroll
     for (int q4 = 0; q4 < HD / 32; ++q4) {
       uint32_t o[32];
@@ -934,7 +970,7 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
     }
     if (store && p.lse) {
       const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-      p.lse[(static_cast<size_t>(im.b) * p.Hq + h) * p.S + tok] = lse;
+      p.lse[im.lse0 + static_cast<long long>(h) * im.lse_hs + tok] = lse;
     }
   }
 }
@@ -974,6 +1010,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = static_cast<uint32_t>(ld_shared_s32(sh.tmem_slot()));
+  if (p.cu_seqlens) total_items = *p.n_items * (p.Hq / NQ);
 
   if (warp >= WARP_PRODUCER) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
@@ -994,15 +1031,70 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// Work items of a packed variable-length batch: the query tiles (qt, b) of
+// every sequence, ordered by qt descending (longest causal rows first).  The
+// position of (v, b) is the number of tiles with a larger qt plus the number
+// of earlier sequences that also have a tile v.  One CTA.
+__global__ void __launch_bounds__(1024) varlen_items_kernel(const int32_t *cu, int B, int max_items,
+                                                            int32_t *n_items, int32_t *items,
+                                                            int32_t *status) {
+  __shared__ int nq[4096];
+  __shared__ int red_max[32], red_sum[32];
+  int my_max = 0, my_sum = 0;
+  for (int b = threadIdx.x; b < B; b += 1024) {
+    const int L = cu[b + 1] - cu[b];
+    const int q = L > 0 ? (L + BM - 1) / BM : 0;
+    if (L < 0) report(status, FA_DEV_BAD_INDEX);
+    nq[b] = q;
+    my_max = max(my_max, q);
+    my_sum += q;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, off));
+    my_sum += __shfl_xor_sync(0xffffffffu, my_sum, off);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red_max[threadIdx.x >> 5] = my_max;
+    red_sum[threadIdx.x >> 5] = my_sum;
+  }
+  __syncthreads();
+  int max_nq = 0, total = 0;
+  for (int w = 0; w < 32; ++w) {
+    max_nq = max(max_nq, red_max[w]);
+    total += red_sum[w];
+  }
+  if (total > max_items) {  // cannot happen with consistent cu_seqlens and total_tokens
+    if (threadIdx.x == 0) report(status, FA_DEV_BAD_INDEX);
+    total = 0;
+  }
+  if (threadIdx.x == 0) *n_items = total;
+  if (total == 0) return;
+  for (int v = threadIdx.x; v < max_nq; v += 1024) {
+    int pos = 0;
+    for (int b = 0; b < B; ++b) pos += max(0, nq[b] - v - 1);
+    for (int b = 0; b < B; ++b)
+      if (nq[b] > v) items[pos++] = (v << 12) | b;
+  }
+}
+
 }  // namespace prefill2
 
 // ----------------------------------------------------------------- host ---
+size_t varlen_workspace_bytes(int B, int total_tokens) {
+  const size_t max_items = static_cast<size_t>(total_tokens) / prefill2::BM + B + 1;
+  return 256 + 4 * max_items;
+}
+
 int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   using namespace prefill;
+  const bool varlen = a.cu_seqlens != nullptr;
   CUtensorMap tmQ, tmK, tmV;
-  if (make_tmap_bhsd(&tmQ, a.q, a.B, a.S, a.Hq, 64, BM) != 0) return FA_ERR_CUDA;
-  if (make_tmap_bhsd(&tmK, a.k, a.B, a.S, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
-  if (make_tmap_bhsd(&tmV, a.v, a.B, a.S, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
+  // A packed batch is one sequence of total_tokens rows for the TMA maps.
+  const int mB = varlen ? 1 : a.B, mS = varlen ? a.total_tokens : a.S;
+  if (make_tmap_bhsd(&tmQ, a.q, mB, mS, a.Hq, 64, BM) != 0) return FA_ERR_CUDA;
+  if (make_tmap_bhsd(&tmK, a.k, mB, mS, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
+  if (make_tmap_bhsd(&tmV, a.v, mB, mS, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
   const int G = a.Hq / a.Hkv;
   const bool two_tiles = (G % 2) == 0;
   if (two_tiles) {
@@ -1028,6 +1120,10 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   p.mode = a.mode_dev;
   p.mix_r = a.mix_r;
   p.status = a.status;
+  p.cu_seqlens = a.cu_seqlens;
+  p.total_tokens = a.total_tokens;
+  p.items = nullptr;
+  p.n_items = nullptr;
   p.B = a.B;
   p.S = a.S;
   p.Hq = a.Hq;
@@ -1036,8 +1132,20 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   p.nqb = (a.S + 63) / 64;
   p.mode_default = a.mode_default;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  const long long grid =
+  long long grid =
       static_cast<long long>(p.n_qtiles) * a.B * (two_tiles ? a.Hq / 2 : a.Hq);
+  if (varlen) {
+    if (!two_tiles || !a.varlen_ws) return FA_ERR_UNSUPPORTED;
+    const long long max_items = static_cast<long long>(a.total_tokens) / BM + a.B + 1;
+    if (max_items >= (1ll << 19) || a.B > 4096) return FA_ERR_UNSUPPORTED;
+    int32_t *ws = reinterpret_cast<int32_t *>(a.varlen_ws);
+    p.n_items = ws;
+    p.items = ws + 64;
+    prefill2::varlen_items_kernel<<<1, 1024, 0, stream>>>(
+        a.cu_seqlens, a.B, static_cast<int>(max_items), ws, ws + 64, a.status);
+    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+    grid = max_items * (a.Hq / 2);   // upper bound; the kernel reads the real count
+  }
   if (grid <= 0 || grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   if (two_tiles) {
     // Persistent: one CTA per SM walks the work items.

@@ -20,19 +20,24 @@ constexpr int kPoolSlices = 5;     // token slices per (head, batch)
 // Partial sums of the selected tokens: slice z of (head h, batch b) adds
 // up its share of the n_head + n_tail selected tokens for all 128 dims.
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *q, float *part, int S,
-                                                   int Hq, int n_head, int n_tail) {
+                                                   int Hq, int n_head, int n_tail,
+                                                   const int32_t *cu) {
   __shared__ float red[16][HD];
   const int h = blockIdx.x, b = blockIdx.y, z = blockIdx.z, B = gridDim.y;
   const int chunk = threadIdx.x & 15, grp = threadIdx.x >> 4;
   const int n_sel = n_head + n_tail;
   const int per = (n_sel + kPoolSlices - 1) / kPoolSlices;
   const int i0 = z * per, i1 = min(n_sel, i0 + per);
+  // Sequence b: rows row0 .. row0 + len - 1 (packed batch: from cu_seqlens).
+  const size_t row0 = cu ? static_cast<size_t>(cu[b]) : static_cast<size_t>(b) * S;
+  const int len = cu ? cu[b + 1] - cu[b] : S;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
   for (int i = i0 + grp; i < i1; i += 16) {
-    const int t = i < n_head ? i : S - n_tail + (i - n_head);
+    const int t = i < n_head ? i : len - n_tail + (i - n_head);
+    if (t < 0 || t >= len) continue;       // a sequence shorter than n_head + n_tail
     const uint4 v = *reinterpret_cast<const uint4 *>(
-        q + ((static_cast<size_t>(b) * S + t) * Hq + h) * HD + chunk * 8);
+        q + ((row0 + t) * Hq + h) * HD + chunk * 8);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -154,7 +159,8 @@ int launch_router(const RouterLaunch &a, cudaStream_t stream) {
                            static_cast<int>(xs_bytes)) != cudaSuccess)
     return FA_ERR_CUDA;
   pool_kernel<<<dim3(a.Hq, a.B, kPoolSlices), 256, 0, stream>>>(
-      reinterpret_cast<const __nv_bfloat16 *>(a.q), part, a.S, a.Hq, a.n_head, a.n_tail);
+      reinterpret_cast<const __nv_bfloat16 *>(a.q), part, a.S, a.Hq, a.n_head, a.n_tail,
+      a.cu_seqlens);
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   hidden_kernel<<<dim3(a.hidden, a.B), 256, xs_bytes, stream>>>(
       part, a.w1, a.b1, hid, in_f, a.hidden, 1.0f / static_cast<float>(a.n_head + a.n_tail));

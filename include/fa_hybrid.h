@@ -148,6 +148,51 @@ FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
                    fa_sparse_cfg cfg, void *o, float *lse, void *workspace,
                    size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/* ------------------------------------------- variable-length batches ---
+ * Serving form of the routed layer ("Flux Attention": the router decides per
+ * request, before each layer's attention): B sequences of different lengths
+ * packed along the token axis, sequence b = tokens [cu_seqlens[b],
+ * cu_seqlens[b+1]).  One persistent launch covers every query tile of every
+ * sequence, longest causal rows first, each sequence in its own mode.
+ *   q, o bf16 [total_tokens, Hq, D]; k, v bf16 [total_tokens, Hkv, D];
+ *   lse fp32 [Hq, total_tokens] or NULL; cu_seqlens int32 [B + 1], device,
+ *   non-decreasing, cu_seqlens[0] = 0, cu_seqlens[B] = total_tokens;
+ *   max_seqlen = the longest sequence (host).  Hq / Hkv must be even.
+ *   Sparse sequences use one CSR built for max_seqlen (row i of the block
+ *   rule does not depend on the length).
+ * fa_attn_prefill_varlen: mode_dev (device int32 [B]) or, if NULL, `mode`
+ *   for all; row_ptr/col_idx required unless every sequence is FULL.
+ *   workspace >= fa_varlen_workspace_size(B, total_tokens) bytes.
+ * fa_hybrid_layer_varlen: the router per sequence (its first and last 100
+ *   tokens; every sequence needs >= 200 tokens), then the attention reading
+ *   mode_out on the device.  workspace >=
+ *   fa_hybrid_varlen_workspace_size(B, total_tokens, Hq, D, hidden). */
+FA_API size_t fa_varlen_workspace_size(int B, int total_tokens);
+FA_API int fa_attn_prefill_varlen(const void *q, const void *k, const void *v,
+                                  void *o, float *lse,
+                                  const int32_t *cu_seqlens, int B,
+                                  int total_tokens, int max_seqlen, int Hq,
+                                  int Hkv, int D, float scale,
+                                  const int32_t *row_ptr,
+                                  const int32_t *col_idx,
+                                  const int32_t *mode_dev, int mode,
+                                  void *workspace, size_t ws_bytes,
+                                  int32_t *dev_status, void *stream);
+FA_API size_t fa_hybrid_varlen_workspace_size(int B, int total_tokens, int Hq,
+                                              int D, int hidden);
+FA_API int fa_hybrid_layer_varlen(const void *q, const void *k, const void *v,
+                                  void *o, float *lse,
+                                  const int32_t *cu_seqlens, int B,
+                                  int total_tokens, int max_seqlen, int Hq,
+                                  int Hkv, int D, float scale, const float *w1,
+                                  const float *b1, int hidden, const float *w2,
+                                  const float *b2, fa_sparse_cfg cfg,
+                                  const int32_t *row_ptr,
+                                  const int32_t *col_idx, float *logits_out,
+                                  int32_t *mode_out, void *workspace,
+                                  size_t ws_bytes, int32_t *dev_status,
+                                  void *stream);
+
 /* ------------------------------------------------------ soft routing ---
  * "Flux Attention", router paragraph on training: the Gumbel-softmax
  * relaxation r = exp((pi_FA + g_FA)/tau) / sum_i exp((pi_i + g_i)/tau) and
