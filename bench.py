@@ -584,6 +584,100 @@ def run_decode(args, wl):
     return line
 
 
+# ------------------------------------------------ variable-length serving
+def run_varlen(args, wl):
+    """One routed layer over a packed batch of requests of different lengths:
+    CSR + fa_hybrid_layer_varlen (router per request on the device, then one
+    persistent attention launch over every request in its own mode)."""
+    import oracle  # pair counting only (host arithmetic of the pattern)
+    from block_sparse_attention_layerrouter_b200 import capi, inputs
+    ws, rank, dev = setup_device(args)
+    lengths = inputs.varlen_lengths(wl.B, wl.S, wl.seed)
+    T = int(lengths.sum())
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32, device=dev)
+    q = inputs.randn_bf16((T, wl.Hq, 128), wl.seed, device=dev)
+    k = inputs.randn_bf16((T, wl.Hkv, 128), wl.seed + 100, device=dev)
+    v = inputs.randn_bf16((T, wl.Hkv, 128), wl.seed + 200, device=dev)
+    o = torch.empty_like(q)
+    w1, b1, w2, b2 = [t.to(dev) for t in inputs.router_weights(wl.Hq * 128, wl.hidden, wl.seed)]
+    c = capi.cfg(64, wl.sink, wl.window)
+    rows, nnz = capi.blocksparse_index_size(wl.S, c)
+    rp = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    ci = torch.empty(nnz, dtype=torch.int32, device=dev)
+    logits = torch.empty(wl.B, 2, device=dev)
+    mode = torch.empty(wl.B, dtype=torch.int32, device=dev)
+    wsb = torch.empty(int(capi.lib().fa_hybrid_varlen_workspace_size(wl.B, T, wl.Hq, 128,
+                                                                      wl.hidden)),
+                      dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(ev=None):
+        capi._check("fa_blocksparse_index", capi.lib().fa_blocksparse_index(
+            wl.S, c, capi._ptr(rp), capi._ptr(ci), capi._stream(dev)))
+        if ev is not None:
+            ev[0].record()
+        capi.hybrid_layer_varlen(q, k, v, cu, wl.S, w1, b1, w2, b2, rp, ci, c, o=o,
+                                 logits=logits, mode=mode, workspace=wsb, status=status)
+        if ev is not None:
+            ev[1].record()
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    sync_all(ws)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record()
+    sync_all(ws)
+    sampler.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
+    layer_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    modes = mode.cpu().tolist()
+    # The same packed batch with every request in FULL mode (one varlen launch):
+    # what the routing saves on this batch.
+    vws = torch.empty(int(capi.lib().fa_varlen_workspace_size(wl.B, T)), dtype=torch.uint8,
+                      device=dev)
+    full_ms = time_kernel_alone(lambda: capi.attn_prefill_varlen(
+        q, k, v, cu, wl.S, mode=0, o=o, workspace=vws, status=status))
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    if rank != 0:
+        return None
+    flops = 0.0
+    for L, m in zip(lengths.tolist(), modes):
+        pairs = L * (L + 1) / 2 if m == 0 else oracle.attended_pairs_sparse(L, 64, wl.sink,
+                                                                          wl.window)
+        flops += 4.0 * 128 * wl.Hq * pairs
+    _, peak_burst, peak_sust, peak_kind = measured_peaks()
+    value = ws * flops / (ms / args.steps * 1e-3) / 1e12
+    achieved = flops / (layer_ms * 1e-3) / 1e12
+    line = base_line(args, wl, ws, ms, "TFLOP/s", value)
+    line["config"] = {"workload": wl.name, "requests": wl.B, "lengths": lengths.tolist(),
+                      "total_tokens": T, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": 128, "sink": wl.sink,
+                      "window": wl.window, "routed_modes": modes,
+                      "step": "CSR + router per request + one packed attention launch",
+                      "l2": "inputs larger than L2 (%.2f GB)" % (
+                          (q.numel() * 2 * 2 + k.numel() * 2 * 2) / 1e9)}
+    line["roofline"] = {"bound": "tensor", "kernel": "router + varlen prefill2_kernel",
+                        "achieved": round(achieved, 2), "peak": peak_sust, "unit": "TFLOP/s",
+                        "frac": round(achieved / peak_sust, 4),
+                        "peak_kind": "%s bf16 sustained" % peak_kind,
+                        "frac_of_burst_peak": round(achieved / peak_burst, 4), "traffic": None,
+                        "algorithmic_flops_per_launch": flops,
+                        "avg_launch_ms": round(layer_ms, 4)}
+    line["all_full_ms"] = round(full_ms, 4)
+    line["routed_speedup_vs_all_full"] = round(full_ms / (ms / args.steps), 3)
+    line["e2e"] = None
+    line["gpu_launches"] = 6 * args.steps
+    line["clocks"] = sampler.report()
+    return line
+
+
 # ------------------------------------------------------- one kernel alone
 def run_only(args, wl):
     """Runs a single kernel of the path `warmup + steps` times on the
@@ -684,6 +778,8 @@ def main():
         line = run_only(args, wl)
     elif wl.decode_len:
         line = run_decode(args, wl)
+    elif wl.varlen:
+        line = run_varlen(args, wl)
     else:
         line = run_ours(args, wl)
     if line is not None:

@@ -36,6 +36,7 @@ class Workload:
     block: int = 64            # sparsity block, tokens
     hidden: int = 64           # router MLP hidden width
     decode_len: int = 0        # >0: decode workload with this cache length
+    varlen: bool = False       # packed batch of B requests of seeded lengths <= S
     seed: int = 1000
     notes: str = field(default="", compare=False)
 
@@ -58,6 +59,12 @@ WORKLOADS = {
                                       layers=32, window=2048, hidden=256,
                                       decode_len=131072, seed=1004,
                                       notes="decode, 16 full + 16 sparse layers"),
+    # Serving batch: 8 requests of seeded lengths in [1024, 32768] packed along
+    # the token axis, one Qwen3-4B-shaped layer, each request routed by the
+    # layer router on its own prompt.
+    "serving-varlen-qwen3-4b": Workload("serving-varlen-qwen3-4b", B=8, S=32768, Hq=32, Hkv=8,
+                                        window=1024, hidden=256, varlen=True, seed=1006,
+                                        notes="packed variable-length batch, routed per request"),
     # Profiling shape: the decode workload at a quarter of the context
     # (1 GiB of K/V, still far above the 126 MB L2).
     "decode-b8-l32768": Workload("decode-b8-l32768", B=8, S=1, Hq=32, Hkv=8, layers=2,
@@ -111,6 +118,14 @@ def gumbel(B: int, seed: int) -> torch.Tensor:
     g = _gen("cpu", seed)
     u = torch.rand(B, 2, generator=g, dtype=torch.float64).clamp_(1e-12, 1 - 1e-12)
     return (-torch.log(-torch.log(u))).float()
+
+
+def varlen_lengths(B: int, max_len: int, seed: int, min_len: int = 1024) -> np.ndarray:
+    """Seeded request lengths in [min_len, max_len] (the longest is max_len)."""
+    rng = np.random.default_rng(seed)
+    L = rng.integers(min_len, max_len + 1, size=B)
+    L[int(rng.integers(0, B))] = max_len
+    return L.astype(np.int64)
 
 
 def bits(t: torch.Tensor) -> np.ndarray:

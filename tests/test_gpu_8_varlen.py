@@ -108,3 +108,52 @@ def test_hybrid_layer_varlen_routes_each_sequence():
             assert mode[b] == ref_mode[0]
         ref, _ = _oracle_seq(q, k, v, cu, b, mode[b] == 1, W)
         assert_close_attention(to_f64(o[t0:t0 + L]), ref[0], "hybrid varlen seq %d" % b)
+
+
+def test_serving_varlen_full_size_sampled():
+    """The packed serving batch at its full size (8 requests of seeded
+    lengths up to 32768, Qwen3-4B heads), through the hybrid varlen entry in
+    the benchmark's launch configuration: every routing decision matches the
+    oracle's, and seeded sampled rows of each request match the oracle in the
+    mode the router chose for that request."""
+    wl = inputs.WORKLOADS["serving-varlen-qwen3-4b"]
+    lengths = inputs.varlen_lengths(wl.B, wl.S, wl.seed)
+    T = int(lengths.sum())
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    q = inputs.randn_bf16((T, wl.Hq, 128), wl.seed, device="cuda")
+    k = inputs.randn_bf16((T, wl.Hkv, 128), wl.seed + 100, device="cuda")
+    v = inputs.randn_bf16((T, wl.Hkv, 128), wl.seed + 200, device="cuda")
+    w1, b1, w2, b2 = inputs.router_weights(wl.Hq * 128, wl.hidden, wl.seed)
+    c = capi.cfg(64, wl.sink, wl.window)
+    rp, ci = capi.blocksparse_index(wl.S, c)
+    lse = torch.empty(wl.Hq, T, device="cuda")
+    status = zero_status()
+    o, logits, mode = capi.hybrid_layer_varlen(q, k, v, torch.from_numpy(cu).cuda(), wl.S,
+                                               w1.cuda(), b1.cuda(), w2.cuda(), b2.cuda(), rp, ci,
+                                               c, lse=lse, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    mode = mode.cpu().numpy()
+    qh, kh, vh = q.cpu(), k.cpu(), v.cpu()
+    for b, L in enumerate(lengths.tolist()):
+        t0 = int(cu[b])
+        qb = inputs.bits(qh[t0:t0 + L][None])
+        ref_logits, ref_mode, _ = oracle.router_decide(qb, w1.double().numpy(), b1.double().numpy(),
+                                                       w2.double().numpy(), b2.double().numpy())
+        np.testing.assert_allclose(logits[b].cpu().double().numpy(), ref_logits[0], atol=1e-5)
+        assert mode[b] == ref_mode[0], "request %d routed differently" % b
+        rows = inputs.sample_rows(1, L, wl.Hq, wl.Hkv, seed=wl.seed + b, n_random=24,
+                                  n_boundary=4, n_groups=1)
+        if mode[b] == 0:
+            rng = np.random.default_rng(wl.seed + b)
+            rows = rows[np.sort(rng.choice(len(rows), size=min(96, len(rows)), replace=False))]
+            mask = None
+        else:
+            mask = oracle.rows_to_dense_mask(oracle.blocksparse_rows(L, 64, wl.sink, wl.window))
+        ref, ref_lse = oracle.attention_rows(qb, inputs.bits(kh[t0:t0 + L][None]),
+                                             inputs.bits(vh[t0:t0 + L][None]), SCALE, rows, mask)
+        rt = torch.from_numpy(rows).cuda()
+        got = o[t0 + rt[:, 2], rt[:, 1]]
+        got_lse = lse[rt[:, 1], t0 + rt[:, 2]]
+        assert_close_attention(to_f64(got), ref, "serving request %d mode %d" % (b, mode[b]))
+        np.testing.assert_allclose(to_f64(got_lse), ref_lse, atol=LSE_ABS_TOL)
