@@ -27,6 +27,9 @@ head-major (x[h*D + d]); a tie pi_SA == pi_FA routes to FULL; the local window
 is counted in whole 64-token blocks including the query's own block; key k is
 allowed for query t only when k <= t; query head h reads KV head h // G.
 
+The backward functions are the chain rule through those definitions (the
+gradients the router's soft-routing relaxation needs for training).
+
 Parity status: every function below is pinned by tests/test_oracle_*.py
 (worked examples, closed forms, invariants, brute force on tiny inputs).
 """
@@ -84,6 +87,21 @@ def _load():
             p, p, p, p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_double, p, ctypes.c_int, p, p]
         lib.oracle_decode.restype = ctypes.c_int
+        for name in ("oracle_attention_backward",):
+            fn = getattr(lib, name)
+            fn.argtypes = [p, p, p, p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_int, ctypes.c_int, ctypes.c_double, p, ctypes.c_int,
+                           p, p, p]
+            fn.restype = ctypes.c_int
+        lib.oracle_attention_backward_qrows.argtypes = [
+            p, p, p, p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_double, p, ctypes.c_int, p, ctypes.c_long, p]
+        lib.oracle_attention_backward_qrows.restype = ctypes.c_int
+        lib.oracle_attention_backward_keyrows.argtypes = [
+            p, p, p, p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_double, p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            p, ctypes.c_long, p, p]
+        lib.oracle_attention_backward_keyrows.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -295,6 +313,124 @@ def attention(q_bits, k_bits, v_bits, scale, block_mask=None, block=BLOCK):
     out, lse = attention_rows(q_bits, k_bits, v_bits, scale, all_rows(B, S, Hq),
                               block_mask, block)
     return out.reshape(B, S, Hq, D), lse.reshape(B, S, Hq).transpose(0, 2, 1)
+
+
+# ----------------------------------------------------------------- backward
+# The gradients below are the reverse-mode chain rule through the forward
+# definitions above -- what training the router through the soft routing
+# relaxation ([FLUX] router paragraphs) differentiates.  The pages print no
+# backward; nothing here goes beyond the chain rule.
+
+def _u16(a):
+    return np.ascontiguousarray(a, dtype=np.uint16)
+
+
+def attention_backward(q_bits, k_bits, v_bits, do_bits, scale, block_mask=None,
+                       block: int = BLOCK):
+    """dQ, dK, dV (fp64, shapes of q, k, v) of the masked causal attention
+    for an upstream gradient dO [B,S,Hq,D] (bf16 bits): dV = P^T dO,
+    dS = P * (dO V^T - rowsum(P * dO V^T)), dQ = scale dS K, dK = scale dS^T Q,
+    a KV head summing over the G query heads that read it."""
+    lib = _load()
+    q_bits, k_bits, v_bits, do_bits = map(_u16, (q_bits, k_bits, v_bits, do_bits))
+    B, S, Hq, D = q_bits.shape
+    Hkv = k_bits.shape[2]
+    dq = np.zeros((B, S, Hq, D))
+    dk = np.zeros((B, S, Hkv, D))
+    dv = np.zeros((B, S, Hkv, D))
+    bm = None if block_mask is None else np.ascontiguousarray(block_mask, dtype=np.uint8)
+    rc = lib.oracle_attention_backward(_ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(do_bits),
+                                       B, S, Hq, Hkv, D, float(scale), _ptr(bm), int(block),
+                                       _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError("oracle_attention_backward rejected its arguments")
+    return dq, dk, dv
+
+
+def attention_backward_qrows(q_bits, k_bits, v_bits, do_bits, scale, rows, block_mask=None,
+                             block: int = BLOCK) -> np.ndarray:
+    """dQ of selected (b, h, t) rows only (each depends on its own row):
+    fp64 [n, D]."""
+    lib = _load()
+    q_bits, k_bits, v_bits, do_bits = map(_u16, (q_bits, k_bits, v_bits, do_bits))
+    B, S, Hq, D = q_bits.shape
+    Hkv = k_bits.shape[2]
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    dq = np.zeros((rows.shape[0], D))
+    bm = None if block_mask is None else np.ascontiguousarray(block_mask, dtype=np.uint8)
+    rc = lib.oracle_attention_backward_qrows(_ptr(q_bits), _ptr(k_bits), _ptr(v_bits),
+                                             _ptr(do_bits), B, S, Hq, Hkv, D, float(scale),
+                                             _ptr(bm), int(block), _ptr(rows), rows.shape[0],
+                                             _ptr(dq))
+    if rc != 0:
+        raise ValueError("oracle_attention_backward_qrows rejected its arguments")
+    return dq
+
+
+def attention_backward_keyrows(q_bits, k_bits, v_bits, do_bits, scale, b, kvh, keys,
+                               block_mask=None, block: int = BLOCK):
+    """dK, dV of selected key positions of one (batch, kv head): fp64 [n, D]
+    each (every query row of the group is evaluated in full)."""
+    lib = _load()
+    q_bits, k_bits, v_bits, do_bits = map(_u16, (q_bits, k_bits, v_bits, do_bits))
+    B, S, Hq, D = q_bits.shape
+    Hkv = k_bits.shape[2]
+    keys = np.ascontiguousarray(keys, dtype=np.int64).ravel()
+    dk = np.zeros((keys.size, D))
+    dv = np.zeros((keys.size, D))
+    bm = None if block_mask is None else np.ascontiguousarray(block_mask, dtype=np.uint8)
+    rc = lib.oracle_attention_backward_keyrows(_ptr(q_bits), _ptr(k_bits), _ptr(v_bits),
+                                               _ptr(do_bits), B, S, Hq, Hkv, D, float(scale),
+                                               _ptr(bm), int(block), int(b), int(kvh),
+                                               _ptr(keys), keys.size, _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError("oracle_attention_backward_keyrows rejected its arguments")
+    return dk, dv
+
+
+def router_pool_backward(dx: np.ndarray, S: int, Hq: int, D: int,
+                         n_head: int = N_HEAD_TOKENS, n_tail: int = N_TAIL_TOKENS) -> np.ndarray:
+    """Gradient of router_pool with respect to Q: each of the n_head + n_tail
+    selected tokens receives dx / (n_head + n_tail); every other token 0.
+    dx [B, Hq*D] -> fp64 [B, S, Hq, D]."""
+    B = dx.shape[0]
+    g = np.zeros((B, S, Hq, D))
+    share = np.asarray(dx, np.float64).reshape(B, Hq, D) / float(n_head + n_tail)
+    g[:, :n_head] += share[:, None]
+    g[:, S - n_tail:] += share[:, None]
+    return g
+
+
+def soft_routed_backward(x, w1, b1, w2, b2, gumbel, tau, o_full, o_sparse, dy):
+    """Chain rule through the soft-routed layer
+        a = W1 x + b1, h = ReLU(a), pi = W2 h + b2, z = pi + g,
+        r = softmax(z / tau)[FA],  y = r O_FA + (1 - r) O_SA
+    for an upstream dy (all fp64; o_full, o_sparse, dy [B, ...]).  ReLU'(0)
+    is taken as 0.  Returns a dict with dr [B], dlogits [B,2], dw1, db1, dw2,
+    db2, dx [B, in], and the output weights r [B] that scale dy into the
+    upstream gradients of the two attention paths (r dy and (1 - r) dy)."""
+    x = np.asarray(x, np.float64)
+    w1, b1 = np.asarray(w1, np.float64), np.asarray(b1, np.float64)
+    w2, b2 = np.asarray(w2, np.float64), np.asarray(b2, np.float64)
+    B = x.shape[0]
+    a = x @ w1.T + b1
+    h = np.maximum(a, 0.0)
+    logits = h @ w2.T + b2
+    r = router_soft(logits, gumbel, tau)
+    diff = (np.asarray(o_full, np.float64) - np.asarray(o_sparse, np.float64)).reshape(B, -1)
+    dr = (np.asarray(dy, np.float64).reshape(B, -1) * diff).sum(axis=1)
+    # r = 1 / (1 + exp((z_SA - z_FA) / tau)): dr/dz_FA = r (1 - r) / tau = -dr/dz_SA
+    dzf = dr * r * (1.0 - r) / float(tau)
+    dlogits = np.stack([dzf, -dzf], axis=1)
+    dw2 = dlogits.T @ h
+    db2 = dlogits.sum(axis=0)
+    dh = dlogits @ w2
+    da = dh * (a > 0.0)
+    dw1 = da.T @ x
+    db1 = da.sum(axis=0)
+    dx = da @ w1
+    return {"r": r, "dr": dr, "dlogits": dlogits, "dw1": dw1, "db1": db1, "dw2": dw2,
+            "db2": db2, "dx": dx}
 
 
 def decode(q_bits, kc_bits, vc_bits, seqlens, scale, mode=MODE_FULL,

@@ -179,6 +179,253 @@ int oracle_decode(const uint16_t *q, const uint16_t *kc, const uint16_t *vc,
     return 0;
 }
 
+/*
+ * Gradients (reverse-mode chain rule through the definition above).  With
+ * an upstream gradient dO_t of the output row o_t:
+ *
+ *   dV_k  += p_k dO_t                       (o_t = sum_k p_k v_k)
+ *   dp_k   = dO_t . v_k
+ *   ds_k   = p_k (dp_k - sum_j p_j dp_j)    (Jacobian of the row softmax)
+ *   dQ_t   = scale * sum_k ds_k k_k         (s_k = scale * q_t . k_k)
+ *   dK_k  += scale * ds_k q_t
+ *
+ * backward_row() fills p[] and ds[] of one query row over its allowed keys;
+ * the three entry points below accumulate what they are asked for.
+ */
+static void backward_row(const uint16_t *q_row, const uint16_t *do_row,
+                         const uint16_t *kbase, const uint16_t *vbase,
+                         long kv_row_stride, int D, long n_keys,
+                         const uint8_t *key_ok, double scale, double *p,
+                         double *ds)
+{
+    double q[512], go[512];
+    for (int d = 0; d < D; ++d) {
+        q[d] = bf16_bits_to_double(q_row[d]);
+        go[d] = bf16_bits_to_double(do_row[d]);
+    }
+    double M = -INFINITY;
+    for (long k = 0; k < n_keys; ++k) {
+        p[k] = 0.0;
+        ds[k] = 0.0;
+        if (!key_ok[k]) continue;
+        const uint16_t *kr = kbase + k * kv_row_stride;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += q[d] * bf16_bits_to_double(kr[d]);
+        p[k] = dot * scale; /* the score, for now */
+        if (p[k] > M) M = p[k];
+    }
+    if (M == -INFINITY) return; /* no key: output 0, all gradients 0 */
+    double denom = 0.0;
+    for (long k = 0; k < n_keys; ++k) {
+        if (!key_ok[k]) continue;
+        p[k] = exp(p[k] - M);
+        denom += p[k];
+    }
+    double pdp = 0.0; /* sum_j p_j dp_j */
+    for (long k = 0; k < n_keys; ++k) {
+        if (!key_ok[k]) continue;
+        p[k] /= denom;
+        const uint16_t *vr = vbase + k * kv_row_stride;
+        double dp = 0.0;
+        for (int d = 0; d < D; ++d) dp += go[d] * bf16_bits_to_double(vr[d]);
+        ds[k] = dp; /* dp, for now */
+        pdp += p[k] * dp;
+    }
+    for (long k = 0; k < n_keys; ++k)
+        if (key_ok[k]) ds[k] = p[k] * (ds[k] - pdp);
+}
+
+static void causal_key_flags(long t, long S, const uint8_t *block_mask, int blk,
+                             long nkb, uint8_t *key_ok)
+{
+    for (long kk = 0; kk < S; ++kk) {
+        int ok = kk <= t;
+        if (ok && block_mask) ok = block_mask[(t / blk) * nkb + kk / blk] != 0;
+        key_ok[kk] = (uint8_t)ok;
+    }
+}
+
+/*
+ * Full backward.  q, dout: [B, S, Hq, D]; k, v: [B, S, Hkv, D] (bf16 bits);
+ * block_mask / blk as in oracle_attention_rows.  dq: [B, S, Hq, D],
+ * dk, dv: [B, S, Hkv, D], fp64, overwritten.  A key/value head's gradient
+ * sums the contributions of all G query heads that read it.
+ */
+int oracle_attention_backward(const uint16_t *q, const uint16_t *k,
+                              const uint16_t *v, const uint16_t *dout, int B,
+                              int S, int Hq, int Hkv, int D, double scale,
+                              const uint8_t *block_mask, int blk, double *dq,
+                              double *dk, double *dv)
+{
+    if (D <= 0 || D > 512 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || B <= 0)
+        return -1;
+    if (block_mask && blk <= 0) return -1;
+    const int G = Hq / Hkv;
+    const long nkb = block_mask ? (S + blk - 1) / blk : 0;
+    const long kvs = (long)Hkv * D;
+
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)S);
+        double *ds = (double *)malloc(sizeof(double) * (size_t)S);
+        uint8_t *key_ok = (uint8_t *)malloc((size_t)S);
+        /* one task per (batch, kv head): it owns that head's dK and dV */
+#pragma omp for schedule(dynamic, 1)
+        for (long bk = 0; bk < (long)B * Hkv; ++bk) {
+            const long b = bk / Hkv, kvh = bk % Hkv;
+            const uint16_t *kb = k + (b * (long)S * Hkv + kvh) * (long)D;
+            const uint16_t *vb = v + (b * (long)S * Hkv + kvh) * (long)D;
+            double *dkb = dk + (b * (long)S * Hkv + kvh) * (long)D;
+            double *dvb = dv + (b * (long)S * Hkv + kvh) * (long)D;
+            for (long kk = 0; kk < S; ++kk)
+                for (int d = 0; d < D; ++d) dkb[kk * kvs + d] = dvb[kk * kvs + d] = 0.0;
+            for (int g = 0; g < G; ++g) {
+                const long h = kvh * G + g;
+                for (long t = 0; t < S; ++t) {
+                    const long row = (b * S + t) * Hq + h;
+                    causal_key_flags(t, S, block_mask, blk, nkb, key_ok);
+                    backward_row(q + row * D, dout + row * D, kb, vb, kvs, D, S,
+                                 key_ok, scale, p, ds);
+                    double *dqr = dq + row * D;
+                    for (int d = 0; d < D; ++d) dqr[d] = 0.0;
+                    for (long kk = 0; kk <= t; ++kk) {
+                        if (!key_ok[kk]) continue;
+                        for (int d = 0; d < D; ++d) {
+                            dqr[d] += scale * ds[kk] * bf16_bits_to_double(kb[kk * kvs + d]);
+                            dkb[kk * kvs + d] +=
+                                scale * ds[kk] * bf16_bits_to_double(q[row * D + d]);
+                            dvb[kk * kvs + d] +=
+                                p[kk] * bf16_bits_to_double(dout[row * D + d]);
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(ds);
+        free(key_ok);
+    }
+    return 0;
+}
+
+/*
+ * dQ of selected query rows (b, h, t) only: each needs its own row alone.
+ * dq: [n_rows, D] fp64.
+ */
+int oracle_attention_backward_qrows(const uint16_t *q, const uint16_t *k,
+                                    const uint16_t *v, const uint16_t *dout,
+                                    int B, int S, int Hq, int Hkv, int D,
+                                    double scale, const uint8_t *block_mask,
+                                    int blk, const int64_t *rows, long n_rows,
+                                    double *dq)
+{
+    if (D <= 0 || D > 512 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || B <= 0)
+        return -1;
+    if (block_mask && blk <= 0) return -1;
+    const int G = Hq / Hkv;
+    const long nkb = block_mask ? (S + blk - 1) / blk : 0;
+    const long kvs = (long)Hkv * D;
+    int bad = 0;
+
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)S);
+        double *ds = (double *)malloc(sizeof(double) * (size_t)S);
+        uint8_t *key_ok = (uint8_t *)malloc((size_t)S);
+#pragma omp for schedule(dynamic, 4)
+        for (long r = 0; r < n_rows; ++r) {
+            const long b = rows[3 * r + 0], h = rows[3 * r + 1], t = rows[3 * r + 2];
+            if (b < 0 || b >= B || h < 0 || h >= Hq || t < 0 || t >= S) {
+                bad = 1;
+                continue;
+            }
+            const long kvh = h / G, row = (b * S + t) * Hq + h;
+            const uint16_t *kb = k + (b * (long)S * Hkv + kvh) * (long)D;
+            const uint16_t *vb = v + (b * (long)S * Hkv + kvh) * (long)D;
+            causal_key_flags(t, S, block_mask, blk, nkb, key_ok);
+            backward_row(q + row * D, dout + row * D, kb, vb, kvs, D, S, key_ok,
+                         scale, p, ds);
+            double *dqr = dq + r * (long)D;
+            for (int d = 0; d < D; ++d) dqr[d] = 0.0;
+            for (long kk = 0; kk <= t; ++kk)
+                if (key_ok[kk])
+                    for (int d = 0; d < D; ++d)
+                        dqr[d] += scale * ds[kk] * bf16_bits_to_double(kb[kk * kvs + d]);
+        }
+        free(p);
+        free(ds);
+        free(key_ok);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * dK and dV of selected key rows of one (batch b, kv head kvh): every query
+ * row of the G heads that read this kv head contributes, so each of those
+ * rows is evaluated in full; only the requested keys are accumulated.
+ * keys: n_keys positions; dk, dv: [n_keys, D] fp64.
+ */
+int oracle_attention_backward_keyrows(const uint16_t *q, const uint16_t *k,
+                                      const uint16_t *v, const uint16_t *dout,
+                                      int B, int S, int Hq, int Hkv, int D,
+                                      double scale, const uint8_t *block_mask,
+                                      int blk, int b, int kvh,
+                                      const int64_t *keys, long n_keys,
+                                      double *dk, double *dv)
+{
+    if (D <= 0 || D > 512 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || B <= 0)
+        return -1;
+    if (block_mask && blk <= 0) return -1;
+    if (b < 0 || b >= B || kvh < 0 || kvh >= Hkv) return -1;
+    for (long i = 0; i < n_keys; ++i)
+        if (keys[i] < 0 || keys[i] >= S) return -1;
+    const int G = Hq / Hkv;
+    const long nkb = block_mask ? (S + blk - 1) / blk : 0;
+    const long kvs = (long)Hkv * D;
+    const uint16_t *kb = k + ((long)b * S * Hkv + kvh) * (long)D;
+    const uint16_t *vb = v + ((long)b * S * Hkv + kvh) * (long)D;
+    for (long i = 0; i < n_keys * D; ++i) dk[i] = dv[i] = 0.0;
+
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)S);
+        double *ds = (double *)malloc(sizeof(double) * (size_t)S);
+        uint8_t *key_ok = (uint8_t *)malloc((size_t)S);
+        double *dk_l = (double *)calloc((size_t)(n_keys * D), sizeof(double));
+        double *dv_l = (double *)calloc((size_t)(n_keys * D), sizeof(double));
+#pragma omp for schedule(dynamic, 8)
+        for (long gt = 0; gt < (long)G * S; ++gt) {
+            const long h = (long)kvh * G + gt / S, t = gt % S;
+            const long row = ((long)b * S + t) * Hq + h;
+            causal_key_flags(t, S, block_mask, blk, nkb, key_ok);
+            int any = 0;
+            for (long i = 0; i < n_keys; ++i) any |= key_ok[keys[i]];
+            if (!any) continue;
+            backward_row(q + row * D, dout + row * D, kb, vb, kvs, D, S, key_ok,
+                         scale, p, ds);
+            for (long i = 0; i < n_keys; ++i) {
+                const long kk = keys[i];
+                if (!key_ok[kk]) continue;
+                for (int d = 0; d < D; ++d) {
+                    dk_l[i * D + d] += scale * ds[kk] * bf16_bits_to_double(q[row * D + d]);
+                    dv_l[i * D + d] += p[kk] * bf16_bits_to_double(dout[row * D + d]);
+                }
+            }
+        }
+#pragma omp critical
+        for (long i = 0; i < n_keys * D; ++i) {
+            dk[i] += dk_l[i];
+            dv[i] += dv_l[i];
+        }
+        free(p);
+        free(ds);
+        free(key_ok);
+        free(dk_l);
+        free(dv_l);
+    }
+    return 0;
+}
+
 /* Number of OpenMP threads the calls above use (for the baseline report). */
 int oracle_num_threads(void)
 {
