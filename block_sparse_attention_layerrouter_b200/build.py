@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa_hybrid.so")
 SOURCES = ["fa_api.cu", "fa_router.cu", "fa_index.cu", "fa_prefill.cu", "fa_decode.cu",
-           "fa_noalloc.cu"]
+           "fa_noalloc.cu", "fa_backward.cu"]
 HEADERS = ["fa_common.cuh", "fa_internal.h", os.path.join("..", "..", "include", "fa_hybrid.h")]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

@@ -71,6 +71,9 @@ _SIGNATURES = {
     "fa_soft_routed_layer": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
                                   _VP, _VP, _F, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
                                   _VP]),
+    "fa_attn_backward_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_attn_prefill_backward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I,
+                                      _I, _F, _VP, _VP, _VP, _I, _VP, _SZ, _VP, _VP]),
     "fa_hybrid_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_hybrid_layer": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
                              _VP, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
@@ -394,3 +397,32 @@ def hybrid_layer_varlen(q, k, v, cu_seqlens, max_seqlen, w1, b1, w2, b2, row_ptr
                                       _ptr(status), _stream(dev))
     _check("fa_hybrid_layer_varlen", rc)
     return o, logits, mode
+
+
+# ------------------------------------------------------------------ backward
+def attn_backward_workspace_size(B, S, Hq, Hkv, D=128) -> int:
+    return int(lib().fa_attn_backward_workspace_size(B, S, Hq, Hkv, D))
+
+
+def attn_prefill_backward(q, k, v, o, lse, dout, row_ptr=None, col_idx=None, mode=FA_MODE_FULL,
+                          mode_dev=None, scale=None, dq=None, dk=None, dv=None, workspace=None,
+                          status=None):
+    """fa_attn_prefill_backward -> (dq, dk, dv), bf16 like q, k, v."""
+    B, S, Hq, Hkv, D, o = _prefill_common(q, k, v, o, None)
+    _need(dout, "dout", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(attn_backward_workspace_size(B, S, Hq, Hkv, D), device=q.device,
+                                dtype=torch.uint8)
+    rc = lib().fa_attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                        _ptr(dq), _ptr(dk), _ptr(dv), B, S, Hq, Hkv, D, scale,
+                                        _ptr(row_ptr), _ptr(col_idx), _ptr(mode_dev), int(mode),
+                                        _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _ptr(status), _stream(q.device))
+    _check("fa_attn_prefill_backward", rc)
+    return dq, dk, dv

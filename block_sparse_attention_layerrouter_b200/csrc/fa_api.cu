@@ -256,6 +256,32 @@ FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v, voi
   return launch_prefill(sparse, st);
 }
 
+FA_API size_t fa_attn_backward_workspace_size(int B, int S, int Hq, int Hkv, int D) {
+  if (B <= 0 || S <= 0 || check_heads(Hq, Hkv, D) != FA_OK) return 0;
+  return backward_workspace_bytes(B, S, Hq);
+}
+
+FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v, const void *o,
+                                    const float *lse, const void *dout, void *dq, void *dk,
+                                    void *dv, int B, int S, int Hq, int Hkv, int D, float scale,
+                                    const int32_t *row_ptr, const int32_t *col_idx,
+                                    const int32_t *mode_dev, int mode, void *workspace,
+                                    size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (int rc = check_prefill(q, k, v, const_cast<void *>(o), B, S, Hq, Hkv, D)) return rc;
+  if (!lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (mode != FA_MODE_FULL && mode != FA_MODE_SPARSE) return FA_ERR_INVALID_ARG;
+  if (mode == FA_MODE_SPARSE && (!row_ptr || !col_idx)) return FA_ERR_INVALID_ARG;
+  if ((row_ptr == nullptr) != (col_idx == nullptr)) return FA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || ws_bytes < backward_workspace_bytes(B, S, Hq))
+    return FA_ERR_WORKSPACE;
+  BackwardLaunch a{q, k, v, o, dout, lse, dq, dk, dv, B, S, Hq, Hkv, scale, row_ptr, col_idx,
+                   mode_dev, mode, dev_status, workspace};
+  return launch_backward(a, static_cast<cudaStream_t>(stream));
+}
+
 FA_API size_t fa_varlen_workspace_size(int B, int total_tokens) {
   if (B <= 0 || total_tokens <= 0) return 0;
   return varlen_workspace_bytes(B, total_tokens);

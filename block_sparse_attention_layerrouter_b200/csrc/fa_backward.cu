@@ -1,0 +1,834 @@
+// fa_backward.cu -- gradients of the causal full and block-sparse attention
+// (dQ, dK, dV) for an upstream gradient dO of the output; what training the
+// router through the soft-routing relaxation ("Flux Attention", router
+// paragraphs) differentiates through both attention paths.
+//
+// With P = softmax(scale * Q K^T) (masked, causal) and O = P V:
+//   dV = P^T dO,   dP = dO V^T,   dS = P * (dP - D),  D_t = dO_t . O_t,
+//   dQ = scale * dS K,   dK = scale * dS^T Q
+// (D_t equals sum_k P_tk dP_tk because O_t = sum_k P_tk v_k.)
+//
+// Kernels:
+//   prep_kernel    D_t and log2(e) * lse_t per (batch, head, token); zeroes
+//                  the fp32 dQ accumulator.                      (HBM-bound)
+//   csc_kernel     for the sparse path: per 128-key tile, the 64-query
+//                  blocks whose CSR rows keep one of its two key blocks.
+//   bwd_kernel     persistent, one CTA per SM; a work item is one 128-key
+//                  tile of one (batch, KV head).  It walks the 64-query
+//                  blocks that attend the tile, for all G query heads of the
+//                  group, with five tcgen05 MMAs per step:
+//                    S^T  = K Q^T      (M=128 keys, N=64 queries, K=D)
+//                    dP^T = V dO^T     (same shape)
+//                    dV  += P^T dO     (A = P^T from TMEM; N=D, K=queries)
+//                    dK  += dS^T Q     (A = dS^T from shared memory)
+//                    dQ^T = K^T dS^T   (M=D, N=64; A and B MN-major)
+//                  dK and dV accumulate in TMEM over the whole item; each
+//                  step's dQ^T goes to an fp32 accumulator in HBM through
+//                  reductions from a separate warpgroup.  TMEM (512 columns):
+//                  S^T x2 (64 each), dP^T/dQ^T x2 (64 each), dV 128, dK 128.
+//   convert_kernel dQ = scale * accumulator (+ the router's pooling term),
+//                  rounded to bf16.
+#include "fa_common.cuh"
+#include "fa_internal.h"
+
+namespace fa {
+namespace backward {
+
+constexpr int BK = 128;                      // keys per work item
+constexpr int BQ = 64;                       // queries per step
+constexpr int HD = 128;
+constexpr int NST = 3;                       // Q/dO stages
+constexpr int NUM_THREADS = 320;             // EW x4 | dQ x4 | producer | MMA
+constexpr int WARP_PRODUCER = 8, WARP_MMA = 9;
+constexpr int KV_BYTES = BK * HD * 2;        // one K or V tile: 32 KB
+constexpr int KV_HALF = KV_BYTES / 2;        // one 64-column TMA box
+constexpr int QT_BYTES = BQ * HD * 2;        // one Q or dO tile: 16 KB
+constexpr int QT_HALF = QT_BYTES / 2;
+constexpr int STAGE_BYTES = 2 * QT_BYTES;    // Q + dO
+constexpr int DS_BYTES = BK * BQ * 2;        // one dS^T tile: 16 KB
+constexpr int VEC_BYTES = BQ * 4;            // lse2 or D of one step
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint64_t kDrainNs = 200000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Shared memory, offsets from one 1024-byte aligned base:
+// K | V | NST x (Q, dO) | 2 x dS^T | NST x (lse2, D) | barriers | TMEM addr | abort.
+struct Smem {
+  uint32_t base;
+  static constexpr uint32_t kK = 0, kV = KV_BYTES, kStages = 2 * KV_BYTES;
+  static constexpr uint32_t kDs = kStages + NST * STAGE_BYTES;
+  static constexpr uint32_t kVec = kDs + 2 * DS_BYTES;
+  static constexpr uint32_t kBars = kVec + NST * 2 * VEC_BYTES;
+  enum : uint32_t {
+    KV_FULL = 0, KV_EMPTY = 1, ST_FULL0 = 2, ST_EMPTY0 = ST_FULL0 + NST,
+    S_FULL0 = ST_EMPTY0 + NST, DP_FULL0 = S_FULL0 + 2, EW_DONE0 = DP_FULL0 + 2,
+    DQ_FULL0 = EW_DONE0 + 2, DQ_FREE0 = DQ_FULL0 + 2, ACC_FULL = DQ_FREE0 + 2,
+    ACC_FREE = ACC_FULL + 1, DRAIN = ACC_FREE + 1, NBARS = DRAIN + 1
+  };
+  FA_DEV uint32_t k() const { return base + kK; }
+  FA_DEV uint32_t v() const { return base + kV; }
+  FA_DEV uint32_t q(int s) const { return base + kStages + s * STAGE_BYTES; }
+  FA_DEV uint32_t dout(int s) const { return q(s) + QT_BYTES; }
+  FA_DEV uint32_t ds(int u) const { return base + kDs + u * DS_BYTES; }
+  FA_DEV uint32_t lse2(int s) const { return base + kVec + s * 2 * VEC_BYTES; }
+  FA_DEV uint32_t dvec(int s) const { return lse2(s) + VEC_BYTES; }
+  FA_DEV uint32_t bar(uint32_t i) const { return base + kBars + 8u * i; }
+  FA_DEV uint32_t tmem_slot() const { return base + kBars + 8u * NBARS; }
+  FA_DEV uint32_t abort_flag() const { return tmem_slot() + 4u; }
+};
+constexpr int SMEM_BYTES = 1024 + Smem::kBars + 8 * Smem::NBARS + 16;
+
+struct Params {
+  const float *lse2, *dvec;          // [B, Hq, Sp]: log2(e) * lse and D (workspace);
+                                     // Sp = S rounded up to 64, pads +inf and 0
+  float *dq_acc;                     // [B, S, Hq, D] fp32 (workspace)
+  __nv_bfloat16 *dk, *dv;            // [B, S, Hkv, D]
+  const int32_t *ct_ptr, *ct_q;      // sparse: per key tile, (qb << 2 | key-block bits)
+  const int32_t *mode;               // per batch, or nullptr
+  int mode_default;
+  const float *gscale;               // per batch output factor, or nullptr (1)
+  int gscale_complement;             // factor = 1 - gscale[b]
+  int accumulate_kv;                 // dK/dV: add into the existing output
+  int32_t *status;
+  int B, S, Sp, Hq, Hkv, G, nqb, nkt;
+  float scale, scale_log2;
+};
+
+FA_DEV Smem carve(uint8_t *raw) {
+  Smem s;
+  s.base = (smem_u32(raw) + 1023u) & ~1023u;
+  return s;
+}
+
+FA_DEV float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+FA_DEV void st_shared_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Work item w -> (key tile, batch, KV head).  Items are numbered key tile
+// first, so the tiles with the most causal query blocks (kt = 0) come first.
+struct Item {
+  int kt, b, kvh, nq, ct0;
+  bool sparse;
+};
+FA_DEV Item item_of(const Params &p, int w) {
+  Item it;
+  const int bh = p.B * p.Hkv;
+  it.kt = w / bh;
+  const int rem = w % bh;
+  it.b = rem / p.Hkv;
+  it.kvh = rem % p.Hkv;
+  const int mode = p.mode ? p.mode[it.b] : p.mode_default;
+  it.sparse = (mode == FA_MODE_SPARSE) && p.ct_ptr != nullptr;
+  if (it.sparse) {
+    it.ct0 = p.ct_ptr[it.kt];
+    it.nq = p.ct_ptr[it.kt + 1] - it.ct0;
+  } else {
+    it.ct0 = 0;
+    it.nq = p.nqb - 2 * it.kt;      // query blocks 2kt .. nqb-1
+  }
+  return it;
+}
+// Query block of the item's qi-th step and which of the tile's two key
+// blocks it keeps (bit 0: keys 0-63 of the tile, bit 1: keys 64-127).
+FA_DEV void q_block(const Params &p, const Item &it, int qi, int &qb, uint32_t &bits) {
+  if (it.sparse) {
+    const int v = p.ct_q[it.ct0 + qi];
+    qb = v >> 2;
+    bits = static_cast<uint32_t>(v) & 3u;
+  } else {
+    qb = 2 * it.kt + qi;
+    bits = 3u;
+  }
+}
+FA_DEV int item_index(int k, int total) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const int w = k * G + ((k & 1) ? (G - 1 - c) : c);
+  return w < total ? w : -1;
+}
+FA_DEV float out_factor(const Params &p, int b) {
+  if (!p.gscale) return 1.0f;
+  return p.gscale_complement ? 1.0f - p.gscale[b] : p.gscale[b];
+}
+
+FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Params &p) {
+  const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
+  return __all_sync(0xffffffffu, done);
+}
+FA_DEV bool warp_aborted(const Smem &sh) {
+  return __any_sync(0xffffffffu, ld_shared_s32(sh.abort_flag()) != 0);
+}
+
+// ------------------------------------------------------------- producer
+FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorMap *tmO,
+                         const CUtensorMap *tmK, const CUtensorMap *tmV, const Params &p,
+                         int total) {
+  int kv_n = 0;   // K/V loads issued
+  int li = 0;     // stage loads issued (continues across items)
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = item_index(k, total);
+    if (w < 0) break;
+    const Item it = item_of(p, w);
+    const int n_it = it.nq * p.G;
+    if (n_it <= 0) continue;
+    if (kv_n > 0 && !warp_wait(sh.bar(Smem::KV_EMPTY), static_cast<uint32_t>(kv_n - 1) & 1u, sh, p))
+      break;
+    {
+      const uint32_t bar = sh.bar(Smem::KV_FULL);
+      mbar_arrive_expect_tx_w(bar, 2 * KV_BYTES);
+      tma_load_4d_w(sh.k(), tmK, bar, 0, it.kvh, it.kt * BK, it.b);
+      tma_load_4d_w(sh.k() + KV_HALF, tmK, bar, 64, it.kvh, it.kt * BK, it.b);
+      tma_load_4d_w(sh.v(), tmV, bar, 0, it.kvh, it.kt * BK, it.b);
+      tma_load_4d_w(sh.v() + KV_HALF, tmV, bar, 64, it.kvh, it.kt * BK, it.b);
+      ++kv_n;
+    }
+    for (int i = 0; i < n_it; ++i) {
+      int qb;
+      uint32_t bits;
+      q_block(p, it, i / p.G, qb, bits);
+      const int h = it.kvh * p.G + i % p.G;
+      const int s = li % NST;
+      const uint32_t round = static_cast<uint32_t>(li / NST);
+      if (!warp_wait(sh.bar(Smem::ST_EMPTY0 + s), (round & 1u) ^ 1u, sh, p)) {
+        ok = false;
+        break;
+      }
+      const uint32_t bar = sh.bar(Smem::ST_FULL0 + s);
+      mbar_arrive_expect_tx_w(bar, STAGE_BYTES + 2 * VEC_BYTES);
+      tma_load_4d_w(sh.q(s), tmQ, bar, 0, h, qb * BQ, it.b);
+      tma_load_4d_w(sh.q(s) + QT_HALF, tmQ, bar, 64, h, qb * BQ, it.b);
+      tma_load_4d_w(sh.dout(s), tmO, bar, 0, h, qb * BQ, it.b);
+      tma_load_4d_w(sh.dout(s) + QT_HALF, tmO, bar, 64, h, qb * BQ, it.b);
+      const size_t vo = (static_cast<size_t>(it.b) * p.Hq + h) * p.Sp + static_cast<size_t>(qb) * BQ;
+      bulk_load_w(sh.lse2(s), p.lse2 + vo, VEC_BYTES, bar);
+      bulk_load_w(sh.dvec(s), p.dvec + vo, VEC_BYTES, bar);
+      ++li;
+    }
+  }
+  if (warp_aborted(sh)) {  // let every copy this warp issued land before exit
+    if (kv_n > 0)
+      mbar_wait_drain_a(sh.bar(Smem::KV_FULL), static_cast<uint32_t>(kv_n - 1) & 1u, kDrainNs);
+    for (int x = (li > NST ? li - NST : 0); x < li; ++x)
+      mbar_wait_drain_a(sh.bar(Smem::ST_FULL0 + x % NST), static_cast<uint32_t>(x / NST) & 1u,
+                        kDrainNs);
+  }
+}
+
+// ------------------------------------------------------------------ MMA
+FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
+  constexpr uint32_t kIdS = idesc_bf16_f32_ab(BK, BQ, false, false);   // S^T, dP^T
+  constexpr uint32_t kIdKV = idesc_bf16_f32_ab(BK, HD, false, true);   // dV, dK
+  constexpr uint32_t kIdQ = idesc_bf16_f32_ab(HD, BQ, true, true);     // dQ^T
+  // K-major operands: 128-byte rows, 8-row atoms 1024 bytes apart; a K step
+  // of 16 elements is 32 bytes inside a 64-column box.  MN-major operands:
+  // 64-element chunks of the M/N dimension one TMA box apart (LBO), groups of
+  // 8 K-rows 1024 bytes apart (SBO); a K step of 16 rows is 2048 bytes.
+  const uint64_t k_kmaj = smem_desc_sw128(sh.k(), 16, 1024);
+  const uint64_t v_kmaj = smem_desc_sw128(sh.v(), 16, 1024);
+  const uint64_t k_mn = smem_desc_sw128(sh.k(), KV_HALF, 1024);
+  const uint64_t q_kmaj = smem_desc_sw128(sh.q(0), 16, 1024);
+  const uint64_t o_kmaj = smem_desc_sw128(sh.dout(0), 16, 1024);
+  const uint64_t q_mn = smem_desc_sw128(sh.q(0), QT_HALF, 1024);
+  const uint64_t o_mn = smem_desc_sw128(sh.dout(0), QT_HALF, 1024);
+  const uint64_t ds_kmaj = smem_desc_sw128(sh.ds(0), 16, 1024);
+  const uint64_t ds_mn = smem_desc_sw128(sh.ds(0), QT_HALF, 1024);
+  const uint32_t t_dv = tmem + 256u, t_dk = tmem + 384u;
+  int nf = 0, nb = 0;      // steps whose front (S, dP) / back half was issued
+  int kv_n = 0, acc_n = 0;
+  bool ok = true;
+
+  auto front = [&]() -> bool {
+    const int s = nf % NST, u = nf & 1;
+    if (!warp_wait(sh.bar(Smem::ST_FULL0 + s), static_cast<uint32_t>(nf / NST) & 1u, sh, p))
+      return false;
+    tc_fence_after_sync();
+    const uint64_t so = static_cast<uint64_t>((s * STAGE_BYTES) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+      const uint64_t ok_ = static_cast<uint64_t>(((kk >> 2) * KV_HALF + (kk & 3) * 32) >> 4);
+      const uint64_t oq = static_cast<uint64_t>(((kk >> 2) * QT_HALF + (kk & 3) * 32) >> 4);
+      mma_bf16_ss_w(tmem + 64u * u, k_kmaj + ok_, q_kmaj + so + oq, kIdS, kk > 0 ? 1u : 0u);
+    }
+    tc_commit_w(sh.bar(Smem::S_FULL0 + u));
+    // dP^T_u is where dQ^T of step nf-2 lives until its readout is done.
+    if (nf >= 2 &&
+        !warp_wait(sh.bar(Smem::DQ_FREE0 + u), static_cast<uint32_t>((nf >> 1) - 1) & 1u, sh, p))
+      return false;
+    tc_fence_after_sync();
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+      const uint64_t ok_ = static_cast<uint64_t>(((kk >> 2) * KV_HALF + (kk & 3) * 32) >> 4);
+      const uint64_t oq = static_cast<uint64_t>(((kk >> 2) * QT_HALF + (kk & 3) * 32) >> 4);
+      mma_bf16_ss_w(tmem + 128u + 64u * u, v_kmaj + ok_, o_kmaj + so + oq, kIdS,
+                    kk > 0 ? 1u : 0u);
+    }
+    tc_commit_w(sh.bar(Smem::DP_FULL0 + u));
+    ++nf;
+    return true;
+  };
+  auto back = [&](bool first, bool last) -> bool {
+    const int s = nb % NST, u = nb & 1;
+    if (!warp_wait(sh.bar(Smem::EW_DONE0 + u), static_cast<uint32_t>(nb >> 1) & 1u, sh, p))
+      return false;
+    if (first && acc_n > 0 &&
+        !warp_wait(sh.bar(Smem::ACC_FREE), static_cast<uint32_t>(acc_n - 1) & 1u, sh, p))
+      return false;
+    tc_fence_after_sync();
+    const uint64_t so = static_cast<uint64_t>((s * STAGE_BYTES) >> 4);
+    const uint64_t du = static_cast<uint64_t>((u * DS_BYTES) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < BQ / 16; ++kk) {   // dV += P^T dO
+      mma_bf16_ts_w(t_dv, tmem + 64u * u + kk * 8, o_mn + so + static_cast<uint64_t>((kk * 2048) >> 4),
+                    kIdKV, (first && kk == 0) ? 0u : 1u);
+    }
+#pragma unroll
+    for (int kk = 0; kk < BQ / 16; ++kk) {   // dK += dS^T Q
+      mma_bf16_ss_w(t_dk, ds_kmaj + du + static_cast<uint64_t>((kk * 32) >> 4),
+                    q_mn + so + static_cast<uint64_t>((kk * 2048) >> 4), kIdKV,
+                    (first && kk == 0) ? 0u : 1u);
+    }
+    tc_commit_w(sh.bar(Smem::ST_EMPTY0 + s));
+#pragma unroll
+    for (int kk = 0; kk < BK / 16; ++kk) {   // dQ^T = K^T dS^T
+      mma_bf16_ss_w(tmem + 128u + 64u * u, k_mn + static_cast<uint64_t>((kk * 2048) >> 4),
+                    ds_mn + du + static_cast<uint64_t>((kk * 2048) >> 4), kIdQ, kk > 0 ? 1u : 0u);
+    }
+    tc_commit_w(sh.bar(Smem::DQ_FULL0 + u));
+    if (last) {
+      tc_commit_w(sh.bar(Smem::ACC_FULL));
+      tc_commit_w(sh.bar(Smem::KV_EMPTY));
+    }
+    ++nb;
+    return true;
+  };
+
+  for (int k = 0; ok; ++k) {
+    const int w = item_index(k, total);
+    if (w < 0) break;
+    const Item it = item_of(p, w);
+    const int n_it = it.nq * p.G;
+    if (n_it <= 0) continue;
+    if (!(ok = warp_wait(sh.bar(Smem::KV_FULL), static_cast<uint32_t>(kv_n) & 1u, sh, p))) break;
+    tc_fence_after_sync();
+    if (!(ok = front())) break;
+    for (int i = 0; i < n_it; ++i) {
+      if (i + 1 < n_it && !(ok = front())) break;
+      if (!(ok = back(i == 0, i + 1 == n_it))) break;
+    }
+    if (!ok) break;
+    ++kv_n;
+    ++acc_n;
+  }
+  if (warp_aborted(sh)) {  // let every MMA this warp issued finish before exit
+    tc_commit_w(sh.bar(Smem::DRAIN));
+    mbar_wait_drain_a(sh.bar(Smem::DRAIN), 0, kDrainNs);
+  }
+}
+
+// Rounds 8 fp32 values to bf16 and writes them as one 16-byte chunk.
+FA_DEV uint4 pack8(const float *x) {
+  return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                    pack_bf16x2(x[6], x[7]));
+}
+FA_DEV void unpack8(uint4 v, float *x) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// One row of dK or dV (128 values in TMEM registers) -> bf16 in HBM.
+FA_DEV void store_grad_row(__nv_bfloat16 *dst, const uint32_t (&r)[128], float f, bool acc) {
+  uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+  for (int c = 0; c < HD / 8; ++c) {
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[8 * c + e]) * f;
+    if (acc) {
+      float old[8];
+      unpack8(d4[c], old);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] += old[e];
+    }
+    d4[c] = pack8(x);
+  }
+}
+
+// ---------------------------------------- elementwise (one key row per thread)
+FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
+  const int r = threadIdx.x;                         // key row within the tile
+  const uint32_t lane = ((static_cast<uint32_t>(r) >> 5) * 32u) << 16;
+  const float c = p.scale_log2;
+  int n = 0, acc_n = 0;
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int w = item_index(k, total);
+    if (w < 0) break;
+    const Item it = item_of(p, w);
+    const int n_it = it.nq * p.G;
+    const int key = it.kt * BK + r;
+    const float f = out_factor(p, it.b);
+    __nv_bfloat16 *dk_row = p.dk + ((static_cast<size_t>(it.b) * p.S + key) * p.Hkv + it.kvh) * HD;
+    __nv_bfloat16 *dv_row = p.dv + ((static_cast<size_t>(it.b) * p.S + key) * p.Hkv + it.kvh) * HD;
+    if (n_it <= 0) {          // no query attends this tile: zero gradients
+      if (key < p.S && !p.accumulate_kv) {
+        uint4 *a = reinterpret_cast<uint4 *>(dk_row), *b = reinterpret_cast<uint4 *>(dv_row);
+        for (int i = 0; i < HD / 8; ++i) a[i] = b[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      continue;
+    }
+    for (int i = 0; i < n_it; ++i, ++n) {
+      int qb;
+      uint32_t bits;
+      q_block(p, it, i / p.G, qb, bits);
+      const int u = n & 1, s = n % NST;
+      const uint32_t ph = static_cast<uint32_t>(n >> 1) & 1u;
+      if (!warp_wait(sh.bar(Smem::S_FULL0 + u), ph, sh, p) ||
+          !warp_wait(sh.bar(Smem::ST_FULL0 + s), static_cast<uint32_t>(n / NST) & 1u, sh, p)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t t_s = tmem + lane + 64u * u;
+      float pv[BQ];
+      {
+        uint32_t a[32], b[32];
+        tmem_ld32(t_s, a);
+        tmem_ld32(t_s + 32u, b);
+        tmem_ld_wait(a);
+        tmem_ld_wait(b);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          pv[j] = __uint_as_float(a[j]);
+          pv[32 + j] = __uint_as_float(b[j]);
+        }
+      }
+      // P = 2^(s * c - lse2) where key <= query and the key block is kept.
+      const bool rowbit = ((bits >> (r >> 6)) & 1u) != 0u;
+      const int rel = qb * BQ - key;                 // query - key at j = 0
+      const bool any = rowbit && (rel + BQ - 1 >= 0);
+      const uint32_t lse_s = sh.lse2(s);
+#pragma unroll
+      for (int j4 = 0; j4 < BQ / 4; ++j4) {
+        const float4 L = ld_shared_f4(lse_s + 16u * j4);
+        const float l4[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * j4 + e;
+          const bool keep = any && (j + rel >= 0);
+          pv[j] = keep ? ex2(fmaf(pv[j], c, -l4[e])) : 0.0f;
+        }
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(pv[2 * j], pv[2 * j + 1]);
+        tmem_st32(t_s, pk);
+      }
+      // dS = P (dP - D), into the dS^T tile once MMAs of step n-2 are done with it.
+      if (!warp_wait(sh.bar(Smem::DP_FULL0 + u), ph, sh, p) ||
+          (n >= 2 && !warp_wait(sh.bar(Smem::DQ_FULL0 + u), static_cast<uint32_t>((n >> 1) - 1) & 1u,
+                                sh, p))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t d_s = sh.dvec(s);
+      const uint32_t ds_row = sh.ds(u) + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane + 128u + 64u * u + 32u * hlf, a);
+        tmem_ld_wait(a);
+        float ds[32];
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 Dv = ld_shared_f4(d_s + 16u * (8 * hlf + j4));
+          const float d4[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * j4 + e;
+            ds[j] = pv[32 * hlf + j] * (__uint_as_float(a[j]) - d4[e]);
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t chunk = static_cast<uint32_t>(4 * hlf + cc);
+          const uint4 v = pack8(ds + 8 * cc);
+          st_shared_u4(ds_row + ((chunk ^ (static_cast<uint32_t>(r) & 7u)) << 4), v.x, v.y, v.z,
+                       v.w);
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      mbar_arrive_a(sh.bar(Smem::EW_DONE0 + u));
+    }
+    if (!ok) break;
+    // Epilogue: dV and scale * dK of this key row.
+    if (!warp_wait(sh.bar(Smem::ACC_FULL), static_cast<uint32_t>(acc_n) & 1u, sh, p)) break;
+    tc_fence_after_sync();
+    const bool store = key < p.S && !ld_shared_s32(sh.abort_flag());
+    {
+      uint32_t a[128];
+      tmem_ld128_wait(tmem + lane + 256u, a);
+      if (store) store_grad_row(dv_row, a, f, p.accumulate_kv != 0);
+    }
+    {
+      uint32_t a[128];
+      tmem_ld128_wait(tmem + lane + 384u, a);
+      if (store) store_grad_row(dk_row, a, f * p.scale, p.accumulate_kv != 0);
+    }
+    tc_fence_before_sync();
+    mbar_arrive_a(sh.bar(Smem::ACC_FREE));
+    ++acc_n;
+  }
+}
+
+// ------------------------------------------- dQ readout (one dim per thread)
+FA_DEV void run_dq(const Smem &sh, uint32_t tmem, const Params &p, int total) {
+  const int d = threadIdx.x - 128;
+  const uint32_t lane = (((static_cast<uint32_t>(threadIdx.x) >> 5) & 3u) * 32u) << 16;
+  int n = 0;
+  for (int k = 0;; ++k) {
+    const int w = item_index(k, total);
+    if (w < 0) return;
+    const Item it = item_of(p, w);
+    const int n_it = it.nq * p.G;
+    const float f = out_factor(p, it.b);
+    for (int i = 0; i < n_it; ++i, ++n) {
+      int qb;
+      uint32_t bits;
+      q_block(p, it, i / p.G, qb, bits);
+      const int h = it.kvh * p.G + i % p.G;
+      const int u = n & 1;
+      if (!warp_wait(sh.bar(Smem::DQ_FULL0 + u), static_cast<uint32_t>(n >> 1) & 1u, sh, p)) return;
+      tc_fence_after_sync();
+      uint32_t a[32], b[32];
+      tmem_ld32(tmem + lane + 128u + 64u * u, a);
+      tmem_ld32(tmem + lane + 160u + 64u * u, b);
+      tmem_ld_wait(a);
+      tmem_ld_wait(b);
+      tc_fence_before_sync();
+      mbar_arrive_a(sh.bar(Smem::DQ_FREE0 + u));
+      float *dst = p.dq_acc + (static_cast<size_t>(it.b) * p.S + static_cast<size_t>(qb) * BQ) *
+                                  p.Hq * HD +
+                   static_cast<size_t>(h) * HD + d;
+      const size_t rs = static_cast<size_t>(p.Hq) * HD;
+      const int valid = p.S - qb * BQ;               // rows past the end are padding
+      if (valid >= BQ) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          atomicAdd(dst + j * rs, __uint_as_float(a[j]) * f);
+          atomicAdd(dst + (32 + j) * rs, __uint_as_float(b[j]) * f);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j < valid) atomicAdd(dst + j * rs, __uint_as_float(a[j]) * f);
+          if (32 + j < valid) atomicAdd(dst + (32 + j) * rs, __uint_as_float(b[j]) * f);
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const Params p, int total_items) {
+  extern __shared__ uint8_t smem_raw[];
+  const Smem sh = carve(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init_a(sh.bar(Smem::KV_FULL), 1);
+    mbar_init_a(sh.bar(Smem::KV_EMPTY), 1);
+    for (int i = 0; i < NST; ++i) {
+      mbar_init_a(sh.bar(Smem::ST_FULL0 + i), 1);
+      mbar_init_a(sh.bar(Smem::ST_EMPTY0 + i), 1);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init_a(sh.bar(Smem::S_FULL0 + u), 1);
+      mbar_init_a(sh.bar(Smem::DP_FULL0 + u), 1);
+      mbar_init_a(sh.bar(Smem::EW_DONE0 + u), 128);
+      mbar_init_a(sh.bar(Smem::DQ_FULL0 + u), 1);
+      mbar_init_a(sh.bar(Smem::DQ_FREE0 + u), 128);
+    }
+    mbar_init_a(sh.bar(Smem::ACC_FULL), 1);
+    mbar_init_a(sh.bar(Smem::ACC_FREE), 128);
+    mbar_init_a(sh.bar(Smem::DRAIN), 1);
+    st_shared_s32(sh.abort_flag(), 0);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc_a(sh.tmem_slot(), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = static_cast<uint32_t>(ld_shared_s32(sh.tmem_slot()));
+  if (warp < 4) {
+    run_ew(sh, tmem, p, total_items);
+  } else if (warp < 8) {
+    run_dq(sh, tmem, p, total_items);
+  } else if (warp == WARP_PRODUCER) {
+    run_producer(sh, &tmQ, &tmO, &tmK, &tmV, p, total_items);
+  } else {
+    run_mma(sh, tmem, p, total_items);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// D_t = dO_t . O_t and lse2_t = log2(e) lse_t for every (batch, token, head),
+// one warp per row; optionally zeroes the row of the dQ accumulator.  Rows
+// t in [S, Sp) of the padded vectors get lse2 = +inf and D = 0, so padded
+// query rows have P = 0.
+__global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16 *o,
+                                                   const __nv_bfloat16 *dout, const float *lse,
+                                                   int B, int S, int Sp, int Hq, float *dvec,
+                                                   float *lse2, float *dq_acc, int zero_acc) {
+  const long long prow = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (prow >= static_cast<long long>(B) * Sp * Hq) return;
+  {
+    const long long h = prow % Hq, bt = prow / Hq, t = bt % Sp, b = bt / Sp;
+    if (t >= S) {
+      if (lane == 0) {
+        dvec[(b * Hq + h) * Sp + t] = 0.f;
+        lse2[(b * Hq + h) * Sp + t] = INFINITY;
+      }
+      return;
+    }
+  }
+  const long long h_ = prow % Hq, bt_ = prow / Hq, t_ = bt_ % Sp, b_ = bt_ / Sp;
+  const long long row = (b_ * S + t_) * Hq + h_;
+  const uint2 a = reinterpret_cast<const uint2 *>(o + row * HD)[lane];
+  const uint2 g = reinterpret_cast<const uint2 *>(dout + row * HD)[lane];
+  float s = __uint_as_float(a.x << 16) * __uint_as_float(g.x << 16);
+  s = fmaf(__uint_as_float(a.x & 0xffff0000u), __uint_as_float(g.x & 0xffff0000u), s);
+  s = fmaf(__uint_as_float(a.y << 16), __uint_as_float(g.y << 16), s);
+  s = fmaf(__uint_as_float(a.y & 0xffff0000u), __uint_as_float(g.y & 0xffff0000u), s);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (zero_acc)
+    reinterpret_cast<float4 *>(dq_acc + row * HD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane == 0) {
+    dvec[(b_ * Hq + h_) * Sp + t_] = s;
+    lse2[(b_ * Hq + h_) * Sp + t_] = lse[(b_ * Hq + h_) * S + t_] * kLog2e;
+  }
+}
+
+// Per 128-key tile kt: the query blocks qb >= 2kt whose CSR row keeps key
+// block 2kt (bit 0) or 2kt+1 (bit 1), ascending, as (qb << 2 | bits).  Rows
+// must be ascending and causal; a row that is not is reported (its entries
+// past the first bad one are ignored).  One CTA.
+FA_DEV bool row_has(const int32_t *col, int lo, int hi, int c) {
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int v = col[mid];
+    if (v == c) return true;
+    if (v < c) lo = mid + 1; else hi = mid;
+  }
+  return false;
+}
+__global__ void __launch_bounds__(1024) csc_kernel(const int32_t *row_ptr, const int32_t *col_idx,
+                                                   int nqb, int nkt, int32_t *ct_ptr,
+                                                   int32_t *ct_q, int32_t *status) {
+  extern __shared__ int32_t cnt[];   // nkt + 1
+  // Row checks (ascending, inside [0, qb]).
+  for (int qb = threadIdx.x; qb < nqb; qb += blockDim.x) {
+    int prev = -1;
+    for (int e = row_ptr[qb]; e < row_ptr[qb + 1]; ++e) {
+      const int c = col_idx[e];
+      if (c <= prev || c > qb) {
+        report(status, FA_DEV_BAD_INDEX);
+        break;
+      }
+      prev = c;
+    }
+  }
+  auto bits_of = [&](int qb, int kt) -> int {
+    const int lo = row_ptr[qb], hi = row_ptr[qb + 1];
+    int b = row_has(col_idx, lo, hi, 2 * kt) ? 1 : 0;
+    if (2 * kt + 1 < nqb && row_has(col_idx, lo, hi, 2 * kt + 1)) b |= 2;
+    return b;
+  };
+  for (int kt = threadIdx.x; kt < nkt; kt += blockDim.x) {
+    int c = 0;
+    for (int qb = 2 * kt; qb < nqb; ++qb) c += bits_of(qb, kt) ? 1 : 0;
+    cnt[kt] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int c = cnt[kt];
+      cnt[kt] = run;
+      ct_ptr[kt] = run;
+      run += c;
+    }
+    ct_ptr[nkt] = run;
+  }
+  __syncthreads();
+  for (int kt = threadIdx.x; kt < nkt; kt += blockDim.x) {
+    int pos = cnt[kt];
+    for (int qb = 2 * kt; qb < nqb; ++qb) {
+      const int b = bits_of(qb, kt);
+      if (b) ct_q[pos++] = (qb << 2) | b;
+    }
+  }
+}
+
+// dQ = scale * accumulator, plus (optionally) the router's pooling gradient
+// dx / (n_head + n_tail) on the first n_head and last n_tail tokens; bf16.
+__global__ void __launch_bounds__(256) convert_kernel(const float *acc, __nv_bfloat16 *dq, int B,
+                                                      int S, int Hq, float scale,
+                                                      const float *pool_dx, int n_head,
+                                                      int n_tail) {
+  const long long n8 = static_cast<long long>(B) * S * Hq * HD / 8;
+  const float inv_n = 1.0f / static_cast<float>(n_head + n_tail > 0 ? n_head + n_tail : 1);
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4 *>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4 *>(acc)[2 * i + 1];
+    float x[8] = {a.x * scale, a.y * scale, a.z * scale, a.w * scale,
+                  b.x * scale, b.y * scale, b.z * scale, b.w * scale};
+    if (pool_dx) {
+      const long long e = i * 8;                 // element index in [B, S, Hq, D]
+      const long long row = e / HD, dd = e % HD;
+      const long long h = row % Hq, bt = row / Hq, t = bt % S, bb = bt / S;
+      if (t < n_head || t >= S - n_tail) {
+        const float *src = pool_dx + (bb * Hq + h) * HD + dd;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] += src[k] * inv_n;
+      }
+    }
+    reinterpret_cast<uint4 *>(dq)[i] = pack8(x);
+  }
+}
+
+}  // namespace backward
+
+// ----------------------------------------------------------------- host ---
+namespace {
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+}  // namespace
+
+size_t backward_workspace_bytes(int B, int S, int Hq) {
+  const size_t nqb = (static_cast<size_t>(S) + 63) / 64, nkt = (nqb + 1) / 2;
+  const size_t acc = static_cast<size_t>(B) * S * Hq * backward::HD * 4;
+  const size_t vec = static_cast<size_t>(B) * Hq * nqb * 64 * 4;
+  return align256(acc) + 2 * align256(vec) + align256((nkt + 1) * 4) + align256(nkt * nqb * 4);
+}
+
+int launch_backward(const BackwardLaunch &a, cudaStream_t stream) {
+  using namespace backward;
+  const int nqb = (a.S + 63) / 64, nkt = (nqb + 1) / 2, Sp = nqb * 64;
+  uint8_t *ws = reinterpret_cast<uint8_t *>(a.workspace);
+  float *acc = reinterpret_cast<float *>(ws);
+  ws += align256(static_cast<size_t>(a.B) * a.S * a.Hq * HD * 4);
+  float *dvec = reinterpret_cast<float *>(ws);
+  ws += align256(static_cast<size_t>(a.B) * a.Hq * Sp * 4);
+  float *lse2 = reinterpret_cast<float *>(ws);
+  ws += align256(static_cast<size_t>(a.B) * a.Hq * Sp * 4);
+  int32_t *ct_ptr = reinterpret_cast<int32_t *>(ws);
+  ws += align256((static_cast<size_t>(nkt) + 1) * 4);
+  int32_t *ct_q = reinterpret_cast<int32_t *>(ws);
+
+  const long long rows = static_cast<long long>(a.B) * a.S * a.Hq;
+  const long long prows = static_cast<long long>(a.B) * Sp * a.Hq;
+  prep_kernel<<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16 *>(a.o), reinterpret_cast<const __nv_bfloat16 *>(a.dout),
+      a.lse, a.B, a.S, Sp, a.Hq, dvec, lse2, acc, a.zero_dq_acc);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const bool maybe_sparse =
+      a.row_ptr != nullptr && (a.mode_dev != nullptr || a.mode_default == FA_MODE_SPARSE);
+  if (maybe_sparse) {
+    const size_t sm = (static_cast<size_t>(nkt) + 1) * 4;
+    if (sm > 200 * 1024) return FA_ERR_UNSUPPORTED;
+    if (sm > 48 * 1024 &&
+        cudaFuncSetAttribute(csc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sm)) != cudaSuccess)
+      return FA_ERR_CUDA;
+    csc_kernel<<<1, 1024, sm, stream>>>(a.row_ptr, a.col_idx, nqb, nkt, ct_ptr, ct_q, a.status);
+    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+
+  CUtensorMap tmQ, tmO, tmK, tmV;
+  if (make_tmap_bhsd(&tmQ, a.q, a.B, a.S, a.Hq, 64, BQ) != 0 ||
+      make_tmap_bhsd(&tmO, a.dout, a.B, a.S, a.Hq, 64, BQ) != 0 ||
+      make_tmap_bhsd(&tmK, a.k, a.B, a.S, a.Hkv, 64, BK) != 0 ||
+      make_tmap_bhsd(&tmV, a.v, a.B, a.S, a.Hkv, 64, BK) != 0)
+    return FA_ERR_CUDA;
+  if (cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  Params p;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.dq_acc = acc;
+  p.dk = reinterpret_cast<__nv_bfloat16 *>(a.dk);
+  p.dv = reinterpret_cast<__nv_bfloat16 *>(a.dv);
+  p.ct_ptr = maybe_sparse ? ct_ptr : nullptr;
+  p.ct_q = maybe_sparse ? ct_q : nullptr;
+  p.mode = a.mode_dev;
+  p.mode_default = a.mode_default;
+  p.gscale = a.gscale;
+  p.gscale_complement = a.gscale_complement;
+  p.accumulate_kv = a.accumulate_kv;
+  p.status = a.status;
+  p.B = a.B;
+  p.S = a.S;
+  p.Sp = Sp;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
+  p.nqb = nqb;
+  p.nkt = nkt;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * kLog2e;
+  const long long total = static_cast<long long>(nkt) * a.B * a.Hkv;
+  if (total <= 0 || total > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const int ctas = static_cast<int>(total < sms ? total : sms);
+  bwd_kernel<<<ctas, NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmO, tmK, tmV, p,
+                                                        static_cast<int>(total));
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (a.convert_dq) {
+    const long long n8 = rows * HD / 8;
+    const long long blocks = (n8 + 255) / 256;
+    convert_kernel<<<static_cast<unsigned>(blocks < 4 * sms ? blocks : 4 * sms), 256, 0, stream>>>(
+        acc, reinterpret_cast<__nv_bfloat16 *>(a.dq), a.B, a.S, a.Hq, a.scale, a.pool_dx,
+        a.n_head, a.n_tail);
+    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+}  // namespace fa

@@ -286,9 +286,25 @@ FA_DEV void tma_load_4d_w(uint32_t dst, const CUtensorMap *map, uint32_t bar, in
 // Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), bf16 A
 // and B (bits 7-9 and 10-12 = 1), A K-major, B K-major or MN-major (bit 16),
 // N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// The same with the A-major bit (15) as well: A MN-major when set.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16_f32(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
+// Untiled bulk copy global -> shared (both 16-byte aligned, size a multiple
+// of 16), completion as transaction bytes on `bar`; one elected lane issues.
+FA_DEV void bulk_load_w(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 // Shared-memory matrix descriptor (sm_100 format: start >> 4 in bits 0-13,

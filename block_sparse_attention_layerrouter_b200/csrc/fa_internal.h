@@ -67,6 +67,30 @@ int launch_router_soft(const float *logits, const float *gumbel, int B, float ta
                        cudaStream_t stream);
 int launch_router(const RouterLaunch &a, cudaStream_t stream);
 
+struct BackwardLaunch {
+  const void *q, *k, *v, *o, *dout;
+  const float *lse;                  // [B, Hq, S] natural-log LSE of the forward
+  void *dq, *dk, *dv;
+  int B, S, Hq, Hkv;
+  float scale;
+  const int32_t *row_ptr, *col_idx;  // nullptr: FULL only
+  const int32_t *mode_dev;           // per batch, or nullptr (mode_default)
+  int mode_default;
+  int32_t *status;
+  void *workspace;
+  // Soft routing: outputs scaled per batch by gscale[b] (or 1 - gscale[b]);
+  // dK/dV added into the existing outputs; dQ accumulated across calls.
+  const float *gscale = nullptr;
+  int gscale_complement = 0;
+  int accumulate_kv = 0;
+  int zero_dq_acc = 1;
+  int convert_dq = 1;
+  const float *pool_dx = nullptr;    // [B, Hq*D] router pooling gradient, or nullptr
+  int n_head = 0, n_tail = 0;
+};
+size_t backward_workspace_bytes(int B, int S, int Hq);
+int launch_backward(const BackwardLaunch &a, cudaStream_t stream);
+
 long long index_nnz(int nrows, int sb, int wb);
 int launch_index(int nrows, int sb, int wb, int32_t *row_ptr, int32_t *col_idx,
                  cudaStream_t stream);

@@ -148,6 +148,35 @@ FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
                    fa_sparse_cfg cfg, void *o, float *lse, void *workspace,
                    size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/* ------------------------------------------------------------ backward ---
+ * Gradients of the causal attention of fa_attn_prefill_full / _blocksparse
+ * for an upstream gradient dO of the output: what training the router through
+ * the soft-routing relaxation ("Flux Attention", router paragraphs) needs
+ * from each attention path.  With P the masked softmax of scale * Q K^T:
+ *   dV = P^T dO,  dS = P * (dO V^T - D),  D_t = dO_t . O_t,
+ *   dQ = scale * dS K,  dK = scale * dS^T Q
+ * (a KV head's dK/dV sum over the G query heads that read it).
+ *   q, o, dout bf16 [B, S, Hq, D]; k, v bf16 [B, S, Hkv, D]; lse fp32
+ *   [B, Hq, S] = the forward's LSE (natural log), all device, caller-owned.
+ *   dq bf16 [B, S, Hq, D]; dk, dv bf16 [B, S, Hkv, D]: overwritten.
+ *   mode: FA_MODE_FULL or FA_MODE_SPARSE for every batch element, or
+ *   mode_dev (device int32 [B], e.g. the router's mode_out) when non-NULL;
+ *   row_ptr/col_idx: the CSR of fa_blocksparse_index for S (required when
+ *   any element may be SPARSE; rows ascending and causal, else the
+ *   offending rows are reported as FA_DEV_BAD_INDEX).
+ *   workspace >= fa_attn_backward_workspace_size(B, S, Hq, Hkv, D) bytes,
+ *   16-byte aligned device memory: an fp32 dQ accumulator [B, S, Hq, D], the
+ *   row terms D and the LSE in base 2, and the transposed block pattern.
+ * D must be 128.  Returns FA_OK or an fa_status; enqueues only. */
+FA_API size_t fa_attn_backward_workspace_size(int B, int S, int Hq, int Hkv, int D);
+FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v,
+                                    const void *o, const float *lse, const void *dout,
+                                    void *dq, void *dk, void *dv, int B, int S, int Hq,
+                                    int Hkv, int D, float scale, const int32_t *row_ptr,
+                                    const int32_t *col_idx, const int32_t *mode_dev,
+                                    int mode, void *workspace, size_t ws_bytes,
+                                    int32_t *dev_status, void *stream);
+
 /* ------------------------------------------- variable-length batches ---
  * Serving form of the routed layer ("Flux Attention": the router decides per
  * request, before each layer's attention): B sequences of different lengths
