@@ -709,6 +709,24 @@ def run_only(args, wl):
         elif args.only == "prefill_sparse":
             fn = lambda: capi.attn_prefill_blocksparse(q, k, v, rp, ci, o=o)  # noqa: E731
             work = 4.0 * 128 * Hq * B * csr_nnz(S, wl.sink, wl.window) * 4096 / 1e12
+        elif args.only in ("backward_full", "backward_sparse"):
+            sparse = args.only == "backward_sparse"
+            lse = torch.empty(B, Hq, S, device=dev)
+            if sparse:
+                capi.attn_prefill_blocksparse(q, k, v, rp, ci, o=o, lse=lse)
+            else:
+                capi.attn_prefill_full(q, k, v, o=o, lse=lse)
+            do = inputs.randn_bf16((B, S, Hq, 128), wl.seed + 400, device=dev)
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            bws = torch.empty(capi.attn_backward_workspace_size(B, S, Hq, Hkv), dtype=torch.uint8,
+                              device=dev)
+            fn = lambda: capi.attn_prefill_backward(  # noqa: E731
+                q, k, v, o, lse, do, rp, ci, mode=int(sparse), dq=dq, dk=dk, dv=dv, workspace=bws)
+            # 2.5x the forward's FLOPs: S, dP, dV, dK and dQ products per pair.
+            if sparse:
+                work = 10.0 * 128 * Hq * B * csr_nnz(S, wl.sink, wl.window) * 4096 / 1e12
+            else:
+                work = 2.5 * flops_full(wl) / 1e12
         elif args.only == "router":
             fn = lambda: capi.router_decide(q, w1, b1, w2, b2)  # noqa: E731
             work = (B * 200 * Hq * 128 * 2 + w1.numel() * 4) / 1e9

@@ -74,6 +74,11 @@ _SIGNATURES = {
     "fa_attn_backward_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_attn_prefill_backward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I,
                                       _I, _F, _VP, _VP, _VP, _I, _VP, _SZ, _VP, _VP]),
+    "fa_soft_routed_backward_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "fa_soft_routed_layer_backward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I,
+                                           _I, _F, _VP, _VP, _I, _VP, _VP, _VP, _F, _VP, _VP, _VP,
+                                           _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
+                                           _VP]),
     "fa_hybrid_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_hybrid_layer": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
                              _VP, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
@@ -426,3 +431,32 @@ def attn_prefill_backward(q, k, v, o, lse, dout, row_ptr=None, col_idx=None, mod
                                         _ptr(status), _stream(q.device))
     _check("fa_attn_prefill_backward", rc)
     return dq, dk, dv
+
+
+def soft_routed_layer_backward(q, k, v, o_full, lse_full, o_sparse, lse_sparse, dy, w1, b1, w2,
+                               b2, row_ptr, col_idx, gumbel=None, tau=1.0, scale=None,
+                               workspace=None, status=None):
+    """fa_soft_routed_layer_backward -> dict of dq, dk, dv (bf16), dw1, db1,
+    dw2, db2 (fp32) and r."""
+    B, S, Hq, Hkv, D, _ = _prefill_common(q, k, v, o_full, None)
+    _need(dy, "dy", torch.bfloat16, 4)
+    hidden = w1.shape[0]
+    dev = q.device
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+           "dw1": torch.empty_like(w1), "db1": torch.empty(hidden, device=dev),
+           "dw2": torch.empty_like(w2), "db2": torch.empty(2, device=dev),
+           "r": torch.empty(B, device=dev)}
+    if workspace is None:
+        workspace = torch.empty(int(lib().fa_soft_routed_backward_workspace_size(B, S, Hq, Hkv, D,
+                                                                                 hidden)),
+                                device=dev, dtype=torch.uint8)
+    rc = lib().fa_soft_routed_layer_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o_full), _ptr(lse_full), _ptr(o_sparse), _ptr(lse_sparse),
+        _ptr(dy), B, S, Hq, Hkv, D, scale, _ptr(w1), _ptr(b1), hidden, _ptr(w2), _ptr(b2),
+        _ptr(gumbel), float(tau), _ptr(row_ptr), _ptr(col_idx), _ptr(out["dq"]), _ptr(out["dk"]),
+        _ptr(out["dv"]), _ptr(out["dw1"]), _ptr(out["db1"]), _ptr(out["dw2"]), _ptr(out["db2"]),
+        _ptr(out["r"]), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(status), _stream(dev))
+    _check("fa_soft_routed_layer_backward", rc)
+    return out

@@ -282,6 +282,37 @@ FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v,
   return launch_backward(a, static_cast<cudaStream_t>(stream));
 }
 
+FA_API size_t fa_soft_routed_backward_workspace_size(int B, int S, int Hq, int Hkv, int D,
+                                                     int hidden) {
+  if (B <= 0 || S <= 0 || hidden <= 0 || check_heads(Hq, Hkv, D) != FA_OK) return 0;
+  return soft_backward_workspace_bytes(B, S, Hq, hidden);
+}
+
+FA_API int fa_soft_routed_layer_backward(
+    const void *q, const void *k, const void *v, const void *o_full, const float *lse_full,
+    const void *o_sparse, const float *lse_sparse, const void *dy, int B, int S, int Hq, int Hkv,
+    int D, float scale, const float *w1, const float *b1, int hidden, const float *w2,
+    const float *b2, const float *gumbel, float tau, const int32_t *row_ptr,
+    const int32_t *col_idx, void *dq, void *dk, void *dv, float *dw1, float *db1, float *dw2,
+    float *db2, float *r_out, void *workspace, size_t ws_bytes, int32_t *dev_status,
+    void *stream) {
+  if (int rc = check_prefill(q, k, v, const_cast<void *>(o_full), B, S, Hq, Hkv, D)) return rc;
+  if (int rc = check_router(q, B, S, Hq, D, 100, 100, w1, hidden, w2)) return rc;
+  if (!o_sparse || !lse_full || !lse_sparse || !dy || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(o_sparse) || !aligned16(dy) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (!dw1 || !db1 || !dw2 || !db2 || !row_ptr || !col_idx) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !(tau > 0.f)) return FA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) ||
+      ws_bytes < soft_backward_workspace_bytes(B, S, Hq, hidden))
+    return FA_ERR_WORKSPACE;
+  SoftBackwardLaunch a{q, k, v, o_full, o_sparse, dy, lse_full, lse_sparse, B, S, Hq, Hkv, scale,
+                       w1, b1, w2, b2, hidden, gumbel, tau, row_ptr, col_idx, dq, dk, dv, dw1,
+                       db1, dw2, db2, r_out, workspace, dev_status};
+  return launch_soft_backward(a, static_cast<cudaStream_t>(stream));
+}
+
 FA_API size_t fa_varlen_workspace_size(int B, int total_tokens) {
   if (B <= 0 || total_tokens <= 0) return 0;
   return varlen_workspace_bytes(B, total_tokens);

@@ -730,53 +730,107 @@ __global__ void __launch_bounds__(256) convert_kernel(const float *acc, __nv_bfl
   }
 }
 
+// dr[b] += sign * sum over (head, token) of D (the padded entries are 0):
+// with D = dy . O per row, the FULL pass adds and the SPARSE pass subtracts,
+// leaving dr[b] = sum dy * (O_FA - O_SA).
+__global__ void __launch_bounds__(256) dsum_kernel(const float *dvec, long long per_b, float sign,
+                                                   float *dr) {
+  const int b = blockIdx.y;
+  const float *src = dvec + b * per_b;
+  float s = 0.f;
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < per_b;
+       i += static_cast<long long>(gridDim.x) * 256)
+    s += src[i];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += red[w];
+    atomicAdd(dr + b, sign * t);
+  }
+}
+
+__global__ void zero_kernel(float *x, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) x[i] = 0.f;
+}
+
 }  // namespace backward
 
 // ----------------------------------------------------------------- host ---
 namespace {
-size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-}  // namespace
 
-size_t backward_workspace_bytes(int B, int S, int Hq) {
-  const size_t nqb = (static_cast<size_t>(S) + 63) / 64, nkt = (nqb + 1) / 2;
-  const size_t acc = static_cast<size_t>(B) * S * Hq * backward::HD * 4;
-  const size_t vec = static_cast<size_t>(B) * Hq * nqb * 64 * 4;
-  return align256(acc) + 2 * align256(vec) + align256((nkt + 1) * 4) + align256(nkt * nqb * 4);
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace carve-up of one backward: dQ accumulator, D and lse2 vectors
+// (padded to Sp = 64 * nqb per (batch, head)), transposed block pattern.
+struct Plan {
+  int nqb, nkt, Sp;
+  float *acc, *dvec, *lse2;
+  int32_t *ct_ptr, *ct_q;
+  size_t bytes;
+};
+Plan make_plan(int B, int S, int Hq, void *workspace) {
+  Plan pl;
+  pl.nqb = (S + 63) / 64;
+  pl.nkt = (pl.nqb + 1) / 2;
+  pl.Sp = pl.nqb * 64;
+  uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t *p = ws ? ws + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  pl.acc = reinterpret_cast<float *>(take(static_cast<size_t>(B) * S * Hq * backward::HD * 4));
+  pl.dvec = reinterpret_cast<float *>(take(static_cast<size_t>(B) * Hq * pl.Sp * 4));
+  pl.lse2 = reinterpret_cast<float *>(take(static_cast<size_t>(B) * Hq * pl.Sp * 4));
+  pl.ct_ptr = reinterpret_cast<int32_t *>(take((static_cast<size_t>(pl.nkt) + 1) * 4));
+  pl.ct_q = reinterpret_cast<int32_t *>(
+      take(static_cast<size_t>(pl.nkt) * static_cast<size_t>(pl.nqb) * 4));
+  pl.bytes = off;
+  return pl;
 }
 
-int launch_backward(const BackwardLaunch &a, cudaStream_t stream) {
-  using namespace backward;
-  const int nqb = (a.S + 63) / 64, nkt = (nqb + 1) / 2, Sp = nqb * 64;
-  uint8_t *ws = reinterpret_cast<uint8_t *>(a.workspace);
-  float *acc = reinterpret_cast<float *>(ws);
-  ws += align256(static_cast<size_t>(a.B) * a.S * a.Hq * HD * 4);
-  float *dvec = reinterpret_cast<float *>(ws);
-  ws += align256(static_cast<size_t>(a.B) * a.Hq * Sp * 4);
-  float *lse2 = reinterpret_cast<float *>(ws);
-  ws += align256(static_cast<size_t>(a.B) * a.Hq * Sp * 4);
-  int32_t *ct_ptr = reinterpret_cast<int32_t *>(ws);
-  ws += align256((static_cast<size_t>(nkt) + 1) * 4);
-  int32_t *ct_q = reinterpret_cast<int32_t *>(ws);
+int sm_count(int *sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
 
-  const long long rows = static_cast<long long>(a.B) * a.S * a.Hq;
-  const long long prows = static_cast<long long>(a.B) * Sp * a.Hq;
+int run_prep(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
+  using namespace backward;
+  const long long prows = static_cast<long long>(a.B) * pl.Sp * a.Hq;
   prep_kernel<<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16 *>(a.o), reinterpret_cast<const __nv_bfloat16 *>(a.dout),
-      a.lse, a.B, a.S, Sp, a.Hq, dvec, lse2, acc, a.zero_dq_acc);
-  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
-  const bool maybe_sparse =
-      a.row_ptr != nullptr && (a.mode_dev != nullptr || a.mode_default == FA_MODE_SPARSE);
-  if (maybe_sparse) {
-    const size_t sm = (static_cast<size_t>(nkt) + 1) * 4;
-    if (sm > 200 * 1024) return FA_ERR_UNSUPPORTED;
-    if (sm > 48 * 1024 &&
-        cudaFuncSetAttribute(csc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sm)) != cudaSuccess)
-      return FA_ERR_CUDA;
-    csc_kernel<<<1, 1024, sm, stream>>>(a.row_ptr, a.col_idx, nqb, nkt, ct_ptr, ct_q, a.status);
-    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
-  }
+      a.lse, a.B, a.S, pl.Sp, a.Hq, pl.dvec, pl.lse2, pl.acc, a.zero_dq_acc);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
+bool may_be_sparse(const BackwardLaunch &a) {
+  return a.row_ptr != nullptr && (a.mode_dev != nullptr || a.mode_default == FA_MODE_SPARSE);
+}
+
+int run_csc(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
+  using namespace backward;
+  const size_t sm = (static_cast<size_t>(pl.nkt) + 1) * 4;
+  if (sm > 200 * 1024) return FA_ERR_UNSUPPORTED;
+  if (sm > 48 * 1024 &&
+      cudaFuncSetAttribute(csc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sm)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  csc_kernel<<<1, 1024, sm, stream>>>(a.row_ptr, a.col_idx, pl.nqb, pl.nkt, pl.ct_ptr, pl.ct_q,
+                                      a.status);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int run_main(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
+  using namespace backward;
   CUtensorMap tmQ, tmO, tmK, tmV;
   if (make_tmap_bhsd(&tmQ, a.q, a.B, a.S, a.Hq, 64, BQ) != 0 ||
       make_tmap_bhsd(&tmO, a.dout, a.B, a.S, a.Hq, 64, BQ) != 0 ||
@@ -786,14 +840,15 @@ int launch_backward(const BackwardLaunch &a, cudaStream_t stream) {
   if (cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
       cudaSuccess)
     return FA_ERR_CUDA;
+  const bool sparse = may_be_sparse(a);
   Params p;
-  p.lse2 = lse2;
-  p.dvec = dvec;
-  p.dq_acc = acc;
+  p.lse2 = pl.lse2;
+  p.dvec = pl.dvec;
+  p.dq_acc = pl.acc;
   p.dk = reinterpret_cast<__nv_bfloat16 *>(a.dk);
   p.dv = reinterpret_cast<__nv_bfloat16 *>(a.dv);
-  p.ct_ptr = maybe_sparse ? ct_ptr : nullptr;
-  p.ct_q = maybe_sparse ? ct_q : nullptr;
+  p.ct_ptr = sparse ? pl.ct_ptr : nullptr;
+  p.ct_q = sparse ? pl.ct_q : nullptr;
   p.mode = a.mode_dev;
   p.mode_default = a.mode_default;
   p.gscale = a.gscale;
@@ -802,33 +857,142 @@ int launch_backward(const BackwardLaunch &a, cudaStream_t stream) {
   p.status = a.status;
   p.B = a.B;
   p.S = a.S;
-  p.Sp = Sp;
+  p.Sp = pl.Sp;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.G = a.Hq / a.Hkv;
-  p.nqb = nqb;
-  p.nkt = nkt;
+  p.nqb = pl.nqb;
+  p.nkt = pl.nkt;
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
-  const long long total = static_cast<long long>(nkt) * a.B * a.Hkv;
+  const long long total = static_cast<long long>(pl.nkt) * a.B * a.Hkv;
   if (total <= 0 || total > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return FA_ERR_CUDA;
+  int sms = 148;
+  if (int rc = sm_count(&sms)) return rc;
   const int ctas = static_cast<int>(total < sms ? total : sms);
   bwd_kernel<<<ctas, NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmO, tmK, tmV, p,
                                                         static_cast<int>(total));
-  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
-  if (a.convert_dq) {
-    const long long n8 = rows * HD / 8;
-    const long long blocks = (n8 + 255) / 256;
-    convert_kernel<<<static_cast<unsigned>(blocks < 4 * sms ? blocks : 4 * sms), 256, 0, stream>>>(
-        acc, reinterpret_cast<__nv_bfloat16 *>(a.dq), a.B, a.S, a.Hq, a.scale, a.pool_dx,
-        a.n_head, a.n_tail);
-    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
-  }
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int run_convert(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
+  using namespace backward;
+  int sms = 148;
+  if (int rc = sm_count(&sms)) return rc;
+  const long long n8 = static_cast<long long>(a.B) * a.S * a.Hq * HD / 8;
+  const long long blocks = (n8 + 255) / 256;
+  convert_kernel<<<static_cast<unsigned>(blocks < 4 * sms ? blocks : 4 * sms), 256, 0, stream>>>(
+      pl.acc, reinterpret_cast<__nv_bfloat16 *>(a.dq), a.B, a.S, a.Hq, a.scale, a.pool_dx,
+      a.n_head, a.n_tail);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int B, int S, int Hq) {
+  return make_plan(B, S, Hq, nullptr).bytes;
+}
+
+int launch_backward(const BackwardLaunch &a, cudaStream_t stream) {
+  const Plan pl = make_plan(a.B, a.S, a.Hq, a.workspace);
+  if (int rc = run_prep(a, pl, stream)) return rc;
+  if (may_be_sparse(a))
+    if (int rc = run_csc(a, pl, stream)) return rc;
+  if (int rc = run_main(a, pl, stream)) return rc;
+  if (a.convert_dq)
+    if (int rc = run_convert(a, pl, stream)) return rc;
   return FA_OK;
+}
+
+// Soft-routed layer: y = r O_FA + (1 - r) O_SA, r from the router.  Workspace:
+// one attention-backward plan (reused by both passes), the router's forward
+// workspace, then x, logits, r, dr, dlogits, da and dx.
+namespace {
+struct SoftPlan {
+  Plan att;
+  void *router_ws;
+  float *x, *logits, *r, *dr, *dlogits, *da, *dx;
+  size_t bytes;
+};
+SoftPlan make_soft_plan(int B, int S, int Hq, int hidden, void *workspace) {
+  SoftPlan sp;
+  sp.att = make_plan(B, S, Hq, workspace);
+  uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+  size_t off = sp.att.bytes;
+  auto take = [&](size_t bytes) {
+    uint8_t *p = ws ? ws + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  const size_t in_f = static_cast<size_t>(Hq) * backward::HD;
+  sp.router_ws = take(router_workspace_bytes(B, Hq, backward::HD, hidden));
+  sp.x = reinterpret_cast<float *>(take(B * in_f * 4));
+  sp.logits = reinterpret_cast<float *>(take(static_cast<size_t>(B) * 2 * 4));
+  sp.r = reinterpret_cast<float *>(take(static_cast<size_t>(B) * 4));
+  sp.dr = reinterpret_cast<float *>(take(static_cast<size_t>(B) * 4));
+  sp.dlogits = reinterpret_cast<float *>(take(static_cast<size_t>(B) * 2 * 4));
+  sp.da = reinterpret_cast<float *>(take(static_cast<size_t>(B) * hidden * 4));
+  sp.dx = reinterpret_cast<float *>(take(B * in_f * 4));
+  sp.bytes = off;
+  return sp;
+}
+}  // namespace
+
+size_t soft_backward_workspace_bytes(int B, int S, int Hq, int hidden) {
+  return make_soft_plan(B, S, Hq, hidden, nullptr).bytes;
+}
+
+int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream) {
+  using namespace backward;
+  const SoftPlan sp = make_soft_plan(a.B, a.S, a.Hq, a.hidden, a.workspace);
+  constexpr int kHead = 100, kTail = 100;
+  // Router forward again: pooling slices, ReLU outputs, logits, r.
+  RouterLaunch rl{a.q, a.B, a.S, a.Hq, kHead, kTail, a.w1, a.b1, a.w2, a.b2, a.hidden,
+                  sp.logits, nullptr, sp.router_ws};
+  if (int rc = launch_router(rl, stream)) return rc;
+  float *r = a.r_out ? a.r_out : sp.r;
+  if (int rc = launch_router_soft(sp.logits, a.gumbel, a.B, a.tau, r, stream)) return rc;
+  zero_kernel<<<(a.B + 255) / 256, 256, 0, stream>>>(sp.dr, a.B);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const long long per_b = static_cast<long long>(a.Hq) * sp.att.Sp;
+  const unsigned dsum_blocks = static_cast<unsigned>(per_b / 4096 + 1 < 64 ? per_b / 4096 + 1 : 64);
+
+  // FULL path, upstream r dy: dK/dV written, dQ accumulated (zeroed first).
+  BackwardLaunch fa{a.q, a.k, a.v, a.o_full, a.dy, a.lse_full, a.dq, a.dk, a.dv, a.B, a.S, a.Hq,
+                    a.Hkv, a.scale, nullptr, nullptr, nullptr, FA_MODE_FULL, a.status,
+                    a.workspace};
+  fa.gscale = r;
+  fa.zero_dq_acc = 1;
+  if (int rc = run_prep(fa, sp.att, stream)) return rc;
+  dsum_kernel<<<dim3(dsum_blocks, a.B), 256, 0, stream>>>(sp.att.dvec, per_b, 1.0f, sp.dr);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (int rc = run_main(fa, sp.att, stream)) return rc;
+
+  // SPARSE path, upstream (1 - r) dy: dK/dV added, dQ accumulated.
+  BackwardLaunch sa{a.q, a.k, a.v, a.o_sparse, a.dy, a.lse_sparse, a.dq, a.dk, a.dv, a.B, a.S,
+                    a.Hq, a.Hkv, a.scale, a.row_ptr, a.col_idx, nullptr, FA_MODE_SPARSE,
+                    a.status, a.workspace};
+  sa.gscale = r;
+  sa.gscale_complement = 1;
+  sa.accumulate_kv = 1;
+  sa.zero_dq_acc = 0;
+  if (int rc = run_prep(sa, sp.att, stream)) return rc;
+  dsum_kernel<<<dim3(dsum_blocks, a.B), 256, 0, stream>>>(sp.att.dvec, per_b, -1.0f, sp.dr);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (int rc = run_csc(sa, sp.att, stream)) return rc;
+  if (int rc = run_main(sa, sp.att, stream)) return rc;
+
+  // Router: dr -> dlogits -> dW2, db2, dW1, db1 and the pooled-input gradient.
+  RouterBwdLaunch rb{sp.logits, a.gumbel, a.tau, sp.dr, sp.router_ws, a.w1, a.w2, a.B, a.Hq,
+                     a.hidden, kHead + kTail, sp.x, sp.dlogits, sp.da, sp.dx, a.dw1, a.db1,
+                     a.dw2, a.db2};
+  if (int rc = launch_router_backward(rb, stream)) return rc;
+
+  // dQ = scale * (accumulated r dQ_FA + (1 - r) dQ_SA) + pooling term.
+  sa.pool_dx = sp.dx;
+  sa.n_head = kHead;
+  sa.n_tail = kTail;
+  return run_convert(sa, sp.att, stream);
 }
 
 }  // namespace fa

@@ -91,6 +91,43 @@ struct BackwardLaunch {
 size_t backward_workspace_bytes(int B, int S, int Hq);
 int launch_backward(const BackwardLaunch &a, cudaStream_t stream);
 
+// Router backward (soft routing): gradients of W1, b1, W2, b2 and of the
+// pooled input x, from dr = dL/dr per sequence.  `router_ws` holds a router
+// forward of the same inputs (pooling slices and ReLU outputs).
+struct RouterBwdLaunch {
+  const float *logits, *gumbel;
+  float tau;
+  const float *dr;
+  void *router_ws;
+  const float *w1, *w2;
+  int B, Hq, hidden, n_sel;
+  float *x, *dlogits, *da, *dx;        // workspace: [B, Hq*D], [B, 2], [B, hidden], [B, Hq*D]
+  float *dw1, *db1, *dw2, *db2;        // outputs
+};
+void router_ws_parts(void *workspace, int B, int Hq, float **part, float **hid);
+int launch_router_backward(const RouterBwdLaunch &a, cudaStream_t stream);
+
+// Soft-routed layer backward: both attention paths (upstream r dy and
+// (1 - r) dy), the router, and the pooling term of dQ.
+struct SoftBackwardLaunch {
+  const void *q, *k, *v, *o_full, *o_sparse, *dy;
+  const float *lse_full, *lse_sparse;
+  int B, S, Hq, Hkv;
+  float scale;
+  const float *w1, *b1, *w2, *b2;
+  int hidden;
+  const float *gumbel;
+  float tau;
+  const int32_t *row_ptr, *col_idx;
+  void *dq, *dk, *dv;
+  float *dw1, *db1, *dw2, *db2;
+  float *r_out;                        // nullable
+  void *workspace;
+  int32_t *status;
+};
+size_t soft_backward_workspace_bytes(int B, int S, int Hq, int hidden);
+int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream);
+
 long long index_nnz(int nrows, int sb, int wb);
 int launch_index(int nrows, int sb, int wb, int32_t *row_ptr, int32_t *col_idx,
                  cudaStream_t stream);

@@ -132,7 +132,149 @@ __global__ void soft_kernel(const float *logits, const float *gumbel, float inv_
   r[b] = 1.0f / (1.0f + expf((zs - zf) * inv_tau));
 }
 
+// ---------------------------------------------------------------- backward
+// Chain rule through the soft-routed layer, for an upstream dr = dL/dr per
+// sequence (r the weight of the FULL output):
+//   dz_FA = dr r (1 - r) / tau = -dz_SA          (r = sigmoid((z_FA - z_SA)/tau))
+//   dW2 = dz^T h, db2 = sum_b dz, da = (dz W2) * [h > 0], db1 = sum_b da,
+//   dW1 = da^T x, dx = da W1
+// (h = ReLU(a) > 0 exactly where a > 0; ReLU'(0) = 0).
+
+// x[b, i] = (sum of the pooling slices) / n_sel, materialised for dW1.
+__global__ void __launch_bounds__(256) pooled_kernel(const float *part, float *x, int B, int in_f,
+                                                     float inv_n) {
+  const long long n = static_cast<long long>(B) * in_f;
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * 256) {
+    float v = 0.f;
+#pragma unroll
+    for (int z = 0; z < kPoolSlices; ++z) v += part[z * n + i];
+    x[i] = v * inv_n;
+  }
+}
+
+// One CTA per hidden unit u: dz per sequence (recomputed from logits, noise
+// and dr), dW2[:, u], da[:, u], db1[u]; unit 0 also writes db2 and dz.
+__global__ void __launch_bounds__(128) head_bwd_kernel(const float *logits, const float *gumbel,
+                                                       float inv_tau, const float *dr,
+                                                       const float *hid, const float *w2, int B,
+                                                       int hidden, float *dlogits, float *da,
+                                                       float *dw2, float *db1, float *db2) {
+  const int u = blockIdx.x;
+  float g2a = 0.f, g2b = 0.f, g1 = 0.f;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    float zf = logits[2 * b], zs = logits[2 * b + 1];
+    if (gumbel) {
+      zf += gumbel[2 * b];
+      zs += gumbel[2 * b + 1];
+    }
+    const float r = 1.0f / (1.0f + expf((zs - zf) * inv_tau));
+    const float dzf = dr[b] * r * (1.0f - r) * inv_tau;
+    const float h = hid[static_cast<size_t>(b) * hidden + u];
+    g2a += dzf * h;                  // dW2[0, u] (pi_FA row)
+    g2b -= dzf * h;                  // dW2[1, u] (pi_SA row): dz_SA = -dz_FA
+    const float dh = dzf * (w2[u] - w2[hidden + u]);
+    const float a = h > 0.f ? dh : 0.f;
+    da[static_cast<size_t>(b) * hidden + u] = a;
+    g1 += a;
+    if (u == 0) {
+      dlogits[2 * b] = dzf;
+      dlogits[2 * b + 1] = -dzf;
+    }
+  }
+  __shared__ float red[3][4];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    g2a += __shfl_xor_sync(0xffffffffu, g2a, off);
+    g2b += __shfl_xor_sync(0xffffffffu, g2b, off);
+    g1 += __shfl_xor_sync(0xffffffffu, g1, off);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red[0][w] = g2a;
+    red[1][w] = g2b;
+    red[2][w] = g1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+    for (int i = 0; i < 4; ++i) {
+      s0 += red[0][i];
+      s1 += red[1][i];
+      s2 += red[2][i];
+    }
+    dw2[u] = s0;
+    dw2[hidden + u] = s1;
+    db1[u] = s2;
+  }
+  if (u == 0 && threadIdx.x == 0 && db2) {
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) {
+      float zf = logits[2 * b], zs = logits[2 * b + 1];
+      if (gumbel) {
+        zf += gumbel[2 * b];
+        zs += gumbel[2 * b + 1];
+      }
+      const float r = 1.0f / (1.0f + expf((zs - zf) * inv_tau));
+      s += dr[b] * r * (1.0f - r) * inv_tau;
+    }
+    db2[0] = s;
+    db2[1] = -s;
+  }
+}
+
+// dW1[u, i] = sum_b da[b, u] x[b, i]: one CTA per row u of W1.
+__global__ void __launch_bounds__(256) dw1_kernel(const float *da, const float *x, int B, int in_f,
+                                                  int hidden, float *dw1) {
+  const int u = blockIdx.x;
+  for (int i = threadIdx.x; i < in_f; i += 256) {
+    float s = 0.f;
+    for (int b = 0; b < B; ++b)
+      s = fmaf(da[static_cast<size_t>(b) * hidden + u], x[static_cast<size_t>(b) * in_f + i], s);
+    dw1[static_cast<size_t>(u) * in_f + i] = s;
+  }
+}
+
+// dx[b, i] = sum_u da[b, u] W1[u, i]: one thread per (i, b), W1 read by
+// columns (coalesced across threads).
+__global__ void __launch_bounds__(256) dx_kernel(const float *da, const float *w1, int B, int in_f,
+                                                 int hidden, float *dx) {
+  const int i = blockIdx.x * 256 + threadIdx.x, b = blockIdx.y;
+  if (i >= in_f) return;
+  const float *dab = da + static_cast<size_t>(b) * hidden;
+  float s = 0.f;
+  for (int u = 0; u < hidden; ++u) s = fmaf(dab[u], w1[static_cast<size_t>(u) * in_f + i], s);
+  dx[static_cast<size_t>(b) * in_f + i] = s;
+}
+
 }  // namespace router
+
+void router_ws_parts(void *workspace, int B, int Hq, float **part, float **hid) {
+  const size_t pbytes = static_cast<size_t>(router::kPoolSlices) * B * Hq * router::HD * sizeof(float);
+  *part = reinterpret_cast<float *>(workspace);
+  *hid = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) +
+                                   ((pbytes + 255) & ~static_cast<size_t>(255)));
+}
+
+int launch_router_backward(const RouterBwdLaunch &a, cudaStream_t stream) {
+  using namespace router;
+  const int in_f = a.Hq * HD;
+  float *part = nullptr, *hid = nullptr;
+  router_ws_parts(a.router_ws, a.B, a.Hq, &part, &hid);
+  const long long n = static_cast<long long>(a.B) * in_f;
+  pooled_kernel<<<static_cast<unsigned>((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184), 256, 0,
+                  stream>>>(part, a.x, a.B, in_f, 1.0f / static_cast<float>(a.n_sel));
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  head_bwd_kernel<<<a.hidden, 128, 0, stream>>>(a.logits, a.gumbel, 1.0f / a.tau, a.dr, hid, a.w2,
+                                                a.B, a.hidden, a.dlogits, a.da, a.dw2, a.db1,
+                                                a.db2);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  dw1_kernel<<<a.hidden, 256, 0, stream>>>(a.da, a.x, a.B, in_f, a.hidden, a.dw1);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  dx_kernel<<<dim3((in_f + 255) / 256, a.B), 256, 0, stream>>>(a.da, a.w1, a.B, in_f, a.hidden,
+                                                                a.dx);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 int launch_router_soft(const float *logits, const float *gumbel, int B, float tau, float *r,
                        cudaStream_t stream) {

@@ -177,6 +177,33 @@ FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v,
                                     int mode, void *workspace, size_t ws_bytes,
                                     int32_t *dev_status, void *stream);
 
+/* Backward of the soft-routed layer y = r O_FA + (1 - r) O_SA (see
+ * fa_soft_routed_layer), for an upstream dy bf16 [B, S, Hq, D]: the router's
+ * weight gradients and the attention inputs' gradients through both paths,
+ * the pooling included.  By the chain rule:
+ *   dr_b = sum dy . (O_FA - O_SA),  dz_FA = -dz_SA = dr r (1 - r) / tau,
+ *   dW2 = dz^T h, db2 = sum_b dz, da = (dz W2) * [h > 0] (h = ReLU(W1 x + b1)),
+ *   dW1 = da^T x, db1 = sum_b da, dx = da W1,
+ *   dQ = r dQ_FA(dy) + (1 - r) dQ_SA(dy) + dx / 200 on the first and last
+ *   100 tokens (x is their mean), dK and dV = r d*_FA + (1 - r) d*_SA.
+ *   o_full / lse_full, o_sparse / lse_sparse: the outputs and LSE of
+ *   fa_attn_prefill_full and fa_attn_prefill_blocksparse on q, k, v.
+ *   dq, dk, dv bf16 like q, k, v; dw1 [hidden, Hq*D], db1 [hidden], dw2 [2,
+ *   hidden], db2 [2]: fp32, overwritten.  r_out fp32 [B] or NULL.
+ *   row_ptr / col_idx: the CSR of the sparse path.  gumbel, tau as in
+ *   fa_router_soft.  workspace >= fa_soft_routed_backward_workspace_size(...).
+ * ReLU'(0) is taken as 0. */
+FA_API size_t fa_soft_routed_backward_workspace_size(int B, int S, int Hq, int Hkv,
+                                                     int D, int hidden);
+FA_API int fa_soft_routed_layer_backward(
+    const void *q, const void *k, const void *v, const void *o_full,
+    const float *lse_full, const void *o_sparse, const float *lse_sparse,
+    const void *dy, int B, int S, int Hq, int Hkv, int D, float scale,
+    const float *w1, const float *b1, int hidden, const float *w2, const float *b2,
+    const float *gumbel, float tau, const int32_t *row_ptr, const int32_t *col_idx,
+    void *dq, void *dk, void *dv, float *dw1, float *db1, float *dw2, float *db2,
+    float *r_out, void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+
 /* ------------------------------------------- variable-length batches ---
  * Serving form of the routed layer ("Flux Attention": the router decides per
  * request, before each layer's attention): B sequences of different lengths

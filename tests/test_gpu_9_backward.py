@@ -135,3 +135,45 @@ def test_backward_qwen3_4b_layer_sampled(mode):
     kt = torch.from_numpy(keys).cuda()
     assert_close_grad(to_f64(dk[0, kt, kvh]), want_k, "%s dk rows" % mode)
     assert_close_grad(to_f64(dv[0, kt, kvh]), want_v, "%s dv rows" % mode)
+
+
+def test_soft_routed_layer_backward_matches_oracle():
+    """Router weights and attention inputs' gradients through the soft-routed
+    layer y = r O_FA + (1 - r) O_SA, against the oracle's chain rule."""
+    B, S, Hq, Hkv, H1, W, tau = 2, 384, 4, 2, 32, 128, 1.5
+    c = capi.cfg(64, 64, W)
+    q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, 641, device="cuda")
+    dy = inputs.randn_bf16((B, S, Hq, 128), 1041, device="cuda")
+    rp, ci = capi.blocksparse_index(S, c)
+    status = zero_status()
+    lse_f = torch.empty(B, Hq, S, device="cuda")
+    lse_s = torch.empty(B, Hq, S, device="cuda")
+    o_f = capi.attn_prefill_full(q, k, v, lse=lse_f, status=status)
+    o_s = capi.attn_prefill_blocksparse(q, k, v, rp, ci, lse=lse_s, status=status)
+    w1, b1, w2, b2 = inputs.router_weights(Hq * 128, H1, 641, b2=(0.02, -0.01), std=0.05)
+    g = inputs.gumbel(B, 641)
+    out = capi.soft_routed_layer_backward(q, k, v, o_f, lse_f, o_s, lse_s, dy, w1.cuda(),
+                                          b1.cuda(), w2.cuda(), b2.cuda(), rp, ci,
+                                          gumbel=g.cuda(), tau=tau, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+    qb, kb, vb, dyb = (inputs.bits(t) for t in (q, k, v, dy))
+    mask = oracle.rows_to_dense_mask(oracle.blocksparse_rows(S, 64, 64, W))
+    x = oracle.router_pool(qb)
+    o_full, _ = oracle.attention(qb, kb, vb, SCALE)
+    o_sparse, _ = oracle.attention(qb, kb, vb, SCALE, mask)
+    rb = oracle.soft_routed_backward(x, w1.double().numpy(), b1.double().numpy(),
+                                     w2.double().numpy(), b2.double().numpy(),
+                                     g.double().numpy(), tau, o_full, o_sparse,
+                                     oracle.bf16_bits_to_f64(dyb))
+    np.testing.assert_allclose(out["r"].cpu().double().numpy(), rb["r"], atol=1e-5)
+    for name in ("dw1", "db1", "dw2", "db2"):
+        assert_close_grad(to_f64(out[name]), rb[name], "soft " + name)
+    gf = oracle.attention_backward(qb, kb, vb, dyb, SCALE)
+    gs = oracle.attention_backward(qb, kb, vb, dyb, SCALE, mask)
+    r = rb["r"][:, None, None, None]
+    want = [r * a + (1 - r) * b for a, b in zip(gf, gs)]
+    want[0] = want[0] + oracle.router_pool_backward(rb["dx"], S, Hq, 128)
+    for name, w in zip(("dq", "dk", "dv"), want):
+        assert_close_grad(to_f64(out[name]), w, "soft " + name)
