@@ -50,6 +50,20 @@ int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int 
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
+int make_tmap_rows_f32(CUtensorMap *map, void *base, long long rows, int box_cols,
+                       int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return -1;
+  const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {128 * 4};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
 namespace {
 
 constexpr int kHeadDim = 128;
@@ -258,7 +272,7 @@ FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v, voi
 
 FA_API size_t fa_attn_backward_workspace_size(int B, int S, int Hq, int Hkv, int D) {
   if (B <= 0 || S <= 0 || check_heads(Hq, Hkv, D) != FA_OK) return 0;
-  return backward_workspace_bytes(B, S, Hq);
+  return backward_workspace_bytes(B, S, Hq, Hkv);
 }
 
 FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v, const void *o,
@@ -275,7 +289,7 @@ FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v,
   if (mode != FA_MODE_FULL && mode != FA_MODE_SPARSE) return FA_ERR_INVALID_ARG;
   if (mode == FA_MODE_SPARSE && (!row_ptr || !col_idx)) return FA_ERR_INVALID_ARG;
   if ((row_ptr == nullptr) != (col_idx == nullptr)) return FA_ERR_INVALID_ARG;
-  if (!workspace || !aligned16(workspace) || ws_bytes < backward_workspace_bytes(B, S, Hq))
+  if (!workspace || !aligned16(workspace) || ws_bytes < backward_workspace_bytes(B, S, Hq, Hkv))
     return FA_ERR_WORKSPACE;
   BackwardLaunch a{q, k, v, o, dout, lse, dq, dk, dv, B, S, Hq, Hkv, scale, row_ptr, col_idx,
                    mode_dev, mode, dev_status, workspace};
@@ -285,7 +299,7 @@ FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v,
 FA_API size_t fa_soft_routed_backward_workspace_size(int B, int S, int Hq, int Hkv, int D,
                                                      int hidden) {
   if (B <= 0 || S <= 0 || hidden <= 0 || check_heads(Hq, Hkv, D) != FA_OK) return 0;
-  return soft_backward_workspace_bytes(B, S, Hq, hidden);
+  return soft_backward_workspace_bytes(B, S, Hq, Hkv, hidden);
 }
 
 FA_API int fa_soft_routed_layer_backward(
@@ -305,7 +319,7 @@ FA_API int fa_soft_routed_layer_backward(
   if (!dw1 || !db1 || !dw2 || !db2 || !row_ptr || !col_idx) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !(tau > 0.f)) return FA_ERR_INVALID_ARG;
   if (!workspace || !aligned16(workspace) ||
-      ws_bytes < soft_backward_workspace_bytes(B, S, Hq, hidden))
+      ws_bytes < soft_backward_workspace_bytes(B, S, Hq, Hkv, hidden))
     return FA_ERR_WORKSPACE;
   SoftBackwardLaunch a{q, k, v, o_full, o_sparse, dy, lse_full, lse_sparse, B, S, Hq, Hkv, scale,
                        w1, b1, w2, b2, hidden, gumbel, tau, row_ptr, col_idx, dq, dk, dv, dw1,

@@ -23,8 +23,9 @@
 //                    dK  += dS^T Q     (A = dS^T from shared memory)
 //                    dQ^T = K^T dS^T   (M=D, N=64; A and B MN-major)
 //                  dK and dV accumulate in TMEM over the whole item; each
-//                  step's dQ^T goes to an fp32 accumulator in HBM through
-//                  reductions from a separate warpgroup.  TMEM (512 columns):
+//                  step's dQ^T goes to an fp32 accumulator in HBM through TMA
+//                  reduce-adds issued by a separate warpgroup (each warp
+//                  stages its 64 x 32 slice in shared memory).  TMEM (512 columns):
 //                  S^T x2 (64 each), dP^T/dQ^T x2 (64 each), dV 128, dK 128.
 //   convert_kernel dQ = scale * accumulator (+ the router's pooling term),
 //                  rounded to bf16.
@@ -47,17 +48,20 @@ constexpr int QT_HALF = QT_BYTES / 2;
 constexpr int STAGE_BYTES = 2 * QT_BYTES;    // Q + dO
 constexpr int DS_BYTES = BK * BQ * 2;        // one dS^T tile: 16 KB
 constexpr int VEC_BYTES = BQ * 4;            // lse2 or D of one step
+constexpr int STG_BYTES = BQ * 32 * 4;       // one dQ warp's staging box: 64 x 32 fp32
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kDrainNs = 200000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Shared memory, offsets from one 1024-byte aligned base:
-// K | V | NST x (Q, dO) | 2 x dS^T | NST x (lse2, D) | barriers | TMEM addr | abort.
+// K | V | NST x (Q, dO) | 2 x dS^T | 4 x dQ staging | NST x (lse2, D) | barriers |
+// TMEM addr | abort.
 struct Smem {
   uint32_t base;
   static constexpr uint32_t kK = 0, kV = KV_BYTES, kStages = 2 * KV_BYTES;
   static constexpr uint32_t kDs = kStages + NST * STAGE_BYTES;
-  static constexpr uint32_t kVec = kDs + 2 * DS_BYTES;
+  static constexpr uint32_t kStg = kDs + 2 * DS_BYTES;
+  static constexpr uint32_t kVec = kStg + 4 * STG_BYTES;
   static constexpr uint32_t kBars = kVec + NST * 2 * VEC_BYTES;
   enum : uint32_t {
     KV_FULL = 0, KV_EMPTY = 1, ST_FULL0 = 2, ST_EMPTY0 = ST_FULL0 + NST,
@@ -70,6 +74,7 @@ struct Smem {
   FA_DEV uint32_t q(int s) const { return base + kStages + s * STAGE_BYTES; }
   FA_DEV uint32_t dout(int s) const { return q(s) + QT_BYTES; }
   FA_DEV uint32_t ds(int u) const { return base + kDs + u * DS_BYTES; }
+  FA_DEV uint32_t stg(int w) const { return base + kStg + w * STG_BYTES; }
   FA_DEV uint32_t lse2(int s) const { return base + kVec + s * 2 * VEC_BYTES; }
   FA_DEV uint32_t dvec(int s) const { return lse2(s) + VEC_BYTES; }
   FA_DEV uint32_t bar(uint32_t i) const { return base + kBars + 8u * i; }
@@ -77,11 +82,12 @@ struct Smem {
   FA_DEV uint32_t abort_flag() const { return tmem_slot() + 4u; }
 };
 constexpr int SMEM_BYTES = 1024 + Smem::kBars + 8 * Smem::NBARS + 16;
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 
 struct Params {
   const float *lse2, *dvec;          // [B, Hq, Sp]: log2(e) * lse and D (workspace);
                                      // Sp = S rounded up to 64, pads +inf and 0
-  float *dq_acc;                     // [B, S, Hq, D] fp32 (workspace)
+  float *dq_acc;                     // [B, Hq, Sp, D] fp32 (workspace)
   __nv_bfloat16 *dk, *dv;            // [B, S, Hkv, D]
   const int32_t *ct_ptr, *ct_q;      // sparse: per key tile, (qb << 2 | key-block bits)
   const int32_t *mode;               // per batch, or nullptr
@@ -89,8 +95,10 @@ struct Params {
   const float *gscale;               // per batch output factor, or nullptr (1)
   int gscale_complement;             // factor = 1 - gscale[b]
   int accumulate_kv;                 // dK/dV: add into the existing output
+  float *dkv_acc;                    // [2, B, Hkv, nkt*128, D] fp32 for split tiles
   int32_t *status;
   int B, S, Sp, Hq, Hkv, G, nqb, nkt;
+  int cq_full, cq_sparse, cmax;      // query blocks per chunk (per mode), chunks per tile
   float scale, scale_log2;
 };
 
@@ -114,39 +122,58 @@ FA_DEV void st_shared_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint
                : "memory");
 }
 
-// Work item w -> (key tile, batch, KV head).  Items are numbered key tile
-// first, so the tiles with the most causal query blocks (kt = 0) come first.
+// Work item w -> (chunk c, key tile, batch, KV head).  A tile's query blocks
+// (a descending list) are cut into chunks of at most cq blocks, so no item is
+// much longer than the others (the sink tile of the sparse path attends every
+// query block); chunk 0 of every tile comes first, key tile first within a
+// chunk index.  A tile with more than one chunk is "split": its chunks add
+// fp32 partial dK/dV into dkv_acc, converted after the kernel.
 struct Item {
-  int kt, b, kvh, nq, ct0;
-  bool sparse;
+  int kt, b, kvh, nq, ct0, q0, nq_total;
+  bool sparse, split;
 };
+FA_DEV int tile_nq(const Params &p, int kt, bool sparse, int &ct0) {
+  if (sparse) {
+    ct0 = p.ct_ptr[kt];
+    return p.ct_ptr[kt + 1] - ct0;
+  }
+  ct0 = 0;
+  return p.nqb - 2 * kt;            // query blocks 2kt .. nqb-1
+}
+FA_DEV bool batch_sparse(const Params &p, int b) {
+  const int mode = p.mode ? p.mode[b] : p.mode_default;
+  return (mode == FA_MODE_SPARSE) && p.ct_ptr != nullptr;
+}
 FA_DEV Item item_of(const Params &p, int w) {
   Item it;
-  const int bh = p.B * p.Hkv;
-  it.kt = w / bh;
-  const int rem = w % bh;
+  const int bh = p.B * p.Hkv, per_c = p.nkt * bh;
+  const int c = w / per_c;
+  int rem = w % per_c;
+  it.kt = rem / bh;
+  rem %= bh;
   it.b = rem / p.Hkv;
   it.kvh = rem % p.Hkv;
-  const int mode = p.mode ? p.mode[it.b] : p.mode_default;
-  it.sparse = (mode == FA_MODE_SPARSE) && p.ct_ptr != nullptr;
-  if (it.sparse) {
-    it.ct0 = p.ct_ptr[it.kt];
-    it.nq = p.ct_ptr[it.kt + 1] - it.ct0;
-  } else {
-    it.ct0 = 0;
-    it.nq = p.nqb - 2 * it.kt;      // query blocks 2kt .. nqb-1
-  }
+  it.sparse = batch_sparse(p, it.b);
+  it.nq_total = tile_nq(p, it.kt, it.sparse, it.ct0);
+  const int cq = it.sparse ? p.cq_sparse : p.cq_full;
+  it.q0 = c * cq;
+  it.nq = max(0, min(cq, it.nq_total - it.q0));
+  it.split = it.nq_total > cq;
   return it;
 }
 // Query block of the item's qi-th step and which of the tile's two key
-// blocks it keeps (bit 0: keys 0-63 of the tile, bit 1: keys 64-127).
+// blocks it keeps (bit 0: keys 0-63 of the tile, bit 1: keys 64-127).  Steps
+// walk the query blocks from the last one down, so the CTAs running at the
+// same time sweep the same query rows together and their dQ reductions and
+// Q/dO reads stay in L2.
 FA_DEV void q_block(const Params &p, const Item &it, int qi, int &qb, uint32_t &bits) {
+  const int pos = it.q0 + qi;       // position in the tile's descending list
   if (it.sparse) {
-    const int v = p.ct_q[it.ct0 + qi];
+    const int v = p.ct_q[it.ct0 + it.nq_total - 1 - pos];
     qb = v >> 2;
     bits = static_cast<uint32_t>(v) & 3u;
   } else {
-    qb = 2 * it.kt + qi;
+    qb = p.nqb - 1 - pos;
     bits = 3u;
   }
 }
@@ -367,6 +394,17 @@ FA_DEV void store_grad_row(__nv_bfloat16 *dst, const uint32_t (&r)[128], float f
   }
 }
 
+// One row of a split tile's dK or dV: fp32 partial sums added into the
+// accumulator with 16-byte vector reductions.
+FA_DEV void add_grad_row(float *dst, const uint32_t (&r)[128], float f) {
+  float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+  for (int c = 0; c < HD / 4; ++c)
+    atomicAdd(d4 + c, make_float4(__uint_as_float(r[4 * c]) * f, __uint_as_float(r[4 * c + 1]) * f,
+                                  __uint_as_float(r[4 * c + 2]) * f,
+                                  __uint_as_float(r[4 * c + 3]) * f));
+}
+
 // ---------------------------------------- elementwise (one key row per thread)
 FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   const int r = threadIdx.x;                         // key row within the tile
@@ -384,7 +422,7 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     __nv_bfloat16 *dk_row = p.dk + ((static_cast<size_t>(it.b) * p.S + key) * p.Hkv + it.kvh) * HD;
     __nv_bfloat16 *dv_row = p.dv + ((static_cast<size_t>(it.b) * p.S + key) * p.Hkv + it.kvh) * HD;
     if (n_it <= 0) {          // no query attends this tile: zero gradients
-      if (key < p.S && !p.accumulate_kv) {
+      if (it.nq_total == 0 && key < p.S && !p.accumulate_kv) {
         uint4 *a = reinterpret_cast<uint4 *>(dk_row), *b = reinterpret_cast<uint4 *>(dv_row);
         for (int i = 0; i < HD / 8; ++i) a[i] = b[i] = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -482,15 +520,23 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     if (!warp_wait(sh.bar(Smem::ACC_FULL), static_cast<uint32_t>(acc_n) & 1u, sh, p)) break;
     tc_fence_after_sync();
     const bool store = key < p.S && !ld_shared_s32(sh.abort_flag());
+    const size_t acc_row = ((static_cast<size_t>(it.b) * p.Hkv + it.kvh) * p.nkt * BK + key) * HD;
+    const size_t acc_half = static_cast<size_t>(p.B) * p.Hkv * p.nkt * BK * HD;
     {
       uint32_t a[128];
       tmem_ld128_wait(tmem + lane + 256u, a);
-      if (store) store_grad_row(dv_row, a, f, p.accumulate_kv != 0);
+      if (store) {
+        if (it.split) add_grad_row(p.dkv_acc + acc_half + acc_row, a, f);
+        else store_grad_row(dv_row, a, f, p.accumulate_kv != 0);
+      }
     }
     {
       uint32_t a[128];
       tmem_ld128_wait(tmem + lane + 384u, a);
-      if (store) store_grad_row(dk_row, a, f * p.scale, p.accumulate_kv != 0);
+      if (store) {
+        if (it.split) add_grad_row(p.dkv_acc + acc_row, a, f * p.scale);
+        else store_grad_row(dk_row, a, f * p.scale, p.accumulate_kv != 0);
+      }
     }
     tc_fence_before_sync();
     mbar_arrive_a(sh.bar(Smem::ACC_FREE));
@@ -499,13 +545,20 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
 }
 
 // ------------------------------------------- dQ readout (one dim per thread)
-FA_DEV void run_dq(const Smem &sh, uint32_t tmem, const Params &p, int total) {
-  const int d = threadIdx.x - 128;
-  const uint32_t lane = (((static_cast<uint32_t>(threadIdx.x) >> 5) & 3u) * 32u) << 16;
+// Warp w (of 4) holds dims 32w .. 32w+31 of the step's 64 x 128 dQ tile: it
+// writes them into its own 64 x 32 staging box and one lane issues a TMA
+// reduce-add into the accumulator [B, Hq, Sp, 128]; before the next step
+// overwrites the box, the warp waits until that reduce has read it.
+FA_DEV void run_dq(const Smem &sh, uint32_t tmem, const CUtensorMap *tmA, const Params &p,
+                   int total) {
+  const int wq = (threadIdx.x >> 5) & 3, lane_id = threadIdx.x & 31;
+  const uint32_t lane = (static_cast<uint32_t>(wq) * 32u) << 16;
+  const uint32_t stg = sh.stg(wq) + 4u * static_cast<uint32_t>(lane_id);
   int n = 0;
-  for (int k = 0;; ++k) {
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
     const int w = item_index(k, total);
-    if (w < 0) return;
+    if (w < 0) break;
     const Item it = item_of(p, w);
     const int n_it = it.nq * p.G;
     const float f = out_factor(p, it.b);
@@ -515,7 +568,10 @@ FA_DEV void run_dq(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       q_block(p, it, i / p.G, qb, bits);
       const int h = it.kvh * p.G + i % p.G;
       const int u = n & 1;
-      if (!warp_wait(sh.bar(Smem::DQ_FULL0 + u), static_cast<uint32_t>(n >> 1) & 1u, sh, p)) return;
+      if (!warp_wait(sh.bar(Smem::DQ_FULL0 + u), static_cast<uint32_t>(n >> 1) & 1u, sh, p)) {
+        ok = false;
+        break;
+      }
       tc_fence_after_sync();
       uint32_t a[32], b[32];
       tmem_ld32(tmem + lane + 128u + 64u * u, a);
@@ -524,32 +580,30 @@ FA_DEV void run_dq(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       tmem_ld_wait(b);
       tc_fence_before_sync();
       mbar_arrive_a(sh.bar(Smem::DQ_FREE0 + u));
-      float *dst = p.dq_acc + (static_cast<size_t>(it.b) * p.S + static_cast<size_t>(qb) * BQ) *
-                                  p.Hq * HD +
-                   static_cast<size_t>(h) * HD + d;
-      const size_t rs = static_cast<size_t>(p.Hq) * HD;
-      const int valid = p.S - qb * BQ;               // rows past the end are padding
-      if (valid >= BQ) {
+      bulk_wait_read0();          // the previous reduce has read the staging box
+      __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          atomicAdd(dst + j * rs, __uint_as_float(a[j]) * f);
-          atomicAdd(dst + (32 + j) * rs, __uint_as_float(b[j]) * f);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j < valid) atomicAdd(dst + j * rs, __uint_as_float(a[j]) * f);
-          if (32 + j < valid) atomicAdd(dst + (32 + j) * rs, __uint_as_float(b[j]) * f);
-        }
+      for (int j = 0; j < 32; ++j) {
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + 128u * j),
+                     "f"(__uint_as_float(a[j]) * f)
+                     : "memory");
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + 128u * (32 + j)),
+                     "f"(__uint_as_float(b[j]) * f)
+                     : "memory");
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int row = (it.b * p.Hq + h) * p.Sp + qb * BQ;
+      tma_reduce_add_2d_w(tmA, sh.stg(wq), 32 * wq, row);
     }
   }
+  bulk_wait_all0();               // every reduce of this warp has completed
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const Params p, int total_items) {
+               const __grid_constant__ CUtensorMap tmA, const Params p, int total_items) {
   extern __shared__ uint8_t smem_raw[];
   const Smem sh = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -576,6 +630,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmO);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmA);
   }
   if (warp == WARP_MMA) {
     tmem_alloc_a(sh.tmem_slot(), TMEM_COLS);
@@ -588,7 +643,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp < 4) {
     run_ew(sh, tmem, p, total_items);
   } else if (warp < 8) {
-    run_dq(sh, tmem, p, total_items);
+    run_dq(sh, tmem, &tmA, p, total_items);
   } else if (warp == WARP_PRODUCER) {
     run_producer(sh, &tmQ, &tmO, &tmK, &tmV, p, total_items);
   } else {
@@ -620,6 +675,9 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16 *o,
         dvec[(b * Hq + h) * Sp + t] = 0.f;
         lse2[(b * Hq + h) * Sp + t] = INFINITY;
       }
+      if (zero_acc)
+        reinterpret_cast<float4 *>(dq_acc + ((b * Hq + h) * Sp + t) * HD)[lane] =
+            make_float4(0.f, 0.f, 0.f, 0.f);
       return;
     }
   }
@@ -634,7 +692,8 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16 *o,
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (zero_acc)
-    reinterpret_cast<float4 *>(dq_acc + row * HD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4 *>(dq_acc + ((b_ * Hq + h_) * Sp + t_) * HD)[lane] =
+        make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane == 0) {
     dvec[(b_ * Hq + h_) * Sp + t_] = s;
     lse2[(b_ * Hq + h_) * Sp + t_] = lse[(b_ * Hq + h_) * S + t_] * kLog2e;
@@ -704,30 +763,67 @@ __global__ void __launch_bounds__(1024) csc_kernel(const int32_t *row_ptr, const
 
 // dQ = scale * accumulator, plus (optionally) the router's pooling gradient
 // dx / (n_head + n_tail) on the first n_head and last n_tail tokens; bf16.
+// The accumulator is [B, Hq, Sp, D]; dQ is [B, S, Hq, D].
 __global__ void __launch_bounds__(256) convert_kernel(const float *acc, __nv_bfloat16 *dq, int B,
-                                                      int S, int Hq, float scale,
+                                                      int S, int Sp, int Hq, float scale,
                                                       const float *pool_dx, int n_head,
                                                       int n_tail) {
   const long long n8 = static_cast<long long>(B) * S * Hq * HD / 8;
   const float inv_n = 1.0f / static_cast<float>(n_head + n_tail > 0 ? n_head + n_tail : 1);
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const float4 a = reinterpret_cast<const float4 *>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4 *>(acc)[2 * i + 1];
+    const long long e = i * 8;                   // element index in [B, S, Hq, D]
+    const long long row = e / HD, dd = e % HD;
+    const long long h = row % Hq, bt = row / Hq, t = bt % S, bb = bt / S;
+    const float *src = acc + ((bb * Hq + h) * Sp + t) * HD + dd;
+    const float4 a = reinterpret_cast<const float4 *>(src)[0];
+    const float4 b = reinterpret_cast<const float4 *>(src)[1];
     float x[8] = {a.x * scale, a.y * scale, a.z * scale, a.w * scale,
                   b.x * scale, b.y * scale, b.z * scale, b.w * scale};
-    if (pool_dx) {
-      const long long e = i * 8;                 // element index in [B, S, Hq, D]
-      const long long row = e / HD, dd = e % HD;
-      const long long h = row % Hq, bt = row / Hq, t = bt % S, bb = bt / S;
-      if (t < n_head || t >= S - n_tail) {
-        const float *src = pool_dx + (bb * Hq + h) * HD + dd;
+    if (pool_dx && (t < n_head || t >= S - n_tail)) {
+      const float *px = pool_dx + (bb * Hq + h) * HD + dd;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] += src[k] * inv_n;
-      }
+      for (int k = 0; k < 8; ++k) x[k] += px[k] * inv_n;
     }
     reinterpret_cast<uint4 *>(dq)[i] = pack8(x);
   }
+}
+
+// dK / dV of split tiles: bf16 of the fp32 accumulator (added to the
+// existing output when accumulating).  One warp per (batch, key, KV head).
+__global__ void __launch_bounds__(256) dkv_convert_kernel(const Params p) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(p.B) * p.S * p.Hkv) return;
+  const int kvh = static_cast<int>(row % p.Hkv);
+  const long long bt = row / p.Hkv;
+  const int key = static_cast<int>(bt % p.S), b = static_cast<int>(bt / p.S);
+  int ct0;
+  const bool sparse = batch_sparse(p, b);
+  if (tile_nq(p, key / BK, sparse, ct0) <= (sparse ? p.cq_sparse : p.cq_full)) return;
+  const size_t acc_row = ((static_cast<size_t>(b) * p.Hkv + kvh) * p.nkt * BK + key) * HD;
+  const size_t acc_half = static_cast<size_t>(p.B) * p.Hkv * p.nkt * BK * HD;
+  __nv_bfloat16 *outs[2] = {p.dk, p.dv};
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const float4 a = reinterpret_cast<const float4 *>(p.dkv_acc + t * acc_half + acc_row)[lane];
+    float x[4] = {a.x, a.y, a.z, a.w};
+    uint2 *dst = reinterpret_cast<uint2 *>(outs[t] + static_cast<size_t>(row) * HD) + lane;
+    if (p.accumulate_kv) {
+      const uint2 o = *dst;
+      x[0] += __uint_as_float(o.x << 16);
+      x[1] += __uint_as_float(o.x & 0xffff0000u);
+      x[2] += __uint_as_float(o.y << 16);
+      x[3] += __uint_as_float(o.y & 0xffff0000u);
+    }
+    *dst = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+  }
+}
+
+__global__ void __launch_bounds__(256) zero4_kernel(float4 *x, long long n4) {
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * 256)
+    x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dr[b] += sign * sum over (head, token) of D (the padded entries are 0):
@@ -769,11 +865,11 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // (padded to Sp = 64 * nqb per (batch, head)), transposed block pattern.
 struct Plan {
   int nqb, nkt, Sp;
-  float *acc, *dvec, *lse2;
+  float *acc, *dvec, *lse2, *dkv_acc;
   int32_t *ct_ptr, *ct_q;
   size_t bytes;
 };
-Plan make_plan(int B, int S, int Hq, void *workspace) {
+Plan make_plan(int B, int S, int Hq, int Hkv, void *workspace) {
   Plan pl;
   pl.nqb = (S + 63) / 64;
   pl.nkt = (pl.nqb + 1) / 2;
@@ -785,12 +881,14 @@ Plan make_plan(int B, int S, int Hq, void *workspace) {
     off += align256(bytes);
     return p;
   };
-  pl.acc = reinterpret_cast<float *>(take(static_cast<size_t>(B) * S * Hq * backward::HD * 4));
+  pl.acc = reinterpret_cast<float *>(take(static_cast<size_t>(B) * Hq * pl.Sp * backward::HD * 4));
   pl.dvec = reinterpret_cast<float *>(take(static_cast<size_t>(B) * Hq * pl.Sp * 4));
   pl.lse2 = reinterpret_cast<float *>(take(static_cast<size_t>(B) * Hq * pl.Sp * 4));
   pl.ct_ptr = reinterpret_cast<int32_t *>(take((static_cast<size_t>(pl.nkt) + 1) * 4));
   pl.ct_q = reinterpret_cast<int32_t *>(
       take(static_cast<size_t>(pl.nkt) * static_cast<size_t>(pl.nqb) * 4));
+  pl.dkv_acc = reinterpret_cast<float *>(
+      take(2 * static_cast<size_t>(B) * Hkv * pl.nkt * backward::BK * backward::HD * 4));
   pl.bytes = off;
   return pl;
 }
@@ -831,11 +929,12 @@ int run_csc(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
 
 int run_main(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
   using namespace backward;
-  CUtensorMap tmQ, tmO, tmK, tmV;
+  CUtensorMap tmQ, tmO, tmK, tmV, tmA;
   if (make_tmap_bhsd(&tmQ, a.q, a.B, a.S, a.Hq, 64, BQ) != 0 ||
       make_tmap_bhsd(&tmO, a.dout, a.B, a.S, a.Hq, 64, BQ) != 0 ||
       make_tmap_bhsd(&tmK, a.k, a.B, a.S, a.Hkv, 64, BK) != 0 ||
-      make_tmap_bhsd(&tmV, a.v, a.B, a.S, a.Hkv, 64, BK) != 0)
+      make_tmap_bhsd(&tmV, a.v, a.B, a.S, a.Hkv, 64, BK) != 0 ||
+      make_tmap_rows_f32(&tmA, pl.acc, static_cast<long long>(a.B) * a.Hq * pl.Sp, 32, BQ) != 0)
     return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
       cudaSuccess)
@@ -865,14 +964,44 @@ int run_main(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
   p.nkt = pl.nkt;
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
-  const long long total = static_cast<long long>(pl.nkt) * a.B * a.Hkv;
-  if (total <= 0 || total > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   int sms = 148;
   if (int rc = sm_count(&sms)) return rc;
+  // Chunks of at most 32 query blocks (a sixteenth of the sequence's blocks
+  // for long sequences).  The sparse path always cuts (its sink tile attends
+  // every query block).  The full path keeps whole tiles when its longest
+  // tile (nqb blocks) is within one SM's share of all the tiles' blocks and
+  // the dQ accumulator is small; with a large accumulator, chunk-major order
+  // keeps the CTAs on the same query rows (L2 hits for the reductions).
+  const int cq = pl.nqb / 16 > 32 ? pl.nqb / 16 : 32;
+  const long long full_blocks =
+      static_cast<long long>(a.B) * a.Hkv * (static_cast<long long>(pl.nkt) * pl.nqb -
+                                             static_cast<long long>(pl.nkt) * (pl.nkt - 1));
+  const long long acc_bytes = static_cast<long long>(a.B) * a.Hq * pl.Sp * HD * 4;
+  const bool balanced = static_cast<long long>(pl.nqb) * sms <= full_blocks;
+  p.cq_full = (balanced && acc_bytes <= (256ll << 20)) ? pl.nqb : cq;
+  p.cq_sparse = cq;
+  const bool any_sparse = sparse && (a.mode_dev != nullptr || a.mode_default == FA_MODE_SPARSE);
+  const int cq_min = any_sparse ? (p.cq_full < cq ? p.cq_full : cq) : p.cq_full;
+  p.cmax = (pl.nqb + cq_min - 1) / cq_min;
+  p.dkv_acc = pl.dkv_acc;
+  const long long total = static_cast<long long>(p.cmax) * pl.nkt * a.B * a.Hkv;
+  if (total <= 0 || total > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  const long long n4 = 2ll * a.B * a.Hkv * pl.nkt * BK * HD / 4;
+  if (p.cmax > 1) {
+    zero4_kernel<<<static_cast<unsigned>(4 * sms), 256, 0, stream>>>(
+        reinterpret_cast<float4 *>(pl.dkv_acc), n4);
+    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
   const int ctas = static_cast<int>(total < sms ? total : sms);
-  bwd_kernel<<<ctas, NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmO, tmK, tmV, p,
+  bwd_kernel<<<ctas, NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmO, tmK, tmV, tmA, p,
                                                         static_cast<int>(total));
-  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (p.cmax > 1) {
+    const long long rows = static_cast<long long>(a.B) * a.S * a.Hkv;
+    dkv_convert_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
 }
 
 int run_convert(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
@@ -882,19 +1011,19 @@ int run_convert(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
   const long long n8 = static_cast<long long>(a.B) * a.S * a.Hq * HD / 8;
   const long long blocks = (n8 + 255) / 256;
   convert_kernel<<<static_cast<unsigned>(blocks < 4 * sms ? blocks : 4 * sms), 256, 0, stream>>>(
-      pl.acc, reinterpret_cast<__nv_bfloat16 *>(a.dq), a.B, a.S, a.Hq, a.scale, a.pool_dx,
+      pl.acc, reinterpret_cast<__nv_bfloat16 *>(a.dq), a.B, a.S, pl.Sp, a.Hq, a.scale, a.pool_dx,
       a.n_head, a.n_tail);
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // namespace
 
-size_t backward_workspace_bytes(int B, int S, int Hq) {
-  return make_plan(B, S, Hq, nullptr).bytes;
+size_t backward_workspace_bytes(int B, int S, int Hq, int Hkv) {
+  return make_plan(B, S, Hq, Hkv, nullptr).bytes;
 }
 
 int launch_backward(const BackwardLaunch &a, cudaStream_t stream) {
-  const Plan pl = make_plan(a.B, a.S, a.Hq, a.workspace);
+  const Plan pl = make_plan(a.B, a.S, a.Hq, a.Hkv, a.workspace);
   if (int rc = run_prep(a, pl, stream)) return rc;
   if (may_be_sparse(a))
     if (int rc = run_csc(a, pl, stream)) return rc;
@@ -914,9 +1043,9 @@ struct SoftPlan {
   float *x, *logits, *r, *dr, *dlogits, *da, *dx;
   size_t bytes;
 };
-SoftPlan make_soft_plan(int B, int S, int Hq, int hidden, void *workspace) {
+SoftPlan make_soft_plan(int B, int S, int Hq, int Hkv, int hidden, void *workspace) {
   SoftPlan sp;
-  sp.att = make_plan(B, S, Hq, workspace);
+  sp.att = make_plan(B, S, Hq, Hkv, workspace);
   uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
   size_t off = sp.att.bytes;
   auto take = [&](size_t bytes) {
@@ -938,13 +1067,13 @@ SoftPlan make_soft_plan(int B, int S, int Hq, int hidden, void *workspace) {
 }
 }  // namespace
 
-size_t soft_backward_workspace_bytes(int B, int S, int Hq, int hidden) {
-  return make_soft_plan(B, S, Hq, hidden, nullptr).bytes;
+size_t soft_backward_workspace_bytes(int B, int S, int Hq, int Hkv, int hidden) {
+  return make_soft_plan(B, S, Hq, Hkv, hidden, nullptr).bytes;
 }
 
 int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream) {
   using namespace backward;
-  const SoftPlan sp = make_soft_plan(a.B, a.S, a.Hq, a.hidden, a.workspace);
+  const SoftPlan sp = make_soft_plan(a.B, a.S, a.Hq, a.Hkv, a.hidden, a.workspace);
   constexpr int kHead = 100, kTail = 100;
   // Router forward again: pooling slices, ReLU outputs, logits, r.
   RouterLaunch rl{a.q, a.B, a.S, a.Hq, kHead, kTail, a.w1, a.b1, a.w2, a.b2, a.hidden,

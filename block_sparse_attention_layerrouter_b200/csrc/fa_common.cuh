@@ -307,6 +307,23 @@ FA_DEV void bulk_load_w(uint32_t dst, const void *src, uint32_t bytes, uint32_t 
       : "memory");
 }
 
+// TMA reduce-add of a shared-memory box into a 2-D global tensor (bulk
+// group completion); one elected lane issues.  Coordinates are >= 0 and the
+// innermost one is 16-byte aligned.
+FA_DEV void tma_reduce_add_2d_w(const CUtensorMap *map, uint32_t src, int c0, int c1) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];\n\t"
+      "@e cp.async.bulk.commit_group;\n\t}\n" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(src)
+      : "memory");
+}
+// Wait until this thread's committed bulk groups have finished reading their
+// shared-memory sources (all but `n` most recent).
+FA_DEV void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+FA_DEV void bulk_wait_all0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Shared-memory matrix descriptor (sm_100 format: start >> 4 in bits 0-13,
 // leading byte offset >> 4 in 16-29, stride byte offset >> 4 in 32-45,
 // version 1 in 46-47, layout type in 61-63 with 2 = 128-byte swizzle).

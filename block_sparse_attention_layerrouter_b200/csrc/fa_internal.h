@@ -14,6 +14,10 @@ namespace fa {
 int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols,
                    int box_rows);
 
+// 2-D TMA map over an fp32 tensor [rows, 128] (row-major), boxes of
+// box_cols x box_rows, no swizzle.  Returns 0 on success.
+int make_tmap_rows_f32(CUtensorMap *map, void *base, long long rows, int box_cols, int box_rows);
+
 struct PrefillLaunch {
   const void *q, *k, *v;
   void *o;
@@ -88,7 +92,7 @@ struct BackwardLaunch {
   const float *pool_dx = nullptr;    // [B, Hq*D] router pooling gradient, or nullptr
   int n_head = 0, n_tail = 0;
 };
-size_t backward_workspace_bytes(int B, int S, int Hq);
+size_t backward_workspace_bytes(int B, int S, int Hq, int Hkv);
 int launch_backward(const BackwardLaunch &a, cudaStream_t stream);
 
 // Router backward (soft routing): gradients of W1, b1, W2, b2 and of the
@@ -125,7 +129,7 @@ struct SoftBackwardLaunch {
   void *workspace;
   int32_t *status;
 };
-size_t soft_backward_workspace_bytes(int B, int S, int Hq, int hidden);
+size_t soft_backward_workspace_bytes(int B, int S, int Hq, int Hkv, int hidden);
 int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream);
 
 long long index_nnz(int nrows, int sb, int wb);

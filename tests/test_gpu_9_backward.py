@@ -48,7 +48,8 @@ def _check_all(got, want, tag):
         assert_close_grad(to_f64(g), w, "%s %s" % (tag, name))
 
 
-@pytest.mark.parametrize("B,S,Hq,Hkv", [(2, 320, 8, 2), (1, 200, 2, 2), (1, 1024, 4, 1)])
+@pytest.mark.parametrize("B,S,Hq,Hkv", [(2, 320, 8, 2), (1, 200, 2, 2), (1, 1024, 4, 1),
+                                         (1, 2560, 2, 1)])
 def test_backward_full(B, S, Hq, Hkv):
     q, k, v, do, o, lse, _, _, status = _setup(B, S, Hq, Hkv, seed=601 + S)
     # Attention of the full path: recompute the forward into o/lse first.
@@ -61,7 +62,8 @@ def test_backward_full(B, S, Hq, Hkv):
 
 @pytest.mark.parametrize("B,S,Hq,Hkv,sink,window", [(2, 320, 8, 2, 64, 128),
                                                     (1, 1000, 4, 2, 128, 256),
-                                                    (1, 640, 2, 1, 0, 64)])
+                                                    (1, 640, 2, 1, 0, 64),
+                                                    (1, 2560, 2, 1, 128, 256)])
 def test_backward_sparse(B, S, Hq, Hkv, sink, window):
     c = capi.cfg(64, sink, window)
     q, k, v, do, o, lse, rp, ci, status = _setup(B, S, Hq, Hkv, seed=611 + S, cfg=c)
@@ -91,8 +93,10 @@ def test_backward_per_batch_modes_on_device():
 
 
 def test_backward_is_deterministic_in_dk_dv():
-    """dK/dV accumulate in one CTA's TMEM in a fixed order: repeat calls give
-    identical bits (dQ is summed with reductions in varying order)."""
+    """With no key tile split into chunks (S = 512: at most 32 query blocks
+    per tile), dK/dV accumulate in one CTA's TMEM in a fixed order: repeat
+    calls give identical bits (dQ is summed with reductions in varying
+    order)."""
     q, k, v, do, o, lse, _, _, status = _setup(1, 512, 4, 2, seed=631)
     capi.attn_prefill_full(q, k, v, o=o, lse=lse, status=status)
     a = capi.attn_prefill_backward(q, k, v, o, lse, do, status=status)
