@@ -678,6 +678,88 @@ def run_varlen(args, wl):
     return line
 
 
+# ------------------------------------------------------ training step
+def run_train(args, wl):
+    """One training step of a soft-routed layer: router logits and the soft
+    weight r, FULL and SPARSE attention with their LSE (forward), then
+    fa_soft_routed_layer_backward for an upstream gradient of the mixed
+    output (router weights, Q, K, V through both paths)."""
+    from block_sparse_attention_layerrouter_b200 import capi, inputs
+    ws, rank, dev = setup_device(args)
+    B, S, Hq, Hkv = wl.B, wl.S, wl.Hq, wl.Hkv
+    q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, wl.seed, device=dev)
+    dy = inputs.randn_bf16((B, S, Hq, 128), wl.seed + 400, device=dev)
+    w1, b1, w2, b2 = [t.to(dev) for t in inputs.router_weights(Hq * 128, wl.hidden, wl.seed)]
+    g = inputs.gumbel(B, wl.seed).to(dev)
+    c = capi.cfg(64, wl.sink, wl.window)
+    rp, ci = capi.blocksparse_index(S, c, device=dev)
+    o_f, o_s = torch.empty_like(q), torch.empty_like(q)
+    lse_f = torch.empty(B, Hq, S, device=dev)
+    lse_s = torch.empty(B, Hq, S, device=dev)
+    logits = torch.empty(B, 2, device=dev)
+    r = torch.empty(B, device=dev)
+    mode = torch.empty(B, dtype=torch.int32, device=dev)
+    rws = torch.empty(capi.router_workspace_size(B, Hq, 128, wl.hidden), dtype=torch.uint8,
+                      device=dev)
+    bws = torch.empty(int(capi.lib().fa_soft_routed_backward_workspace_size(B, S, Hq, Hkv, 128,
+                                                                             wl.hidden)),
+                      dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        capi.router_decide(q, w1, b1, w2, b2, logits=logits, mode=mode, workspace=rws)
+        capi.router_soft(logits, g, tau=1.0, r=r)
+        capi.attn_prefill_full(q, k, v, o=o_f, lse=lse_f, status=status)
+        capi.attn_prefill_blocksparse(q, k, v, rp, ci, o=o_s, lse=lse_s, status=status)
+        return capi.soft_routed_layer_backward(q, k, v, o_f, lse_f, o_s, lse_s, dy, w1, b1, w2, b2,
+                                               rp, ci, gumbel=g, tau=1.0, workspace=bws,
+                                               status=status)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    sync_all(ws)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    sync_all(ws)
+    sampler.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    if rank != 0:
+        return None
+    f_full = flops_full(wl)
+    f_sparse = 4.0 * 128 * Hq * B * csr_nnz(S, wl.sink, wl.window) * 4096
+    flops = 3.5 * (f_full + f_sparse)      # forward 1x, backward 2.5x of each path
+    bwd_full_ms = time_kernel_alone(lambda: capi.attn_prefill_backward(
+        q, k, v, o_f, lse_f, dy, mode=0))
+    _, peak_burst, peak_sust, peak_kind = measured_peaks()
+    value = ws * flops / (ms / args.steps * 1e-3) / 1e12
+    bwd_achieved = 2.5 * f_full / (bwd_full_ms * 1e-3) / 1e12
+    line = base_line(args, wl, ws, ms, "TFLOP/s", value)
+    line["config"] = {"workload": wl.name, "B": B, "S": S, "Hq": Hq, "Hkv": Hkv, "D": 128,
+                      "sink": wl.sink, "window": wl.window, "hidden": wl.hidden,
+                      "step": "router + r + FULL and SPARSE forward with LSE + soft-routed "
+                              "backward (router grads, dQ/dK/dV through both paths)",
+                      "flops": "forward 4*D*Hq*pairs per path (SPARSE: executed 64x64 "
+                               "blocks), backward 2.5x the forward",
+                      "l2": "Q/K/V/O/dy/accumulators 0.6 GB per step > L2"}
+    line["roofline"] = {"bound": "tensor", "kernel": "backward::bwd_kernel (FULL, alone)",
+                        "achieved": round(bwd_achieved, 2), "peak": peak_burst,
+                        "unit": "TFLOP/s", "frac": round(bwd_achieved / peak_burst, 4),
+                        "peak_kind": "%s bf16 burst" % peak_kind,
+                        "frac_of_sustained_peak": round(bwd_achieved / peak_sust, 4),
+                        "traffic": None, "algorithmic_flops_per_launch": 2.5 * f_full,
+                        "avg_launch_ms": round(bwd_full_ms, 4)}
+    line["e2e"] = None
+    line["gpu_launches"] = None
+    line["clocks"] = sampler.report()
+    return line
+
+
 # ------------------------------------------------------- one kernel alone
 def run_only(args, wl):
     """Runs a single kernel of the path `warmup + steps` times on the
@@ -798,6 +880,8 @@ def main():
         line = run_decode(args, wl)
     elif wl.varlen:
         line = run_varlen(args, wl)
+    elif wl.train:
+        line = run_train(args, wl)
     else:
         line = run_ours(args, wl)
     if line is not None:

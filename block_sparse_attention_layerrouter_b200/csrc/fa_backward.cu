@@ -11,7 +11,7 @@
 // Kernels:
 //   prep_kernel    D_t and log2(e) * lse_t per (batch, head, token); zeroes
 //                  the fp32 dQ accumulator.                      (HBM-bound)
-//   csc_kernel     for the sparse path: per 128-key tile, the 64-query
+//   csc_*_kernel   for the sparse path: per 128-key tile, the 64-query
 //                  blocks whose CSR rows keep one of its two key blocks.
 //   bwd_kernel     persistent, one CTA per SM; a work item is one 128-key
 //                  tile of one (batch, KV head).  It walks the 64-query
@@ -125,9 +125,10 @@ FA_DEV void st_shared_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint
 // Work item w -> (chunk c, key tile, batch, KV head).  A tile's query blocks
 // (a descending list) are cut into chunks of at most cq blocks, so no item is
 // much longer than the others (the sink tile of the sparse path attends every
-// query block); chunk 0 of every tile comes first, key tile first within a
-// chunk index.  A tile with more than one chunk is "split": its chunks add
-// fp32 partial dK/dV into dkv_acc, converted after the kernel.
+// query block); items are numbered chunk index first, key tile next, so the
+// CTAs running together work on the same (top) query rows of their lists.  A
+// tile with more than one chunk is "split": its chunks add fp32 partial dK/dV
+// into dkv_acc, converted after the kernel.
 struct Item {
   int kt, b, kvh, nq, ct0, q0, nq_total;
   bool sparse, split;
@@ -701,9 +702,11 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16 *o,
 }
 
 // Per 128-key tile kt: the query blocks qb >= 2kt whose CSR row keeps key
-// block 2kt (bit 0) or 2kt+1 (bit 1), ascending, as (qb << 2 | bits).  Rows
-// must be ascending and causal; a row that is not is reported (its entries
-// past the first bad one are ignored).  One CTA.
+// block 2kt (bit 0) or 2kt+1 (bit 1), ascending, as (qb << 2 | bits).  Three
+// passes: count per tile (one warp per tile, 32 rows at a time, each lane a
+// binary search of its row), an exclusive scan plus the row checks (rows
+// must be ascending and inside [0, qb]; a bad row is reported), and the fill
+// (the same search, lanes' hits placed in row order with a ballot).
 FA_DEV bool row_has(const int32_t *col, int lo, int hi, int c) {
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
@@ -713,11 +716,28 @@ FA_DEV bool row_has(const int32_t *col, int lo, int hi, int c) {
   }
   return false;
 }
-__global__ void __launch_bounds__(1024) csc_kernel(const int32_t *row_ptr, const int32_t *col_idx,
-                                                   int nqb, int nkt, int32_t *ct_ptr,
-                                                   int32_t *ct_q, int32_t *status) {
-  extern __shared__ int32_t cnt[];   // nkt + 1
-  // Row checks (ascending, inside [0, qb]).
+FA_DEV int csc_bits(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int qb, int kt) {
+  const int lo = row_ptr[qb], hi = row_ptr[qb + 1];
+  int b = row_has(col_idx, lo, hi, 2 * kt) ? 1 : 0;
+  if (2 * kt + 1 < nqb && row_has(col_idx, lo, hi, 2 * kt + 1)) b |= 2;
+  return b;
+}
+__global__ void __launch_bounds__(256) csc_count_kernel(const int32_t *row_ptr,
+                                                        const int32_t *col_idx, int nqb, int nkt,
+                                                        int32_t *cnt) {
+  const int kt = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (kt >= nkt) return;
+  int c = 0;
+  for (int q0 = 2 * kt; q0 < nqb; q0 += 32) {
+    const int qb = q0 + lane;
+    const bool hit = qb < nqb && csc_bits(row_ptr, col_idx, nqb, qb, kt) != 0;
+    c += __popc(__ballot_sync(0xffffffffu, hit));
+  }
+  if (lane == 0) cnt[kt] = c;
+}
+__global__ void __launch_bounds__(1024) csc_scan_kernel(const int32_t *row_ptr,
+                                                        const int32_t *col_idx, int nqb, int nkt,
+                                                        int32_t *ct_ptr, int32_t *status) {
   for (int qb = threadIdx.x; qb < nqb; qb += blockDim.x) {
     int prev = -1;
     for (int e = row_ptr[qb]; e < row_ptr[qb + 1]; ++e) {
@@ -729,35 +749,31 @@ __global__ void __launch_bounds__(1024) csc_kernel(const int32_t *row_ptr, const
       prev = c;
     }
   }
-  auto bits_of = [&](int qb, int kt) -> int {
-    const int lo = row_ptr[qb], hi = row_ptr[qb + 1];
-    int b = row_has(col_idx, lo, hi, 2 * kt) ? 1 : 0;
-    if (2 * kt + 1 < nqb && row_has(col_idx, lo, hi, 2 * kt + 1)) b |= 2;
-    return b;
-  };
-  for (int kt = threadIdx.x; kt < nkt; kt += blockDim.x) {
-    int c = 0;
-    for (int qb = 2 * kt; qb < nqb; ++qb) c += bits_of(qb, kt) ? 1 : 0;
-    cnt[kt] = c;
-  }
+  // ct_ptr holds the counts on entry; exclusive scan in place (one thread:
+  // nkt is at most a few thousand).
   __syncthreads();
   if (threadIdx.x == 0) {
     int run = 0;
     for (int kt = 0; kt < nkt; ++kt) {
-      const int c = cnt[kt];
-      cnt[kt] = run;
+      const int c = ct_ptr[kt];
       ct_ptr[kt] = run;
       run += c;
     }
     ct_ptr[nkt] = run;
   }
-  __syncthreads();
-  for (int kt = threadIdx.x; kt < nkt; kt += blockDim.x) {
-    int pos = cnt[kt];
-    for (int qb = 2 * kt; qb < nqb; ++qb) {
-      const int b = bits_of(qb, kt);
-      if (b) ct_q[pos++] = (qb << 2) | b;
-    }
+}
+__global__ void __launch_bounds__(256) csc_fill_kernel(const int32_t *row_ptr,
+                                                       const int32_t *col_idx, int nqb, int nkt,
+                                                       const int32_t *ct_ptr, int32_t *ct_q) {
+  const int kt = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (kt >= nkt) return;
+  int pos = ct_ptr[kt];
+  for (int q0 = 2 * kt; q0 < nqb; q0 += 32) {
+    const int qb = q0 + lane;
+    const int b = qb < nqb ? csc_bits(row_ptr, col_idx, nqb, qb, kt) : 0;
+    const uint32_t m = __ballot_sync(0xffffffffu, b != 0);
+    if (b) ct_q[pos + __popc(m & ((1u << lane) - 1u))] = (qb << 2) | b;
+    pos += __popc(m);
   }
 }
 
@@ -916,14 +932,14 @@ bool may_be_sparse(const BackwardLaunch &a) {
 
 int run_csc(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
   using namespace backward;
-  const size_t sm = (static_cast<size_t>(pl.nkt) + 1) * 4;
-  if (sm > 200 * 1024) return FA_ERR_UNSUPPORTED;
-  if (sm > 48 * 1024 &&
-      cudaFuncSetAttribute(csc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sm)) != cudaSuccess)
-    return FA_ERR_CUDA;
-  csc_kernel<<<1, 1024, sm, stream>>>(a.row_ptr, a.col_idx, pl.nqb, pl.nkt, pl.ct_ptr, pl.ct_q,
-                                      a.status);
+  const unsigned blocks = static_cast<unsigned>((pl.nkt + 7) / 8);
+  csc_count_kernel<<<blocks, 256, 0, stream>>>(a.row_ptr, a.col_idx, pl.nqb, pl.nkt, pl.ct_ptr);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  csc_scan_kernel<<<1, 1024, 0, stream>>>(a.row_ptr, a.col_idx, pl.nqb, pl.nkt, pl.ct_ptr,
+                                          a.status);
+  if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+  csc_fill_kernel<<<blocks, 256, 0, stream>>>(a.row_ptr, a.col_idx, pl.nqb, pl.nkt, pl.ct_ptr,
+                                              pl.ct_q);
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

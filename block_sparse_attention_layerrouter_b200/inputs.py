@@ -37,6 +37,7 @@ class Workload:
     hidden: int = 64           # router MLP hidden width
     decode_len: int = 0        # >0: decode workload with this cache length
     varlen: bool = False       # packed batch of B requests of seeded lengths <= S
+    train: bool = False        # soft-routed training step (forward + backward)
     seed: int = 1000
     notes: str = field(default="", compare=False)
 
@@ -65,6 +66,13 @@ WORKLOADS = {
     "serving-varlen-qwen3-4b": Workload("serving-varlen-qwen3-4b", B=8, S=32768, Hq=32, Hkv=8,
                                         window=1024, hidden=256, varlen=True, seed=1006,
                                         notes="packed variable-length batch, routed per request"),
+    # Training step of one soft-routed Qwen3-4B-shaped layer: router, both
+    # attention paths with their LSE, then the backward of the mixed output
+    # (router weights and Q/K/V gradients through both paths).
+    "train-soft-qwen3-4b-layer-s8192": Workload("train-soft-qwen3-4b-layer-s8192", B=1, S=8192,
+                                                Hq=32, Hkv=8, window=1024, hidden=256,
+                                                train=True, seed=1007,
+                                                notes="soft-routed layer, forward + backward"),
     # Profiling shape: the decode workload at a quarter of the context
     # (1 GiB of K/V, still far above the 126 MB L2).
     "decode-b8-l32768": Workload("decode-b8-l32768", B=8, S=1, Hq=32, Hkv=8, layers=2,
