@@ -464,6 +464,103 @@ def decode(q_bits, kc_bits, vc_bits, seqlens, scale, mode=MODE_FULL,
     return out, lse
 
 
+# ------------------------------------------------------- FP8 KV cache codec
+# OCP 8-bit floating point E4M3 (the "FN" variant): 1 sign bit, 4 exponent
+# bits with bias 7, 3 mantissa bits; no infinities; S.1111.111 is NaN; the
+# largest finite magnitude is 448 (S.1111.110).  The pages note that their
+# B200 kernel is BF16-only; an FP8 cache is the adjacent decode variant.
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Exact value of each E4M3 code (uint8) as fp64; NaN codes give NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    normal = sign * np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64))
+    sub = sign * np.ldexp(m / 8.0, -6)
+    val = np.where(e == 0, sub, normal)
+    return np.where((c & 0x7F) == 0x7F, np.nan, val)
+
+
+_E4M3_CODES = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+_E4M3_VALUES = e4m3_decode(_E4M3_CODES)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest E4M3 code to each finite value (ties to the even code, i.e.
+    mantissa bit 0 clear), saturating at +-448; -0 and +0 keep their sign.
+    Brute force over the 254 finite codes."""
+    x = np.asarray(x, dtype=np.float64)
+    flat = x.ravel()
+    out = np.empty(flat.size, dtype=np.uint8)
+    for i, v in enumerate(flat):
+        if not np.isfinite(v):
+            raise ValueError("e4m3_encode takes finite values")
+        v = min(max(v, -448.0), 448.0)
+        d = np.abs(_E4M3_VALUES - v)
+        best = np.flatnonzero(d == d.min())
+        cands = _E4M3_CODES[best]
+        if len(cands) > 1:           # a tie (or +-0): even mantissa, then the sign of v
+            even = cands[(cands & 1) == 0]
+            cands = even if len(even) else cands
+            if len(cands) > 1:
+                cands = cands[((cands & 0x80) != 0) == bool(np.signbit(v))]
+        out[i] = cands[0]
+    return out.reshape(x.shape)
+
+
+def kv_quantize(x_bits: np.ndarray, scale) -> np.ndarray:
+    """E4M3 codes of a bf16 tensor divided by a per-head scale, the quotient
+    rounded to fp32 first (IEEE division): code = RN_e4m3(fp32(x / s)).
+    x_bits [..., H, D] bf16 bits; scale [H] fp32."""
+    x = bf16_bits_to_f64(x_bits).astype(np.float32)
+    s = np.asarray(scale, dtype=np.float32)
+    q = (x / s[:, None]).astype(np.float32)
+    return e4m3_encode(q.astype(np.float64))
+
+
+def decode_values(q, k, v, seqlens, scale, mode=MODE_FULL, block=BLOCK, sink=SINK_TOKENS,
+                  window=2 * BLOCK):
+    """decode() on fp64 values instead of bf16 bits (for dequantized FP8
+    caches): q [B,Hq,D], k, v [B,Lmax,Hkv,D].  Same key rule, plain numpy."""
+    q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
+    B, Hq, D = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        L = int(seqlens[b])
+        if mode == MODE_SPARSE:
+            keep = np.zeros(L, bool)
+            for j in blocksparse_rows(L, block, sink, window)[-1]:
+                keep[j * block:min(L, (j + 1) * block)] = True
+        else:
+            keep = np.ones(L, bool)
+        for h in range(Hq):
+            s = (k[b, :L, h // G] @ q[b, h]) * scale
+            s = np.where(keep, s, -np.inf)
+            m = s.max()
+            p = np.exp(s - m)
+            out[b, h] = (p @ v[b, :L, h // G]) / p.sum()
+            lse[b, h] = m + np.log(p.sum())
+    return out, lse
+
+
+def paged_gather(pages: np.ndarray, block_table: np.ndarray, seqlens, page_size: int = BLOCK):
+    """The tokens of each sequence, in order, from a paged cache
+    pages [num_pages, page_size, H, D] and block_table [B, max_pages]
+    (token t of sequence b sits in page block_table[b, t // page_size] at slot
+    t % page_size).  Returns [B, Lmax, H, D] (zeros past each length)."""
+    B, max_pages = block_table.shape
+    Lmax = max_pages * page_size
+    out = np.zeros((B, Lmax) + pages.shape[2:], dtype=pages.dtype)
+    for b in range(B):
+        for t in range(int(seqlens[b])):
+            out[b, t] = pages[block_table[b, t // page_size], t % page_size]
+    return out
+
+
 # --------------------------------------------------------------- accounting
 def attended_pairs_full(S: int) -> int:
     """Causal (query, key) pairs of one head: S(S+1)/2."""
