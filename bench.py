@@ -486,8 +486,21 @@ def run_decode(args, wl):
     ws, rank, dev = setup_device(args)
     B, L, Hq, Hkv = wl.B, wl.decode_len, wl.Hq, wl.Hkv
     caches = []
+    max_pages = L // 64
+    bt = inputs.page_table(B, max_pages, wl.seed).to(dev) if wl.paged else None
+    ksc = inputs.fp8_scales(Hkv, wl.seed).to(dev) if wl.kv_fp8 else None
+    vsc = inputs.fp8_scales(Hkv, wl.seed + 1).to(dev) if wl.kv_fp8 else None
+    kv_dtype = capi.FA_KV_FP8_E4M3 if wl.kv_fp8 else capi.FA_KV_BF16
     for i in range(DECODE_CACHE_SETS):
+        if wl.kv_fp8:
+            shape = (B * max_pages, 64, Hkv, 128)
+            caches.append((inputs.fp8_codes(shape, wl.seed + 17 * i, device=dev),
+                           inputs.fp8_codes(shape, wl.seed + 17 * i + 5, device=dev)))
+            continue
         _, kc, vc = inputs.decode_inputs(B, L, Hq, Hkv, 128, wl.seed + 17 * i, device=dev)
+        if wl.paged:
+            kc = kc.view(B * max_pages, 64, Hkv, 128)
+            vc = vc.view(B * max_pages, 64, Hkv, 128)
         caches.append((kc, vc))
     qs = [inputs.randn_bf16((B, Hq, 128), wl.seed + 1000 + li, device=dev)
           for li in range(wl.layers)]
@@ -503,8 +516,12 @@ def run_decode(args, wl):
             kc, vc = caches[li % DECODE_CACHE_SETS]
             if ev is not None and li == 0:
                 ev[0].record()
-            capi.attn_decode(qs[li], kc, vc, sl, modes[li], c, o=outs[li], workspace=wsb,
-                             status=status)
+            if wl.paged:
+                capi.attn_decode_paged(qs[li], kc, vc, bt, sl, kv_dtype, ksc, vsc, modes[li], c,
+                                       o=outs[li], workspace=wsb, status=status)
+            else:
+                capi.attn_decode(qs[li], kc, vc, sl, modes[li], c, o=outs[li], workspace=wsb,
+                                 status=status)
             if ev is not None and li == 0:
                 ev[1].record()
 
@@ -524,8 +541,18 @@ def run_decode(args, wl):
     sampler.stop()
     ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
     full_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    sparse_ms = time_kernel_alone(lambda: capi.attn_decode(qs[1], *caches[1], sl, 1, c, o=outs[1],
-                                                           workspace=wsb))
+    if wl.paged:
+        sparse_ms = time_kernel_alone(lambda: capi.attn_decode_paged(
+            qs[1], *caches[1], bt, sl, kv_dtype, ksc, vsc, 1, c, o=outs[1], workspace=wsb))
+        # KV append of one token for all sequences, alone (positions L-9 ..).
+        sl_app = torch.full((B,), L - 9, dtype=torch.int32, device=dev)
+        kn = inputs.randn_bf16((B, Hkv, 128), wl.seed + 2, device=dev)
+        append_ms = time_kernel_alone(lambda: capi.kv_append_paged(
+            kn, kn, caches[0][0], caches[0][1], bt, sl_app, kv_dtype, ksc, vsc), reps=5)
+    else:
+        sparse_ms = time_kernel_alone(lambda: capi.attn_decode(qs[1], *caches[1], sl, 1, c,
+                                                               o=outs[1], workspace=wsb))
+        append_ms = None
     # e2e: the caches are device-resident state; per step the 32 layers'
     # query tokens go up from pinned host memory and their outputs come back.
     hq = [q.cpu().pin_memory() for q in qs]
@@ -552,7 +579,7 @@ def run_decode(args, wl):
     if rank != 0:
         return None
     hbm, _, _, peak_kind = measured_peaks()
-    kv_row = 2 * Hkv * 128 * 2                               # K and V bytes per token
+    kv_row = 2 * Hkv * 128 * (1 if wl.kv_fp8 else 2)         # K and V bytes per token
     qo = 2 * B * Hq * 128 * 2
     full_bytes = B * kv_row * decode_keys(L, 0, wl.sink, wl.window) + qo
     sparse_bytes = B * kv_row * decode_keys(L, 1, wl.sink, wl.window) + qo
@@ -562,8 +589,12 @@ def run_decode(args, wl):
     line["config"] = {"workload": wl.name, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv, "D": 128,
                       "layers": wl.layers, "split": "16 FULL + 16 SPARSE (alternating)",
                       "sink": wl.sink, "window": wl.window,
+                      "cache": ("paged (64-token pages, seeded random order), " if wl.paged
+                                else "contiguous, ") + ("E4M3 + per-head scales" if wl.kv_fp8
+                                                        else "bf16"),
                       "l2": "inputs larger than L2: %d cache sets of %.2f GB rotated" % (
-                          DECODE_CACHE_SETS, 2 * caches[0][0].numel() * 2 / 1e9)}
+                          DECODE_CACHE_SETS,
+                          2 * caches[0][0].numel() * caches[0][0].element_size() / 1e9)}
     achieved = full_bytes / (full_ms * 1e-3) / 1e9
     line["roofline"] = {"bound": "hbm", "kernel": "decode_kernel + combine (a FULL layer)",
                         "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
@@ -581,6 +612,8 @@ def run_decode(args, wl):
         "decode_sparse_gbs": round(sparse_bytes / (sparse_ms * 1e-3) / 1e9, 1),
         "all_full_step_ms_est": round(wl.layers * full_ms, 3),
         "hybrid_vs_all_full": round(wl.layers * full_ms / (ms / args.steps), 3)}
+    if append_ms is not None:
+        line["components"]["kv_append_ms"] = round(append_ms, 4)
     return line
 
 

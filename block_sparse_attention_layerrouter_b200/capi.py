@@ -79,6 +79,11 @@ _SIGNATURES = {
                                            _I, _F, _VP, _VP, _I, _VP, _VP, _VP, _F, _VP, _VP, _VP,
                                            _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
                                            _VP]),
+    "fa_kv_append_paged": (_I, [_VP, _VP, _VP, _VP, _I, _VP, _VP, _VP, _I, _I, _VP, _I, _I, _I,
+                                _VP, _VP]),
+    "fa_decode_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_attn_decode_paged": (_I, [_VP, _VP, _VP, _I, _VP, _VP, _VP, _I, _I, _VP, _I, _I, _I, _I,
+                                  _F, _I, _VP, SparseCfg, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "fa_hybrid_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_hybrid_layer": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
                              _VP, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
@@ -460,3 +465,57 @@ def soft_routed_layer_backward(q, k, v, o_full, lse_full, o_sparse, lse_sparse, 
         _ptr(status), _stream(dev))
     _check("fa_soft_routed_layer_backward", rc)
     return out
+
+
+# ----------------------------------------------------- paged / FP8 KV cache
+FA_KV_BF16 = 0
+FA_KV_FP8_E4M3 = 1
+
+
+def kv_append_paged(k_new, v_new, k_pages, v_pages, block_table, seqlens, kv_dtype=FA_KV_BF16,
+                    k_scale=None, v_scale=None, status=None):
+    """fa_kv_append_paged: writes the token at seqlens[b], then seqlens += 1
+    (in place, on the device)."""
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    B, Hkv, D = k_new.shape
+    num_pages = k_pages.shape[0]
+    rc = lib().fa_kv_append_paged(_ptr(k_new), _ptr(v_new), _ptr(k_pages), _ptr(v_pages),
+                                  int(kv_dtype), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
+                                  block_table.shape[1], num_pages, _ptr(seqlens), B, Hkv, D,
+                                  _ptr(status), _stream(k_new.device))
+    _check("fa_kv_append_paged", rc)
+
+
+def decode_paged_workspace_size(B, Hq, Hkv, max_pages, D=128) -> int:
+    return int(lib().fa_decode_paged_workspace_size(B, Hq, Hkv, max_pages, D))
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seqlens, kv_dtype=FA_KV_BF16,
+                      k_scale=None, v_scale=None, mode=FA_MODE_FULL, c: Optional[SparseCfg] = None,
+                      mode_dev=None, scale=None, o=None, lse=None, workspace=None, status=None):
+    """fa_attn_decode_paged: q bf16 [B,Hq,D]; pools [num_pages,64,Hkv,D]."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, D = q.shape
+    num_pages, page, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    if page != 64:
+        raise ValueError("pages hold 64 tokens")
+    max_pages = block_table.shape[1]
+    c = cfg() if c is None else c
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    o = torch.empty_like(q) if o is None else o
+    if workspace is None:
+        workspace = torch.empty(decode_paged_workspace_size(B, Hq, Hkv, max_pages, D),
+                                device=q.device, dtype=torch.uint8)
+    rc = lib().fa_attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), int(kv_dtype),
+                                    _ptr(k_scale), _ptr(v_scale), _ptr(block_table), max_pages,
+                                    num_pages, _ptr(seqlens), B, Hq, Hkv, D, scale, int(mode),
+                                    _ptr(mode_dev), c, _ptr(o), _ptr(lse), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _ptr(status),
+                                    _stream(q.device))
+    _check("fa_attn_decode_paged", rc)
+    return o

@@ -50,6 +50,22 @@ int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int 
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
+int make_tmap_bhsd_u8(CUtensorMap *map, const void *base, int B, int S, int H, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return -1;
+  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128,
+                                 static_cast<cuuint64_t>(S) * H * 128};
+  const cuuint32_t box[4] = {128, 1, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
 int make_tmap_rows_f32(CUtensorMap *map, void *base, long long rows, int box_cols,
                        int box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -210,6 +226,64 @@ FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
     return FA_ERR_WORKSPACE;
   DecodeLaunch a{q, kcache, vcache, seqlens, B, Lmax, Hq, Hkv, scale, mode, mode_dev,
                  cfg.sink, cfg.window, o, lse, workspace, dev_status};
+  return launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+FA_API int fa_kv_append_paged(const void *k_new, const void *v_new, void *k_pages,
+                              void *v_pages, int kv_dtype, const float *k_scale,
+                              const float *v_scale, const int32_t *block_table, int max_pages,
+                              int num_pages, int32_t *seqlens, int B, int Hkv, int D,
+                              int32_t *dev_status, void *stream) {
+  if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !seqlens)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pages) || !aligned16(v_pages))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || max_pages <= 0 || num_pages <= 0) return FA_ERR_INVALID_ARG;
+  if (D != kHeadDim) return FA_ERR_UNSUPPORTED;
+  if (kv_dtype != FA_KV_BF16 && kv_dtype != FA_KV_FP8_E4M3) return FA_ERR_INVALID_ARG;
+  if (kv_dtype == FA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return FA_ERR_INVALID_ARG;
+  KvAppendLaunch a{k_new, v_new, k_pages, v_pages, kv_dtype == FA_KV_FP8_E4M3 ? 1 : 0,
+                   k_scale, v_scale, block_table, max_pages, num_pages, seqlens, B, Hkv,
+                   dev_status};
+  return launch_kv_append(a, static_cast<cudaStream_t>(stream));
+}
+
+FA_API size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_pages, int D) {
+  if (max_pages <= 0 || max_pages > (1 << 24)) return 0;
+  return fa_decode_workspace_size(B, Hq, Hkv, 64 * max_pages, D);
+}
+
+FA_API int fa_attn_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                                int kv_dtype, const float *k_scale, const float *v_scale,
+                                const int32_t *block_table, int max_pages, int num_pages,
+                                const int32_t *seqlens, int B, int Hq, int Hkv, int D,
+                                float scale, int mode, const int32_t *mode_dev,
+                                fa_sparse_cfg cfg, void *o, float *lse, void *workspace,
+                                size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seqlens || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || max_pages <= 0 || num_pages <= 0 || max_pages > (1 << 24))
+    return FA_ERR_INVALID_ARG;
+  if (int rc = check_heads(Hq, Hkv, D)) return rc;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
+  if (mode != FA_MODE_FULL && mode != FA_MODE_SPARSE) return FA_ERR_INVALID_ARG;
+  if (kv_dtype != FA_KV_BF16 && kv_dtype != FA_KV_FP8_E4M3) return FA_ERR_INVALID_ARG;
+  if (kv_dtype == FA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (int rc = check_cfg(cfg)) return rc;
+  const int Lmax = 64 * max_pages;
+  if (!workspace || !aligned16(workspace) || ws_bytes < decode_workspace_bytes(B, Hq, Hkv, Lmax))
+    return FA_ERR_WORKSPACE;
+  DecodeLaunch a{q, k_pages, v_pages, seqlens, B, Lmax, Hq, Hkv, scale, mode, mode_dev,
+                 cfg.sink, cfg.window, o, lse, workspace, dev_status};
+  a.block_table = block_table;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  a.fp8 = kv_dtype == FA_KV_FP8_E4M3 ? 1 : 0;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   return launch_decode(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -9,30 +9,55 @@
 // Grid (split, kv head, batch).  A CTA owns one KV head (all G query heads
 // of its group share each K/V tile) and a contiguous share of the sequence's
 // 64-key tiles.  Thread 0 streams the tiles with 4-D TMA loads (128-byte
-// swizzle, 4 boxes of 64 keys x 64 dims per tile) into a 3-stage ring; all
-// threads compute from shared memory:
+// swizzle; bf16: 2 boxes of 64 keys x 64 dims per K or V tile, 3 stages;
+// fp8: 1 box of 64 keys x 128 dims, 6 stages) into a ring; all threads
+// compute from shared memory:
 //   QK^T   thread = (key, 1/PARTS of the head dim), dot products for the G
 //          heads, reduced across the PARTS lanes with shuffles;
 //   softmax one warp per query head: running max / sum in log2 units;
 //   PV     thread = (8 output dims, one of 16 key streams), G accumulators.
 // Each CTA writes its partial (max, sum, unnormalised output) per head; the
 // combine kernel merges the splits by log-sum-exp.
+//
+// Paged cache: with a block table, tile n of sequence b is page
+// block_table[b][n] of a pool [num_pages, 64, Hkv, 128] (one page = one
+// 64-token block, so the sparse mode skips whole pages).  FP8 cache: E4M3
+// codes with one dequantisation scale per KV head for K and for V; the K
+// scale is folded into the query, the V scale into the partial outputs.
 #include "fa_common.cuh"
 #include "fa_internal.h"
 
+#include <cuda_fp8.h>
+#include <climits>
 #include <math.h>
 
 namespace fa {
 namespace decode {
 
-constexpr int KT = 64;                         // keys per tile = one block
+constexpr int KT = 64;                         // keys per tile = one block = one page
 constexpr int HD = 128;
-constexpr int NSTAGE = 3;
 constexpr int BOX_BYTES = KT * 64 * 2;         // 64 keys x 64 dims bf16
-constexpr int STAGE_BYTES = 4 * BOX_BYTES;     // K (2 boxes) + V (2 boxes)
 constexpr int NT = 256;
-constexpr int SMEM_BYTES = 1024 + NSTAGE * STAGE_BYTES + 8 * NSTAGE + 16 +
-                           /* scores */ 8 * KT * 4 + /* probs */ KT * 8 * 4 + 8 * 4;
+constexpr int RING_BYTES = 3 * 4 * BOX_BYTES;  // 96 KB of K/V in flight per CTA
+constexpr int MAX_STAGES = 6;
+constexpr int PAGE_CACHE = 256;                // page ids of a CTA's tiles kept in smem
+constexpr int SMEM_BYTES = 1024 + RING_BYTES + 8 * MAX_STAGES + 16 +
+                           /* scores */ 8 * 2 * KT * 4 + /* probs */ 2 * KT * 8 * 4 + 8 * 4 +
+                           /* page ids */ PAGE_CACHE * 4;
+
+// Per KV type: blocks (pages) per iteration, bytes of one block of K or V,
+// ring stages.  FP8 takes two blocks (128 keys) per iteration: half the
+// bytes per key, so the per-iteration work (barriers, the softmax step) is
+// spread over twice the keys.
+template <bool FP8>
+struct KvT {
+  static constexpr int NB = FP8 ? 2 : 1;
+  static constexpr int TK = NB * KT;                  // keys per iteration
+  static constexpr int BLK = FP8 ? KT * HD : KT * HD * 2;
+  static constexpr int KBYTES = NB * BLK;             // K (or V) of one iteration
+  static constexpr int STAGE = 2 * KBYTES;
+  static constexpr int NST = RING_BYTES / STAGE;
+};
 
 struct Params {
   const __nv_bfloat16 *q;
@@ -44,6 +69,9 @@ struct Params {
   int B, Lmax, Hq, Hkv, nsplit;
   int mode_default, sink_blocks, win_blocks;
   float scale_log2;
+  const int32_t *block_table;   // [B, max_pages] or nullptr (contiguous cache)
+  int max_pages, num_pages;
+  const float *k_scale, *v_scale;   // [Hkv] (FP8 cache) or nullptr
 };
 
 // Tiles (64-key blocks) a sequence of length L attends, as a virtual list:
@@ -72,7 +100,6 @@ struct Cfg {
   static constexpr int PARTS = (G <= 4) ? 8 : 16;       // threads per key in QK^T
   static constexpr int DPT = HD / PARTS;                 // dims per thread
   static constexpr int KPP = NT / PARTS;                 // keys per pass
-  static constexpr int PASSES = KT / KPP;
   static constexpr int MIN_BLOCKS = (G <= 4) ? 2 : 1;
 };
 
@@ -101,20 +128,70 @@ FA_DEV uint32_t tile_offset(int key, int chunk16) {
   return static_cast<uint32_t>(box * BOX_BYTES + key * 128 + phys * 16);
 }
 
-template <int G>
+// The same for an FP8 tile (one 128-byte row per key): byte offset of the
+// 8 codes of dims [8*g8, 8*g8+8).
+FA_DEV uint32_t tile_offset_fp8(int key, int g8) {
+  const int phys = (g8 >> 1) ^ (key & 7);
+  return static_cast<uint32_t>(key * 128 + phys * 16 + (g8 & 1) * 8);
+}
+
+// Eight E4M3 codes (8 bytes) -> four packed fp32 pairs, exact.
+FA_DEV void fp8x8_to_f2(const uint2 &v, uint64_t (&f)[4]) {
+  const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * j)) & 0xffffu), __NV_E4M3);
+      const float2 fl = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+      f[2 * i + j] = f2_make(fl.x, fl.y);
+    }
+  }
+}
+
+// K or V of eight dims of one key (0 .. TK-1) from a stage's K or V part, as
+// four fp32 pairs.
+template <bool FP8>
+FA_DEV void load8(const uint8_t *tile, int key, int g8, uint64_t (&f)[4]) {
+  if constexpr (FP8) {
+    const uint8_t *blk = tile + (key >> 6) * KvT<true>::BLK;
+    fp8x8_to_f2(*reinterpret_cast<const uint2 *>(blk + tile_offset_fp8(key & 63, g8)), f);
+  } else {
+    bf16x8_to_f2(*reinterpret_cast<const uint4 *>(tile + tile_offset(key, g8)), f);
+  }
+}
+
+// Page id of block `blk` of sequence b; an id outside the pool is reported
+// and replaced by num_pages (a TMA load there reads zeros).
+__device__ __noinline__ int page_of(const int32_t *block_table, int max_pages, int num_pages,
+                                    int32_t *status, int b, int blk) {
+  int pg = block_table[static_cast<size_t>(b) * max_pages + blk];
+  if (pg < 0 || pg >= num_pages) {
+    report(status, FA_DEV_BAD_INDEX);
+    pg = num_pages;
+  }
+  return pg;
+}
+
+template <int G, bool FP8, bool PAGED>
 __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const Params p) {
   using C = Cfg<G>;
+  using T = KvT<FP8>;
+  constexpr int NSTAGE = T::NST, STAGE_BYTES = T::STAGE, TK = T::TK, NB = T::NB;
+  constexpr int PASSES = TK / C::KPP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *stages = base;
-  uint64_t *full = reinterpret_cast<uint64_t *>(base + NSTAGE * STAGE_BYTES);
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + RING_BYTES);
   volatile int *abort = reinterpret_cast<volatile int *>(full + NSTAGE);
-  float *s_sm = reinterpret_cast<float *>(base + NSTAGE * STAGE_BYTES + 8 * NSTAGE + 16);
-  float *p_sm = s_sm + 8 * KT;          // [KT][G]
-  float *alpha_sm = p_sm + KT * 8;      // [G]
+  float *s_sm = reinterpret_cast<float *>(base + RING_BYTES + 8 * NSTAGE + 16);
+  float *p_sm = s_sm + 8 * TK;          // [TK][G]
+  float *alpha_sm = p_sm + TK * 8;      // [G]
+  int *page_sm = reinterpret_cast<int *>(alpha_sm + 8);   // [PAGE_CACHE]
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -124,36 +201,66 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
   const int mode = p.mode ? p.mode[b] : p.mode_default;
   TileList tl;
   tl.init(L, mode == FA_MODE_SPARSE, p.sink_blocks, p.win_blocks);
-  const int per = (tl.count + p.nsplit - 1) / p.nsplit;
+  const int per = ((tl.count + p.nsplit - 1) / p.nsplit + NB - 1) / NB * NB;
   const int pos0 = min(tl.count, split * per);
   const int pos1 = min(tl.count, pos0 + per);
-  const int ntiles = pos1 - pos0;
+  const int nblocks = pos1 - pos0;
+  const int ntiles = (nblocks + NB - 1) / NB;      // iterations
 
   if (tid == 0) {
     for (int i = 0; i < NSTAGE; ++i) mbar_init(&full[i], 1);
     *abort = 0;
     fence_mbar_init();
   }
+  // Page ids of this CTA's tiles (paged cache), read once by all threads.
+  if constexpr (PAGED) {
+    for (int i = tid; i < nblocks && i < PAGE_CACHE; i += NT)
+      page_sm[i] = page_of(p.block_table, p.max_pages, p.num_pages, p.status, b,
+                           tl.block(pos0 + i));
+  }
   __syncthreads();
 
   int issued = 0;            // tiles whose copies thread 0 has started
-  auto issue = [&](int i) {  // tile i of this CTA into stage i % NSTAGE
+  auto issue = [&](int i) {  // iteration i of this CTA into stage i % NSTAGE
     const int st = i % NSTAGE;
-    const int key0 = tl.block(pos0 + i) * KT;
     uint8_t *dst = stages + st * STAGE_BYTES;
     mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
-    tma_load_4d(dst, &tmK, &full[st], 0, kvh, key0, b);
-    tma_load_4d(dst + BOX_BYTES, &tmK, &full[st], 64, kvh, key0, b);
-    tma_load_4d(dst + 2 * BOX_BYTES, &tmV, &full[st], 0, kvh, key0, b);
-    tma_load_4d(dst + 3 * BOX_BYTES, &tmV, &full[st], 64, kvh, key0, b);
+    if constexpr (FP8) {     // paged: NB pages; a missing last one reads zeros
+#pragma unroll
+      for (int h = 0; h < NB; ++h) {
+        const int j = NB * i + h;
+        int pg = p.num_pages;
+        if (j < nblocks)
+          pg = j < PAGE_CACHE ? page_sm[j]
+                              : page_of(p.block_table, p.max_pages, p.num_pages, p.status, b,
+                                        tl.block(pos0 + j));
+        tma_load_4d(dst + h * T::BLK, &tmK, &full[st], 0, kvh, 0, pg);
+        tma_load_4d(dst + T::KBYTES + h * T::BLK, &tmV, &full[st], 0, kvh, 0, pg);
+      }
+    } else {
+      int tok = tl.block(pos0 + i) * KT, bidx = b;
+      if constexpr (PAGED) {
+        bidx = i < PAGE_CACHE ? page_sm[i]
+                              : page_of(p.block_table, p.max_pages, p.num_pages, p.status, b,
+                                        tl.block(pos0 + i));
+        tok = 0;
+      }
+      tma_load_4d(dst, &tmK, &full[st], 0, kvh, tok, bidx);
+      tma_load_4d(dst + BOX_BYTES, &tmK, &full[st], 64, kvh, tok, bidx);
+      tma_load_4d(dst + 2 * BOX_BYTES, &tmV, &full[st], 0, kvh, tok, bidx);
+      tma_load_4d(dst + 3 * BOX_BYTES, &tmV, &full[st], 64, kvh, tok, bidx);
+    }
     issued = i + 1;
   };
   if (tid == 0) {
     for (int i = 0; i < NSTAGE && i < ntiles; ++i) issue(i);
   }
 
-  // Query slice of this thread for QK^T, pre-scaled by scale*log2(e).
+  // Query slice of this thread for QK^T, pre-scaled by scale*log2(e) (and
+  // by the K dequantisation scale of this KV head).
   const int part = tid % C::PARTS;
+  float qscale = p.scale_log2;
+  if constexpr (FP8) qscale *= p.k_scale[kvh];
   uint64_t qr[G][C::DPT / 2];   // packed pairs of dims
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -164,7 +271,7 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
       bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + c8 * 8), f);
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        qr[g][c8 * 4 + e] = f2_make(f[2 * e] * p.scale_log2, f[2 * e + 1] * p.scale_log2);
+        qr[g][c8 * 4 + e] = f2_make(f[2 * e] * qscale, f[2 * e + 1] * qscale);
     }
   }
   const int dc = tid & 15;     // PV: output dims [8*dc, 8*dc+8)
@@ -181,12 +288,17 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>(i / NSTAGE) & 1u, abort, p.status);
     if (__syncthreads_or(!ok)) break;
     const uint8_t *sK = stages + st * STAGE_BYTES;
-    const uint8_t *sV = sK + 2 * BOX_BYTES;
-    const int key_base = tl.block(pos0 + i) * KT;
+    const uint8_t *sV = sK + T::KBYTES;
+    // Token position of key 0 of each block of this iteration (a missing
+    // block: past every length, so its keys are masked).
+    int key_base[NB];
+#pragma unroll
+    for (int h = 0; h < NB; ++h)
+      key_base[h] = (NB * i + h < nblocks) ? tl.block(pos0 + NB * i + h) * KT : INT_MAX / 2;
 
     // ---- scores
 #pragma unroll
-    for (int pass = 0; pass < C::PASSES; ++pass) {
+    for (int pass = 0; pass < PASSES; ++pass) {
       const int key = pass * C::KPP + tid / C::PARTS;
       uint64_t d2[G];
 #pragma unroll
@@ -194,7 +306,7 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 #pragma unroll
       for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
         uint64_t k2[4];
-        bf16x8_to_f2(*reinterpret_cast<const uint4 *>(sK + tile_offset(key, part * (C::DPT / 8) + c8)), k2);
+        load8<FP8>(sK, key, part * (C::DPT / 8) + c8, k2);
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -212,30 +324,38 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 #pragma unroll
         for (int g = 0; g < G; ++g) d[g] += __shfl_xor_sync(0xffffffffu, d[g], off);
       if (part == 0) {
-        const bool valid = key_base + key < L;
+        const bool valid = key_base[key / KT] + (key % KT) < L;
 #pragma unroll
-        for (int g = 0; g < G; ++g) s_sm[g * KT + key] = valid ? d[g] : -INFINITY;
+        for (int g = 0; g < G; ++g) s_sm[g * TK + key] = valid ? d[g] : -INFINITY;
       }
     }
     __syncthreads();
 
-    // ---- online softmax, one warp per query head
+    // ---- online softmax, one warp per query head (TK / 32 keys per lane)
     if (warp < G) {
-      const float v0 = s_sm[warp * KT + lane], v1 = s_sm[warp * KT + lane + 32];
-      float mt = fmaxf(v0, v1);
+      constexpr int KL = TK / 32;
+      float v[KL];
+#pragma unroll
+      for (int j = 0; j < KL; ++j) v[j] = s_sm[warp * TK + lane + 32 * j];
+      float mt = v[0];
+#pragma unroll
+      for (int j = 1; j < KL; ++j) mt = fmaxf(mt, v[j]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
       const float m_new = fmaxf(m_run, mt);
       const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float p0 = ex2(v0 - m_use), p1 = ex2(v1 - m_use);
-      float ps = p0 + p1;
+      float ps = 0.f;
+#pragma unroll
+      for (int j = 0; j < KL; ++j) {
+        const float pj = ex2(v[j] - m_use);
+        ps += pj;
+        p_sm[(lane + 32 * j) * G + warp] = pj;
+      }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
       l_run = l_run * alpha + ps;
       m_run = m_new;
-      p_sm[lane * G + warp] = p0;
-      p_sm[(lane + 32) * G + warp] = p1;
       if (lane == 0) alpha_sm[warp] = alpha;
     }
     __syncthreads();
@@ -248,10 +368,10 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
       for (int e = 0; e < 4; ++e) acc[g][e] = f2_mul(acc[g][e], a2);
     }
 #pragma unroll
-    for (int kk = 0; kk < KT / 16; ++kk) {
+    for (int kk = 0; kk < TK / 16; ++kk) {
       const int key = ks + 16 * kk;
       uint64_t v2[4];
-      bf16x8_to_f2(*reinterpret_cast<const uint4 *>(sV + tile_offset(key, dc)), v2);
+      load8<FP8>(sV, key, dc, v2);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float pg = p_sm[key * G + g];
@@ -275,6 +395,8 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 
   // ---- reduce the 16 key streams through shared memory (stage buffers free)
   float *red = reinterpret_cast<float *>(stages);   // [16][G][HD]
+  float vs = 1.0f;
+  if constexpr (FP8) vs = p.v_scale[kvh];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -291,7 +413,7 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     float sum = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) sum += red[(s * G + g) * HD + dd];
-    p.o_part[(row0 + static_cast<size_t>(g) * p.nsplit) * HD + dd] = sum;
+    p.o_part[(row0 + static_cast<size_t>(g) * p.nsplit) * HD + dd] = sum * vs;
   }
   if (warp < G && lane == 0) {
     float *ml = p.ml_part + (row0 + static_cast<size_t>(warp) * p.nsplit) * 2;
@@ -383,8 +505,17 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax) {
 int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
   using namespace decode;
   CUtensorMap tmK, tmV;
-  if (make_tmap_bhsd(&tmK, a.kcache, a.B, a.Lmax, a.Hkv, 64, KT) != 0) return FA_ERR_CUDA;
-  if (make_tmap_bhsd(&tmV, a.vcache, a.B, a.Lmax, a.Hkv, 64, KT) != 0) return FA_ERR_CUDA;
+  const bool paged = a.block_table != nullptr;
+  // The cache as a 4-D tensor (D, Hkv, tokens, batch); a page pool is
+  // (D, Hkv, 64, num_pages).
+  const int mB = paged ? a.num_pages : a.B, mS = paged ? KT : a.Lmax;
+  if (a.fp8) {
+    if (make_tmap_bhsd_u8(&tmK, a.kcache, mB, mS, a.Hkv, KT) != 0) return FA_ERR_CUDA;
+    if (make_tmap_bhsd_u8(&tmV, a.vcache, mB, mS, a.Hkv, KT) != 0) return FA_ERR_CUDA;
+  } else {
+    if (make_tmap_bhsd(&tmK, a.kcache, mB, mS, a.Hkv, 64, KT) != 0) return FA_ERR_CUDA;
+    if (make_tmap_bhsd(&tmV, a.vcache, mB, mS, a.Hkv, 64, KT) != 0) return FA_ERR_CUDA;
+  }
   const int G = a.Hq / a.Hkv;
   // Splits: sized for FULL unless every sequence is known to be SPARSE.
   int ns = decode_num_splits(a.B, a.Hkv, a.Lmax);
@@ -410,13 +541,28 @@ int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
   p.sink_blocks = a.sink / KT;
   p.win_blocks = a.window / KT;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.block_table = a.block_table;
+  p.max_pages = a.max_pages;
+  p.num_pages = a.num_pages;
+  p.k_scale = a.fp8 ? a.k_scale : nullptr;
+  p.v_scale = a.fp8 ? a.v_scale : nullptr;
   const dim3 grid(ns, a.Hkv, a.B);
   void (*kern)(const CUtensorMap, const CUtensorMap, const Params) = nullptr;
-  switch (G) {
-    case 1: kern = decode_kernel<1>; break;
-    case 2: kern = decode_kernel<2>; break;
-    case 4: kern = decode_kernel<4>; break;
-    case 8: kern = decode_kernel<8>; break;
+  // FP8 caches are always paged (a contiguous cache is the identity table).
+  if (a.fp8 && !paged) return FA_ERR_UNSUPPORTED;
+  switch (G * 4 + (a.fp8 ? 2 : 0) + (paged ? 1 : 0)) {
+    case 4: kern = decode_kernel<1, false, false>; break;
+    case 8: kern = decode_kernel<2, false, false>; break;
+    case 16: kern = decode_kernel<4, false, false>; break;
+    case 32: kern = decode_kernel<8, false, false>; break;
+    case 5: kern = decode_kernel<1, false, true>; break;
+    case 9: kern = decode_kernel<2, false, true>; break;
+    case 17: kern = decode_kernel<4, false, true>; break;
+    case 33: kern = decode_kernel<8, false, true>; break;
+    case 7: kern = decode_kernel<1, true, true>; break;
+    case 11: kern = decode_kernel<2, true, true>; break;
+    case 19: kern = decode_kernel<4, true, true>; break;
+    case 35: kern = decode_kernel<8, true, true>; break;
     default: return FA_ERR_UNSUPPORTED;
   }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
@@ -426,6 +572,61 @@ int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   combine_kernel<<<dim3(a.Hq, a.B), 128, 0, stream>>>(
       p.o_part, p.ml_part, reinterpret_cast<__nv_bfloat16 *>(a.o), a.lse, a.Hq, ns);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ KV append
+// Writes token position seqlens[b] of every sequence (K and V of all KV
+// heads) into its page, quantising to E4M3 (code = RN(fp32(x / scale)),
+// saturating) for an FP8 cache, then advances seqlens[b].  A position past
+// the block table or a page id outside the pool is reported and skipped.
+// One CTA per sequence.
+__global__ void __launch_bounds__(256) kv_append_kernel(const __nv_bfloat16 *k_new,
+                                                        const __nv_bfloat16 *v_new,
+                                                        uint8_t *k_pages, uint8_t *v_pages, int fp8,
+                                                        const float *k_scale, const float *v_scale,
+                                                        const int32_t *block_table, int max_pages,
+                                                        int num_pages, int32_t *seqlens, int Hkv,
+                                                        int32_t *status) {
+  const int b = blockIdx.x;
+  const int pos = seqlens[b];
+  const int pi = pos / decode::KT, slot = pos % decode::KT;
+  int page = -1;
+  if (pos >= 0 && pi < max_pages) page = block_table[static_cast<size_t>(b) * max_pages + pi];
+  const bool ok = page >= 0 && page < num_pages;
+  if (!ok) {
+    if (threadIdx.x == 0) report(status, FA_DEV_BAD_INDEX);
+    return;
+  }
+  const size_t row = (static_cast<size_t>(page) * decode::KT + slot) * Hkv;   // token row
+  const int n = Hkv * decode::HD;
+  for (int t = 0; t < 2; ++t) {
+    const __nv_bfloat16 *src = (t ? v_new : k_new) + static_cast<size_t>(b) * n;
+    uint8_t *dst = (t ? v_pages : k_pages);
+    const float *sc = t ? v_scale : k_scale;
+    for (int i = threadIdx.x * 2; i < n; i += 2 * blockDim.x) {
+      if (fp8) {
+        const float s = sc[i / decode::HD];
+        const float2 x = make_float2(__fdiv_rn(__bfloat162float(src[i]), s),
+                                     __fdiv_rn(__bfloat162float(src[i + 1]), s));
+        const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+        *reinterpret_cast<__nv_fp8x2_storage_t *>(dst + row * decode::HD + i) = c;
+      } else {
+        *reinterpret_cast<uint32_t *>(dst + (row * decode::HD + i) * 2) =
+            *reinterpret_cast<const uint32_t *>(src + i);
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) seqlens[b] = pos + 1;
+}
+
+int launch_kv_append(const KvAppendLaunch &a, cudaStream_t stream) {
+  kv_append_kernel<<<a.B, 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16 *>(a.k_new),
+      reinterpret_cast<const __nv_bfloat16 *>(a.v_new), reinterpret_cast<uint8_t *>(a.k_pages),
+      reinterpret_cast<uint8_t *>(a.v_pages), a.fp8, a.k_scale, a.v_scale, a.block_table,
+      a.max_pages, a.num_pages, a.seqlens, a.Hkv, a.status);
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

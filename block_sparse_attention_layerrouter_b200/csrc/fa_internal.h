@@ -50,7 +50,28 @@ struct DecodeLaunch {
   float *lse;
   void *workspace;
   int32_t *status;
+  // Paged cache: pool [num_pages, 64, Hkv, D]; Lmax = 64 * max_pages.
+  const int32_t *block_table = nullptr;
+  int max_pages = 0, num_pages = 0;
+  // FP8 (E4M3) cache with per-KV-head dequantisation scales.
+  int fp8 = 0;
+  const float *k_scale = nullptr, *v_scale = nullptr;
 };
+struct KvAppendLaunch {
+  const void *k_new, *v_new;        // bf16 [B, Hkv, D]
+  void *k_pages, *v_pages;
+  int fp8;
+  const float *k_scale, *v_scale;
+  const int32_t *block_table;
+  int max_pages, num_pages;
+  int32_t *seqlens;                 // in: positions to write; out: + 1
+  int B, Hkv;
+  int32_t *status;
+};
+int launch_kv_append(const KvAppendLaunch &a, cudaStream_t stream);
+// 4-D TMA map over a byte tensor [B, S, H, 128] (an FP8 cache), boxes of
+// 128 x 1 x box_rows x 1 with the 128-byte swizzle.
+int make_tmap_bhsd_u8(CUtensorMap *map, const void *base, int B, int S, int H, int box_rows);
 int decode_num_splits(int B, int Hkv, int Lmax);
 int decode_splits_for_tiles(int B, int Hkv, int tiles);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax);

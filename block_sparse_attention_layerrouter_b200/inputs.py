@@ -38,6 +38,8 @@ class Workload:
     decode_len: int = 0        # >0: decode workload with this cache length
     varlen: bool = False       # packed batch of B requests of seeded lengths <= S
     train: bool = False        # soft-routed training step (forward + backward)
+    paged: bool = False        # decode through a paged cache (64-token pages)
+    kv_fp8: bool = False       # E4M3 KV cache (paged)
     seed: int = 1000
     notes: str = field(default="", compare=False)
 
@@ -73,6 +75,16 @@ WORKLOADS = {
                                                 Hq=32, Hkv=8, window=1024, hidden=256,
                                                 train=True, seed=1007,
                                                 notes="soft-routed layer, forward + backward"),
+    # The decode workload through a paged cache (pages in a seeded random
+    # order), bf16 and FP8 E4M3 with per-head scales.
+    "decode-paged-b8-l131072-32l": Workload("decode-paged-b8-l131072-32l", B=8, S=1, Hq=32,
+                                            Hkv=8, layers=32, window=2048, hidden=256,
+                                            decode_len=131072, paged=True, seed=1008,
+                                            notes="paged bf16 decode"),
+    "decode-fp8-b8-l131072-32l": Workload("decode-fp8-b8-l131072-32l", B=8, S=1, Hq=32, Hkv=8,
+                                          layers=32, window=2048, hidden=256, decode_len=131072,
+                                          paged=True, kv_fp8=True, seed=1009,
+                                          notes="paged FP8 (E4M3) decode"),
     # Profiling shape: the decode workload at a quarter of the context
     # (1 GiB of K/V, still far above the 126 MB L2).
     "decode-b8-l32768": Workload("decode-b8-l32768", B=8, S=1, Hq=32, Hkv=8, layers=2,
@@ -134,6 +146,30 @@ def varlen_lengths(B: int, max_len: int, seed: int, min_len: int = 1024) -> np.n
     L = rng.integers(min_len, max_len + 1, size=B)
     L[int(rng.integers(0, B))] = max_len
     return L.astype(np.int64)
+
+
+def fp8_codes(shape, seed: int, device="cpu") -> torch.Tensor:
+    """Seeded E4M3 codes (uint8) with random sign and mantissa and exponent
+    field 4..10 (magnitudes 1/8 .. 15): a stand-in for a quantised cache."""
+    g = _gen(device, seed)
+    sign = torch.randint(0, 2, shape, generator=g, device=device, dtype=torch.int32)
+    e = torch.randint(4, 11, shape, generator=g, device=device, dtype=torch.int32)
+    m = torch.randint(0, 8, shape, generator=g, device=device, dtype=torch.int32)
+    return ((sign << 7) | (e << 3) | m).to(torch.uint8)
+
+
+def fp8_scales(H: int, seed: int) -> torch.Tensor:
+    """Per-head dequantisation scales, fp32 uniform in [1/48, 1/24]."""
+    rng = np.random.default_rng(seed)
+    return torch.from_numpy(rng.uniform(1 / 48, 1 / 24, size=H).astype(np.float32))
+
+
+def page_table(B: int, max_pages: int, seed: int, extra: int = 0) -> torch.Tensor:
+    """Block table [B, max_pages] int32: a seeded permutation of the pool's
+    B * max_pages + extra pages (the first B * max_pages entries)."""
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(B * max_pages + extra)[:B * max_pages]
+    return torch.from_numpy(perm.reshape(B, max_pages).astype(np.int32))
 
 
 def bits(t: torch.Tensor) -> np.ndarray:

@@ -61,6 +61,9 @@ typedef enum {
 
 typedef enum { FA_MODE_FULL = 0, FA_MODE_SPARSE = 1 } fa_mode;
 
+/* KV cache element type of the paged decode path. */
+typedef enum { FA_KV_BF16 = 0, FA_KV_FP8_E4M3 = 1 } fa_kv_dtype;
+
 /* Sparse pattern, in tokens: block = 64 ("Flux Attention", implementation
  * paragraph: 64-token blocks), sink = 128 sink tokens, window = local window
  * counted in whole blocks and including the query's own block.  sink and
@@ -203,6 +206,42 @@ FA_API int fa_soft_routed_layer_backward(
     const float *gumbel, float tau, const int32_t *row_ptr, const int32_t *col_idx,
     void *dq, void *dk, void *dv, float *dw1, float *db1, float *dw2, float *db2,
     float *r_out, void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ----------------------------------------------- paged / FP8 KV cache ---
+ * Decode over a paged KV cache, and the append of the current token.  A page
+ * holds 64 consecutive tokens of one sequence (one block of the sparse rule,
+ * so a SPARSE layer reads only the pages of its sink and window blocks and
+ * never loads any other page: "Flux Attention", KV-cache bypass paragraph).
+ *   k_pages, v_pages: device pools [num_pages, 64, Hkv, D] of bf16
+ *   (FA_KV_BF16) or E4M3 bytes (FA_KV_FP8_E4M3); token t of sequence b is
+ *   slot t % 64 of page block_table[b * max_pages + t / 64].
+ *   block_table: device int32 [B, max_pages]; page ids must lie in
+ *   [0, num_pages) (an id outside is reported as FA_DEV_BAD_INDEX and its
+ *   tokens read as zeros).  A contiguous cache [B, Lmax, Hkv, D] is the
+ *   pool with num_pages = B * Lmax / 64 and block_table[b][i] = b * Lmax/64 + i.
+ *   k_scale, v_scale: device fp32 [Hkv], FP8 only: stored code c of value x is
+ *   RN_e4m3(fp32(x / scale)) (saturating at +-448); x is read back as
+ *   e4m3(c) * scale.  Ignored (may be NULL) for bf16.
+ * fa_kv_append_paged: writes k_new, v_new (bf16 [B, Hkv, D], device) at
+ *   position seqlens[b] of every sequence, quantising for FP8, then sets
+ *   seqlens[b] += 1 on the device (seqlens: device int32 [B], in/out).  A
+ *   position past max_pages * 64 is reported (FA_DEV_BAD_INDEX) and skipped.
+ * fa_attn_decode_paged: as fa_attn_decode (query at position L-1, L =
+ *   seqlens[b] <= 64 * max_pages), reading the cache through the block table.
+ *   workspace >= fa_decode_paged_workspace_size(B, Hq, Hkv, max_pages, D). */
+FA_API int fa_kv_append_paged(const void *k_new, const void *v_new, void *k_pages,
+                              void *v_pages, int kv_dtype, const float *k_scale,
+                              const float *v_scale, const int32_t *block_table,
+                              int max_pages, int num_pages, int32_t *seqlens, int B,
+                              int Hkv, int D, int32_t *dev_status, void *stream);
+FA_API size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_pages, int D);
+FA_API int fa_attn_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                                int kv_dtype, const float *k_scale, const float *v_scale,
+                                const int32_t *block_table, int max_pages, int num_pages,
+                                const int32_t *seqlens, int B, int Hq, int Hkv, int D,
+                                float scale, int mode, const int32_t *mode_dev,
+                                fa_sparse_cfg cfg, void *o, float *lse, void *workspace,
+                                size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /* ------------------------------------------- variable-length batches ---
  * Serving form of the routed layer ("Flux Attention": the router decides per
