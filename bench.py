@@ -802,7 +802,23 @@ def run_only(args, wl):
     B, Hq, Hkv = wl.B, wl.Hq, wl.Hkv
     S = wl.decode_len or wl.S
     c = capi.cfg(64, wl.sink, wl.window)
-    if args.only.startswith("decode"):
+    if args.only.startswith("decode_fp8"):
+        max_pages = S // 64
+        q = inputs.randn_bf16((B, Hq, 128), wl.seed, device=dev)
+        kc = inputs.fp8_codes((B * max_pages, 64, Hkv, 128), wl.seed + 100, device=dev)
+        vc = inputs.fp8_codes((B * max_pages, 64, Hkv, 128), wl.seed + 200, device=dev)
+        bt = inputs.page_table(B, max_pages, wl.seed).to(dev)
+        ksc, vsc = inputs.fp8_scales(Hkv, wl.seed).to(dev), inputs.fp8_scales(Hkv, 1).to(dev)
+        sl = torch.full((B,), S, dtype=torch.int32, device=dev)
+        wsb = torch.empty(capi.decode_workspace_size(B, Hq, Hkv, S), dtype=torch.uint8,
+                          device=dev)
+        md = 0 if args.only == "decode_fp8_full" else 1
+        o = torch.empty_like(q)
+        fn = lambda: capi.attn_decode_paged(  # noqa: E731
+            q, kc, vc, bt, sl, capi.FA_KV_FP8_E4M3, ksc, vsc, md, c, o=o, workspace=wsb)
+        work = B * 2 * Hkv * 128 * 1 * decode_keys(S, md, wl.sink, wl.window) / 1e9
+        unit = "GB/s"
+    elif args.only.startswith("decode"):
         q, kc, vc = inputs.decode_inputs(B, S, Hq, Hkv, 128, wl.seed, device=dev)
         sl = torch.full((B,), S, dtype=torch.int32, device=dev)
         wsb = torch.empty(capi.decode_workspace_size(B, Hq, Hkv, S), dtype=torch.uint8,
@@ -899,7 +915,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
-                    help="prefill_full | prefill_sparse | decode_full | decode_sparse | router")
+                    help="prefill_full | prefill_sparse | decode_full | decode_sparse | "
+                         "decode_fp8_full | decode_fp8_sparse | backward_full | "
+                         "backward_sparse | router")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

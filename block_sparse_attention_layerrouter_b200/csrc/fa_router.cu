@@ -235,16 +235,26 @@ __global__ void __launch_bounds__(256) dw1_kernel(const float *da, const float *
   }
 }
 
-// dx[b, i] = sum_u da[b, u] W1[u, i]: one thread per (i, b), W1 read by
-// columns (coalesced across threads).
+// dx[b, i] = sum_u da[b, u] W1[u, i]: a CTA covers 32 columns i; its 8 warps
+// take every 8th hidden unit (each warp reads 128 contiguous bytes of a W1
+// row) and the partial sums meet in shared memory.
 __global__ void __launch_bounds__(256) dx_kernel(const float *da, const float *w1, int B, int in_f,
                                                  int hidden, float *dx) {
-  const int i = blockIdx.x * 256 + threadIdx.x, b = blockIdx.y;
-  if (i >= in_f) return;
+  __shared__ float part[8][32];
+  const int lane = threadIdx.x & 31, ug = threadIdx.x >> 5;
+  const int i = blockIdx.x * 32 + lane, b = blockIdx.y;
   const float *dab = da + static_cast<size_t>(b) * hidden;
   float s = 0.f;
-  for (int u = 0; u < hidden; ++u) s = fmaf(dab[u], w1[static_cast<size_t>(u) * in_f + i], s);
-  dx[static_cast<size_t>(b) * in_f + i] = s;
+  if (i < in_f)
+    for (int u = ug; u < hidden; u += 8) s = fmaf(dab[u], w1[static_cast<size_t>(u) * in_f + i], s);
+  part[ug][lane] = s;
+  __syncthreads();
+  if (ug == 0 && i < in_f) {
+    float t = 0.f;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) t += part[g][lane];
+    dx[static_cast<size_t>(b) * in_f + i] = t;
+  }
 }
 
 }  // namespace router
@@ -271,8 +281,8 @@ int launch_router_backward(const RouterBwdLaunch &a, cudaStream_t stream) {
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   dw1_kernel<<<a.hidden, 256, 0, stream>>>(a.da, a.x, a.B, in_f, a.hidden, a.dw1);
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
-  dx_kernel<<<dim3((in_f + 255) / 256, a.B), 256, 0, stream>>>(a.da, a.w1, a.B, in_f, a.hidden,
-                                                                a.dx);
+  dx_kernel<<<dim3((in_f + 31) / 32, a.B), 256, 0, stream>>>(a.da, a.w1, a.B, in_f, a.hidden,
+                                                              a.dx);
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
