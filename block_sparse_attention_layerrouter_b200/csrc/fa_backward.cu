@@ -20,7 +20,7 @@
 //                    S^T  = K Q^T      (M=128 keys, N=64 queries, K=D)
 //                    dP^T = V dO^T     (same shape)
 //                    dV  += P^T dO     (A = P^T from TMEM; N=D, K=queries)
-//                    dK  += dS^T Q     (A = dS^T from shared memory)
+//                    dK  += dS^T Q     (A = dS^T from TMEM)
 //                    dQ^T = K^T dS^T   (M=D, N=64; A and B MN-major)
 //                  dK and dV accumulate in TMEM over the whole item; each
 //                  step's dQ^T goes to an fp32 accumulator in HBM through TMA
@@ -268,7 +268,6 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   const uint64_t o_kmaj = smem_desc_sw128(sh.dout(0), 16, 1024);
   const uint64_t q_mn = smem_desc_sw128(sh.q(0), QT_HALF, 1024);
   const uint64_t o_mn = smem_desc_sw128(sh.dout(0), QT_HALF, 1024);
-  const uint64_t ds_kmaj = smem_desc_sw128(sh.ds(0), 16, 1024);
   const uint64_t ds_mn = smem_desc_sw128(sh.ds(0), QT_HALF, 1024);
   const uint32_t t_dv = tmem + 256u, t_dk = tmem + 384u;
   int nf = 0, nb = 0;      // steps whose front (S, dP) / back half was issued
@@ -320,8 +319,8 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
                     kIdKV, (first && kk == 0) ? 0u : 1u);
     }
 #pragma unroll
-    for (int kk = 0; kk < BQ / 16; ++kk) {   // dK += dS^T Q
-      mma_bf16_ss_w(t_dk, ds_kmaj + du + static_cast<uint64_t>((kk * 32) >> 4),
+    for (int kk = 0; kk < BQ / 16; ++kk) {   // dK += dS^T Q (dS^T from TMEM)
+      mma_bf16_ts_w(t_dk, tmem + 128u + 64u * u + kk * 8,
                     q_mn + so + static_cast<uint64_t>((kk * 2048) >> 4), kIdKV,
                     (first && kk == 0) ? 0u : 1u);
     }
@@ -503,13 +502,21 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
             ds[j] = pv[32 * hlf + j] * (__uint_as_float(a[j]) - d4[e]);
           }
         }
+        uint32_t pk[16];
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           const uint32_t chunk = static_cast<uint32_t>(4 * hlf + cc);
           const uint4 v = pack8(ds + 8 * cc);
           st_shared_u4(ds_row + ((chunk ^ (static_cast<uint32_t>(r) & 7u)) << 4), v.x, v.y, v.z,
                        v.w);
+          pk[4 * cc] = v.x;
+          pk[4 * cc + 1] = v.y;
+          pk[4 * cc + 2] = v.z;
+          pk[4 * cc + 3] = v.w;
         }
+        // dS (bf16 pairs) also into the dP columns just read, as the TMEM A
+        // operand of dK += dS^T Q.
+        tmem_st16(tmem + lane + 128u + 64u * u + 16u * hlf, pk);
       }
       tmem_st_wait();
       fence_proxy_async_smem();
