@@ -726,7 +726,7 @@ def run_train(args, wl):
     g = inputs.gumbel(B, wl.seed).to(dev)
     c = capi.cfg(64, wl.sink, wl.window)
     rp, ci = capi.blocksparse_index(S, c, device=dev)
-    o_f, o_s = torch.empty_like(q), torch.empty_like(q)
+    o_f, o_s, y = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     lse_f = torch.empty(B, Hq, S, device=dev)
     lse_s = torch.empty(B, Hq, S, device=dev)
     logits = torch.empty(B, 2, device=dev)
@@ -744,6 +744,7 @@ def run_train(args, wl):
         capi.router_soft(logits, g, tau=1.0, r=r)
         capi.attn_prefill_full(q, k, v, o=o_f, lse=lse_f, status=status)
         capi.attn_prefill_blocksparse(q, k, v, rp, ci, o=o_s, lse=lse_s, status=status)
+        capi.soft_mix(o_f, o_s, r, y=y)
         return capi.soft_routed_layer_backward(q, k, v, o_f, lse_f, o_s, lse_s, dy, w1, b1, w2, b2,
                                                rp, ci, gumbel=g, tau=1.0, workspace=bws,
                                                status=status)
@@ -775,8 +776,9 @@ def run_train(args, wl):
     line = base_line(args, wl, ws, ms, "TFLOP/s", value)
     line["config"] = {"workload": wl.name, "B": B, "S": S, "Hq": Hq, "Hkv": Hkv, "D": 128,
                       "sink": wl.sink, "window": wl.window, "hidden": wl.hidden,
-                      "step": "router + r + FULL and SPARSE forward with LSE + soft-routed "
-                              "backward (router grads, dQ/dK/dV through both paths)",
+                      "step": "router + r + FULL and SPARSE forward with LSE + y = r O_FA + "
+                              "(1-r) O_SA + soft-routed backward (router grads, dQ/dK/dV "
+                              "through both paths)",
                       "flops": "forward 4*D*Hq*pairs per path (SPARSE: executed 64x64 "
                                "blocks), backward 2.5x the forward",
                       "l2": "Q/K/V/O/dy/accumulators 0.6 GB per step > L2"}

@@ -84,6 +84,7 @@ _SIGNATURES = {
     "fa_decode_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_attn_decode_paged": (_I, [_VP, _VP, _VP, _I, _VP, _VP, _VP, _I, _I, _VP, _I, _I, _I, _I,
                                   _F, _I, _VP, SparseCfg, _VP, _VP, _VP, _SZ, _VP, _VP]),
+    "fa_soft_mix": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "fa_hybrid_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_hybrid_layer": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _VP, _I, _VP,
                              _VP, SparseCfg, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
@@ -519,3 +520,15 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seqlens, kv_dtype=FA_KV_
                                     _stream(q.device))
     _check("fa_attn_decode_paged", rc)
     return o
+
+
+def soft_mix(o_full, o_sparse, r, y=None) -> torch.Tensor:
+    """fa_soft_mix: y = r O_FA + (1 - r) O_SA per sequence (bf16)."""
+    _need(o_full, "o_full", torch.bfloat16, 4)
+    _need(o_sparse, "o_sparse", torch.bfloat16, 4)
+    _need(r, "r", torch.float32, 1)
+    B, S, Hq, D = o_full.shape
+    y = torch.empty_like(o_full) if y is None else y
+    _check("fa_soft_mix", lib().fa_soft_mix(_ptr(o_full), _ptr(o_sparse), _ptr(r), _ptr(y), B, S,
+                                            Hq, D, _stream(o_full.device)))
+    return y

@@ -344,6 +344,15 @@ FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v, voi
   return launch_prefill(sparse, st);
 }
 
+FA_API int fa_soft_mix(const void *o_full, const void *o_sparse, const float *r, void *y, int B,
+                       int S, int Hq, int D, void *stream) {
+  if (!o_full || !o_sparse || !r || !y || B <= 0 || S <= 0 || Hq <= 0) return FA_ERR_INVALID_ARG;
+  if (!aligned16(o_full) || !aligned16(o_sparse) || !aligned16(y)) return FA_ERR_INVALID_ARG;
+  if (D != kHeadDim) return FA_ERR_UNSUPPORTED;
+  return launch_soft_mix(o_full, o_sparse, r, y, B, static_cast<long long>(S) * Hq * D,
+                         static_cast<cudaStream_t>(stream));
+}
+
 FA_API size_t fa_attn_backward_workspace_size(int B, int S, int Hq, int Hkv, int D) {
   if (B <= 0 || S <= 0 || check_heads(Hq, Hkv, D) != FA_OK) return 0;
   return backward_workspace_bytes(B, S, Hq, Hkv);

@@ -130,6 +130,8 @@ struct RouterBwdLaunch {
   float *dw1, *db1, *dw2, *db2;        // outputs
 };
 void router_ws_parts(void *workspace, int B, int Hq, float **part, float **hid);
+int launch_soft_mix(const void *o_full, const void *o_sparse, const float *r, void *y, int B,
+                    long long per_b, cudaStream_t stream);
 int launch_router_backward(const RouterBwdLaunch &a, cudaStream_t stream);
 
 // Soft-routed layer backward: both attention paths (upstream r dy and

@@ -257,7 +257,46 @@ __global__ void __launch_bounds__(256) dx_kernel(const float *da, const float *w
   }
 }
 
+// y = r O_FA + (1 - r) O_SA per sequence (bf16 rows of 8 elements per thread;
+// the products in fp32, rounded once).
+__global__ void __launch_bounds__(256) mix_kernel(const __nv_bfloat16 *of, const __nv_bfloat16 *os,
+                                                  const float *r, __nv_bfloat16 *y,
+                                                  long long per_b, int B) {
+  const long long n8 = per_b * B / 8;
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * 256) {
+    const float rb = r[(i * 8) / per_b];
+    const uint4 a = reinterpret_cast<const uint4 *>(of)[i];
+    const uint4 b = reinterpret_cast<const uint4 *>(os)[i];
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = rb * __uint_as_float(wa[k] << 16) + (1.0f - rb) * __uint_as_float(wb[k] << 16);
+      const float hi = rb * __uint_as_float(wa[k] & 0xffff0000u) +
+                       (1.0f - rb) * __uint_as_float(wb[k] & 0xffff0000u);
+      w[k] = pack_bf16x2(lo, hi);
+    }
+    reinterpret_cast<uint4 *>(y)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 }  // namespace router
+
+int launch_soft_mix(const void *o_full, const void *o_sparse, const float *r, void *y, int B,
+                    long long per_b, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const long long n8 = per_b * B / 8;
+  const long long blocks = (n8 + 255) / 256;
+  router::mix_kernel<<<static_cast<unsigned>(blocks < 4 * sms ? blocks : 4 * sms), 256, 0,
+                       stream>>>(reinterpret_cast<const __nv_bfloat16 *>(o_full),
+                                 reinterpret_cast<const __nv_bfloat16 *>(o_sparse), r,
+                                 reinterpret_cast<__nv_bfloat16 *>(y), per_b, B);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 void router_ws_parts(void *workspace, int B, int Hq, float **part, float **hid) {
   const size_t pbytes = static_cast<size_t>(router::kPoolSlices) * B * Hq * router::HD * sizeof(float);

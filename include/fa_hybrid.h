@@ -299,6 +299,12 @@ FA_API int fa_hybrid_layer_varlen(const void *q, const void *k, const void *v,
  * it (O_FA is rounded to bf16 in between).  Forward only; no LSE.
  *   logits_out fp32 [B, 2], r_out fp32 [B]: device, required.
  *   workspace >= fa_router_workspace_size(B, Hq, D, hidden). */
+/* fa_soft_mix: y = r * O_FA + (1 - r) * O_SA per sequence, for a training
+ * forward that keeps both outputs (and their LSE) for the backward.
+ * o_full, o_sparse, y: bf16 [B, S, Hq, D] (y may alias neither input); r fp32
+ * [B]; all device.  Rounded to bf16 once. */
+FA_API int fa_soft_mix(const void *o_full, const void *o_sparse, const float *r, void *y,
+                       int B, int S, int Hq, int D, void *stream);
 FA_API int fa_router_soft(const float *logits, const float *gumbel, int B,
                           float tau, float *r_out, void *stream);
 FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v,

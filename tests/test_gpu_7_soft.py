@@ -54,3 +54,17 @@ def test_soft_routed_layer_matches_oracle(B, S, Hq, Hkv, W):
     assert_close_attention(to_f64(y), ref, "soft routed layer")
     # the mix is not either endpoint
     assert np.abs(to_f64(y) - o_full).max() > 1e-2 and np.abs(to_f64(y) - o_sparse).max() > 1e-2
+
+
+def test_soft_mix_matches_oracle():
+    """fa_soft_mix against the oracle's mix of the same bf16 outputs."""
+    of = inputs.randn_bf16((3, 200, 4, 128), 851, device="cuda")
+    osp = inputs.randn_bf16((3, 200, 4, 128), 852, device="cuda")
+    r = torch.tensor([0.1, 0.5, 0.93], device="cuda")
+    y = capi.soft_mix(of, osp, r)
+    torch.cuda.synchronize()
+    want = oracle.soft_mix(oracle.bf16_bits_to_f64(inputs.bits(of)),
+                           oracle.bf16_bits_to_f64(inputs.bits(osp)), r.cpu().double().numpy())
+    got = y.float().cpu().double().numpy()
+    # one bf16 rounding of the fp32 result: half an ulp, relative 2^-9
+    assert np.all(np.abs(got - want) <= np.abs(want) * 2.0 ** -8 + 1e-6)
