@@ -285,8 +285,10 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 
   for (int i = 0; i < ntiles; ++i) {
     const int st = i % NSTAGE;
+    // Every thread runs the scores even if its wait failed (the shuffles need
+    // the whole warp; the reads stay inside shared memory); the barrier after
+    // them agrees on leaving.
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>(i / NSTAGE) & 1u, abort, p.status);
-    if (__syncthreads_or(!ok)) break;
     const uint8_t *sK = stages + st * STAGE_BYTES;
     const uint8_t *sV = sK + T::KBYTES;
     // Token position of key 0 of each block of this iteration (a missing
@@ -329,7 +331,10 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
         for (int g = 0; g < G; ++g) s_sm[g * TK + key] = valid ? d[g] : -INFINITY;
       }
     }
-    __syncthreads();
+    // Past this barrier every thread is done with tile i-1 (its PV came before
+    // these scores), so its stage takes tile i-1+NSTAGE.
+    if (__syncthreads_or(!ok)) break;
+    if (tid == 0 && i >= 1 && i - 1 + NSTAGE < ntiles) issue(i - 1 + NSTAGE);
 
     // ---- online softmax, one warp per query head (TK / 32 keys per lane)
     if (warp < G) {
@@ -380,9 +385,8 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
         for (int e = 0; e < 4; ++e) acc[g][e] = f2_fma(p2, v2[e], acc[g][e]);
       }
     }
-    __syncthreads();
-    if (tid == 0 && i + NSTAGE < ntiles) issue(i + NSTAGE);
   }
+  __syncthreads();   // every thread is done with the stages (reused below) and p_sm
 
   if (*abort) {  // let the copies still in flight land, then leave
     if (tid == 0) {
