@@ -105,3 +105,50 @@ def test_product_path_has_no_cpu_fallback(monkeypatch, tmp_path):
     monkeypatch.setattr(capi, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not found"):
         capi.lib()
+
+
+# ---- host-side checks of the backward, paged/FP8 decode and soft-mix entries
+_P = ctypes.c_void_p(16)      # an aligned non-null pointer that is never dereferenced
+_N = None
+
+
+def test_backward_entries_reject_on_host(lib):
+    b = lib.fa_attn_prefill_backward
+    args = [_P] * 9 + [1, 256, 4, 2, 128, 0.088, _N, _N, _N, 0, _P, 1 << 30, _N, _N]
+    assert b(*args[:3], _N, *args[4:]) == -1                  # o missing
+    bad = list(args); bad[13] = 64                             # D != 128
+    assert b(*bad) == -2
+    bad = list(args); bad[18] = 1                              # SPARSE without a CSR
+    assert b(*bad) == -1
+    bad = list(args); bad[20] = 16                             # workspace too small
+    assert b(*bad) == -3
+    assert lib.fa_attn_backward_workspace_size(1, 256, 4, 2, 128) > 4 * 256 * 4 * 128
+    assert lib.fa_attn_backward_workspace_size(1, 256, 4, 3, 128) == 0
+    assert lib.fa_soft_routed_backward_workspace_size(1, 256, 4, 2, 128, 64) > \
+        lib.fa_attn_backward_workspace_size(1, 256, 4, 2, 128)
+
+
+def test_paged_decode_entries_reject_on_host(lib):
+    c = capi.cfg(64, 128, 256)
+    d = lib.fa_attn_decode_paged
+    good = [_P, _P, _P, 0, _N, _N, _P, 4, 8, _P, 2, 8, 2, 128, 0.088, 0, _N, c, _P, _N, _P,
+            1 << 30, _N, _N]
+    bad = list(good); bad[3] = 7                               # unknown cache type
+    assert d(*bad) == -1
+    bad = list(good); bad[3] = 1                               # FP8 without scales
+    assert d(*bad) == -1
+    bad = list(good); bad[11] = 7                              # Hq % Hkv != 0
+    assert d(*bad) == -1
+    bad = list(good); bad[21] = 8                              # workspace too small
+    assert d(*bad) == -3
+    assert lib.fa_decode_paged_workspace_size(2, 8, 2, 4, 128) == \
+        lib.fa_decode_workspace_size(2, 8, 2, 256, 128)
+    a = lib.fa_kv_append_paged
+    assert a(_P, _P, _P, _P, 0, _N, _N, _P, 4, 8, _P, 2, 2, 64, _N, _N) == -2   # D != 128
+    assert a(_P, _P, _P, _P, 1, _N, _N, _P, 4, 8, _P, 2, 2, 128, _N, _N) == -1  # FP8, no scales
+    assert a(_P, _P, _P, _P, 0, _N, _N, _N, 4, 8, _P, 2, 2, 128, _N, _N) == -1  # no block table
+
+
+def test_soft_mix_rejects_on_host(lib):
+    assert lib.fa_soft_mix(_P, _P, _P, _N, 1, 8, 2, 128, _N) == -1
+    assert lib.fa_soft_mix(_P, _P, _P, _P, 1, 8, 2, 64, _N) == -2
