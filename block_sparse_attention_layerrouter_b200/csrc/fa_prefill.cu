@@ -541,8 +541,16 @@ constexpr int WARP_PRODUCER = 8, WARP_MMA = 9;   // warps 10-11 idle
 // must not exceed what the block was launched with (384 x the compiled
 // count); the launcher checks it before every launch.
 constexpr int kSoftmaxRegs = 184, kOtherRegs = 136;
-constexpr int NUM_BARS = 2 + 2 * NSLOT + 4 * NQ + 1;
-constexpr int SMEM_BYTES = 1024 + NQ * TILE_BYTES + NSLOT * TILE_BYTES + NUM_BARS * 8 + 16;
+constexpr int NUM_BARS = 2 + 2 * NSLOT + 4 * NQ + 1 + 16;
+// For a sparse item the producer, which walks the CSR ahead of everyone to
+// load the KV tiles, hands each tile to the MMA and softmax warps through an
+// 8-entry ring in shared memory, so they do not walk it themselves:
+// (tile << 8) | last << 5 | valid << 4 | 4-bit block mask (0: an item without
+// tiles).  A full item's tiles 0..qt need no list.
+constexpr int NINFO = 8;
+constexpr int SMEM_BYTES =
+    1024 + NQ * TILE_BYTES + NSLOT * TILE_BYTES + NUM_BARS * 8 + 16 + 4 * NINFO;
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint64_t kDrainNs = 200000000ull;
@@ -597,13 +605,16 @@ struct Smem {
   enum : uint32_t {
     Q_FULL = 0, Q_EMPTY = 1, FULL0 = 2, EMPTY0 = FULL0 + NSLOT, S_FULL0 = EMPTY0 + NSLOT,
     P_FULL0 = S_FULL0 + NQ, O_DONE0 = P_FULL0 + NQ, O_FREE0 = O_DONE0 + NQ, DRAIN = O_FREE0 + NQ,
-    NBARS = DRAIN + 1
+    INFO_FULL0 = DRAIN + 1, INFO_EMPTY0 = INFO_FULL0 + NINFO, NBARS = INFO_EMPTY0 + NINFO
   };
   FA_DEV uint32_t q(int t) const { return base + t * TILE_BYTES; }
   FA_DEV uint32_t ring(int slot) const { return base + kRing + slot * TILE_BYTES; }
   FA_DEV uint32_t bar(uint32_t i) const { return base + kBars + 8u * i; }
   FA_DEV uint32_t tmem_slot() const { return base + kBars + 8u * NBARS; }
   FA_DEV uint32_t abort_flag() const { return tmem_slot() + 4u; }
+  FA_DEV uint32_t info(int slot) const {
+    return base + kBars + 8u * NBARS + 16u + 4u * static_cast<uint32_t>(slot);
+  }
 };
 
 FA_DEV Smem carve(uint8_t *raw) {
@@ -684,6 +695,7 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
                          const CUtensorMap *tmV, const Params &p, int total) {
   int li = 0;       // ring loads issued (continues across items)
   int nq = 0;       // Q loads issued
+  int ig = 0;       // tile entries handed to the MMA and softmax warps
   bool ok = true;
   for (int k = 0; ok; ++k) {
     const int w = item_index(k, total);
@@ -702,6 +714,18 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
     ++nq;
     TileIter it;
     it.init(p, im.qt, im.sparse, nqb_of(im));
+    auto publish = [&](int v) -> bool {
+      const int slot = ig & (NINFO - 1);
+      if (ig >= NINFO &&
+          !warp_wait(sh.bar(Smem::INFO_EMPTY0 + slot), static_cast<uint32_t>(ig / NINFO - 1) & 1u,
+                     sh, p))
+        return false;
+      if ((threadIdx.x & 31) == 0) st_shared_s32(sh.info(slot), v);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive_a(sh.bar(Smem::INFO_FULL0 + slot));
+      ++ig;
+      return true;
+    };
     auto load = [&](const CUtensorMap *map, int n) -> bool {
       const int slot = li % NSLOT;
       const uint32_t round = static_cast<uint32_t>(li / NSLOT);
@@ -713,13 +737,20 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
       ++li;
       return true;
     };
-    int n = 0;
-    uint32_t bits;
-    while (it.next(n, bits)) {
-      if (!load(tmK, n) || !load(tmV, n)) {
+    int n = 0, n2 = 0;
+    uint32_t bits = 0, bits2 = 0;
+    bool has = it.next(n, bits);
+    if (!has && im.sparse && !(ok = publish(0))) break;
+    while (has) {
+      const bool has2 = it.next(n2, bits2);
+      if ((im.sparse && !publish((n << 8) | (has2 ? 0 : 0x20) | 0x10 | static_cast<int>(bits))) ||
+          !load(tmK, n) || !load(tmV, n)) {
         ok = false;
         break;
       }
+      n = n2;
+      bits = bits2;
+      has = has2;
     }
   }
   if (warp_aborted(sh)) {  // let every copy this warp issued land before exit
@@ -741,6 +772,20 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   const uint64_t k_desc_base = smem_desc_sw128(sh.ring(0), 16, 1024);
   const uint64_t v_desc_base = smem_desc_sw128(sh.ring(0), HALF_BYTES, 1024);
   int ci = 0;         // ring slots consumed
+  int ig = 0;         // tile entries taken from the producer
+  // The next tile entry (0 on an abort, with ok = false).
+  auto take_info = [&](bool &okk) -> int {
+    const int slot = ig & (NINFO - 1);
+    if (!warp_wait(sh.bar(Smem::INFO_FULL0 + slot), static_cast<uint32_t>(ig / NINFO) & 1u, sh, p)) {
+      okk = false;
+      return 0;
+    }
+    const int v = ld_shared_s32(sh.info(slot));
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive_a(sh.bar(Smem::INFO_EMPTY0 + slot));
+    ++ig;
+    return v;
+  };
   int jp = 0;         // P tiles consumed (per tile index, both advance together)
   int done_items = 0; // items that produced an output (o_done / o_free phases)
   bool ok = true;
@@ -785,25 +830,33 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     const Item im = item_of(p, w);
     if (!(ok = warp_wait(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(k) & 1u, sh, p))) break;
     tc_fence_after_sync();
-    TileIter it;
-    it.init(p, im.qt, im.sparse, nqb_of(im));
-    int n = 0;
-    uint32_t bits;
-    if (!it.next(n, bits)) {          // no KV tile: Q is free again at once
-      tc_commit_w(sh.bar(Smem::Q_EMPTY));
-      continue;
+    bool has_next = im.qt > 0, has_next2 = false;     // full item: tiles 0..qt
+    if (im.sparse) {
+      const int e0 = take_info(ok);
+      if (!ok) break;
+      if (!(e0 & 0x10)) {             // no KV tile: Q is free again at once
+        tc_commit_w(sh.bar(Smem::Q_EMPTY));
+        continue;
+      }
+      has_next = (e0 & 0x20) == 0;
     }
     int k_slot = 0, v_slot = 0;
     if (!(ok = take(k_slot))) break;
     qk(0, k_slot);
     qk(1, k_slot);
     tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
-    bool has_next = it.next(n, bits);
     if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));     // the last QK of this item is issued
     for (int j = 0;; ++j) {
       if (!(ok = take(v_slot))) break;
       if (!(ok = pv(0, j == 0, v_slot))) break;
       if (has_next) {
+        if (im.sparse) {                      // tile j+1: is it the last?
+          const int e = take_info(ok);
+          if (!ok) break;
+          has_next2 = (e & 0x20) == 0;
+        } else {
+          has_next2 = j + 1 < im.qt;
+        }
         if (!(ok = take(k_slot))) break;
         qk(0, k_slot);
       } else {
@@ -818,7 +871,7 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       }
       qk(1, k_slot);
       tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
-      has_next = it.next(n, bits);
+      has_next = has_next2;
       if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));
     }
     ++done_items;
@@ -837,6 +890,7 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
   const uint32_t o_base = s_base + 128u;
   const float c = p.scale_log2;
   int js = 0;           // S tiles consumed (continues across items)
+  int ig = 0;           // tile entries taken from the producer
   int done_items = 0;   // items whose O this warpgroup has read
   bool ok = true;
   for (int k = 0; ok; ++k) {
@@ -845,11 +899,30 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
     const Item im = item_of(p, w);
     const int h = im.h0 + t;
     float m_run = -INFINITY, l_run = 0.f;
-    TileIter it;
-    it.init(p, im.qt, im.sparse, nqb_of(im));
     int j = 0, n = 0;
     uint32_t bits = 0;
-    while (it.next(n, bits)) {
+    bool last = false;
+    while (!last) {
+      if (!im.sparse) {   // a full item: tiles 0..qt
+        n = j;
+        bits = 0xFu;
+        last = j == im.qt;
+      } else {   // the next tile from the producer
+        const int slot = ig & (NINFO - 1);
+        if (!warp_wait(sh.bar(Smem::INFO_FULL0 + slot), static_cast<uint32_t>(ig / NINFO) & 1u, sh,
+                       p)) {
+          ok = false;
+          break;
+        }
+        const int v = ld_shared_s32(sh.info(slot));
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive_a(sh.bar(Smem::INFO_EMPTY0 + slot));
+        ++ig;
+        if (!(v & 0x10)) break;       // an item without tiles
+        n = v >> 8;
+        bits = static_cast<uint32_t>(v) & 15u;
+        last = (v & 0x20) != 0;
+      }
       if (!warp_wait(sh.bar(Smem::S_FULL0 + t), static_cast<uint32_t>(js) & 1u, sh, p)) {
         ok = false;
         break;
@@ -996,6 +1069,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init_a(sh.bar(Smem::O_FREE0 + t), 128);
     }
     mbar_init_a(sh.bar(Smem::DRAIN), 1);
+    for (int i = 0; i < NINFO; ++i) {
+      mbar_init_a(sh.bar(Smem::INFO_FULL0 + i), 1);
+      mbar_init_a(sh.bar(Smem::INFO_EMPTY0 + i), 1 + 8);   // the MMA warp + 8 softmax warps
+    }
     st_shared_s32(sh.abort_flag(), 0);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
