@@ -13,11 +13,15 @@
 // fp8: 1 box of 64 keys x 128 dims, 6 stages) into a ring; all threads
 // compute from shared memory:
 //   QK^T   thread = (key, 1/PARTS of the head dim), dot products for the G
-//          heads, reduced across the PARTS lanes with shuffles;
-//   softmax one warp per query head: running max / sum in log2 units;
+//          heads, reduced across the PARTS lanes by a butterfly that leaves
+//          each head's score on one lane, which also forms its probability
+//          2^(s - m) against a per-head reference max m (log2 units);
 //   PV     thread = (8 output dims, one of 16 key streams), G accumulators.
-// Each CTA writes its partial (max, sum, unnormalised output) per head; the
-// combine kernel merges the splits by log-sum-exp.
+// The reference only moves, for the whole CTA, on a tile holding a score more
+// than 16 above it (always the first): then the accumulators and row sums
+// are rescaled and the tile's probabilities redone.  One block barrier per
+// tile otherwise.  Each CTA writes its partial (reference, sum, unnormalised
+// output) per head; the combine kernel merges the splits by log-sum-exp.
 //
 // Paged cache: with a block table, tile n of sequence b is page
 // block_table[b][n] of a pool [num_pages, 64, Hkv, 128] (one page = one
@@ -41,9 +45,6 @@ constexpr int NT = 256;
 constexpr int RING_BYTES = 3 * 4 * BOX_BYTES;  // 96 KB of K/V in flight per CTA
 constexpr int MAX_STAGES = 6;
 constexpr int PAGE_CACHE = 256;                // page ids of a CTA's tiles kept in smem
-constexpr int SMEM_BYTES = 1024 + RING_BYTES + 8 * MAX_STAGES + 16 +
-                           /* scores */ 8 * 2 * KT * 4 + /* probs */ 2 * KT * 8 * 4 + 8 * 4 +
-                           /* page ids */ PAGE_CACHE * 4;
 
 // Per KV type: blocks (pages) per iteration, bytes of one block of K or V,
 // ring stages.  FP8 takes two blocks (128 keys) per iteration: half the
@@ -174,24 +175,55 @@ __device__ __noinline__ int page_of(const int32_t *block_table, int max_pages, i
   return pg;
 }
 
+// Shared memory of one decode CTA (offsets from a 1024-byte aligned base):
+// K/V ring | stage barriers | abort and re-reference flags | P pairs
+// (double-buffered [2][TK][G], each probability stored twice so a packed
+// FMA reads it as one 64-bit operand) | raw scores of a re-referenced tile
+// [G][TK] | per-head reference max and rescale factor, per-warp row sums |
+// page ids.
+template <int G, bool FP8>
+struct Lay {
+  static constexpr int TK = KvT<FP8>::TK;
+  static constexpr int FULL = RING_BYTES;
+  static constexpr int FLAGS = FULL + 8 * MAX_STAGES;
+  static constexpr int P2 = FLAGS + 16;
+  static constexpr int SRAW = P2 + 2 * TK * G * 8;
+  static constexpr int REF = SRAW + TK * G * 4;
+  static constexpr int PAGES = REF + (8 + 8 + 8 * 8) * 4;
+  static constexpr int BYTES = 1024 + PAGES + PAGE_CACHE * 4;
+};
+
+// A tile is scored against a fixed per-head reference max; only a score
+// more than kRefSlack (log2 units) above it, or the first tile, makes the
+// whole CTA move the reference (the rare path).  p <= 2^kRefSlack keeps
+// every fp32 sum far from overflow.
+constexpr float kRefSlack = 16.0f;
+
 template <int G, bool FP8, bool PAGED>
 __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const Params p) {
   using C = Cfg<G>;
   using T = KvT<FP8>;
+  using Y = Lay<G, FP8>;
   constexpr int NSTAGE = T::NST, STAGE_BYTES = T::STAGE, TK = T::TK, NB = T::NB;
   constexpr int PASSES = TK / C::KPP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *stages = base;
-  uint64_t *full = reinterpret_cast<uint64_t *>(base + RING_BYTES);
-  volatile int *abort = reinterpret_cast<volatile int *>(full + NSTAGE);
-  float *s_sm = reinterpret_cast<float *>(base + RING_BYTES + 8 * NSTAGE + 16);
-  float *p_sm = s_sm + 8 * TK;          // [TK][G]
-  float *alpha_sm = p_sm + TK * 8;      // [G]
-  int *page_sm = reinterpret_cast<int *>(alpha_sm + 8);   // [PAGE_CACHE]
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + Y::FULL);
+  volatile int *abort = reinterpret_cast<volatile int *>(base + Y::FLAGS);
+  // reref[i & 1]: some score of tile i passed its reference.  One flag per
+  // tile parity: a thread may already be scoring tile i+1 (and raising its
+  // flag) while another still reads tile i's.
+  volatile int *reref = abort + 1;
+  uint64_t *p2_sm = reinterpret_cast<uint64_t *>(base + Y::P2);
+  float *sraw_sm = reinterpret_cast<float *>(base + Y::SRAW);
+  float *mref_sm = reinterpret_cast<float *>(base + Y::REF);   // [8]
+  float *alpha_sm = mref_sm + 8;                                // [8]
+  float *lsum_sm = alpha_sm + 8;                                // [8 warps][G]
+  int *page_sm = reinterpret_cast<int *>(base + Y::PAGES);     // [PAGE_CACHE]
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -210,8 +242,11 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
   if (tid == 0) {
     for (int i = 0; i < NSTAGE; ++i) mbar_init(&full[i], 1);
     *abort = 0;
+    reref[0] = 0;
+    reref[1] = 0;
     fence_mbar_init();
   }
+  if (tid < 8) mref_sm[tid] = -INFINITY;
   // Page ids of this CTA's tiles (paged cache), read once by all threads.
   if constexpr (PAGED) {
     for (int i = tid; i < nblocks && i < PAGE_CACHE; i += NT)
@@ -256,15 +291,26 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     for (int i = 0; i < NSTAGE && i < ntiles; ++i) issue(i);
   }
 
-  // Query slice of this thread for QK^T, pre-scaled by scale*log2(e) (and
-  // by the K dequantisation scale of this KV head).
+  // QK^T: the PARTS threads of a key each hold G partial dot products.  Slot
+  // j of this thread accumulates query head j ^ hsel, where bit s of `part`
+  // contributes G >> (s+1) to hsel: then a butterfly that at each step keeps
+  // the lower half of the slots and sends the upper half sums every head with
+  // G - 1 shuffles and no selects, leaving head hsel's total in slot 0.
   const int part = tid % C::PARTS;
+  int hsel = 0;
+#pragma unroll
+  for (int s = 0; (G >> (s + 1)) > 0; ++s)
+    if ((part >> s) & 1) hsel |= G >> (s + 1);
+  const bool writer = part < G;   // one thread per (key, head) scores it
+  // Query slice of this thread, pre-scaled by scale*log2(e) (and by the K
+  // dequantisation scale of this KV head).
   float qscale = p.scale_log2;
   if constexpr (FP8) qscale *= p.k_scale[kvh];
   uint64_t qr[G][C::DPT / 2];   // packed pairs of dims
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const __nv_bfloat16 *qrow = p.q + (static_cast<size_t>(b) * p.Hq + kvh * G + g) * HD + part * C::DPT;
+    const __nv_bfloat16 *qrow =
+        p.q + (static_cast<size_t>(b) * p.Hq + kvh * G + (g ^ hsel)) * HD + part * C::DPT;
 #pragma unroll
     for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
       float f[8];
@@ -281,7 +327,8 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[g][e] = 0ull;
-  float m_run = -INFINITY, l_run = 0.f;  // meaningful in warp g < G
+  float mref = -INFINITY;       // writer: reference max of head hsel (log2 units)
+  float l_part = 0.f;           // writer: its share of head hsel's row sum
 
   for (int i = 0; i < ntiles; ++i) {
     const int st = i % NSTAGE;
@@ -291,6 +338,7 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>(i / NSTAGE) & 1u, abort, p.status);
     const uint8_t *sK = stages + st * STAGE_BYTES;
     const uint8_t *sV = sK + T::KBYTES;
+    uint64_t *p2b = p2_sm + (i & 1) * TK * G;
     // Token position of key 0 of each block of this iteration (a missing
     // block: past every length, so its keys are masked).
     int key_base[NB];
@@ -298,7 +346,10 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     for (int h = 0; h < NB; ++h)
       key_base[h] = (NB * i + h < nblocks) ? tl.block(pos0 + NB * i + h) * KT : INT_MAX / 2;
 
-    // ---- scores
+    // ---- scores and probabilities against the reference
+    float s_keep[PASSES];
+    float l_tile = 0.f;           // writer: this tile's share, added once the reference holds
+    bool over = false;
 #pragma unroll
     for (int pass = 0; pass < PASSES; ++pass) {
       const int key = pass * C::KPP + tid / C::PARTS;
@@ -322,71 +373,102 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
         d[g] = lo + hi;
       }
 #pragma unroll
-      for (int off = 1; off < C::PARTS; off <<= 1)
+      for (int half = G / 2; half >= 1; half >>= 1)
 #pragma unroll
-        for (int g = 0; g < G; ++g) d[g] += __shfl_xor_sync(0xffffffffu, d[g], off);
-      if (part == 0) {
-        const bool valid = key_base[key / KT] + (key % KT) < L;
+        for (int j = 0; j < half; ++j)
+          d[j] += __shfl_xor_sync(0xffffffffu, d[j + half], G / (2 * half));
 #pragma unroll
-        for (int g = 0; g < G; ++g) s_sm[g * TK + key] = valid ? d[g] : -INFINITY;
+      for (int off = G; off < C::PARTS; off <<= 1)
+        d[0] += __shfl_xor_sync(0xffffffffu, d[0], off);
+      const bool valid = key_base[key / KT] + (key % KT) < L;
+      const float s = valid ? d[0] : -INFINITY;
+      s_keep[pass] = s;
+      if (writer) {
+        const bool up = s > mref + kRefSlack;
+        over |= up;
+        const float pj = (up || s == -INFINITY) ? 0.f : ex2(s - mref);
+        l_tile += pj;
+        p2b[key * G + hsel] = f2_make(pj, pj);
       }
     }
+    if (over) reref[i & 1] = 1;
     // Past this barrier every thread is done with tile i-1 (its PV came before
     // these scores), so its stage takes tile i-1+NSTAGE.
     if (__syncthreads_or(!ok)) break;
     if (tid == 0 && i >= 1 && i - 1 + NSTAGE < ntiles) issue(i - 1 + NSTAGE);
 
-    // ---- online softmax, one warp per query head (TK / 32 keys per lane)
-    if (warp < G) {
-      constexpr int KL = TK / 32;
-      float v[KL];
+    // ---- rare: move the reference to the running max, rescale, redo P
+    if (reref[i & 1]) {
+      if (writer) {
 #pragma unroll
-      for (int j = 0; j < KL; ++j) v[j] = s_sm[warp * TK + lane + 32 * j];
-      float mt = v[0];
-#pragma unroll
-      for (int j = 1; j < KL; ++j) mt = fmaxf(mt, v[j]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-      const float m_new = fmaxf(m_run, mt);
-      const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      float ps = 0.f;
-#pragma unroll
-      for (int j = 0; j < KL; ++j) {
-        const float pj = ex2(v[j] - m_use);
-        ps += pj;
-        p_sm[(lane + 32 * j) * G + warp] = pj;
+        for (int pass = 0; pass < PASSES; ++pass)
+          sraw_sm[hsel * TK + pass * C::KPP + tid / C::PARTS] = s_keep[pass];
       }
+      __syncthreads();
+      if (tid == 0) reref[i & 1] = 0;   // every thread read it before this barrier; the
+                                        // next write to it comes after the next tile's barrier
+      if (warp < G) {
+        float mt = -INFINITY;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-      l_run = l_run * alpha + ps;
-      m_run = m_new;
-      if (lane == 0) alpha_sm[warp] = alpha;
+        for (int j = lane; j < TK; j += 32) mt = fmaxf(mt, sraw_sm[warp * TK + j]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        if (lane == 0) {
+          const float mo = mref_sm[warp];
+          const float mn = fmaxf(mo, mt);
+          alpha_sm[warp] = (mo == -INFINITY) ? 0.f : ex2(mo - mn);
+          mref_sm[warp] = mn;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const uint64_t a2 = f2_make(alpha_sm[g], alpha_sm[g]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[g][e] = f2_mul(acc[g][e], a2);
+      }
+      if (writer) {
+        l_part *= alpha_sm[hsel];
+        mref = mref_sm[hsel];
+#pragma unroll
+        for (int pass = 0; pass < PASSES; ++pass) {
+          const float s = s_keep[pass];
+          const float pj = (s == -INFINITY) ? 0.f : ex2(s - mref);
+          l_part += pj;
+          p2b[(pass * C::KPP + tid / C::PARTS) * G + hsel] = f2_make(pj, pj);
+        }
+      }
+      __syncthreads();
+    } else {
+      l_part += l_tile;
     }
-    __syncthreads();
 
-    // ---- O += P V
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const uint64_t a2 = f2_make(alpha_sm[g], alpha_sm[g]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[g][e] = f2_mul(acc[g][e], a2);
-    }
+    // ---- O += P V (P of the G heads of a key: G packed pairs, 16-byte loads)
 #pragma unroll
     for (int kk = 0; kk < TK / 16; ++kk) {
       const int key = ks + 16 * kk;
       uint64_t v2[4];
       load8<FP8>(sV, key, dc, v2);
+      if constexpr (G == 1) {
+        const uint64_t pg = p2b[key];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float pg = p_sm[key * G + g];
-        const uint64_t p2 = f2_make(pg, pg);
+        for (int e = 0; e < 4; ++e) acc[0][e] = f2_fma(pg, v2[e], acc[0][e]);
+      } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[g][e] = f2_fma(p2, v2[e], acc[g][e]);
+        for (int g2 = 0; g2 < G / 2; ++g2) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(p2b + key * G + 2 * g2);
+          const uint64_t pa = (static_cast<uint64_t>(w.y) << 32) | w.x;
+          const uint64_t pb = (static_cast<uint64_t>(w.w) << 32) | w.z;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * g2][e] = f2_fma(pa, v2[e], acc[2 * g2][e]);
+            acc[2 * g2 + 1][e] = f2_fma(pb, v2[e], acc[2 * g2 + 1][e]);
+          }
+        }
       }
     }
   }
-  __syncthreads();   // every thread is done with the stages (reused below) and p_sm
+  __syncthreads();   // every thread is done with the stages (reused below)
 
   if (*abort) {  // let the copies still in flight land, then leave
     if (tid == 0) {
@@ -396,6 +478,11 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     __syncthreads();
     return;
   }
+
+  // ---- row sums: the writers of a head share `part`; one total per warp
+#pragma unroll
+  for (int off = C::PARTS; off < 32; off <<= 1) l_part += __shfl_xor_sync(0xffffffffu, l_part, off);
+  if (lane < G) lsum_sm[warp * G + hsel] = l_part;   // lane < G: part = lane, a writer
 
   // ---- reduce the 16 key streams through shared memory (stage buffers free)
   float *red = reinterpret_cast<float *>(stages);   // [16][G][HD]
@@ -419,10 +506,13 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     for (int s = 0; s < 16; ++s) sum += red[(s * G + g) * HD + dd];
     p.o_part[(row0 + static_cast<size_t>(g) * p.nsplit) * HD + dd] = sum * vs;
   }
-  if (warp < G && lane == 0) {
-    float *ml = p.ml_part + (row0 + static_cast<size_t>(warp) * p.nsplit) * 2;
-    ml[0] = m_run;
-    ml[1] = l_run;
+  if (tid < G) {
+    float l = 0.f;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) l += lsum_sm[w * G + tid];
+    float *ml = p.ml_part + (row0 + static_cast<size_t>(tid) * p.nsplit) * 2;
+    ml[0] = mref_sm[tid];
+    ml[1] = l;
   }
 }
 
@@ -552,27 +642,28 @@ int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
   p.v_scale = a.fp8 ? a.v_scale : nullptr;
   const dim3 grid(ns, a.Hkv, a.B);
   void (*kern)(const CUtensorMap, const CUtensorMap, const Params) = nullptr;
+  int smem = 0;
   // FP8 caches are always paged (a contiguous cache is the identity table).
   if (a.fp8 && !paged) return FA_ERR_UNSUPPORTED;
   switch (G * 4 + (a.fp8 ? 2 : 0) + (paged ? 1 : 0)) {
-    case 4: kern = decode_kernel<1, false, false>; break;
-    case 8: kern = decode_kernel<2, false, false>; break;
-    case 16: kern = decode_kernel<4, false, false>; break;
-    case 32: kern = decode_kernel<8, false, false>; break;
-    case 5: kern = decode_kernel<1, false, true>; break;
-    case 9: kern = decode_kernel<2, false, true>; break;
-    case 17: kern = decode_kernel<4, false, true>; break;
-    case 33: kern = decode_kernel<8, false, true>; break;
-    case 7: kern = decode_kernel<1, true, true>; break;
-    case 11: kern = decode_kernel<2, true, true>; break;
-    case 19: kern = decode_kernel<4, true, true>; break;
-    case 35: kern = decode_kernel<8, true, true>; break;
+    case 4: kern = decode_kernel<1, false, false>, smem = Lay<1, false>::BYTES; break;
+    case 8: kern = decode_kernel<2, false, false>, smem = Lay<2, false>::BYTES; break;
+    case 16: kern = decode_kernel<4, false, false>, smem = Lay<4, false>::BYTES; break;
+    case 32: kern = decode_kernel<8, false, false>, smem = Lay<8, false>::BYTES; break;
+    case 5: kern = decode_kernel<1, false, true>, smem = Lay<1, false>::BYTES; break;
+    case 9: kern = decode_kernel<2, false, true>, smem = Lay<2, false>::BYTES; break;
+    case 17: kern = decode_kernel<4, false, true>, smem = Lay<4, false>::BYTES; break;
+    case 33: kern = decode_kernel<8, false, true>, smem = Lay<8, false>::BYTES; break;
+    case 7: kern = decode_kernel<1, true, true>, smem = Lay<1, true>::BYTES; break;
+    case 11: kern = decode_kernel<2, true, true>, smem = Lay<2, true>::BYTES; break;
+    case 19: kern = decode_kernel<4, true, true>, smem = Lay<4, true>::BYTES; break;
+    case 35: kern = decode_kernel<8, true, true>, smem = Lay<8, true>::BYTES; break;
     default: return FA_ERR_UNSUPPORTED;
   }
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FA_ERR_CUDA;
-  kern<<<grid, NT, SMEM_BYTES, stream>>>(tmK, tmV, p);
+  kern<<<grid, NT, smem, stream>>>(tmK, tmV, p);
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   combine_kernel<<<dim3(a.Hq, a.B), 128, 0, stream>>>(
       p.o_part, p.ml_part, reinterpret_cast<__nv_bfloat16 *>(a.o), a.lse, a.Hq, ns);

@@ -13,8 +13,12 @@ from tests.gpu_util import LSE_ABS_TOL, assert_close_attention, to_f64, zero_sta
 pytestmark = pytest.mark.gpu
 
 
-def _decode_case(B, Lmax, Hq, Hkv, seqlens, mode, sink, window, seed, mode_dev=None):
+def _decode_case(B, Lmax, Hq, Hkv, seqlens, mode, sink, window, seed, mode_dev=None, spikes=()):
     q, kc, vc = inputs.decode_inputs(B, Lmax, Hq, Hkv, 128, seed)
+    G = Hq // Hkv
+    for b, lo, hi, g, factor in spikes:   # keys lo..hi-1 of batch b pulled towards query head g
+        kc[b, lo:hi, g // G] = (kc[b, lo:hi, g // G].float()
+                                + factor * q[b, g].float()).to(torch.bfloat16)
     sl = torch.tensor(seqlens, dtype=torch.int32)
     status = zero_status()
     lse = torch.empty(B, Hq, device="cuda", dtype=torch.float32)
@@ -72,3 +76,17 @@ def test_decode_sparse_reads_only_its_blocks():
     torch.cuda.synchronize()
     assert torch.equal(clean, dirty)
     assert (full.float() - clean_full.float()).abs().max() > 100.0
+
+
+@pytest.mark.parametrize("mode", [capi.FA_MODE_FULL, capi.FA_MODE_SPARSE])
+def test_decode_rising_score_plateaus(mode):
+    """Runs of keys pulled towards one query head so that their scores sit
+    about 26 and then 45 (log2 units) above the rest, starting in the middle
+    of a split and lasting to the end, plus one sink key at about 33: the
+    splits meet scores far above what they have seen on later tiles, not only
+    the first, and every key after the jump still carries weight; the other
+    heads of the group see moderately raised scores.  Against the oracle."""
+    L = 3000
+    plateaus = [(0, 700, L, 1, 1.6), (0, 2050, L, 1, 1.2),       # 1.6, then 2.8 in all
+                (1, 140, L, 6, 1.6), (1, 5, 6, 6, 2.0)]
+    _decode_case(2, L, 8, 2, [L, L - 74], mode, 128, 512, seed=24, spikes=plateaus)
