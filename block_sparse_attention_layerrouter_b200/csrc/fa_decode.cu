@@ -302,6 +302,14 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
   for (int s = 0; (G >> (s + 1)) > 0; ++s)
     if ((part >> s) & 1) hsel |= G >> (s + 1);
   const bool writer = part < G;   // one thread per (key, head) scores it
+  // Chunk (8 dims) of the head dim for step c8 of this thread's QK^T.  bf16:
+  // chunk c8*PARTS + part, so the 8 lanes of a key that share a shared-memory
+  // phase read 8 different swizzled slots of one box (no bank conflicts).
+  // FP8: the thread's chunks are adjacent (a conflict-free order measured
+  // slower there: it costs registers).
+  auto chunk_of = [&](int c8) {
+    return FP8 ? part * (C::DPT / 8) + c8 : c8 * C::PARTS + part;
+  };
   // Query slice of this thread, pre-scaled by scale*log2(e) (and by the K
   // dequantisation scale of this KV head).
   float qscale = p.scale_log2;
@@ -310,11 +318,11 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const __nv_bfloat16 *qrow =
-        p.q + (static_cast<size_t>(b) * p.Hq + kvh * G + (g ^ hsel)) * HD + part * C::DPT;
+        p.q + (static_cast<size_t>(b) * p.Hq + kvh * G + (g ^ hsel)) * HD;
 #pragma unroll
     for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
       float f[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + c8 * 8), f);
+      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + chunk_of(c8) * 8), f);
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         qr[g][c8 * 4 + e] = f2_make(f[2 * e] * qscale, f[2 * e + 1] * qscale);
@@ -359,7 +367,7 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 #pragma unroll
       for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
         uint64_t k2[4];
-        load8<FP8>(sK, key, part * (C::DPT / 8) + c8, k2);
+        load8<FP8>(sK, key, chunk_of(c8), k2);
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll

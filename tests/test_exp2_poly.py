@@ -1,4 +1,5 @@
-"""The FMA-pipe exp2 used for a share of the softmax in the prefill kernel:
+"""The FMA-pipe exp2 the prefill kernel can use for a share of the softmax
+(a compile-time share, 0 by default):
 range reduction x = n + f with the 1.5*2^23 shifter, a degree-3 polynomial
 for 2^f on [-1/2, 1/2], n added to the exponent field.  The constants are
 read from the kernel source and the routine is replayed in fp32 numpy, op
