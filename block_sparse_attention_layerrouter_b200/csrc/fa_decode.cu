@@ -63,7 +63,7 @@ struct KvT {
 struct Params {
   const __nv_bfloat16 *q;
   float *o_part;    // [B, Hq, nsplit, HD]
-  float *ml_part;   // [B, Hq, nsplit, 2] (max, sum) in log2 units
+  float *ml_part;   // [B, Hq, nsplit, 2] (reference max, sum relative to it), log2 units
   const int32_t *seqlens;
   const int32_t *mode;
   int32_t *status;

@@ -143,7 +143,9 @@ FA_API int fa_attn_prefill_blocksparse(const void *q, const void *k, const void 
  *   (e.g. the router's mode_out) read on the device.
  *   o bf16 [B, Hq, D]; lse fp32 [B, Hq] or NULL.
  *   workspace >= fa_decode_workspace_size(B, Hq, Hkv, Lmax, D) bytes, device.
- * Split-KV: partial (max, sum, output) per split, merged by log-sum-exp. */
+ * Split-KV: each split keeps (reference max, sum, output) with sums relative
+ * to its reference; the splits are merged by log-sum-exp, which is exact for
+ * any reference at or below the split's true max. */
 FA_API size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
 FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
                    const int32_t *seqlens, int B, int Lmax, int Hq, int Hkv,
