@@ -236,7 +236,6 @@ class Step:
         self.seqlens = torch.full((B,), S, dtype=torch.int32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.capi = capi
-        self.launches = 1 + 4 * n_layers + (2 * n_layers if with_decode else 0)
 
     def run(self, ev=None):
         """Enqueue one step.  ev: optional {layer: (start, end)} events
@@ -376,10 +375,12 @@ def run_ours(args, wl):
     ev_full = [{full_layer: (torch.cuda.Event(enable_timing=True),
                              torch.cuda.Event(enable_timing=True))} for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_launch0 = capi.kernel_launches()
     t0.record()
     for i in range(args.steps):
         sets[i % n_sets].run(ev_full[i])
     t1.record()
+    n_launch = capi.kernel_launches() - n_launch0   # kernels enqueued in the timed loop
     sync_all(ws)
     sampler.stop()
     ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
@@ -450,7 +451,7 @@ def run_ours(args, wl):
         traffic_workload=traffic_wl, algorithmic_flops_per_launch=f_full,
         avg_launch_ms=round(avg_full_ms, 4))
     line["e2e"] = e2e
-    line["gpu_launches"] = s0.launches * args.steps
+    line["gpu_launches"] = n_launch
     line["components"] = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in comp.items()}
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
@@ -583,10 +584,12 @@ def run_decode(args, wl):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_launch0 = capi.kernel_launches()
     t0.record()
     for i in range(args.steps):
         step(evs[i])
     t1.record()
+    n_launch = capi.kernel_launches() - n_launch0   # kernels enqueued in the timed loop
     sync_all(ws)
     sampler.stop()
     ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
@@ -655,7 +658,7 @@ def run_decode(args, wl):
                    "unit": "GB/s", "h2d_bytes_per_step": sum(t.numel() * 2 for t in hq),
                    "d2h_bytes_per_step": sum(t.numel() * 2 for t in ho),
                    "note": "KV caches are device-resident decode state"}
-    line["gpu_launches"] = 2 * wl.layers * args.steps
+    line["gpu_launches"] = n_launch
     line["clocks"] = sampler.report()
     line["components"] = {
         "decode_full_layer_ms": round(full_ms, 4), "decode_sparse_layer_ms": round(sparse_ms, 4),
@@ -712,10 +715,12 @@ def run_varlen(args, wl):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_launch0 = capi.kernel_launches()
     t0.record()
     for i in range(args.steps):
         step(evs[i])
     t1.record()
+    n_launch = capi.kernel_launches() - n_launch0   # kernels enqueued in the timed loop
     sync_all(ws)
     sampler.stop()
     ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
@@ -754,7 +759,7 @@ def run_varlen(args, wl):
     line["all_full_ms"] = round(full_ms, 4)
     line["routed_speedup_vs_all_full"] = round(full_ms / (ms / args.steps), 3)
     line["e2e"] = None
-    line["gpu_launches"] = 6 * args.steps
+    line["gpu_launches"] = n_launch
     return line
 
 
@@ -802,10 +807,12 @@ def run_train(args, wl):
         step()
     sync_all(ws)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_launch0 = capi.kernel_launches()
     t0.record()
     for _ in range(args.steps):
         step()
     t1.record()
+    n_launch = capi.kernel_launches() - n_launch0   # kernels enqueued in the timed loop
     sync_all(ws)
     sampler.stop()
     ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
@@ -835,7 +842,7 @@ def run_train(args, wl):
         kernel="backward::bwd_kernel (FULL, alone)", traffic=None,
         algorithmic_flops_per_launch=2.5 * f_full, avg_launch_ms=round(bwd_full_ms, 4))
     line["e2e"] = None
-    line["gpu_launches"] = None
+    line["gpu_launches"] = n_launch
     return line
 
 

@@ -46,6 +46,7 @@ _SZ = ctypes.c_size_t
 _SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
+    "fa_kernel_launches": (ctypes.c_ulonglong, []),
     "fa_router_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_router_decide": (_I, [_VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _I, _VP, _VP, _VP, _VP,
                               _VP, _SZ, _VP]),
@@ -111,6 +112,12 @@ def lib():
 
 def status_string(status: int) -> str:
     return lib().fa_status_string(int(status)).decode()
+
+
+def kernel_launches() -> int:
+    """Kernels this library has enqueued in this process so far (host-side
+    count; no GPU access)."""
+    return int(lib().fa_kernel_launches())
 
 
 def _check(name: str, rc: int):

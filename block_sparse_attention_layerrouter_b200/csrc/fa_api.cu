@@ -4,9 +4,14 @@
 #include "fa_common.cuh"
 #include "fa_internal.h"
 
+#include <atomic>
 #include <mutex>
 
 namespace fa {
+
+static std::atomic<unsigned long long> g_kernel_launches{0};
+void note_launch() { g_kernel_launches.fetch_add(1, std::memory_order_relaxed); }
+
 namespace {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -142,6 +147,10 @@ FA_API const char *fa_status_string(int status) {
 }
 
 FA_API int fa_version(void) { return 100; }
+
+FA_API unsigned long long fa_kernel_launches(void) {
+  return g_kernel_launches.load(std::memory_order_relaxed);
+}
 
 FA_API size_t fa_router_workspace_size(int B, int Hq, int D, int hidden) {
   if (B <= 0 || Hq <= 0 || D <= 0 || hidden <= 0) return 0;

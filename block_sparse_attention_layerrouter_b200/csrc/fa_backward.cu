@@ -930,6 +930,7 @@ int run_prep(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
   prep_kernel<<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16 *>(a.o), reinterpret_cast<const __nv_bfloat16 *>(a.dout),
       a.lse, a.B, a.S, pl.Sp, a.Hq, pl.dvec, pl.lse2, pl.acc, a.zero_dq_acc);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -941,12 +942,15 @@ int run_csc(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
   using namespace backward;
   const unsigned blocks = static_cast<unsigned>((pl.nkt + 7) / 8);
   csc_count_kernel<<<blocks, 256, 0, stream>>>(a.row_ptr, a.col_idx, pl.nqb, pl.nkt, pl.ct_ptr);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   csc_scan_kernel<<<1, 1024, 0, stream>>>(a.row_ptr, a.col_idx, pl.nqb, pl.nkt, pl.ct_ptr,
                                           a.status);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   csc_fill_kernel<<<blocks, 256, 0, stream>>>(a.row_ptr, a.col_idx, pl.nqb, pl.nkt, pl.ct_ptr,
                                               pl.ct_q);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -1013,15 +1017,18 @@ int run_main(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
   if (p.cmax > 1) {
     zero4_kernel<<<static_cast<unsigned>(4 * sms), 256, 0, stream>>>(
         reinterpret_cast<float4 *>(pl.dkv_acc), n4);
+    note_launch();
     if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   const int ctas = static_cast<int>(total < sms ? total : sms);
   bwd_kernel<<<ctas, NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmO, tmK, tmV, tmA, p,
                                                         static_cast<int>(total));
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (p.cmax > 1) {
     const long long rows = static_cast<long long>(a.B) * a.S * a.Hkv;
     dkv_convert_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+    note_launch();
     if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
@@ -1036,6 +1043,7 @@ int run_convert(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
   convert_kernel<<<static_cast<unsigned>(blocks < 4 * sms ? blocks : 4 * sms), 256, 0, stream>>>(
       pl.acc, reinterpret_cast<__nv_bfloat16 *>(a.dq), a.B, a.S, pl.Sp, a.Hq, a.scale, a.pool_dx,
       a.n_head, a.n_tail);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -1105,6 +1113,7 @@ int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream) {
   float *r = a.r_out ? a.r_out : sp.r;
   if (int rc = launch_router_soft(sp.logits, a.gumbel, a.B, a.tau, r, stream)) return rc;
   zero_kernel<<<(a.B + 255) / 256, 256, 0, stream>>>(sp.dr, a.B);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   const long long per_b = static_cast<long long>(a.Hq) * sp.att.Sp;
   const unsigned dsum_blocks = static_cast<unsigned>(per_b / 4096 + 1 < 64 ? per_b / 4096 + 1 : 64);
@@ -1117,6 +1126,7 @@ int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream) {
   fa.zero_dq_acc = 1;
   if (int rc = run_prep(fa, sp.att, stream)) return rc;
   dsum_kernel<<<dim3(dsum_blocks, a.B), 256, 0, stream>>>(sp.att.dvec, per_b, 1.0f, sp.dr);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (int rc = run_main(fa, sp.att, stream)) return rc;
 
@@ -1130,6 +1140,7 @@ int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream) {
   sa.zero_dq_acc = 0;
   if (int rc = run_prep(sa, sp.att, stream)) return rc;
   dsum_kernel<<<dim3(dsum_blocks, a.B), 256, 0, stream>>>(sp.att.dvec, per_b, -1.0f, sp.dr);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (int rc = run_csc(sa, sp.att, stream)) return rc;
   if (int rc = run_main(sa, sp.att, stream)) return rc;

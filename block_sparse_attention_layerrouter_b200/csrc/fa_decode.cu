@@ -672,9 +672,11 @@ int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
       cudaSuccess)
     return FA_ERR_CUDA;
   kern<<<grid, NT, smem, stream>>>(tmK, tmV, p);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   combine_kernel<<<dim3(a.Hq, a.B), 128, 0, stream>>>(
       p.o_part, p.ml_part, reinterpret_cast<__nv_bfloat16 *>(a.o), a.lse, a.Hq, ns);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -730,6 +732,7 @@ int launch_kv_append(const KvAppendLaunch &a, cudaStream_t stream) {
       reinterpret_cast<const __nv_bfloat16 *>(a.v_new), reinterpret_cast<uint8_t *>(a.k_pages),
       reinterpret_cast<uint8_t *>(a.v_pages), a.fp8, a.k_scale, a.v_scale, a.block_table,
       a.max_pages, a.num_pages, a.seqlens, a.Hkv, a.status);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

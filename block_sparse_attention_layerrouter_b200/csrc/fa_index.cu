@@ -68,6 +68,7 @@ long long index_nnz(int nrows, int sb, int wb) {
 int launch_index(int nrows, int sb, int wb, int32_t *row_ptr, int32_t *col_idx,
                  cudaStream_t stream) {
   index::csr_kernel<<<1, index::NT, 0, stream>>>(nrows, sb, wb, row_ptr, col_idx);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

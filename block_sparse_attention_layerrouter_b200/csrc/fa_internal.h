@@ -155,6 +155,9 @@ struct SoftBackwardLaunch {
 size_t soft_backward_workspace_bytes(int B, int S, int Hq, int Hkv, int hidden);
 int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream);
 
+// Counts one kernel launch (the total is fa_kernel_launches()).
+void note_launch();
+
 long long index_nnz(int nrows, int sb, int wb);
 int launch_index(int nrows, int sb, int wb, int32_t *row_ptr, int32_t *col_idx,
                  cudaStream_t stream);

@@ -1224,6 +1224,7 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
     p.items = ws + 64;
     prefill2::varlen_items_kernel<<<1, 1024, 0, stream>>>(
         a.cu_seqlens, a.B, static_cast<int>(max_items), ws, ws + 64, a.status);
+    note_launch();
     if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
     grid = max_items * (a.Hq / 2);   // upper bound; the kernel reads the real count
   }
@@ -1241,10 +1242,12 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
     const int ctas = static_cast<int>(grid < cap ? grid : cap);
     prefill2::prefill2_kernel<<<ctas, prefill2::NUM_THREADS, prefill2::SMEM_BYTES, stream>>>(
         tmQ, tmK, tmV, p, static_cast<int>(grid));
-  }
-  else
+    note_launch();
+  } else {
     prefill_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmK,
                                                                                     tmV, p);
+    note_launch();
+  }
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -295,6 +295,7 @@ int launch_soft_mix(const void *o_full, const void *o_sparse, const float *r, vo
                        stream>>>(reinterpret_cast<const __nv_bfloat16 *>(o_full),
                                  reinterpret_cast<const __nv_bfloat16 *>(o_sparse), r,
                                  reinterpret_cast<__nv_bfloat16 *>(y), per_b, B);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -313,21 +314,26 @@ int launch_router_backward(const RouterBwdLaunch &a, cudaStream_t stream) {
   const long long n = static_cast<long long>(a.B) * in_f;
   pooled_kernel<<<static_cast<unsigned>((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184), 256, 0,
                   stream>>>(part, a.x, a.B, in_f, 1.0f / static_cast<float>(a.n_sel));
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   head_bwd_kernel<<<a.hidden, 128, 0, stream>>>(a.logits, a.gumbel, 1.0f / a.tau, a.dr, hid, a.w2,
                                                 a.B, a.hidden, a.dlogits, a.da, a.dw2, a.db1,
                                                 a.db2);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   dw1_kernel<<<a.hidden, 256, 0, stream>>>(a.da, a.x, a.B, in_f, a.hidden, a.dw1);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   dx_kernel<<<dim3((in_f + 31) / 32, a.B), 256, 0, stream>>>(a.da, a.w1, a.B, in_f, a.hidden,
                                                               a.dx);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int launch_router_soft(const float *logits, const float *gumbel, int B, float tau, float *r,
                        cudaStream_t stream) {
   router::soft_kernel<<<(B + 127) / 128, 128, 0, stream>>>(logits, gumbel, 1.0f / tau, r, B);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -352,11 +358,14 @@ int launch_router(const RouterLaunch &a, cudaStream_t stream) {
   pool_kernel<<<dim3(a.Hq, a.B, kPoolSlices), 256, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16 *>(a.q), part, a.S, a.Hq, a.n_head, a.n_tail,
       a.cu_seqlens);
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   hidden_kernel<<<dim3(a.hidden, a.B), 256, xs_bytes, stream>>>(
       part, a.w1, a.b1, hid, in_f, a.hidden, 1.0f / static_cast<float>(a.n_head + a.n_tail));
+  note_launch();
   if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
   head_kernel<<<a.B, 64, 0, stream>>>(hid, a.w2, a.b2, a.logits, a.mode, a.hidden);
+  note_launch();
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

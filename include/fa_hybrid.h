@@ -80,6 +80,13 @@ FA_API const char *fa_status_string(int status);
 /* Library ABI version (major * 100 + minor). */
 FA_API int fa_version(void);
 
+/* Number of kernels this library has enqueued in this process so far, on
+ * any stream and device (a host-side count taken at each launch; calls
+ * rejected by their host-side checks launch nothing and add nothing).  For
+ * callers that report how many kernels a step ran: read it before and after.
+ * Thread-safe; never touches the GPU. */
+FA_API unsigned long long fa_kernel_launches(void);
+
 /* ------------------------------------------------------------ router ---
  * "Flux Attention", router paragraphs: pool tokens [0, n_head) and
  * [S - n_tail, S) of Q (mean, fp32), flatten head-major to x[h*D + d],

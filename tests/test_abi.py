@@ -152,3 +152,17 @@ def test_paged_decode_entries_reject_on_host(lib):
 def test_soft_mix_rejects_on_host(lib):
     assert lib.fa_soft_mix(_P, _P, _P, _N, 1, 8, 2, 128, _N) == -1
     assert lib.fa_soft_mix(_P, _P, _P, _P, 1, 8, 2, 64, _N) == -2
+
+
+def test_host_rejections_launch_nothing(lib):
+    """The launch counter is host-side (readable without a GPU) and calls
+    rejected by their host-side checks add nothing to it."""
+    before = capi.kernel_launches()
+    p = ctypes.c_void_p(4096)
+    c = capi.cfg(64, 128, 2048)
+    assert lib.fa_attn_prefill_full(None, p, p, p, None, 1, 128, 4, 4, 128, 0.1, None,
+                                    None) == -1
+    ws = lib.fa_decode_workspace_size(8, 32, 8, 131072, 128)
+    assert lib.fa_attn_decode(p, p, p, p, 8, 131072, 32, 8, 128, 0.1, 0, None, c, p, None, p,
+                              ws - 1, None, None) == -3
+    assert capi.kernel_launches() == before
