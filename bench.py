@@ -133,6 +133,12 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- helpers
+# Spec figures, reported beside the measured-peak fractions: dense bf16 tensor
+# throughput of one B200 and its HBM3e bandwidth (~8 TB/s).
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+
+
 def tensor_peak(clocks, peak_burst, peak_sust, peak_kind):
     """The bf16 denominator that matches the clocks the kernel ran at: the
     sustained GEMM figure (measured back to back under the power cap) only
@@ -153,7 +159,16 @@ def roofline_tensor(achieved, clocks, peaks, **extra):
     alt_name, alt_peak = next(iter(other.items()))
     line = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4), "peak_kind": kind,
-            alt_name.replace("_at", ""): round(achieved / alt_peak, 4)}
+            alt_name.replace("_at", ""): round(achieved / alt_peak, 4),
+            "frac_of_nominal": round(achieved / NOMINAL_BF16_TFLOPS, 4)}
+    line.update(extra)
+    return line
+
+
+def roofline_hbm(achieved, hbm, peak_kind, **extra):
+    line = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "peak_kind": "%s HBM copy" % peak_kind,
+            "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4)}
     line.update(extra)
     return line
 
@@ -649,11 +664,9 @@ def run_decode(args, wl):
                           DECODE_CACHE_SETS,
                           2 * caches[0][0].numel() * caches[0][0].element_size() / 1e9)}
     achieved = full_bytes / (full_ms * 1e-3) / 1e9
-    line["roofline"] = {"bound": "hbm", "kernel": "decode_kernel + combine (a FULL layer)",
-                        "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                        "frac": round(achieved / hbm, 4), "peak_kind": "%s HBM copy" % peak_kind,
-                        "traffic": None, "algorithmic_bytes_per_launch": full_bytes,
-                        "avg_launch_ms": round(full_ms, 4)}
+    line["roofline"] = roofline_hbm(
+        achieved, hbm, peak_kind, kernel="decode_kernel + combine (a FULL layer)", traffic=None,
+        algorithmic_bytes_per_launch=full_bytes, avg_launch_ms=round(full_ms, 4))
     line["e2e"] = {"value": round(ws * step_bytes / (ms_e2e / args.steps * 1e-3) / 1e9, 1),
                    "unit": "GB/s", "h2d_bytes_per_step": sum(t.numel() * 2 for t in hq),
                    "d2h_bytes_per_step": sum(t.numel() * 2 for t in ho),

@@ -27,3 +27,11 @@ def test_sustained_peak_only_when_power_capped_and_slow():
     # No clock record at all: burst.
     assert bench.roofline_tensor(1000.0, {"sm_mhz": None, "sm_max_mhz": None, "reasons": []},
                                  PEAKS)["peak"] == 1676.5
+
+
+def test_nominal_fractions_reported_beside_measured():
+    r = bench.roofline_tensor(1125.0, {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}, PEAKS)
+    assert r["frac_of_nominal"] == 0.5
+    h = bench.roofline_hbm(6000.0, 6546.9, "measured", kernel="k", traffic=None)
+    assert h["bound"] == "hbm" and h["frac"] == round(6000 / 6546.9, 4)
+    assert h["frac_of_nominal"] == 0.75 and h["kernel"] == "k" and h["traffic"] is None
