@@ -1,6 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the layer-routed hybrid attention hot path on B200.
 
+Default run (the headline): the 256K-context Qwen3-8B-shaped layer pair.
 One step = one pass of the whole hot path over one batch of the workload:
   * the CSR of the block pattern (fa_blocksparse_index),
   * two routed layers (fa_hybrid_layer: router pool -> MLP -> argmax on the
@@ -9,12 +10,15 @@ One step = one pass of the whole hot path over one batch of the workload:
   * one decode token per layer in that layer's mode (fa_attn_decode).
 value = algorithmic FLOPs of the step / time: full layer 4*D*Hq*B*S(S+1)/2,
 sparse layer 4*D*Hq*B*(exact attended pairs), decode 4*D*Hq*B*(keys read).
+The same line carries the 36-layer hybrid-vs-full projection, the 32-layer
+decode step in HBM GB/s ("decode") and the 8K-context layer's kernels
+("qwen3-4b-layer-s8192").
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                       [--workload NAME]
-Multi-GPU (torchrun): every rank runs an independent replica of the step on
-its own GPU (the path has no exchange step); value = all ranks' FLOPs / the
-slowest rank's time.
+                       [--workload NAME] [--dry-run]
+Multi-GPU: every rank runs an independent replica of the step on its own GPU
+(the path has no exchange step); value = all ranks' FLOPs / the slowest
+rank's time.  `--gpus N` outside torchrun starts the N ranks itself.
 """
 from __future__ import annotations
 
@@ -35,11 +39,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "prefill attn TFLOP/s & % bf16 peak; decode HBM GB/s; hybrid vs full at 256K"
-DEFAULT_WORKLOAD = "qwen3-4b-layer-s8192"
+DEFAULT_WORKLOAD = "qwen3-8b-layer-s262144"       # 256K prefill, one layer per mode
+DECODE_WORKLOAD = "decode-b8-l131072-32l"          # 32-layer decode step
+LAYER8K_WORKLOAD = "qwen3-4b-layer-s8192"          # Qwen3-4B layer at 8K
 N_INPUT_SETS = 4           # rotated so each step reads inputs not resident in L2
-KERNEL_SRC = os.path.join(ROOT, "block_sparse_attention_layerrouter_b200", "csrc",
-                          "fa_prefill.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "prefill_full_dram_traffic.txt")
+CSRC = os.path.join(ROOT, "block_sparse_attention_layerrouter_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "prefill2_kernel_full_dram_traffic.txt")
 
 
 # ------------------------------------------------------------ accounting
@@ -182,23 +187,40 @@ def measured_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def kernel_traffic():
-    """DRAM bytes per full-prefill launch from the committed ncu summary, only
-    if it was taken on the current kernel source."""
+HOST_MARK = "// ----------------------------------------------------------------- host ---"
+
+
+def prefill_device_sha():
+    """Hash of the prefill kernels' device code: fa_prefill.cu up to its host
+    section, plus the shared device helpers (fa_common.cuh).  A DRAM traffic
+    record taken with ncu is only reported while this hash is unchanged."""
+    h = hashlib.sha256()
+    src = open(os.path.join(CSRC, "fa_prefill.cu"), "rb").read()
+    cut = src.find(HOST_MARK.encode())
+    h.update(src[:cut] if cut >= 0 else src)
+    h.update(open(os.path.join(CSRC, "fa_common.cuh"), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def kernel_traffic(workload):
+    """DRAM bytes per FULL prefill launch of `workload` from the committed ncu
+    record (profiles/), if it was taken on the current device code and on
+    this workload; else None.  Returns (bytes, record's workload, reason)."""
     if not os.path.exists(TRAFFIC_FILE):
-        return None, None
+        return None, None, "no ncu record"
     kv = {}
     for line in open(TRAFFIC_FILE):
-        if ":" in line:
+        if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    src_sha = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
-    if kv.get("kernel_src_sha256_16") != src_sha:
-        return None, kv.get("workload")
+    if kv.get("device_code_sha256_16") != prefill_device_sha():
+        return None, kv.get("workload"), "ncu record is of other device code"
+    if kv.get("workload", "").split(" ")[0] != workload:
+        return None, kv.get("workload"), "ncu record is of another workload"
     try:
-        return float(kv["dram_bytes_per_full_launch"]), kv.get("workload")
+        return float(kv["dram_bytes_per_full_launch"]), kv.get("workload"), "ncu, same code"
     except (KeyError, ValueError):
-        return None, kv.get("workload")
+        return None, kv.get("workload"), "ncu record unreadable"
 
 
 def dist_env():
@@ -216,8 +238,8 @@ def stack_plan(wl):
         rng = np.random.default_rng(wl.seed)
         sparse = set(rng.choice(wl.layers, size=wl.layers // 2, replace=False).tolist())
         return wl.layers, sparse, False, 1
-    if wl.S >= 65536:     # one layer per mode at long context
-        return 2, {1}, False, 1
+    if wl.S >= 65536:     # one layer per mode at long context (5 GiB per layer > L2)
+        return 2, {1}, True, 1
     return 2, {1}, True, N_INPUT_SETS
 
 
@@ -275,17 +297,6 @@ class Step:
                                  mode_dev=lay["mode"], c=c, o=lay["od"], workspace=self.dws,
                                  status=self.status)
 
-    def flops(self):
-        wl = self.wl
-        nf = sum(1 for l in self.layers if not l["sparse"])
-        ns = len(self.layers) - nf
-        f = nf * flops_full(wl) + ns * flops_sparse_exact(wl)
-        if self.with_decode:
-            keys = nf * decode_keys(wl.S, 0, wl.sink, wl.window) + \
-                ns * decode_keys(wl.S, 1, wl.sink, wl.window)
-            f += 4.0 * 128 * wl.Hq * wl.B * keys
-        return f
-
 
 def time_kernel_alone(fn, reps=5):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -299,18 +310,28 @@ def time_kernel_alone(fn, reps=5):
     return s.elapsed_time(e) / reps
 
 
-def cpu_baseline(wl, budget_s=15.0):
-    """The oracle as it stands, on the host cores, on a bounded sample of the
-    workload: seeded query rows of the full and the sparse layer; scaled to
-    TFLOP/s by the algorithmic FLOPs of the rows computed."""
+def cpu_inputs(wl, qkv_bits=None):
+    """Host data of the oracle's sample: the bf16 bits of Q/K/V (given, or
+    drawn on the CPU with the workload's seeds) and the dense block mask."""
     import oracle
     from block_sparse_attention_layerrouter_b200 import inputs
-    B, S, Hq, Hkv = wl.B, wl.S, wl.Hq, wl.Hkv
-    q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, wl.seed, device="cpu")
-    qb, kb, vb = inputs.bits(q), inputs.bits(k), inputs.bits(v)
-    del q, k, v
-    mask = oracle.rows_to_dense_mask(oracle.blocksparse_rows(S, 64, wl.sink, wl.window))
-    rng = np.random.default_rng(wl.seed)
+    if qkv_bits is None:
+        q, k, v = inputs.qkv(wl.B, wl.S, wl.Hq, wl.Hkv, 128, wl.seed, device="cpu")
+        qkv_bits = (inputs.bits(q), inputs.bits(k), inputs.bits(v))
+        del q, k, v
+    mask = oracle.rows_to_dense_mask(oracle.blocksparse_rows(wl.S, 64, wl.sink, wl.window))
+    return qkv_bits + (mask,)
+
+
+def cpu_baseline(wl, budget_s=15.0, data=None, seed=None):
+    """The oracle as it stands, on the host cores, on a bounded sample of the
+    workload: seeded query rows, each computed once as a row of the FULL
+    layer and once as a row of the SPARSE layer; scaled to TFLOP/s by the
+    algorithmic FLOPs of the rows computed (4*D*(attended pairs))."""
+    import oracle
+    qb, kb, vb, mask = data if data is not None else cpu_inputs(wl)
+    S, Hq = wl.S, wl.Hq
+    rng = np.random.default_rng(wl.seed if seed is None else seed)
     flops, elapsed, nrows = 0.0, 0.0, 0
     chunk = 64 if S <= 32768 else 16
     oracle.attention_rows(qb, kb, vb, 0.1, np.array([[0, 0, 0]]))   # load + warm
@@ -332,7 +353,8 @@ def cpu_baseline(wl, budget_s=15.0):
     return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": "%d query rows (random head and position; each row once in the full and "
-                      "once in the sparse layer) of %s, %.1f s" % (nrows, wl.name, elapsed)}
+                      "once in the sparse layer) of %s, %.1f s of oracle time; TFLOP/s from the "
+                      "rows' attended pairs" % (nrows, wl.name, elapsed)}
 
 
 def setup_device(args):
@@ -352,10 +374,12 @@ def setup_device(args):
 
 
 def sync_all(ws):
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(ms, ws, dev):
@@ -374,6 +398,23 @@ def base_line(args, wl, ws, ms, unit, value):
                     "for LongBench-E/RULER prompts of this shape"}
 
 
+def prefill_config(wl, ws):
+    """The `config` of a prefill workload's line; both arms print this dict."""
+    n_layers, sparse_layers, with_decode, n_sets = stack_plan(wl)
+    layer_bytes = wl.B * wl.S * 128 * 2 * (2 * wl.Hq + 2 * wl.Hkv)    # Q, O, K, V
+    return {
+        "workload": wl.name, "B": wl.B, "S": wl.S, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": 128,
+        "block": 64, "sink": wl.sink, "window": wl.window,
+        "router": "%d->%d->2" % (wl.Hq * 128, wl.hidden),
+        "step": "index + %d routed layers (%d FULL, %d SPARSE)%s" % (
+            n_layers, n_layers - len(sparse_layers), len(sparse_layers),
+            " + 1 decode token each" if with_decode else ""),
+        "parallelism": "replicas (dp%d, no collective)" % ws if ws > 1 else "single GPU",
+        "l2": "inputs %s than L2 (126 MB): %d input set(s) of %.2f GB, rotated" % (
+            "larger" if n_layers * layer_bytes > 126e6 else "SMALLER", n_sets,
+            n_layers * layer_bytes / 1e9)}
+
+
 def run_ours(args, wl):
     from block_sparse_attention_layerrouter_b200 import capi, inputs
     ws, rank, dev = setup_device(args)
@@ -381,114 +422,187 @@ def run_ours(args, wl):
     sets = [Step(wl, wl.seed + 101 * i, dev, capi, inputs, n_layers, sparse_layers, with_decode)
             for i in range(n_sets)]
     full_layer = min(li for li in range(n_layers) if li not in sparse_layers)
+    sparse_layer = min(sparse_layers)
     torch.cuda.synchronize()
     sampler = ClockSampler(dev)
     sampler.start()
     for i in range(args.warmup):
         sets[i % n_sets].run()
     sync_all(ws)
-    ev_full = [{full_layer: (torch.cuda.Event(enable_timing=True),
-                             torch.cuda.Event(enable_timing=True))} for _ in range(args.steps)]
+    ev = [{li: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for li in (full_layer, sparse_layer)} for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_launch0 = capi.kernel_launches()
     t0.record()
     for i in range(args.steps):
-        sets[i % n_sets].run(ev_full[i])
+        sets[i % n_sets].run(ev[i])
     t1.record()
     n_launch = capi.kernel_launches() - n_launch0   # kernels enqueued in the timed loop
     sync_all(ws)
     sampler.stop()
     ms = max_over_ranks(t0.elapsed_time(t1), ws, dev)
-    ms_full = [e[full_layer][0].elapsed_time(e[full_layer][1]) for e in ev_full]
+    ms_full = [e[full_layer][0].elapsed_time(e[full_layer][1]) for e in ev]
+    ms_sparse = [e[sparse_layer][0].elapsed_time(e[sparse_layer][1]) for e in ev]
     status = max(int(s.status.item()) for s in sets)
     modes = [int(l["mode"][0].item()) for l in sets[0].layers]
     want = [1 if li in sparse_layers else 0 for li in range(n_layers)]
+    assert status == 0, "device status %d" % status
 
-    e2e = run_e2e(args, wl, dev, capi, inputs, ws) if with_decode else None
-
-    # ---- components, each timed alone (breakdown only, not the headline)
+    # ---- the layer kernels each timed alone (breakdown only, not the headline)
     s0 = sets[0]
-    lay_f = s0.layers[full_layer]
-    lay_s = s0.layers[min(sparse_layers)]
+    lay_f, lay_s = s0.layers[full_layer], s0.layers[sparse_layer]
+    reps = 3 if wl.S >= 65536 else 10
     comp = {}
     comp["prefill_full_ms"] = time_kernel_alone(
-        lambda: capi.attn_prefill_full(lay_f["q"], lay_f["k"], lay_f["v"], o=lay_f["o"]))
+        lambda: capi.attn_prefill_full(lay_f["q"], lay_f["k"], lay_f["v"], o=lay_f["o"]), reps)
     comp["prefill_sparse_ms"] = time_kernel_alone(
         lambda: capi.attn_prefill_blocksparse(lay_s["q"], lay_s["k"], lay_s["v"], s0.row_ptr,
-                                              s0.col_idx, o=lay_s["o"]))
+                                              s0.col_idx, o=lay_s["o"]), reps)
     comp["router_ms"] = time_kernel_alone(
         lambda: capi.router_decide(lay_f["q"], lay_f["w1"], lay_f["b1"], lay_f["w2"],
                                    lay_f["b2"], logits=lay_f["logits"], mode=lay_f["mode"],
                                    workspace=s0.ws))
-    torch.cuda.synchronize()
+    headline = wl.name == DEFAULT_WORKLOAD and not args.no_sections
+    cpu_data = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        from block_sparse_attention_layerrouter_b200 import inputs as _in
+        cpu_data = cpu_inputs(wl, (_in.bits(lay_f["q"]), _in.bits(lay_f["k"]),
+                                   _in.bits(lay_f["v"])))
+    del sets, s0, lay_f, lay_s
+    torch.cuda.empty_cache()
+
+    e2e = run_e2e(args, wl, dev, capi, inputs, ws) if with_decode else None
+    torch.cuda.empty_cache()
+    sections = {}
+    if headline:
+        sections["decode"] = decode_section(args, WORKLOADS_()[DECODE_WORKLOAD], dev, ws, rank)
+        torch.cuda.empty_cache()
+        sections[LAYER8K_WORKLOAD] = layer_kernels_section(WORKLOADS_()[LAYER8K_WORKLOAD], dev)
+        torch.cuda.empty_cache()
     if rank != 0:
         return None
     hbm, peak_burst, peak_sust, peak_kind = measured_peaks()
     f_full = flops_full(wl)
     f_sparse = flops_sparse_exact(wl)
     f_sparse_exec = 4.0 * 128 * wl.Hq * wl.B * csr_nnz(wl.S, wl.sink, wl.window) * 64 * 64
-    value = ws * s0.flops() / (ms / args.steps * 1e-3) / 1e12
-    avg_full_ms = statistics.mean(ms_full)
+    step_flops = step_flops_of(wl, n_layers, sparse_layers, with_decode)
+    value = ws * step_flops / (ms / args.steps * 1e-3) / 1e12
+    avg_full_ms, avg_sparse_ms = statistics.mean(ms_full), statistics.mean(ms_sparse)
     achieved = f_full / (avg_full_ms * 1e-3) / 1e12
-    traffic, traffic_wl = kernel_traffic()
+    traffic, traffic_wl, traffic_note = kernel_traffic(wl.name)
     comp.update({
+        "prefill_full_in_step_ms": avg_full_ms,
+        "prefill_sparse_in_step_ms": avg_sparse_ms,
         "prefill_full_tflops": f_full / (comp["prefill_full_ms"] * 1e-3) / 1e12,
         "prefill_sparse_exec_tflops": f_sparse_exec / (comp["prefill_sparse_ms"] * 1e-3) / 1e12,
         "prefill_sparse_exec_frac_of_burst": f_sparse_exec / (comp["prefill_sparse_ms"] * 1e-3)
         / 1e12 / peak_burst,
+        "prefill_sparse_exec_in_step_tflops": f_sparse_exec / (avg_sparse_ms * 1e-3) / 1e12,
         "prefill_sparse_exact_tflops": f_sparse / (comp["prefill_sparse_ms"] * 1e-3) / 1e12,
         "routed_modes_match_plan": modes == want,
         "device_status": status,
     })
-    if wl.S >= 65536 or n_layers > 2:
-        tf, tsp = comp["prefill_full_ms"], comp["prefill_sparse_ms"]
-        nl = 36 if wl.S >= 65536 else n_layers
-        comp["hybrid_vs_full"] = {
-            "layers": nl, "split": "50/50", "t_full_layer_ms": tf, "t_sparse_layer_ms": tsp,
-            "hybrid_ms": nl / 2 * (tf + tsp), "all_full_ms": nl * tf,
-            "speedup": (nl * tf) / (nl / 2 * (tf + tsp))}
     line = base_line(args, wl, ws, ms, "TFLOP/s", value)
-    line["config"] = {
-        "workload": wl.name, "B": wl.B, "S": wl.S, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": 128,
-        "block": 64, "sink": wl.sink, "window": wl.window,
-        "router": "%d->%d->2" % (wl.Hq * 128, wl.hidden),
-        "step": "index + %d routed layers (%d FULL, %d SPARSE)%s" % (
-            n_layers, n_layers - len(sparse_layers), len(sparse_layers),
-            " + 1 decode token each" if with_decode else ""),
-        "parallelism": "replicas" if ws > 1 else "single GPU",
-        "l2": "inputs larger than L2: %d input set(s) of %.2f GB" % (
-            n_sets, sum(t.numel() * t.element_size() for l in s0.layers
-                        for t in (l["q"], l["k"], l["v"], l["o"])) / 1e9)}
+    line["config"] = prefill_config(wl, ws)
     line["clocks"] = sampler.report()
     line["roofline"] = roofline_tensor(
         achieved, line["clocks"], (hbm, peak_burst, peak_sust, peak_kind),
-        kernel="prefill_kernel (a FULL layer of the step)", traffic=traffic,
-        traffic_workload=traffic_wl, algorithmic_flops_per_launch=f_full,
-        avg_launch_ms=round(avg_full_ms, 4))
+        kernel="prefill2::prefill2_kernel, FULL layer of the step (CUDA events around "
+               "fa_hybrid_layer: router kernels included, %.3f ms of it alone)" % comp["router_ms"],
+        traffic=traffic, traffic_source=traffic_note, traffic_workload=traffic_wl,
+        algorithmic_flops_per_launch=f_full, avg_launch_ms=round(avg_full_ms, 4),
+        sparse_layer={"kernel": "prefill2::prefill2_kernel, SPARSE layer of the step",
+                      "avg_launch_ms": round(avg_sparse_ms, 4),
+                      "executed_flops_per_launch": f_sparse_exec,
+                      "achieved_exec_tflops": round(f_sparse_exec / (avg_sparse_ms * 1e-3)
+                                                    / 1e12, 2)})
+    if wl.S >= 65536 or n_layers > 2:
+        nl = 36 if wl.S >= 65536 else n_layers
+        tf, tsp = avg_full_ms, avg_sparse_ms
+        tfa, tspa = comp["prefill_full_ms"], comp["prefill_sparse_ms"]
+        line["hybrid_vs_full"] = {
+            "layers": nl, "split": "50/50",
+            "t_full_layer_ms": round(tf, 3), "t_sparse_layer_ms": round(tsp, 3),
+            "hybrid_ms": round(nl / 2 * (tf + tsp), 2), "all_full_ms": round(nl * tf, 2),
+            "speedup": round((nl * tf) / (nl / 2 * (tf + tsp)), 4),
+            "speedup_layers_alone": round((nl * tfa) / (nl / 2 * (tfa + tspa)), 4),
+            "note": "layer times from the timed steps (routed layers, router included); "
+                    "projection = %d/2 FULL + %d/2 SPARSE layers vs %d FULL" % (nl, nl, nl),
+            "pages_context": "up to 2.8x prefill at 256K (hardware not stated)"}
     line["e2e"] = e2e
     line["gpu_launches"] = n_launch
     line["components"] = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in comp.items()}
-    if ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl)
+    line.update(sections)
+    if cpu_data is not None:
+        line["cpu_baseline"] = cpu_baseline(wl, data=cpu_data)
     return line
+
+
+def WORKLOADS_():
+    from block_sparse_attention_layerrouter_b200.inputs import WORKLOADS
+    return WORKLOADS
+
+
+def step_flops_of(wl, n_layers, sparse_layers, with_decode):
+    ns = len(sparse_layers)
+    nf = n_layers - ns
+    f = nf * flops_full(wl) + ns * flops_sparse_exact(wl)
+    if with_decode:
+        keys = nf * decode_keys(wl.S, 0, wl.sink, wl.window) + \
+            ns * decode_keys(wl.S, 1, wl.sink, wl.window)
+        f += 4.0 * 128 * wl.Hq * wl.B * keys
+    return f
+
+
+def layer_kernels_section(wl, dev):
+    """FULL and SPARSE prefill of one layer of `wl`, each launched alone
+    (the 8K-context layer: several full waves of work items per launch)."""
+    from block_sparse_attention_layerrouter_b200 import capi, inputs
+    q, k, v = inputs.qkv(wl.B, wl.S, wl.Hq, wl.Hkv, 128, wl.seed, device=dev)
+    o = torch.empty_like(q)
+    c = capi.cfg(64, wl.sink, wl.window)
+    rp, ci = capi.blocksparse_index(wl.S, c, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    tf = time_kernel_alone(lambda: capi.attn_prefill_full(q, k, v, o=o, status=status), 20)
+    ts = time_kernel_alone(lambda: capi.attn_prefill_blocksparse(q, k, v, rp, ci, o=o,
+                                                                 status=status), 20)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
+    _, peak_burst, peak_sust, _ = measured_peaks()
+    f_full = flops_full(wl)
+    f_exec = 4.0 * 128 * wl.Hq * wl.B * csr_nnz(wl.S, wl.sink, wl.window) * 64 * 64
+    return {"config": {"B": wl.B, "S": wl.S, "Hq": wl.Hq, "Hkv": wl.Hkv, "window": wl.window,
+                       "sink": wl.sink},
+            "timing": "each kernel alone, 20 launches on one input set (0.34 GB), CUDA events",
+            "prefill_full_ms": round(tf, 4),
+            "prefill_full_tflops": round(f_full / (tf * 1e-3) / 1e12, 2),
+            "prefill_full_frac_of_burst": round(f_full / (tf * 1e-3) / 1e12 / peak_burst, 4),
+            "prefill_sparse_ms": round(ts, 4),
+            "prefill_sparse_exec_tflops": round(f_exec / (ts * 1e-3) / 1e12, 2),
+            "prefill_sparse_exec_frac_of_burst": round(f_exec / (ts * 1e-3) / 1e12 / peak_burst,
+                                                       4),
+            "prefill_sparse_exact_tflops": round(flops_sparse_exact(wl) / (ts * 1e-3) / 1e12, 2)}
 
 
 def run_e2e(args, wl, dev, capi, inputs, ws):
     """Same step through the public API with host buffers: per step, copy
-    the two layers' Q/K/V and decode queries from pinned host memory, run,
-    and read both layers' outputs back.  The copies are pipelined across
-    steps: two device buffer sets, the inputs of step i+1 going up on one
-    copy stream and the outputs of step i-1 coming down on another while
-    step i computes (PCIe is full duplex)."""
-    steps = [Step(wl, wl.seed, dev, capi, inputs), Step(wl, wl.seed, dev, capi, inputs)]
+    the layers' Q/K/V and decode queries from pinned host memory, run, and
+    read the layers' outputs back.  The copies are pipelined across steps:
+    two device buffer sets, the inputs of step i+1 going up on one copy
+    stream and the outputs of step i-1 coming down on another while step i
+    computes (PCIe is full duplex)."""
+    n_layers, sparse_layers, with_decode, _ = stack_plan(wl)
+    steps = [Step(wl, wl.seed, dev, capi, inputs, n_layers, sparse_layers, with_decode)
+             for _ in range(2)]
     host = []
     for lay in steps[0].layers:
         host.append([lay[n].cpu().pin_memory() for n in ("q", "k", "v", "qd")])
-    outs = [[(torch.empty(lay["o"].shape, dtype=lay["o"].dtype).pin_memory(),
-              torch.empty(lay["od"].shape, dtype=lay["od"].dtype).pin_memory())
-             for lay in st.layers] for st in steps]
+    # One host output set: the D2H copies run in order on one stream.
+    outs = [(torch.empty(lay["o"].shape, dtype=lay["o"].dtype).pin_memory(),
+             torch.empty(lay["od"].shape, dtype=lay["od"].dtype).pin_memory())
+            for lay in steps[0].layers]
     h2d = sum(t.numel() * t.element_size() for hs in host for t in hs)
-    d2h = sum(t.numel() * t.element_size() for o in outs[0] for t in o)
+    d2h = sum(t.numel() * t.element_size() for o in outs for t in o)
     s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     s_comp = torch.cuda.current_stream(dev)
     ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("up", "comp", "down")}
@@ -512,8 +626,8 @@ def run_e2e(args, wl, dev, capi, inputs, ws):
         with torch.cuda.stream(s_down):
             s_down.wait_event(ev["comp"][b])
             for li, lay in enumerate(st.layers):
-                outs[b][li][0].copy_(lay["o"], non_blocking=True)
-                outs[b][li][1].copy_(lay["od"], non_blocking=True)
+                outs[li][0].copy_(lay["o"], non_blocking=True)
+                outs[li][1].copy_(lay["od"], non_blocking=True)
             ev["down"][b].record(s_down)
         started[b] = True
 
@@ -531,7 +645,8 @@ def run_e2e(args, wl, dev, capi, inputs, ws):
     e.record(s_comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e), ws, dev)
-    return {"value": round(ws * steps[0].flops() / (ms / args.steps * 1e-3) / 1e12, 3),
+    flops = step_flops_of(wl, n_layers, sparse_layers, with_decode)
+    return {"value": round(ws * flops / (ms / args.steps * 1e-3) / 1e12, 3),
             "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / args.steps, 4),
             "note": "copies pipelined across steps (two device buffer sets, separate H2D "
@@ -542,14 +657,16 @@ def run_e2e(args, wl, dev, capi, inputs, ws):
 DECODE_CACHE_SETS = 8
 
 
-def run_decode(args, wl):
+def decode_measure(wl, dev, ws, steps, warmup, min_seconds=0.0):
     """Decode step of a 32-layer model: one token per sequence per layer,
     layers alternating FULL / SPARSE (16 + 16, fixed by the router at
     prefill).  Each layer reads its own KV cache; 8 distinct cache sets (4 GiB
     each) are rotated over the 32 layers, so consecutive reads of one set are
-    8 layers (>= 16 GiB of other traffic) apart and come from HBM."""
+    8 layers (>= 16 GiB of other traffic) apart and come from HBM.  With
+    min_seconds > 0 the timed step count is raised until the timed region
+    lasts at least that long (estimated from the warm-up steps).  Returns a
+    dict of measurements (every rank) or raises on a device error."""
     from block_sparse_attention_layerrouter_b200 import capi, inputs
-    ws, rank, dev = setup_device(args)
     B, L, Hq, Hkv = wl.B, wl.decode_len, wl.Hq, wl.Hkv
     caches = []
     max_pages = L // 64
@@ -593,15 +710,23 @@ def run_decode(args, wl):
 
     sampler = ClockSampler(dev)
     sampler.start()
-    for _ in range(args.warmup):
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step()
+    w0.record()
+    for _ in range(max(1, warmup - 1)):
         step()
+    w1.record()
     sync_all(ws)
+    if min_seconds > 0:
+        est = w0.elapsed_time(w1) / max(1, warmup - 1)
+        est = max_over_ranks(est, ws, dev)       # every rank times the same count
+        steps = max(steps, int(math.ceil(min_seconds * 1e3 / max(est, 1e-3))))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+           for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_launch0 = capi.kernel_launches()
     t0.record()
-    for i in range(args.steps):
+    for i in range(steps):
         step(evs[i])
     t1.record()
     n_launch = capi.kernel_launches() - n_launch0   # kernels enqueued in the timed loop
@@ -621,6 +746,9 @@ def run_decode(args, wl):
         sparse_ms = time_kernel_alone(lambda: capi.attn_decode(qs[1], *caches[1], sl, 1, c,
                                                                o=outs[1], workspace=wsb))
         append_ms = None
+    # FULL layer alone on one cache (a burst, 10 launches): the kernel's own rate.
+    full_alone_ms = time_kernel_alone(lambda: capi.attn_decode(
+        qs[0], *caches[0], sl, 0, c, o=outs[0], workspace=wsb), reps=10) if not wl.paged else None
     # e2e: the caches are device-resident state; per step the 32 layers'
     # query tokens go up from pinned host memory and their outputs come back.
     hq = [q.cpu().pin_memory() for q in qs]
@@ -638,48 +766,76 @@ def run_decode(args, wl):
     sync_all(ws)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
+    for _ in range(steps):
         step_e2e()
     e1.record()
     torch.cuda.synchronize()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), ws, dev)
     assert int(status.item()) == 0, "device status %d" % int(status.item())
-    if rank != 0:
-        return None
     hbm, _, _, peak_kind = measured_peaks()
     kv_row = 2 * Hkv * 128 * (1 if wl.kv_fp8 else 2)         # K and V bytes per token
     qo = 2 * B * Hq * 128 * 2
     full_bytes = B * kv_row * decode_keys(L, 0, wl.sink, wl.window) + qo
     sparse_bytes = B * kv_row * decode_keys(L, 1, wl.sink, wl.window) + qo
     step_bytes = sum(full_bytes if m == 0 else sparse_bytes for m in modes)
-    value = ws * step_bytes / (ms / args.steps * 1e-3) / 1e9
-    line = base_line(args, wl, ws, ms, "GB/s", value)
-    line["config"] = {"workload": wl.name, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv, "D": 128,
-                      "layers": wl.layers, "split": "16 FULL + 16 SPARSE (alternating)",
-                      "sink": wl.sink, "window": wl.window,
-                      "cache": ("paged (64-token pages, seeded random order), " if wl.paged
-                                else "contiguous, ") + ("E4M3 + per-head scales" if wl.kv_fp8
-                                                        else "bf16"),
-                      "l2": "inputs larger than L2: %d cache sets of %.2f GB rotated" % (
-                          DECODE_CACHE_SETS,
-                          2 * caches[0][0].numel() * caches[0][0].element_size() / 1e9)}
-    achieved = full_bytes / (full_ms * 1e-3) / 1e9
-    line["roofline"] = roofline_hbm(
-        achieved, hbm, peak_kind, kernel="decode_kernel + combine (a FULL layer)", traffic=None,
-        algorithmic_bytes_per_launch=full_bytes, avg_launch_ms=round(full_ms, 4))
-    line["e2e"] = {"value": round(ws * step_bytes / (ms_e2e / args.steps * 1e-3) / 1e9, 1),
-                   "unit": "GB/s", "h2d_bytes_per_step": sum(t.numel() * 2 for t in hq),
-                   "d2h_bytes_per_step": sum(t.numel() * 2 for t in ho),
-                   "note": "KV caches are device-resident decode state"}
-    line["gpu_launches"] = n_launch
-    line["clocks"] = sampler.report()
-    line["components"] = {
-        "decode_full_layer_ms": round(full_ms, 4), "decode_sparse_layer_ms": round(sparse_ms, 4),
-        "decode_sparse_gbs": round(sparse_bytes / (sparse_ms * 1e-3) / 1e9, 1),
-        "all_full_step_ms_est": round(wl.layers * full_ms, 3),
-        "hybrid_vs_all_full": round(wl.layers * full_ms / (ms / args.steps), 3)}
+    clocks = sampler.report()
+    out = {
+        "value": round(ws * step_bytes / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "steps": steps, "ms_per_step": round(ms / steps, 4), "timed_s": round(ms / 1e3, 3),
+        "config": {"workload": wl.name, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv, "D": 128,
+                   "layers": wl.layers, "split": "16 FULL + 16 SPARSE (alternating)",
+                   "sink": wl.sink, "window": wl.window,
+                   "cache": ("paged (64-token pages, seeded random order), " if wl.paged
+                             else "contiguous, ") + ("E4M3 + per-head scales" if wl.kv_fp8
+                                                     else "bf16"),
+                   "l2": "inputs larger than L2: %d cache sets of %.2f GB rotated" % (
+                       DECODE_CACHE_SETS,
+                       2 * caches[0][0].numel() * caches[0][0].element_size() / 1e9)},
+        "clocks": clocks,
+        "roofline": roofline_hbm(
+            full_bytes / (full_ms * 1e-3) / 1e9, hbm, peak_kind,
+            kernel="decode::decode_kernel + combine_kernel (FULL layer of the step)",
+            traffic=None, algorithmic_bytes_per_launch=full_bytes,
+            avg_launch_ms=round(full_ms, 4)),
+        "e2e": {"value": round(ws * step_bytes / (ms_e2e / steps * 1e-3) / 1e9, 1),
+                "unit": "GB/s", "h2d_bytes_per_step": sum(t.numel() * 2 for t in hq),
+                "d2h_bytes_per_step": sum(t.numel() * 2 for t in ho),
+                "note": "KV caches are device-resident decode state"},
+        "gpu_launches": n_launch,
+        "components": {
+            "decode_full_layer_ms": round(full_ms, 4),
+            "decode_sparse_layer_ms": round(sparse_ms, 4),
+            "decode_sparse_gbs": round(sparse_bytes / (sparse_ms * 1e-3) / 1e9, 1),
+            "all_full_step_ms_est": round(wl.layers * full_ms, 3),
+            "hybrid_vs_all_full": round(wl.layers * full_ms / (ms / steps), 3),
+            "pages_context": "up to 2.0x decode at 256K (hardware not stated)"}}
+    if full_alone_ms is not None:
+        out["components"]["decode_full_layer_alone_ms"] = round(full_alone_ms, 4)
+        out["components"]["decode_full_layer_alone_gbs"] = round(
+            full_bytes / (full_alone_ms * 1e-3) / 1e9, 1)
+        out["components"]["decode_full_layer_alone_frac_of_hbm"] = round(
+            full_bytes / (full_alone_ms * 1e-3) / 1e9 / hbm, 4)
     if append_ms is not None:
-        line["components"]["kv_append_ms"] = round(append_ms, 4)
+        out["components"]["kv_append_ms"] = round(append_ms, 4)
+    del caches
+    return out
+
+
+def decode_section(args, wl, dev, ws, rank):
+    """The 32-layer decode step inside the headline line, timed for at least
+    one second whatever --steps is, so the clock record covers it."""
+    d = decode_measure(wl, dev, ws, args.steps, args.warmup, min_seconds=1.0)
+    return d if rank == 0 else None
+
+
+def run_decode(args, wl):
+    ws, rank, dev = setup_device(args)
+    d = decode_measure(wl, dev, ws, args.steps, args.warmup)
+    if rank != 0:
+        return None
+    line = base_line(args, wl, ws, d["ms_per_step"] * args.steps, "GB/s", d["value"])
+    for k in ("config", "clocks", "roofline", "e2e", "gpu_launches", "components"):
+        line[k] = d[k]
     return line
 
 
@@ -946,16 +1102,21 @@ def run_only(args, wl):
 
 # --------------------------------------------------------- reference arm
 def run_reference(args, wl):
-    """The oracle as it stands on the host cores, same metric and unit; each
-    step a bounded sample of the workload (see cpu_baseline)."""
+    """The oracle as it stands on the host cores, same metric, unit and
+    config as our arm; each step a bounded sample of the workload (see
+    cpu_baseline).  Under torchrun rank 0 alone runs it."""
     ws, rank, _ = dist_env()
     if rank != 0:
         return None
+    if wl.decode_len or wl.varlen or wl.train:
+        return {"impl": "reference", "unavailable": "the reference arm times the prefill "
+                "workloads only (the oracle's attention rows); %s is not one" % wl.name}
     budget = float(os.environ.get("FA_REF_STEP_S", "4"))
+    data = cpu_inputs(wl)
     vals, t_total = [], 0.0
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        r = cpu_baseline(wl, budget_s=budget)
+        r = cpu_baseline(wl, budget_s=budget, data=data, seed=wl.seed + i)
         if i >= args.warmup:
             vals.append(r["value"])
             t_total += time.perf_counter() - t0
@@ -965,23 +1126,62 @@ def run_reference(args, wl):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * t_total / max(1, args.steps), 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "B": wl.B, "S": wl.S, "Hq": wl.Hq, "Hkv": wl.Hkv,
-                       "D": 128, "block": 64, "sink": wl.sink, "window": wl.window},
+            "config": prefill_config(wl, ws),
             "cpu_baseline": r,
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------- host-only dry run
+def run_dry(args, wl):
+    """The multi-rank host path without a GPU: gloo process group, barrier,
+    a timed host loop, maximum over ranks, one line from rank 0."""
+    ws, rank, _ = dist_env()
+    if ws > 1 and not torch.distributed.is_initialized():
+        from datetime import timedelta
+        torch.distributed.init_process_group("gloo", timeout=timedelta(seconds=120))
+    dev = torch.device("cpu")
+    sync_all(ws)
+    t0 = time.perf_counter()
+    for _ in range(args.warmup + args.steps):
+        torch.ones(64).sum()
+    ms = max_over_ranks((time.perf_counter() - t0) * 1e3, ws, dev)
+    if rank != 0:
+        return None
+    line = base_line(args, wl, ws, ms, "TFLOP/s", 0.0)
+    line.update({"dry_run": True, "config": prefill_config(wl, ws), "e2e": None,
+                 "gpu_launches": 0})
+    return line
+
+
+def relaunch(args) -> int:
+    """`--gpus N` outside torchrun: start N ranks of this script through
+    torch.distributed.run on this node and return their exit status."""
+    import socket
+    import subprocess
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node=%d" % args.gpus, "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: 200 for the sub-millisecond default step, so "
-                         "the clock samples cover the timed region; 20 otherwise)")
+                    help="timed steps (default: 200 for the sub-millisecond 8K step, so the "
+                         "clock samples cover the timed region; 20 otherwise)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sections", action="store_true",
+                    help="headline workload without the decode and 8K sections")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="host path only (gloo, no GPU): ranks, barrier, max over ranks")
     ap.add_argument("--only", default=None,
                     help="prefill_full | prefill_sparse | decode_full | decode_sparse | "
                          "decode_fp8_full | decode_fp8_sparse | backward_full | "
@@ -989,12 +1189,21 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch(args))
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws != args.gpus:
+        ap.error("--gpus %d but WORLD_SIZE=%d" % (args.gpus, ws))
     from block_sparse_attention_layerrouter_b200.inputs import WORKLOADS
     wl = WORKLOADS[args.workload]
     if args.steps is None:
         args.steps = 200 if (args.impl == "ours" and not args.only
-                             and wl.name == DEFAULT_WORKLOAD) else 20
-    if args.impl == "reference":
+                             and wl.name == LAYER8K_WORKLOAD) else 20
+    if args.dry_run:
+        line = run_dry(args, wl)
+    elif args.impl == "reference":
         line = run_reference(args, wl)
     elif args.only:
         line = run_only(args, wl)

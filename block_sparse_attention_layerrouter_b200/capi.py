@@ -47,6 +47,7 @@ _SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
     "fa_kernel_launches": (ctypes.c_ulonglong, []),
+    "fa_debug_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
     "fa_router_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_router_decide": (_I, [_VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _I, _VP, _VP, _VP, _VP,
                               _VP, _SZ, _VP]),
@@ -118,6 +119,13 @@ def kernel_launches() -> int:
     """Kernels this library has enqueued in this process so far (host-side
     count; no GPU access)."""
     return int(lib().fa_kernel_launches())
+
+
+def debug_set_wait_limit_ns(ns: int):
+    """fa_debug_set_wait_limit_ns: the bound of every wait inside the kernels
+    on the current device (default 2e9 ns).  A testing aid: a short bound
+    makes the kernels give up and report FA_DEV_TIMEOUT."""
+    _check("fa_debug_set_wait_limit_ns", lib().fa_debug_set_wait_limit_ns(int(ns)))
 
 
 def _check(name: str, rc: int):

@@ -4,10 +4,22 @@
 #include "fa_common.cuh"
 #include "fa_internal.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <mutex>
 
 namespace fa {
+
+// An NVTX range named after the entry point around each call that enqueues
+// work, so a timeline (nsys, ncu's range filter) shows which library call
+// launched which kernels.  Without a tool attached it costs a no-op call.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 static std::atomic<unsigned long long> g_kernel_launches{0};
 void note_launch() { g_kernel_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -128,6 +140,22 @@ int check_router(const void *q, int B, int S, int Hq, int D, int n_head, int n_t
 }
 
 }  // namespace
+
+int check_decode_args(const void *q, const void *kcache, const void *vcache,
+                      const int32_t *seqlens, int B, int Lmax, int Hq, int Hkv, int D,
+                      float scale, int mode, fa_sparse_cfg cfg, const void *o) {
+  if (!q || !kcache || !vcache || !seqlens || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Lmax <= 0) return FA_ERR_INVALID_ARG;
+  if (int rc = check_heads(Hq, Hkv, D)) return rc;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
+  if (mode != FA_MODE_FULL && mode != FA_MODE_SPARSE) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  return check_cfg(cfg);
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -152,6 +180,13 @@ FA_API unsigned long long fa_kernel_launches(void) {
   return g_kernel_launches.load(std::memory_order_relaxed);
 }
 
+FA_API int fa_debug_set_wait_limit_ns(unsigned long long ns) {
+  if (set_wait_limit_prefill(ns) != 0 || set_wait_limit_decode(ns) != 0 ||
+      set_wait_limit_backward(ns) != 0)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 FA_API size_t fa_router_workspace_size(int B, int Hq, int D, int hidden) {
   if (B <= 0 || Hq <= 0 || D <= 0 || hidden <= 0) return 0;
   return router_workspace_bytes(B, Hq, D, hidden);
@@ -161,6 +196,7 @@ FA_API int fa_router_decide(const void *q, int B, int S, int Hq, int D, int n_he
                      const float *w1, const float *b1, int hidden, const float *w2,
                      const float *b2, float *logits_out, int32_t *mode_out, void *workspace,
                      size_t ws_bytes, void *stream) {
+  NvtxRange range_("fa_router_decide");
   if (int rc = check_router(q, B, S, Hq, D, n_head_tok, n_tail_tok, w1, hidden, w2)) return rc;
   if (!logits_out && !mode_out) return FA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < router_workspace_bytes(B, Hq, D, hidden)) return FA_ERR_WORKSPACE;
@@ -182,6 +218,7 @@ FA_API int fa_blocksparse_index_size(int S, fa_sparse_cfg cfg, int *n_rows, int 
 
 FA_API int fa_blocksparse_index(int S, fa_sparse_cfg cfg, int32_t *row_ptr, int32_t *col_idx,
                          void *stream) {
+  NvtxRange range_("fa_blocksparse_index");
   int rows = 0, nnz = 0;
   if (int rc = fa_blocksparse_index_size(S, cfg, &rows, &nnz)) return rc;
   if (!row_ptr || !col_idx) return FA_ERR_INVALID_ARG;
@@ -192,6 +229,7 @@ FA_API int fa_blocksparse_index(int S, fa_sparse_cfg cfg, int32_t *row_ptr, int3
 FA_API int fa_attn_prefill_full(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                          int S, int Hq, int Hkv, int D, float scale, int32_t *dev_status,
                          void *stream) {
+  NvtxRange range_("fa_attn_prefill_full");
   if (int rc = check_prefill(q, k, v, o, B, S, Hq, Hkv, D)) return rc;
   if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
   PrefillLaunch a{q, k, v, o, lse, B, S, Hq, Hkv, scale, nullptr, nullptr, nullptr,
@@ -203,6 +241,7 @@ FA_API int fa_attn_prefill_blocksparse(const void *q, const void *k, const void 
                                 int B, int S, int Hq, int Hkv, int D, float scale,
                                 const int32_t *row_ptr, const int32_t *col_idx, int block,
                                 int32_t *dev_status, void *stream) {
+  NvtxRange range_("fa_attn_prefill_blocksparse");
   if (int rc = check_prefill(q, k, v, o, B, S, Hq, Hkv, D)) return rc;
   if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
   if (!row_ptr || !col_idx) return FA_ERR_INVALID_ARG;
@@ -221,16 +260,10 @@ FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
                    int B, int Lmax, int Hq, int Hkv, int D, float scale, int mode,
                    const int32_t *mode_dev, fa_sparse_cfg cfg, void *o, float *lse,
                    void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream) {
-  if (!q || !kcache || !vcache || !seqlens || !o) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
-    return FA_ERR_INVALID_ARG;
-  if (B <= 0 || Lmax <= 0) return FA_ERR_INVALID_ARG;
-  if (int rc = check_heads(Hq, Hkv, D)) return rc;
-  const int G = Hq / Hkv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
-  if (mode != FA_MODE_FULL && mode != FA_MODE_SPARSE) return FA_ERR_INVALID_ARG;
-  if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
-  if (int rc = check_cfg(cfg)) return rc;
+  NvtxRange range_("fa_attn_decode");
+  if (int rc = check_decode_args(q, kcache, vcache, seqlens, B, Lmax, Hq, Hkv, D, scale, mode,
+                                 cfg, o))
+    return rc;
   if (!workspace || !aligned16(workspace) || ws_bytes < decode_workspace_bytes(B, Hq, Hkv, Lmax))
     return FA_ERR_WORKSPACE;
   DecodeLaunch a{q, kcache, vcache, seqlens, B, Lmax, Hq, Hkv, scale, mode, mode_dev,
@@ -243,6 +276,7 @@ FA_API int fa_kv_append_paged(const void *k_new, const void *v_new, void *k_page
                               const float *v_scale, const int32_t *block_table, int max_pages,
                               int num_pages, int32_t *seqlens, int B, int Hkv, int D,
                               int32_t *dev_status, void *stream) {
+  NvtxRange range_("fa_kv_append_paged");
   if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !seqlens)
     return FA_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pages) || !aligned16(v_pages))
@@ -269,6 +303,7 @@ FA_API int fa_attn_decode_paged(const void *q, const void *k_pages, const void *
                                 float scale, int mode, const int32_t *mode_dev,
                                 fa_sparse_cfg cfg, void *o, float *lse, void *workspace,
                                 size_t ws_bytes, int32_t *dev_status, void *stream) {
+  NvtxRange range_("fa_attn_decode_paged");
   if (!q || !k_pages || !v_pages || !block_table || !seqlens || !o) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o))
     return FA_ERR_INVALID_ARG;
@@ -306,6 +341,7 @@ FA_API int fa_hybrid_layer(const void *q, const void *k, const void *v, void *o,
                     const int32_t *row_ptr, const int32_t *col_idx, float *logits_out,
                     int32_t *mode_out, void *workspace, size_t ws_bytes, int32_t *dev_status,
                     void *stream) {
+  NvtxRange range_("fa_hybrid_layer");
   if (int rc = check_prefill(q, k, v, o, B, S, Hq, Hkv, D)) return rc;
   if (int rc = check_router(q, B, S, Hq, D, 100, 100, w1, hidden, w2)) return rc;
   if (int rc = check_cfg(cfg)) return rc;
@@ -317,11 +353,14 @@ FA_API int fa_hybrid_layer(const void *q, const void *k, const void *v, void *o,
   if (int rc = launch_router(r, st)) return rc;
   PrefillLaunch a{q, k, v, o, lse, B, S, Hq, Hkv, scale, row_ptr, col_idx, mode_out,
                   FA_MODE_FULL, dev_status};
+  a.expect_nnz = index_nnz((S + cfg.block - 1) / cfg.block, cfg.sink / cfg.block,
+                           cfg.window / cfg.block);
   return launch_prefill(a, st);
 }
 
 FA_API int fa_router_soft(const float *logits, const float *gumbel, int B, float tau,
                           float *r_out, void *stream) {
+  NvtxRange range_("fa_router_soft");
   if (!logits || !r_out || B <= 0) return FA_ERR_INVALID_ARG;
   if (!(tau > 0.f)) return FA_ERR_INVALID_ARG;
   return launch_router_soft(logits, gumbel, B, tau, r_out, static_cast<cudaStream_t>(stream));
@@ -334,6 +373,7 @@ FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v, voi
                                 const int32_t *row_ptr, const int32_t *col_idx, float *logits_out,
                                 float *r_out, void *workspace, size_t ws_bytes,
                                 int32_t *dev_status, void *stream) {
+  NvtxRange range_("fa_soft_routed_layer");
   if (int rc = check_prefill(q, k, v, o, B, S, Hq, Hkv, D)) return rc;
   if (int rc = check_router(q, B, S, Hq, D, 100, 100, w1, hidden, w2)) return rc;
   if (int rc = check_cfg(cfg)) return rc;
@@ -350,11 +390,14 @@ FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v, voi
   PrefillLaunch sparse{q, k, v, o, nullptr, B, S, Hq, Hkv, scale, row_ptr, col_idx, nullptr,
                        FA_MODE_SPARSE, dev_status};
   sparse.mix_r = r_out;
+  sparse.expect_nnz = index_nnz((S + cfg.block - 1) / cfg.block, cfg.sink / cfg.block,
+                                cfg.window / cfg.block);
   return launch_prefill(sparse, st);
 }
 
 FA_API int fa_soft_mix(const void *o_full, const void *o_sparse, const float *r, void *y, int B,
                        int S, int Hq, int D, void *stream) {
+  NvtxRange range_("fa_soft_mix");
   if (!o_full || !o_sparse || !r || !y || B <= 0 || S <= 0 || Hq <= 0) return FA_ERR_INVALID_ARG;
   if (!aligned16(o_full) || !aligned16(o_sparse) || !aligned16(y)) return FA_ERR_INVALID_ARG;
   if (D != kHeadDim) return FA_ERR_UNSUPPORTED;
@@ -373,6 +416,7 @@ FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v,
                                     const int32_t *row_ptr, const int32_t *col_idx,
                                     const int32_t *mode_dev, int mode, void *workspace,
                                     size_t ws_bytes, int32_t *dev_status, void *stream) {
+  NvtxRange range_("fa_attn_prefill_backward");
   if (int rc = check_prefill(q, k, v, const_cast<void *>(o), B, S, Hq, Hkv, D)) return rc;
   if (!lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
@@ -402,6 +446,7 @@ FA_API int fa_soft_routed_layer_backward(
     const int32_t *col_idx, void *dq, void *dk, void *dv, float *dw1, float *db1, float *dw2,
     float *db2, float *r_out, void *workspace, size_t ws_bytes, int32_t *dev_status,
     void *stream) {
+  NvtxRange range_("fa_soft_routed_layer_backward");
   if (int rc = check_prefill(q, k, v, const_cast<void *>(o_full), B, S, Hq, Hkv, D)) return rc;
   if (int rc = check_router(q, B, S, Hq, D, 100, 100, w1, hidden, w2)) return rc;
   if (!o_sparse || !lse_full || !lse_sparse || !dy || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
@@ -441,6 +486,7 @@ FA_API int fa_attn_prefill_varlen(const void *q, const void *k, const void *v, v
                                   const int32_t *row_ptr, const int32_t *col_idx,
                                   const int32_t *mode_dev, int mode, void *workspace,
                                   size_t ws_bytes, int32_t *dev_status, void *stream) {
+  NvtxRange range_("fa_attn_prefill_varlen");
   if (int rc = check_varlen(q, k, v, o, cu_seqlens, B, total_tokens, max_seqlen, Hq, Hkv, D))
     return rc;
   if (!(scale > 0.f)) return FA_ERR_INVALID_ARG;
@@ -472,6 +518,7 @@ FA_API int fa_hybrid_layer_varlen(const void *q, const void *k, const void *v, v
                                   const int32_t *col_idx, float *logits_out, int32_t *mode_out,
                                   void *workspace, size_t ws_bytes, int32_t *dev_status,
                                   void *stream) {
+  NvtxRange range_("fa_hybrid_layer_varlen");
   if (int rc = check_varlen(q, k, v, o, cu_seqlens, B, total_tokens, max_seqlen, Hq, Hkv, D))
     return rc;
   if (int rc = check_router(q, B, max_seqlen, Hq, D, 100, 100, w1, hidden, w2)) return rc;
@@ -491,6 +538,8 @@ FA_API int fa_hybrid_layer_varlen(const void *q, const void *k, const void *v, v
   a.cu_seqlens = cu_seqlens;
   a.total_tokens = total_tokens;
   a.varlen_ws = static_cast<uint8_t *>(workspace) + ((rws + 255) & ~static_cast<size_t>(255));
+  a.expect_nnz = index_nnz((max_seqlen + cfg.block - 1) / cfg.block, cfg.sink / cfg.block,
+                           cfg.window / cfg.block);
   return launch_prefill(a, st);
 }
 

@@ -192,16 +192,14 @@ FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Param
   const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
   return __all_sync(0xffffffffu, done);
 }
-FA_DEV bool warp_aborted(const Smem &sh) {
-  return __any_sync(0xffffffffu, ld_shared_s32(sh.abort_flag()) != 0);
-}
 
 // ------------------------------------------------------------- producer
+// kv_n / li: K/V loads and stage loads issued (the abort path drains them).
 FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorMap *tmO,
                          const CUtensorMap *tmK, const CUtensorMap *tmV, const Params &p,
-                         int total) {
-  int kv_n = 0;   // K/V loads issued
-  int li = 0;     // stage loads issued (continues across items)
+                         int total, int &kv_n, int &li) {
+  kv_n = 0;       // K/V loads issued
+  li = 0;         // stage loads issued (continues across items)
   bool ok = true;
   for (int k = 0; ok; ++k) {
     const int w = item_index(k, total);
@@ -242,13 +240,6 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
       bulk_load_w(sh.dvec(s), p.dvec + vo, VEC_BYTES, bar);
       ++li;
     }
-  }
-  if (warp_aborted(sh)) {  // let every copy this warp issued land before exit
-    if (kv_n > 0)
-      mbar_wait_drain_a(sh.bar(Smem::KV_FULL), static_cast<uint32_t>(kv_n - 1) & 1u, kDrainNs);
-    for (int x = (li > NST ? li - NST : 0); x < li; ++x)
-      mbar_wait_drain_a(sh.bar(Smem::ST_FULL0 + x % NST), static_cast<uint32_t>(x / NST) & 1u,
-                        kDrainNs);
   }
 }
 
@@ -355,10 +346,6 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     if (!ok) break;
     ++kv_n;
     ++acc_n;
-  }
-  if (warp_aborted(sh)) {  // let every MMA this warp issued finish before exit
-    tc_commit_w(sh.bar(Smem::DRAIN));
-    mbar_wait_drain_a(sh.bar(Smem::DRAIN), 0, kDrainNs);
   }
 }
 
@@ -648,18 +635,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = static_cast<uint32_t>(ld_shared_s32(sh.tmem_slot()));
+  int kv_loads = 0, loads = 0;
   if (warp < 4) {
     run_ew(sh, tmem, p, total_items);
   } else if (warp < 8) {
     run_dq(sh, tmem, &tmA, p, total_items);
   } else if (warp == WARP_PRODUCER) {
-    run_producer(sh, &tmQ, &tmO, &tmK, &tmV, p, total_items);
+    run_producer(sh, &tmQ, &tmO, &tmK, &tmV, p, total_items, kv_loads, loads);
   } else {
     run_mma(sh, tmem, p, total_items);
   }
   tc_fence_before_sync();
   __syncthreads();
+  // Every wait of every role is over, so the abort flag is final here.  After
+  // an abort, copies and MMAs issued before it may still be in flight: the
+  // producer waits (bounded) for its last loads to land and the MMA warp for
+  // its MMAs to finish before TMEM is freed and the CTA exits.  (The dQ
+  // warps' reduce-adds completed before they left their loop.)
+  const bool aborted = ld_shared_s32(sh.abort_flag()) != 0;
+  if (aborted && warp == WARP_PRODUCER) {
+    if (kv_loads > 0)
+      mbar_wait_drain_a(sh.bar(Smem::KV_FULL), static_cast<uint32_t>(kv_loads - 1) & 1u,
+                        kDrainNs);
+    for (int x = (loads > NST ? loads - NST : 0); x < loads; ++x)
+      mbar_wait_drain_a(sh.bar(Smem::ST_FULL0 + x % NST), static_cast<uint32_t>(x / NST) & 1u,
+                        kDrainNs);
+  }
   if (warp == WARP_MMA) {
+    if (aborted) {
+      tc_commit_w(sh.bar(Smem::DRAIN));
+      mbar_wait_drain_a(sh.bar(Smem::DRAIN), 0, kDrainNs);
+    }
     tc_fence_after_sync();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -1052,6 +1058,8 @@ int run_convert(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
 size_t backward_workspace_bytes(int B, int S, int Hq, int Hkv) {
   return make_plan(B, S, Hq, Hkv, nullptr).bytes;
 }
+
+int set_wait_limit_backward(uint64_t ns) { return set_wait_limit_local(ns); }
 
 int launch_backward(const BackwardLaunch &a, cudaStream_t stream) {
   const Plan pl = make_plan(a.B, a.S, a.Hq, a.Hkv, a.workspace);

@@ -23,6 +23,17 @@ namespace fa {
 // waits inside one CTA last microseconds; this only bounds a broken case.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
 
+// The bound the kernels use, in constant memory so that a test can shorten
+// it (fa_debug_set_wait_limit_ns) and make a wait run out on purpose.  Each
+// translation unit that includes this header holds its own copy;
+// set_wait_limit_local() sets the copy of the unit it is called from, on the
+// current device.  It is read only after a wait's first try failed.
+static __constant__ uint64_t c_wait_limit_ns = kWaitTimeoutNs;
+
+static inline int set_wait_limit_local(uint64_t ns) {
+  return cudaMemcpyToSymbol(c_wait_limit_ns, &ns, sizeof(ns)) == cudaSuccess ? 0 : -1;
+}
+
 FA_DEV uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -76,7 +87,7 @@ FA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int32
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > c_wait_limit_ns) {
       *abort = 1;
       report(status, FA_DEV_TIMEOUT);
       return false;
@@ -121,7 +132,7 @@ FA_DEV bool mbar_wait_a(uint32_t bar, uint32_t parity, uint32_t abort_flag, int3
   while (true) {
     if (mbar_try_wait_a(bar, parity)) return true;
     if (ld_shared_s32(abort_flag)) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > c_wait_limit_ns) {
       st_shared_s32(abort_flag, 1);
       report(status, FA_DEV_TIMEOUT);
       return false;

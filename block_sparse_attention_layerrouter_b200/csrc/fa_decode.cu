@@ -478,10 +478,18 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
   }
   __syncthreads();   // every thread is done with the stages (reused below)
 
-  if (*abort) {  // let the copies still in flight land, then leave
+  if (*abort) {  // a wait ran out: let the copies still in flight land, then leave
     if (tid == 0) {
       for (int x = (issued > NSTAGE ? issued - NSTAGE : 0); x < issued; ++x)
         mbar_wait_drain(&full[x % NSTAGE], static_cast<uint32_t>(x / NSTAGE) & 1u, 200000000ull);
+    }
+    // Mark this split's partials as missing (NaN reference): the combine then
+    // writes NaN for these heads instead of merging whatever the workspace
+    // held before.
+    if (tid < G) {
+      const size_t r0 = (static_cast<size_t>(b) * p.Hq + kvh * G + tid) * p.nsplit + split;
+      p.ml_part[r0 * 2] = __int_as_float(0x7fc00000);
+      p.ml_part[r0 * 2 + 1] = __int_as_float(0x7fc00000);
     }
     __syncthreads();
     return;
@@ -527,6 +535,8 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
 // Merge the splits of one (batch, head): M = max m_s, w_s = 2^(m_s - M),
 // o = sum w_s o_s / sum w_s l_s.  The weights are computed once into shared
 // memory; then thread d walks the splits for output dim d (coalesced rows).
+// A split that gave up (a bounded wait ran out) left a NaN reference: the
+// head's output and LSE are then NaN.
 constexpr int kMaxSplits = 256;
 __global__ void __launch_bounds__(128) combine_kernel(const float *o_part, const float *ml_part,
                                                       __nv_bfloat16 *o, float *lse, int Hq,
@@ -538,7 +548,13 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *o_part, const
   const size_t row = (static_cast<size_t>(b) * Hq + h);
   const float *ml = ml_part + row * nsplit * 2;
   float mx = -INFINITY;
-  for (int s = d; s < nsplit; s += 128) mx = fmaxf(mx, ml[2 * s]);
+  bool missing = false;
+  for (int s = d; s < nsplit; s += 128) {
+    const float m = ml[2 * s];
+    missing |= (m != m);
+    mx = fmaxf(mx, m);
+  }
+  missing = __syncthreads_or(missing) != 0;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   if (lane == 0) red[warp] = mx;
@@ -565,8 +581,10 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *o_part, const
   const float *op = o_part + row * nsplit * HD + d;
   for (int s = 0; s < nsplit; ++s) num = fmaf(w_sm[s], op[static_cast<size_t>(s) * HD], num);
   const bool any = (M != -INFINITY) && den > 0.f;
-  o[row * HD + d] = __float2bfloat16_rn(any ? num / den : 0.f);
-  if (lse && d == 0) lse[row] = any ? (M + __log2f(den)) * 0.69314718055994531f : -INFINITY;
+  const float nan = __int_as_float(0x7fc00000);
+  o[row * HD + d] = __float2bfloat16_rn(missing ? nan : (any ? num / den : 0.f));
+  if (lse && d == 0)
+    lse[row] = missing ? nan : (any ? (M + __log2f(den)) * 0.69314718055994531f : -INFINITY);
 }
 
 }  // namespace decode
@@ -598,6 +616,8 @@ int decode_splits_for_tiles(int B, int Hkv, int tiles) {
 int decode_num_splits(int B, int Hkv, int Lmax) {
   return decode_splits_for_tiles(B, Hkv, (Lmax + decode::KT - 1) / decode::KT);
 }
+
+int set_wait_limit_decode(uint64_t ns) { return set_wait_limit_local(ns); }
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax) {
   const size_t ns = static_cast<size_t>(decode_num_splits(B, Hkv, Lmax));

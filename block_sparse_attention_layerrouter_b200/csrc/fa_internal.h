@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/fa_hybrid.h"
+
 namespace fa {
 
 // 4-D TMA map over a bf16 tensor [B, S, H, 128] (row-major), boxes of
@@ -34,6 +36,9 @@ struct PrefillLaunch {
   const int32_t *cu_seqlens = nullptr;
   int total_tokens = 0;
   void *varlen_ws = nullptr;
+  // Entry count the CSR must have (the block rule's count for S and the
+  // sparse config), checked on the device; -1: not checked.
+  long long expect_nnz = -1;
 };
 size_t varlen_workspace_bytes(int B, int total_tokens);
 int launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
@@ -72,6 +77,11 @@ int launch_kv_append(const KvAppendLaunch &a, cudaStream_t stream);
 // 4-D TMA map over a byte tensor [B, S, H, 128] (an FP8 cache), boxes of
 // 128 x 1 x box_rows x 1 with the 128-byte swizzle.
 int make_tmap_bhsd_u8(CUtensorMap *map, const void *base, int B, int S, int H, int box_rows);
+// Host-side argument checks of fa_attn_decode (everything but the
+// workspace); FA_OK or an fa_status.
+int check_decode_args(const void *q, const void *kcache, const void *vcache,
+                      const int32_t *seqlens, int B, int Lmax, int Hq, int Hkv, int D,
+                      float scale, int mode, fa_sparse_cfg cfg, const void *o);
 int decode_num_splits(int B, int Hkv, int Lmax);
 int decode_splits_for_tiles(int B, int Hkv, int tiles);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax);
@@ -157,6 +167,12 @@ int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream);
 
 // Counts one kernel launch (the total is fa_kernel_launches()).
 void note_launch();
+
+// Bound of the kernels' waits (ns) in each kernel file's constant memory,
+// on the current device; 0 on success.
+int set_wait_limit_prefill(uint64_t ns);
+int set_wait_limit_decode(uint64_t ns);
+int set_wait_limit_backward(uint64_t ns);
 
 long long index_nnz(int nrows, int sb, int wb);
 int launch_index(int nrows, int sb, int wb, int32_t *row_ptr, int32_t *col_idx,

@@ -64,7 +64,17 @@ struct Params {
   int n_qtiles, nqb;
   int mode_default;
   float scale_log2;        // scale * log2(e)
+  int expect_nnz;          // row_ptr[nqb] the CSR must have, or -1 (unchecked)
 };
+
+// The CSR must start at 0 and hold the entry count of the block rule the
+// caller configured; one thread of the grid checks it (a mismatch is
+// reported; the CSR is still walked as given, entry checks included).
+FA_DEV void check_csr_size(const Params &p) {
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.row_ptr != nullptr && p.expect_nnz >= 0) {
+    if (p.row_ptr[0] != 0 || p.row_ptr[p.nqb] != p.expect_nnz) report(p.status, FA_DEV_BAD_INDEX);
+  }
+}
 
 // Writes 32 output columns of one row: o * inv_l as bf16, or, when mix_r is
 // given, r * (the bf16 already there) + (1 - r) * o * inv_l (the soft-routing
@@ -195,9 +205,10 @@ FA_DEV Shared carve(uint8_t *raw) {
 }
 
 // ------------------------------------------------------------- producer ---
-FA_DEV void run_producer(const Shared &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
-                         const CUtensorMap *tmV, const Params &p, int qt, int b, int h,
-                         int kvh, bool sparse) {
+// Returns the number of ring loads issued (the abort path drains them).
+FA_DEV int run_producer(const Shared &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                        const CUtensorMap *tmV, const Params &p, int qt, int b, int h,
+                        int kvh, bool sparse) {
   mbar_arrive_expect_tx(sh.q_full, TILE_BYTES);
   tma_load_4d(sh.q, tmQ, sh.q_full, 0, h, qt * BM, b);
   tma_load_4d(sh.q + HALF_BYTES, tmQ, sh.q_full, 64, h, qt * BM, b);
@@ -228,11 +239,7 @@ FA_DEV void run_producer(const Shared &sh, const CUtensorMap *tmQ, const CUtenso
     n_cur = n_next;
     has = has_next;
   }
-  if (*sh.abort) {  // let every copy this thread issued land before exit
-    mbar_wait_drain(sh.q_full, 0, kDrainNs);
-    for (int x = (li > NSLOT ? li - NSLOT : 0); x < li; ++x)
-      mbar_wait_drain(&sh.full[x % NSLOT], static_cast<uint32_t>(x / NSLOT) & 1u, kDrainNs);
-  }
+  return li;
 }
 
 // ------------------------------------------------------------------ MMA ---
@@ -298,10 +305,6 @@ FA_DEV void run_mma(const Shared &sh, uint32_t tmem, const Params &p, int qt, bo
     if (has_next && !(ok = qk(j + 1))) break;
     if (!(ok = pv(j))) break;
     has = has_next;
-  }
-  if (*sh.abort) {  // let every MMA this thread issued finish before exit
-    tc_commit(sh.drain);
-    mbar_wait_drain(sh.drain, 0, kDrainNs);
   }
 }
 
@@ -481,6 +484,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
+  check_csr_size(p);
   if (warp == 1) {
     tmem_alloc(sh.tmem_slot, TMEM_COLS);
     tmem_relinquish();
@@ -490,8 +494,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *sh.tmem_slot;
 
+  int loads = 0;
   if (warp == 0) {
-    if (lane == 0) run_producer(sh, &tmQ, &tmK, &tmV, p, qt, b, h, kvh, sparse);
+    if (lane == 0) loads = run_producer(sh, &tmQ, &tmK, &tmV, p, qt, b, h, kvh, sparse);
   } else if (warp == 1) {
     if (lane == 0) run_mma(sh, tmem, p, qt, sparse);
     __syncwarp();
@@ -500,7 +505,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   tc_fence_before_sync();
   __syncthreads();
+  // Every wait of every role is over, so the abort flag is final here.  After
+  // an abort, copies and MMAs issued before it may still be in flight: the
+  // producer waits (bounded) for its last loads to land and the MMA thread
+  // for its MMAs to finish before TMEM is freed and the CTA exits.
+  const bool aborted = *sh.abort != 0;
+  if (aborted && warp == 0 && lane == 0) {
+    mbar_wait_drain(sh.q_full, 0, kDrainNs);
+    for (int x = (loads > NSLOT ? loads - NSLOT : 0); x < loads; ++x)
+      mbar_wait_drain(&sh.full[x % NSLOT], static_cast<uint32_t>(x / NSLOT) & 1u, kDrainNs);
+  }
   if (warp == 1) {
+    if (aborted && lane == 0) {
+      tc_commit(sh.drain);
+      mbar_wait_drain(sh.drain, 0, kDrainNs);
+    }
+    __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -689,16 +709,14 @@ FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Param
   const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
   return __all_sync(0xffffffffu, done);
 }
-FA_DEV bool warp_aborted(const Smem &sh) {
-  return __any_sync(0xffffffffu, ld_shared_s32(sh.abort_flag()) != 0);
-}
-
 // The producer and MMA roles run on all 32 lanes of their warp with
 // warp-uniform state; one elected lane issues each TMA copy, MMA and commit.
+// li / nq: ring loads and Q loads issued (the abort path drains them).
 FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
-                         const CUtensorMap *tmV, const Params &p, int total) {
-  int li = 0;       // ring loads issued (continues across items)
-  int nq = 0;       // Q loads issued
+                         const CUtensorMap *tmV, const Params &p, int total, int &li,
+                         int &nq) {
+  li = 0;           // ring loads issued (continues across items)
+  nq = 0;           // Q loads issued
   int ig = 0;       // tile entries handed to the MMA and softmax warps
   bool ok = true;
   for (int k = 0; ok; ++k) {
@@ -756,12 +774,6 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
       bits = bits2;
       has = has2;
     }
-  }
-  if (warp_aborted(sh)) {  // let every copy this warp issued land before exit
-    if (nq > 0) mbar_wait_drain_a(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(nq - 1) & 1u, kDrainNs);
-    for (int x = (li > NSLOT ? li - NSLOT : 0); x < li; ++x)
-      mbar_wait_drain_a(sh.bar(Smem::FULL0 + x % NSLOT), static_cast<uint32_t>(x / NSLOT) & 1u,
-                        kDrainNs);
   }
 }
 
@@ -879,10 +891,6 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));
     }
     ++done_items;
-  }
-  if (warp_aborted(sh)) {  // let every MMA this warp issued finish before exit
-    tc_commit_w(sh.bar(Smem::DRAIN));
-    mbar_wait_drain_a(sh.bar(Smem::DRAIN), 0, kDrainNs);
   }
 }
 
@@ -1083,6 +1091,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
+  prefill::check_csr_size(p);
   if (warp == WARP_MMA) {
     tmem_alloc_a(sh.tmem_slot(), TMEM_COLS);
     tmem_relinquish();
@@ -1093,10 +1102,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = static_cast<uint32_t>(ld_shared_s32(sh.tmem_slot()));
   if (p.cu_seqlens) total_items = *p.n_items * (p.Hq / NQ);
 
+  int loads = 0, qloads = 0;
   if (warp >= WARP_PRODUCER) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
     if (warp == WARP_PRODUCER) {
-      run_producer(sh, &tmQ, &tmK, &tmV, p, total_items);
+      run_producer(sh, &tmQ, &tmK, &tmV, p, total_items, loads, qloads);
     } else if (warp == WARP_MMA) {
       run_mma(sh, tmem, p, total_items);
     }
@@ -1106,7 +1116,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   tc_fence_before_sync();
   __syncthreads();
+  // Every wait of every role is over, so the abort flag is final here.  After
+  // an abort, copies and MMAs issued before it may still be in flight: the
+  // producer waits (bounded) for its last loads to land and the MMA warp for
+  // its MMAs to finish before TMEM is freed and the CTA exits.
+  const bool aborted = ld_shared_s32(sh.abort_flag()) != 0;
+  if (aborted && warp == WARP_PRODUCER) {
+    if (qloads > 0)
+      mbar_wait_drain_a(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(qloads - 1) & 1u, kDrainNs);
+    for (int x = (loads > NSLOT ? loads - NSLOT : 0); x < loads; ++x)
+      mbar_wait_drain_a(sh.bar(Smem::FULL0 + x % NSLOT), static_cast<uint32_t>(x / NSLOT) & 1u,
+                        kDrainNs);
+  }
   if (warp == WARP_MMA) {
+    if (aborted) {
+      tc_commit_w(sh.bar(Smem::DRAIN));
+      mbar_wait_drain_a(sh.bar(Smem::DRAIN), 0, kDrainNs);
+    }
     tc_fence_after_sync();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -1162,6 +1188,8 @@ __global__ void __launch_bounds__(1024) varlen_items_kernel(const int32_t *cu, i
 }  // namespace prefill2
 
 // ----------------------------------------------------------------- host ---
+int set_wait_limit_prefill(uint64_t ns) { return set_wait_limit_local(ns); }
+
 size_t varlen_workspace_bytes(int B, int total_tokens) {
   const size_t max_items = static_cast<size_t>(total_tokens) / prefill2::BM + B + 1;
   return 256 + 4 * max_items;
@@ -1213,6 +1241,8 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   p.nqb = (a.S + 63) / 64;
   p.mode_default = a.mode_default;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.expect_nnz = (a.expect_nnz >= 0 && a.expect_nnz <= 0x7fffffffLL)
+                     ? static_cast<int>(a.expect_nnz) : -1;
   long long grid =
       static_cast<long long>(p.n_qtiles) * a.B * (two_tiles ? a.Hq / 2 : a.Hq);
   if (varlen) {

@@ -80,6 +80,17 @@ FA_API const char *fa_status_string(int status);
 /* Library ABI version (major * 100 + minor). */
 FA_API int fa_version(void);
 
+/* Testing aid: sets the bound of every wait inside this library's kernels
+ * (default 2 s) on the current device.  Each wait in a kernel is bounded; a
+ * wait that runs out makes the kernel give up (FA_DEV_TIMEOUT in dev_status,
+ * the outputs of that call invalid; a decode head whose split gave up reads
+ * NaN), let its copies and MMAs in flight finish and return, leaving the
+ * device usable.  A short bound (0 works) makes that happen on purpose, so a
+ * test can check the path; put the default back afterwards.  Synchronous (a
+ * copy to device constant memory): not during stream capture or while this
+ * library's kernels run.  Returns FA_OK or FA_ERR_CUDA. */
+FA_API int fa_debug_set_wait_limit_ns(unsigned long long ns);
+
 /* Number of kernels this library has enqueued in this process so far, on
  * any stream and device (a host-side count taken at each launch; calls
  * rejected by their host-side checks launch nothing and add nothing).  For
@@ -331,16 +342,21 @@ FA_API int fa_soft_routed_layer(const void *q, const void *k, const void *v,
  * that cannot allocate device memory where they run decode (a plugin behind
  * a fixed operator interface with no workspace argument, an engine whose
  * memory is all reserved up front, a real-time loop where cudaMalloc is not
- * allowed).  Same arguments and results as fa_attn_decode without the
- * workspace: the split-KV scratch lives in one static device array of
+ * allowed).  Same arguments, checks and results as fa_attn_decode without
+ * the workspace: the split-KV scratch lives in one static device array of
  * fa_noalloc_scratch_bytes() (8 MiB) that every GPU loading this library
  * holds until exit.  The call allocates nothing.
- *  - Returns FA_ERR_UNSUPPORTED when the shape needs more scratch than that
- *    (fa_decode_workspace_size(B, Hq, Hkv, Lmax, D) > 8 MiB).
+ *  - Arguments are checked as by fa_attn_decode first (same status codes);
+ *    then FA_ERR_UNSUPPORTED when the shape needs more scratch than the array
+ *    holds (fa_decode_workspace_size(B, Hq, Hkv, Lmax, D) > 8 MiB).
  *  - The first call on a device (with that device current) looks up the
- *    array's device address once; make it before any stream capture.
- *  - All calls share the array (nothing in it needs to start at zero): calls
- *    whose kernels overlap on the GPU race and must be serialised. */
+ *    array's device address; it is cached with the CUDA context's id and
+ *    looked up again in a new context (after a device reset).  Make the first
+ *    call on a device before any stream capture.
+ *  - All calls share the array.  Nothing in it needs to start at zero: every
+ *    split overwrites its slot before the merge reads it (a split that gave
+ *    up marks its slot, and those heads read NaN).  Calls whose kernels
+ *    overlap on the GPU race on the array and must be serialised. */
 FA_API size_t fa_noalloc_scratch_bytes(void);
 FA_API int fa_attn_decode_noalloc(const void *q, const void *kcache,
                                   const void *vcache, const int32_t *seqlens,
@@ -356,6 +372,13 @@ FA_API int fa_attn_decode_noalloc(const void *q, const void *kcache,
  * and runs exact causal attention (FULL) or block-sparse attention over the
  * caller's CSR (SPARSE; build it once with fa_blocksparse_index for this S and
  * cfg).  Arguments as for the calls above; n_head/n_tail are 100/100.
+ * The CSR is read on the device only, so the host cannot compare it with
+ * cfg: the kernel checks that row_ptr[0] = 0 and that row_ptr[last] is the
+ * entry count of the block rule for (S, cfg), and reports a mismatch as
+ * FA_DEV_BAD_INDEX (then attends the CSR as given; every entry is still
+ * checked against the causal range).  A CSR with the right count but other
+ * entries is attended as given.  The same holds for the varlen and
+ * soft-routed layers (count for max_seqlen, resp. S).
  *   workspace >= fa_hybrid_workspace_size(B, Hq, D, hidden) bytes. */
 FA_API size_t fa_hybrid_workspace_size(int B, int Hq, int D, int hidden);
 FA_API int fa_hybrid_layer(const void *q, const void *k, const void *v, void *o,

@@ -21,7 +21,9 @@ Sources are cited by page title and section:
 * [SELFATTN] "Self-Attention 이후: 트랜스포머 다음에 올 것들", section "셀프
   어텐션이 비싼 이유" (scores = Q K^T / sqrt(d_k), softmax, times V).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent (the router paragraphs of [FLUX]
+state "compress", not the operator, and give no flatten order, tie rule or
+window granularity; [SELFATTN] gives the 1/sqrt(d_k) scale):
 pooling is the arithmetic mean; the pooled [1 x h x d'] tensor is flattened
 head-major (x[h*D + d]); a tie pi_SA == pi_FA routes to FULL; the local window
 is counted in whole 64-token blocks including the query's own block; key k is

@@ -47,3 +47,39 @@ def assert_close_grad(got: np.ndarray, ref: np.ndarray, what: str):
         "%s: max-abs/max|ref| %.3g (tol %.1g), mean-abs/mean|ref| %.3g (tol %.1g)"
         % (what, mx, GRAD_MAX_REL, mean, GRAD_MEAN_REL))
     return mx, mean
+
+
+# ------------------------------------------------------------- canaries
+# The sanitizer's out-of-bounds checks are not available here, so the
+# kernels' writes are fenced by sentinels instead: an output (or workspace)
+# is a view into a larger buffer whose head and tail hold a sentinel bit
+# pattern, and the output itself starts as NaN.  After the call the head and
+# tail must hold the sentinel still (no write past either end) and every
+# output element must be finite (no element left unwritten).
+_SENTINEL = {torch.bfloat16: (torch.int16, 0x7FA5),           # a NaN bit pattern
+             torch.float32: (torch.int32, 0x7FC0A5A5),        # a NaN bit pattern
+             torch.uint8: (torch.uint8, 0xA5)}
+
+
+class Guarded:
+    def __init__(self, shape, dtype, pad=4096, device="cuda"):
+        n = 1
+        for s in shape:
+            n *= int(s)
+        self.n, self.pad = n, pad
+        self.buf = torch.empty(n + 2 * pad, dtype=dtype, device=device)
+        view_dtype, pattern = _SENTINEL[dtype]
+        self.buf.view(view_dtype).fill_(pattern)
+        self.t = self.buf[pad:pad + n].view(*shape)
+        self._pattern = self.buf.view(view_dtype)[:pad].clone()
+
+    def check_fences(self, what):
+        vd = self._pattern.dtype
+        head = self.buf.view(vd)[:self.pad]
+        tail = self.buf.view(vd)[self.pad + self.n:]
+        assert torch.equal(head, self._pattern), "%s: write before the start" % what
+        assert torch.equal(tail, self._pattern), "%s: write past the end" % what
+
+    def check_all_written(self, what):
+        self.check_fences(what)
+        assert bool(torch.isfinite(self.t.float()).all()), "%s: element left unwritten" % what

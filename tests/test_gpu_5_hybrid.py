@@ -47,3 +47,24 @@ def test_hybrid_layer_routes_and_matches(bias, want):
                                   inputs.bits(v[b:b + 1]), 1 / math.sqrt(128),
                                   mask if mode[b] == 1 else None)
         assert_close_attention(to_f64(o[b:b + 1]), ref, "hybrid b=%d" % b)
+
+
+def test_hybrid_layer_reports_a_csr_built_for_another_window():
+    """The routed layer reads the CSR on the device only; one built for
+    another window (a different entry count) is reported as
+    FA_DEV_BAD_INDEX, and the one built for its own window is not."""
+    B, S, Hq, Hkv = 1, 1024, 4, 2
+    q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, seed=62)
+    w1, b1, w2, b2 = [t.cuda() for t in inputs.router_weights(Hq * 128, 64, seed=62,
+                                                               b2=(0.0, 0.1))]
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    c = capi.cfg(64, 128, 256)
+    rp_own, ci_own = capi.blocksparse_index(S, c)
+    rp_other, ci_other = capi.blocksparse_index(S, capi.cfg(64, 128, 512))
+    st = zero_status()
+    capi.hybrid_layer(qd, kd, vd, w1, b1, w2, b2, rp_own, ci_own, c, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    capi.hybrid_layer(qd, kd, vd, w1, b1, w2, b2, rp_other, ci_other, c, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & capi.FA_DEV_BAD_INDEX

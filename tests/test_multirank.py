@@ -59,3 +59,26 @@ def test_reference_arm_under_torchrun_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` run directly (no torchrun) starts two ranks itself;
+    the host-only dry run prints exactly one line, from rank 0, with
+    n_gpus = 2."""
+    cmd = [sys.executable, "bench.py", "--gpus", "2", "--dry-run", "--steps", "1", "--warmup",
+           "3", "--workload", "mha4-s1024"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["dry_run"] is True and d["scaling"] == "weak"
+    assert d["config"]["parallelism"].startswith("replicas")
+
+
+def test_bench_rejects_gpus_that_disagree_with_world_size():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    cmd = [sys.executable, "bench.py", "--gpus", "2", "--dry-run", "--steps", "1", "--warmup",
+           "3", "--workload", "mha4-s1024"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr
