@@ -47,10 +47,10 @@ EncodeTiledFn encode_fn() {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-}  // namespace
-
-int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols,
-                   int box_rows) {
+// 4-D TMA map over a bf16 tensor [B, S, H, 128] with boxes of box_cols x 1 x
+// box_rows x 1.
+int tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols, int box_rows,
+              CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return -1;
   const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
@@ -61,11 +61,23 @@ int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int 
                              static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -1;
 }
+
+}  // namespace
+
+int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols,
+                   int box_rows) {
+  return tmap_bhsd(map, base, B, S, H, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int make_tmap_bhsd_plain(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols,
+                         int box_rows) {
+  return tmap_bhsd(map, base, B, S, H, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 
 int make_tmap_bhsd_u8(CUtensorMap *map, const void *base, int B, int S, int H, int box_rows) {
   EncodeTiledFn fn = encode_fn();

@@ -23,11 +23,14 @@ namespace fa {
 // waits inside one CTA last microseconds; this only bounds a broken case.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
 
-// The bound the kernels use, in constant memory so that a test can shorten
+// The bound the kernels use, in constant memory so that a test can change
 // it (fa_debug_set_wait_limit_ns) and make a wait run out on purpose.  Each
 // translation unit that includes this header holds its own copy;
 // set_wait_limit_local() sets the copy of the unit it is called from, on the
-// current device.  It is read only after a wait's first try failed.
+// current device.  0 is the testing mode: a wait whose phase is not complete
+// at its first (non-blocking) test gives up at once.  (With a positive bound
+// a wait can still outlast it: mbarrier.try_wait may suspend the thread until
+// the phase completes, and the bound is checked between tries.)
 static __constant__ uint64_t c_wait_limit_ns = kWaitTimeoutNs;
 
 static inline int set_wait_limit_local(uint64_t ns) {
@@ -79,9 +82,27 @@ FA_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+FA_DEV bool mbar_test_wait_a(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase of parity `parity` of `bar` has completed.  Returns
 // false (and sets *abort) if the CTA is aborting or the wait ran out.
 FA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *status) {
+  if (c_wait_limit_ns == 0) {   // testing mode: give up unless complete already
+    if (mbar_test_wait_a(smem_u32(bar), parity)) return true;
+    *abort = 1;
+    report(status, FA_DEV_TIMEOUT);
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -127,6 +148,12 @@ FA_DEV void st_shared_s32(uint32_t addr, int v) {
 }
 // Bounded wait; `abort_flag` is the shared address of the CTA's abort word.
 FA_DEV bool mbar_wait_a(uint32_t bar, uint32_t parity, uint32_t abort_flag, int32_t *status) {
+  if (c_wait_limit_ns == 0) {   // testing mode: give up unless complete already
+    if (mbar_test_wait_a(bar, parity)) return true;
+    st_shared_s32(abort_flag, 1);
+    report(status, FA_DEV_TIMEOUT);
+    return false;
+  }
   if (mbar_try_wait_a(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -330,6 +357,21 @@ FA_DEV void tma_reduce_add_2d_w(const CUtensorMap *map, uint32_t src, int c0, in
       "r"(c0), "r"(c1), "r"(src)
       : "memory");
 }
+// 4-D tiled TMA store of a shared-memory box into a global tensor (bulk
+// group completion; the calling thread issues it and commits the group).
+// Coordinates >= 0, the innermost one 16-byte aligned; parts of the box
+// outside the tensor's extent are not written.
+FA_DEV void tma_store_4d_commit(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2,
+                                int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];\n\t"
+      "cp.async.bulk.commit_group;" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src)
+      : "memory");
+}
+// Wait until all but the most recent of this thread's committed bulk groups
+// have finished reading their shared-memory sources.
+FA_DEV void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // Wait until this thread's committed bulk groups have finished reading their
 // shared-memory sources (all but `n` most recent).
 FA_DEV void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
@@ -364,6 +406,19 @@ FA_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[31])
       : "r"(taddr)
       : "memory");
+}
+// TMEM -> registers: 32 lanes x 32 bits, 64 consecutive columns per thread,
+// then one wait.
+FA_DEV void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]),"=r"(r[1]),"=r"(r[2]),"=r"(r[3]),"=r"(r[4]),"=r"(r[5]),"=r"(r[6]),"=r"(r[7]),"=r"(r[8]),"=r"(r[9]),"=r"(r[10]),"=r"(r[11]),"=r"(r[12]),"=r"(r[13]),"=r"(r[14]),"=r"(r[15]),"=r"(r[16]),"=r"(r[17]),"=r"(r[18]),"=r"(r[19]),"=r"(r[20]),"=r"(r[21]),"=r"(r[22]),"=r"(r[23]),"=r"(r[24]),"=r"(r[25]),"=r"(r[26]),"=r"(r[27]),"=r"(r[28]),"=r"(r[29]),"=r"(r[30]),"=r"(r[31]),"=r"(r[32]),"=r"(r[33]),"=r"(r[34]),"=r"(r[35]),"=r"(r[36]),"=r"(r[37]),"=r"(r[38]),"=r"(r[39]),"=r"(r[40]),"=r"(r[41]),"=r"(r[42]),"=r"(r[43]),"=r"(r[44]),"=r"(r[45]),"=r"(r[46]),"=r"(r[47]),"=r"(r[48]),"=r"(r[49]),"=r"(r[50]),"=r"(r[51]),"=r"(r[52]),"=r"(r[53]),"=r"(r[54]),"=r"(r[55]),"=r"(r[56]),"=r"(r[57]),"=r"(r[58]),"=r"(r[59]),"=r"(r[60]),"=r"(r[61]),"=r"(r[62]),"=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]),"+r"(r[1]),"+r"(r[2]),"+r"(r[3]),"+r"(r[4]),"+r"(r[5]),"+r"(r[6]),"+r"(r[7]),"+r"(r[8]),"+r"(r[9]),"+r"(r[10]),"+r"(r[11]),"+r"(r[12]),"+r"(r[13]),"+r"(r[14]),"+r"(r[15]),"+r"(r[16]),"+r"(r[17]),"+r"(r[18]),"+r"(r[19]),"+r"(r[20]),"+r"(r[21]),"+r"(r[22]),"+r"(r[23]),"+r"(r[24]),"+r"(r[25]),"+r"(r[26]),"+r"(r[27]),"+r"(r[28]),"+r"(r[29]),"+r"(r[30]),"+r"(r[31]),"+r"(r[32]),"+r"(r[33]),"+r"(r[34]),"+r"(r[35]),"+r"(r[36]),"+r"(r[37]),"+r"(r[38]),"+r"(r[39]),"+r"(r[40]),"+r"(r[41]),"+r"(r[42]),"+r"(r[43]),"+r"(r[44]),"+r"(r[45]),"+r"(r[46]),"+r"(r[47]),"+r"(r[48]),"+r"(r[49]),"+r"(r[50]),"+r"(r[51]),"+r"(r[52]),"+r"(r[53]),"+r"(r[54]),"+r"(r[55]),"+r"(r[56]),"+r"(r[57]),"+r"(r[58]),"+r"(r[59]),"+r"(r[60]),"+r"(r[61]),"+r"(r[62]),"+r"(r[63])
+               :
+               : "memory");
 }
 // Wait for this thread's TMEM loads; the "+r" operands keep the compiler
 // from using the loaded registers before the wait.

@@ -15,6 +15,9 @@ namespace fa {
 // box_cols x 1 x box_rows x 1 with the 128-byte swizzle.  Returns 0 on success.
 int make_tmap_bhsd(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols,
                    int box_rows);
+// The same without swizzle (a box is stored row-major in shared memory).
+int make_tmap_bhsd_plain(CUtensorMap *map, const void *base, int B, int S, int H, int box_cols,
+                         int box_rows);
 
 // 2-D TMA map over an fp32 tensor [rows, 128] (row-major), boxes of
 // box_cols x box_rows, no swizzle.  Returns 0 on success.

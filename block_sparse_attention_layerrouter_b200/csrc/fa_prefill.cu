@@ -65,6 +65,8 @@ struct Params {
   int mode_default;
   float scale_log2;        // scale * log2(e)
   int expect_nnz;          // row_ptr[nqb] the CSR must have, or -1 (unchecked)
+  int band_q;              // two-tile kernel: q-tiles per band of the KV-head-major item
+                           // order, or 0 for the query-tile-major order
 };
 
 // The CSR must start at 0 and hold the entry count of the block rule the
@@ -554,7 +556,18 @@ namespace prefill2 {
 using prefill::Params;
 using prefill::TileIter;
 constexpr int BM = 128, BN = 128, HD = 128, NQ = 2;
-constexpr int NSLOT = 5;
+// Epilogue: each softmax warp writes its 32 rows x 32 columns of O (bf16)
+// into a staging box in shared memory and one lane stores it with a TMA bulk
+// tensor store, instead of 16-byte stores of single rows (each warp-wide
+// store instruction of the latter touches 32 rows 8 KB apart).  The staging
+// (2 boxes per warp) takes the shared memory of one K/V ring slot.
+#ifndef FA_TMA_EPILOGUE
+#define FA_TMA_EPILOGUE 1
+#endif
+constexpr bool kTmaEpilogue = FA_TMA_EPILOGUE != 0;
+constexpr int NSLOT = kTmaEpilogue ? 4 : 5;
+constexpr int STG_BOX = 32 * 32 * 2;              // 32 rows x 32 bf16 columns
+constexpr int STG_BYTES = kTmaEpilogue ? 8 * 2 * STG_BOX : 0;
 constexpr int TILE_BYTES = BN * HD * 2;
 constexpr int HALF_BYTES = TILE_BYTES / 2;
 constexpr int NUM_THREADS = 384;                 // 3 warpgroups
@@ -572,7 +585,7 @@ constexpr int NUM_BARS = 2 + 2 * NSLOT + 4 * NQ + 1 + 16;
 // tiles).  A full item's tiles 0..qt need no list.
 constexpr int NINFO = 8;
 constexpr int SMEM_BYTES =
-    1024 + NQ * TILE_BYTES + NSLOT * TILE_BYTES + NUM_BARS * 8 + 16 + 4 * NINFO;
+    1024 + NQ * TILE_BYTES + NSLOT * TILE_BYTES + STG_BYTES + NUM_BARS * 8 + 16 + 4 * NINFO;
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;
@@ -621,11 +634,12 @@ FA_DEV void ex2_poly2(uint64_t x2, float &r0, float &r1) {
 }
 
 // Shared-memory layout, as offsets from one 1024-byte aligned base:
-// Q tiles | K/V ring | mbarriers | TMEM address | abort word.
+// Q tiles | K/V ring | epilogue staging | mbarriers | TMEM address | abort word.
 struct Smem {
   uint32_t base;
   static constexpr uint32_t kRing = NQ * TILE_BYTES;
-  static constexpr uint32_t kBars = kRing + NSLOT * TILE_BYTES;
+  static constexpr uint32_t kStg = kRing + NSLOT * TILE_BYTES;
+  static constexpr uint32_t kBars = kStg + STG_BYTES;
   enum : uint32_t {
     Q_FULL = 0, Q_EMPTY = 1, FULL0 = 2, EMPTY0 = FULL0 + NSLOT, S_FULL0 = EMPTY0 + NSLOT,
     P_FULL0 = S_FULL0 + NQ, O_DONE0 = P_FULL0 + NQ, O_FREE0 = O_DONE0 + NQ, DRAIN = O_FREE0 + NQ,
@@ -633,6 +647,8 @@ struct Smem {
   };
   FA_DEV uint32_t q(int t) const { return base + t * TILE_BYTES; }
   FA_DEV uint32_t ring(int slot) const { return base + kRing + slot * TILE_BYTES; }
+  // Staging box `u` (0/1) of softmax warp `w` (0..7).
+  FA_DEV uint32_t stg(int w, int u) const { return base + kStg + (2 * w + u) * STG_BOX; }
   FA_DEV uint32_t bar(uint32_t i) const { return base + kBars + 8u * i; }
   FA_DEV uint32_t tmem_slot() const { return base + kBars + 8u * NBARS; }
   FA_DEV uint32_t abort_flag() const { return tmem_slot() + 4u; }
@@ -648,8 +664,17 @@ FA_DEV Smem carve(uint8_t *raw) {
 }
 
 // Work item -> (query tile, batch, first head of the pair).  Items are
-// numbered longest causal rows first; the head pairs of one KV group are
-// adjacent so K/V tiles are shared through L2.
+// numbered longest causal rows first.  Two orders:
+//  * query-tile-major (band_q = 0): all head pairs of one query tile, then
+//    the next tile down; the head pairs of one KV group are adjacent.  The
+//    CTAs running together cover every KV head.
+//  * KV-head-major bands (long sequences): a band is band_q query tiles; its
+//    items are ordered by KV stream (batch, KV head), then query tile, then
+//    head pair, so the CTAs running together (band_q x pairs-per-KV-head =
+//    one CTA per SM) all stream the K/V tiles of the same KV head and each
+//    tile is read from HBM about once per band rather than once per CTA
+//    that drifted out of L2 reach.  Lengths inside a band differ by at most
+//    band_q tiles.
 struct Item {
   int qt, b, h0, kvh;
   bool sparse;
@@ -676,11 +701,33 @@ FA_DEV Item item_of(const Params &p, int w) {
     it.lse0 = t0;
     it.lse_hs = p.total_tokens;
   } else {
-    const int bh = p.B * hp_count;
-    it.qt = p.n_qtiles - 1 - w / bh;
-    const int rem = w % bh;
-    it.b = rem / hp_count;
-    it.h0 = (rem % hp_count) * NQ;
+    if (p.band_q > 0) {
+      const int ppk = p.G / NQ;                       // head pairs per KV head
+      const int nkv = p.Hq / p.G;
+      const int streams = p.B * nkv;
+      const int full_items = p.band_q * ppk * streams;  // items of a full band
+      const int full_bands = p.n_qtiles / p.band_q;
+      int band, rows, r;
+      if (w < full_bands * full_items) {
+        band = w / full_items;
+        rows = p.band_q;
+        r = w % full_items;
+      } else {                                        // the last, partial band
+        band = full_bands;
+        rows = p.n_qtiles - full_bands * p.band_q;
+        r = w - full_bands * full_items;
+      }
+      const int s = r / (rows * ppk), rr = r % (rows * ppk);
+      it.qt = p.n_qtiles - 1 - band * p.band_q - rr / ppk;
+      it.b = s / nkv;
+      it.h0 = (s % nkv) * p.G + (rr % ppk) * NQ;
+    } else {
+      const int bh = p.B * hp_count;
+      it.qt = p.n_qtiles - 1 - w / bh;
+      const int rem = w % bh;
+      it.b = rem / hp_count;
+      it.h0 = (rem % hp_count) * NQ;
+    }
     it.L = p.S;
     it.row0 = it.b * p.S;
     it.tma_tok0 = 0;
@@ -709,6 +756,18 @@ FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Param
   const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
   return __all_sync(0xffffffffu, done);
 }
+// Which 64-key half of a 128-key tile its 4-bit block mask (bit 2*qs + ks)
+// keeps: 0 both, 1 only keys 0-63 (no ks = 1 bit), 2 only keys 64-127.  A
+// half tile (the first window tile of a sparse row pair, for instance) is
+// computed with N = 64 / K = 64 products and 64 exponentials per row.
+#ifndef FA_HALF_TILES
+#define FA_HALF_TILES 1
+#endif
+FA_DEV int half_of(uint32_t bits) {
+  if (!FA_HALF_TILES) return 0;
+  return (bits & 0xAu) == 0u ? 1 : ((bits & 0x5u) == 0u ? 2 : 0);
+}
+
 // The producer and MMA roles run on all 32 lanes of their warp with
 // warp-uniform state; one elected lane issues each TMA copy, MMA and commit.
 // li / nq: ring loads and Q loads issued (the abort path drains them).
@@ -779,6 +838,7 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
 
 FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
+  constexpr uint32_t kIdescQK64 = idesc_bf16_f32(BM, BN / 2, false);   // half tiles
   constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
   // Descriptors of the Q tiles (fixed) and of ring slot 0; slot s adds
   // s * TILE_BYTES / 16 to the start-address field, a K step kk adds the
@@ -813,17 +873,30 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     tc_fence_after_sync();
     return true;
   };
-  auto qk = [&](int t, int slot) {
+  // S_t = Q_t K^T of one tile; a half tile (half = 1: keys 0-63, 2: keys
+  // 64-127) takes N = 64 and writes S columns 0-63 or 64-127.
+  auto qk = [&](int t, int slot, int half) {
     const uint64_t qd = t ? q_desc1 : q_desc0;
-    const uint64_t kd = k_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
+    uint64_t kd = k_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
+    uint32_t d = tmem + 256u * t;
+    uint32_t idesc = kIdescQK;
+    if (half != 0) {
+      idesc = kIdescQK64;
+      if (half == 2) {
+        kd += static_cast<uint64_t>((64 * 128) >> 4);   // key rows 64.. of each 64-column box
+        d += 64u;
+      }
+    }
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
       const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-      mma_bf16_ss_w(tmem + 256u * t, qd + off, kd + off, kIdescQK, kk > 0 ? 1u : 0u);
+      mma_bf16_ss_w(d, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
     }
     tc_commit_w(sh.bar(Smem::S_FULL0 + t));
   };
-  auto pv = [&](int t, bool first, int slot) -> bool {
+  // O_t (+)= P_t V over the tile's keys, or over the half's 64 keys (K steps
+  // 0-3 or 4-7; P of key k sits in TMEM column k / 2 either way).
+  auto pv = [&](int t, bool first, int slot, int half) -> bool {
     if (!warp_wait(sh.bar(Smem::P_FULL0 + t), static_cast<uint32_t>(jp) & 1u, sh, p))
       return false;
     if (first && done_items > 0 &&
@@ -831,11 +904,13 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       return false;
     tc_fence_after_sync();
     const uint64_t vd = v_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
+    const int kb = half == 2 ? 4 : 0, ke = half == 1 ? 4 : BN / 16;
 #pragma unroll
     for (int kk = 0; kk < BN / 16; ++kk) {
+      if (kk < kb || kk >= ke) continue;
       mma_bf16_ts_w(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
                     vd + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
-                    (!first || kk > 0) ? 1u : 0u);
+                    (!first || kk > kb) ? 1u : 0u);
     }
     return true;
   };
@@ -847,6 +922,7 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     if (!(ok = warp_wait(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(k) & 1u, sh, p))) break;
     tc_fence_after_sync();
     bool has_next = im.qt > 0, has_next2 = false;     // full item: tiles 0..qt
+    int half = 0, half2 = 0;                           // half tiles (sparse items only)
     if (im.sparse) {
       const int e0 = take_info(ok);
       if (!ok) break;
@@ -855,39 +931,42 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
         continue;
       }
       has_next = (e0 & 0x20) == 0;
+      half = half_of(static_cast<uint32_t>(e0) & 15u);
     }
     int k_slot = 0, v_slot = 0;
     if (!(ok = take(k_slot))) break;
-    qk(0, k_slot);
-    qk(1, k_slot);
+    qk(0, k_slot, half);
+    qk(1, k_slot, half);
     tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
     if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));     // the last QK of this item is issued
     for (int j = 0;; ++j) {
       if (!(ok = take(v_slot))) break;
-      if (!(ok = pv(0, j == 0, v_slot))) break;
+      if (!(ok = pv(0, j == 0, v_slot, half))) break;
       if (has_next) {
         if (im.sparse) {                      // tile j+1: is it the last?
           const int e = take_info(ok);
           if (!ok) break;
           has_next2 = (e & 0x20) == 0;
+          half2 = half_of(static_cast<uint32_t>(e) & 15u);
         } else {
           has_next2 = j + 1 < im.qt;
         }
         if (!(ok = take(k_slot))) break;
-        qk(0, k_slot);
+        qk(0, k_slot, half2);
       } else {
         tc_commit_w(sh.bar(Smem::O_DONE0));
       }
-      if (!(ok = pv(1, j == 0, v_slot))) break;
+      if (!(ok = pv(1, j == 0, v_slot, half))) break;
       ++jp;
       tc_commit_w(sh.bar(Smem::EMPTY0 + v_slot));
       if (!has_next) {
         tc_commit_w(sh.bar(Smem::O_DONE0 + 1));
         break;
       }
-      qk(1, k_slot);
+      qk(1, k_slot, half2);
       tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
       has_next = has_next2;
+      half = half2;
       if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));
     }
     ++done_items;
@@ -895,7 +974,98 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
 }
 
 
-FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int total, int t) {
+// Softmax of one S tile of NC columns (128, or 64 for a half tile) starting
+// at column col0 of S_t, for the row r of this thread: mask (the block mask
+// `bits`, causal on the diagonal tile), row max, P = 2^(s*c - m) written as
+// bf16 pairs into columns col0/2 .. of S_t (the A operand of the PV product),
+// O rescaled when the running max grew by more than kRescaleThreshold
+// (`rescale_ok`: a PV product of this item has run), running max and sum.
+template <int NC>
+FA_DEV void softmax_tile(uint32_t s_base, uint32_t o_base, int col0, uint32_t bits, bool diag,
+                         int r, float c, bool rescale_ok, float &m_run, float &l_run) {
+  float s[NC];
+  {
+    uint32_t raw[NC];
+    if constexpr (NC == BN) {
+      tmem_ld128_wait(s_base, raw);
+    } else {
+      tmem_ld64_wait(s_base + static_cast<uint32_t>(col0), raw);
+    }
+#pragma unroll
+    for (int i = 0; i < NC; ++i) s[i] = __uint_as_float(raw[i]);
+  }
+  if (diag || bits != 0xFu) {
+    const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const bool keep = ((rb >> ((col0 + i) >> 6)) & 1u) && (!diag || col0 + i <= r);
+      s[i] = keep ? s[i] : -INFINITY;
+    }
+  }
+  // Row max: 3-input max over pairs, 8 independent chains.
+  float mx8[8];
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmaxf(s[2 * kk], s[2 * kk + 1]);
+#pragma unroll
+  for (int i = 16; i < NC; i += 16)
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmax3(mx8[kk], s[i + 2 * kk], s[i + 2 * kk + 1]);
+  const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                         fmaxf(mx8[6], mx8[7]));
+  const float m_new = fmaxf(m_run, mx * c);
+  const bool need = m_new > m_run + kRescaleThreshold;
+  const float m_next = need ? m_new : m_run;
+  const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
+  // p = 2^(s*c - m), two lanes per instruction (the argument and the
+  // sums); ex2.approx, or the FMA-pipe polynomial for kPolyPer8 keys of 8.
+  const uint64_t c2 = f2_make(c, c), negm2 = f2_make(-m_use, -m_use);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int q2 = 0; q2 < NC / 64; ++q2) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int k0 = q2 * 64 + 2 * i;
+      const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
+      float p0, p1;
+      if ((k0 & 7) >= 8 - kPolyPer8) {
+        ex2_poly2(x, p0, p1);
+      } else {
+        float x0, x1;
+        f2_split(x, x0, x1);
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
+      acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+    tmem_st32(s_base + static_cast<uint32_t>(col0 / 2 + q2 * 32), pk);
+  }
+  // S_t(j) ready implies PV_t(j-1) is done (MMAs complete in order), so
+  // O_t may be rescaled here before P_t(j) is released.
+  if (rescale_ok && __any_sync(0xffffffffu, need)) {
+    const float alpha = need ? ex2(m_run - m_new) : 1.0f;
+#pragma unroll
+    for (int q4 = 0; q4 < HD / 32; ++q4) {
+      uint32_t o[32];
+      tmem_ld32(o_base + q4 * 32, o);
+      tmem_ld_wait(o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+      tmem_st32(o_base + q4 * 32, o);
+    }
+  }
+  if (need) l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
+  m_run = m_next;
+  {
+    float a0, a1;
+    f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+    l_run += a0 + a1;
+  }
+}
+
+FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CUtensorMap *tmO,
+                        int total, int t) {
   const int r = threadIdx.x - 128 * t;                 // row within the tile
   const uint32_t quad = (threadIdx.x >> 5) & 3u;
   const uint32_t s_base = tmem + ((quad * 32u) << 16) + 256u * t;
@@ -940,82 +1110,12 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
         break;
       }
       tc_fence_after_sync();
-      float s[BN];
-      {
-        uint32_t raw[BN];
-        tmem_ld128_wait(s_base, raw);
-#pragma unroll
-        for (int i = 0; i < BN; ++i) s[i] = __uint_as_float(raw[i]);
-      }
-      const bool diag = (n == im.qt);
-      if (diag || bits != 0xFu) {
-        const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
-#pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
-          s[i] = keep ? s[i] : -INFINITY;
-        }
-      }
-      // Row max: 3-input max over pairs, 8 independent chains.
-      float mx8[8];
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmaxf(s[2 * kk], s[2 * kk + 1]);
-#pragma unroll
-      for (int i = 16; i < BN; i += 16)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmax3(mx8[kk], s[i + 2 * kk], s[i + 2 * kk + 1]);
-      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                             fmaxf(mx8[6], mx8[7]));
-      const float m_new = fmaxf(m_run, mx * c);
-      const bool need = m_new > m_run + kRescaleThreshold;
-      const float m_next = need ? m_new : m_run;
-      const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
-      // p = 2^(s*c - m), two lanes per instruction (the argument and the
-      // sums); ex2.approx, or the FMA-pipe polynomial for kPolyPer8 keys of 8.
-      const uint64_t c2 = f2_make(c, c), negm2 = f2_make(-m_use, -m_use);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int k0 = q2 * 64 + 2 * i;
-          const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
-          float p0, p1;
-          if ((k0 & 7) >= 8 - kPolyPer8) {
-            ex2_poly2(x, p0, p1);
-          } else {
-            float x0, x1;
-            f2_split(x, x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(s_base + q2 * 32, pk);
-      }
-      // S_t(j) ready implies PV_t(j-1) is done (MMAs complete in order), so
-      // O_t may be rescaled here before P_t(j) is released.
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2(m_run - m_new) : 1.0f;
-#pragma unroll
-        for (int q4 = 0; q4 < HD / 32; ++q4) {
-          uint32_t o[32];
-          tmem_ld32(o_base + q4 * 32, o);
-          tmem_ld_wait(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(o_base + q4 * 32, o);
-        }
-      }
-      if (need) l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
-      m_run = m_next;
-      {
-        float a0, a1;
-        f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
-        l_run += a0 + a1;
-      }
+      const int half = im.sparse ? half_of(bits) : 0;
+      if (half == 0)
+        softmax_tile<BN>(s_base, o_base, 0, bits, n == im.qt, r, c, j > 0, m_run, l_run);
+      else
+        softmax_tile<BN / 2>(s_base, o_base, half == 2 ? BN / 2 : 0, bits, n == im.qt, r, c,
+                             j > 0, m_run, l_run);
       tmem_st_wait();
       tc_fence_before_sync();
       mbar_arrive_a(sh.bar(Smem::P_FULL0 + t));
@@ -1030,9 +1130,18 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
     if (j > 0 && !have_o) break;
     tc_fence_after_sync();
     const int tok = im.qt * BM + r;
-    const bool store = (tok < im.L) && !ld_shared_s32(sh.abort_flag());
+    const bool aborted = ld_shared_s32(sh.abort_flag()) != 0;
+    const bool store = (tok < im.L) && !aborted;
     const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
     __nv_bfloat16 *orow = p.o + ((static_cast<size_t>(im.row0) + tok) * p.Hq + h) * HD;
+    // Bulk tensor stores unless the output is mixed into the existing one or
+    // the tile of a packed sequence reaches into the next sequence (TMA only
+    // clips at the tensor's own end).  Warp-uniform.
+    const bool tma = __all_sync(0xffffffffu, kTmaEpilogue && p.mix_r == nullptr && !aborted &&
+                                                 (p.cu_seqlens == nullptr ||
+                                                  (im.qt + 1) * BM <= im.L));
+    const int wq = (threadIdx.x >> 5) & 3;        // rows 32wq .. 32wq+31 of the tile
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int q4 = 0; q4 < HD / 32; ++q4) {
       uint32_t o[32];
@@ -1043,7 +1152,30 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
-      if (store) {
+      if (tma) {
+        const uint32_t box = sh.stg(4 * t + wq, q4 & 1);
+        if (lane == 0) bulk_wait_read1();    // the store that last used this box has read it
+        __syncwarp();
+        const uint32_t row = box + 64u * static_cast<uint32_t>(lane);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t w0 = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
+                                          __uint_as_float(o[8 * v + 1]) * inv_l);
+          const uint32_t w1 = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
+                                          __uint_as_float(o[8 * v + 3]) * inv_l);
+          const uint32_t w2 = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
+                                          __uint_as_float(o[8 * v + 5]) * inv_l);
+          const uint32_t w3 = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
+                                          __uint_as_float(o[8 * v + 7]) * inv_l);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + 16u * v), "r"(w0),
+                       "r"(w1), "r"(w2), "r"(w3)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && im.qt * BM + 32 * wq < im.L)   // rows past the end are clipped
+          tma_store_4d_commit(tmO, box, q4 * 32, h, im.tma_tok0 + im.qt * BM + 32 * wq, im.tma_b);
+      } else if (store) {
         uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
         prefill::store_row_chunk(dst, o, inv_l, p.mix_r, im.b);
       }
@@ -1058,11 +1190,15 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, int tota
       p.lse[im.lse0 + static_cast<long long>(h) * im.lse_hs + tok] = lse;
     }
   }
+  // Every bulk store of this warp has completed before the CTA exits.
+  if (kTmaEpilogue && (threadIdx.x & 31) == 0) bulk_wait_all0();
+  __syncwarp();
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const Params p, int total_items) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const Params p, int total_items) {
   extern __shared__ uint8_t smem_raw[];
   const Smem sh = carve(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -1090,6 +1226,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if (kTmaEpilogue) tma_prefetch_desc(&tmO);
   }
   prefill::check_csr_size(p);
   if (warp == WARP_MMA) {
@@ -1112,7 +1249,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
-    run_softmax(sh, tmem, p, total_items, warp >> 2);
+    run_softmax(sh, tmem, p, &tmO, total_items, warp >> 2);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -1204,6 +1341,8 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   if (make_tmap_bhsd(&tmQ, a.q, mB, mS, a.Hq, 64, BM) != 0) return FA_ERR_CUDA;
   if (make_tmap_bhsd(&tmK, a.k, mB, mS, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
   if (make_tmap_bhsd(&tmV, a.v, mB, mS, a.Hkv, 64, BN) != 0) return FA_ERR_CUDA;
+  CUtensorMap tmO;   // epilogue stores of the two-tile kernel: 32 columns x 32 rows
+  if (make_tmap_bhsd_plain(&tmO, a.o, mB, mS, a.Hq, 32, 32) != 0) return FA_ERR_CUDA;
   const int G = a.Hq / a.Hkv;
   const bool two_tiles = (G % 2) == 0;
   if (two_tiles) {
@@ -1243,6 +1382,7 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.expect_nnz = (a.expect_nnz >= 0 && a.expect_nnz <= 0x7fffffffLL)
                      ? static_cast<int>(a.expect_nnz) : -1;
+  p.band_q = 0;
   long long grid =
       static_cast<long long>(p.n_qtiles) * a.B * (two_tiles ? a.Hq / 2 : a.Hq);
   if (varlen) {
@@ -1270,8 +1410,17 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
 #endif
     const long long cap = FA_PREFILL_PERSISTENT ? sms : grid;
     const int ctas = static_cast<int>(grid < cap ? grid : cap);
+    // KV-head-major bands when the sequence is long enough for several bands
+    // of one CTA per SM (the K/V of one head then no longer fits the L2
+    // share the query-tile-major order leaves it).
+#ifndef FA_BAND_ORDER
+#define FA_BAND_ORDER 1
+#endif
+    const int ppk = G / 2;
+    const int band = ctas / ppk;
+    p.band_q = (FA_BAND_ORDER && !varlen && band >= 1 && p.n_qtiles >= 4 * band) ? band : 0;
     prefill2::prefill2_kernel<<<ctas, prefill2::NUM_THREADS, prefill2::SMEM_BYTES, stream>>>(
-        tmQ, tmK, tmV, p, static_cast<int>(grid));
+        tmQ, tmK, tmV, tmO, p, static_cast<int>(grid));
     note_launch();
   } else {
     prefill_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, SMEM_BYTES, stream>>>(tmQ, tmK,

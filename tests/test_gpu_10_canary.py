@@ -138,3 +138,38 @@ def test_backward_split_tiles_write_only_their_gradients(mode):
                                      inputs.bits(do), SCALE, mask)
     for name, g, w in zip(("dq", "dk", "dv"), (dq.t, dk.t, dv.t), want):
         assert_close_grad(to_f64(g), w, "%s %s" % (mode, name))
+
+
+@pytest.mark.parametrize("mode", ["full", "sparse"])
+def test_prefill_long_sequence_item_order_covers_every_row(mode):
+    """S = 40000 with 4 query heads per KV head: long enough for the
+    KV-head-major item order (bands of 74 query tiles and a partial last
+    band; the last tile ragged).  Every output row must be written exactly
+    where it belongs: all rows finite inside the fences, sampled rows equal
+    to the oracle's."""
+    B, S, Hq, Hkv = 2, 40000, 8, 2
+    q, k, v = inputs.qkv(B, S, Hq, Hkv, 128, 991, device="cuda")
+    o = Guarded((B, S, Hq, 128), torch.bfloat16)
+    lse = Guarded((B, Hq, S), torch.float32)
+    status = zero_status()
+    c = capi.cfg(64, 128, 1024)
+    rp, ci = capi.blocksparse_index(S, c)
+    if mode == "full":
+        capi.attn_prefill_full(q, k, v, o=o.t, lse=lse.t, status=status)
+        mask = None
+    else:
+        capi.attn_prefill_blocksparse(q, k, v, rp, ci, o=o.t, lse=lse.t, status=status)
+        mask = oracle.rows_to_dense_mask(oracle.blocksparse_rows(S, 64, 128, 1024))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    o.check_all_written("o")
+    lse.check_all_written("lse")
+    rows = inputs.sample_rows(B, S, Hq, Hkv, seed=991, n_random=48, n_groups=1)
+    rng = np.random.default_rng(991)
+    rows = rows[np.sort(rng.choice(len(rows), size=min(400, len(rows)), replace=False))]
+    ref, ref_lse = oracle.attention_rows(inputs.bits(q), inputs.bits(k), inputs.bits(v), SCALE,
+                                         rows, mask)
+    rt = torch.from_numpy(rows).cuda()
+    assert_close_attention(to_f64(o.t[rt[:, 0], rt[:, 2], rt[:, 1]]), ref, "S=40000 %s" % mode)
+    np.testing.assert_allclose(to_f64(lse.t[rt[:, 0], rt[:, 1], rt[:, 2]]), ref_lse,
+                               atol=LSE_ABS_TOL)
