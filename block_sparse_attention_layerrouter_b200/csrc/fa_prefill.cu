@@ -756,18 +756,6 @@ FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Param
   const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
   return __all_sync(0xffffffffu, done);
 }
-// Which 64-key half of a 128-key tile its 4-bit block mask (bit 2*qs + ks)
-// keeps: 0 both, 1 only keys 0-63 (no ks = 1 bit), 2 only keys 64-127.  A
-// half tile (the first window tile of a sparse row pair, for instance) is
-// computed with N = 64 / K = 64 products and 64 exponentials per row.
-#ifndef FA_HALF_TILES
-#define FA_HALF_TILES 1
-#endif
-FA_DEV int half_of(uint32_t bits) {
-  if (!FA_HALF_TILES) return 0;
-  return (bits & 0xAu) == 0u ? 1 : ((bits & 0x5u) == 0u ? 2 : 0);
-}
-
 // The producer and MMA roles run on all 32 lanes of their warp with
 // warp-uniform state; one elected lane issues each TMA copy, MMA and commit.
 // li / nq: ring loads and Q loads issued (the abort path drains them).
@@ -838,7 +826,6 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
 
 FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
-  constexpr uint32_t kIdescQK64 = idesc_bf16_f32(BM, BN / 2, false);   // half tiles
   constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
   // Descriptors of the Q tiles (fixed) and of ring slot 0; slot s adds
   // s * TILE_BYTES / 16 to the start-address field, a K step kk adds the
@@ -873,30 +860,17 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     tc_fence_after_sync();
     return true;
   };
-  // S_t = Q_t K^T of one tile; a half tile (half = 1: keys 0-63, 2: keys
-  // 64-127) takes N = 64 and writes S columns 0-63 or 64-127.
-  auto qk = [&](int t, int slot, int half) {
+  auto qk = [&](int t, int slot) {
     const uint64_t qd = t ? q_desc1 : q_desc0;
-    uint64_t kd = k_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
-    uint32_t d = tmem + 256u * t;
-    uint32_t idesc = kIdescQK;
-    if (half != 0) {
-      idesc = kIdescQK64;
-      if (half == 2) {
-        kd += static_cast<uint64_t>((64 * 128) >> 4);   // key rows 64.. of each 64-column box
-        d += 64u;
-      }
-    }
+    const uint64_t kd = k_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
       const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-      mma_bf16_ss_w(d, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
+      mma_bf16_ss_w(tmem + 256u * t, qd + off, kd + off, kIdescQK, kk > 0 ? 1u : 0u);
     }
     tc_commit_w(sh.bar(Smem::S_FULL0 + t));
   };
-  // O_t (+)= P_t V over the tile's keys, or over the half's 64 keys (K steps
-  // 0-3 or 4-7; P of key k sits in TMEM column k / 2 either way).
-  auto pv = [&](int t, bool first, int slot, int half) -> bool {
+  auto pv = [&](int t, bool first, int slot) -> bool {
     if (!warp_wait(sh.bar(Smem::P_FULL0 + t), static_cast<uint32_t>(jp) & 1u, sh, p))
       return false;
     if (first && done_items > 0 &&
@@ -904,13 +878,11 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       return false;
     tc_fence_after_sync();
     const uint64_t vd = v_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
-    const int kb = half == 2 ? 4 : 0, ke = half == 1 ? 4 : BN / 16;
 #pragma unroll
     for (int kk = 0; kk < BN / 16; ++kk) {
-      if (kk < kb || kk >= ke) continue;
       mma_bf16_ts_w(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
                     vd + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
-                    (!first || kk > kb) ? 1u : 0u);
+                    (!first || kk > 0) ? 1u : 0u);
     }
     return true;
   };
@@ -922,7 +894,6 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     if (!(ok = warp_wait(sh.bar(Smem::Q_FULL), static_cast<uint32_t>(k) & 1u, sh, p))) break;
     tc_fence_after_sync();
     bool has_next = im.qt > 0, has_next2 = false;     // full item: tiles 0..qt
-    int half = 0, half2 = 0;                           // half tiles (sparse items only)
     if (im.sparse) {
       const int e0 = take_info(ok);
       if (!ok) break;
@@ -931,42 +902,39 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
         continue;
       }
       has_next = (e0 & 0x20) == 0;
-      half = half_of(static_cast<uint32_t>(e0) & 15u);
     }
     int k_slot = 0, v_slot = 0;
     if (!(ok = take(k_slot))) break;
-    qk(0, k_slot, half);
-    qk(1, k_slot, half);
+    qk(0, k_slot);
+    qk(1, k_slot);
     tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
     if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));     // the last QK of this item is issued
     for (int j = 0;; ++j) {
       if (!(ok = take(v_slot))) break;
-      if (!(ok = pv(0, j == 0, v_slot, half))) break;
+      if (!(ok = pv(0, j == 0, v_slot))) break;
       if (has_next) {
         if (im.sparse) {                      // tile j+1: is it the last?
           const int e = take_info(ok);
           if (!ok) break;
           has_next2 = (e & 0x20) == 0;
-          half2 = half_of(static_cast<uint32_t>(e) & 15u);
         } else {
           has_next2 = j + 1 < im.qt;
         }
         if (!(ok = take(k_slot))) break;
-        qk(0, k_slot, half2);
+        qk(0, k_slot);
       } else {
         tc_commit_w(sh.bar(Smem::O_DONE0));
       }
-      if (!(ok = pv(1, j == 0, v_slot, half))) break;
+      if (!(ok = pv(1, j == 0, v_slot))) break;
       ++jp;
       tc_commit_w(sh.bar(Smem::EMPTY0 + v_slot));
       if (!has_next) {
         tc_commit_w(sh.bar(Smem::O_DONE0 + 1));
         break;
       }
-      qk(1, k_slot, half2);
+      qk(1, k_slot);
       tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
       has_next = has_next2;
-      half = half2;
       if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));
     }
     ++done_items;
@@ -974,23 +942,19 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
 }
 
 
-// Softmax of one S tile of NC columns (128, or 64 for a half tile) starting
-// at column col0 of S_t, for the row r of this thread: mask (the block mask
-// `bits`, causal on the diagonal tile), row max, P = 2^(s*c - m) written as
-// bf16 pairs into columns col0/2 .. of S_t (the A operand of the PV product),
-// O rescaled when the running max grew by more than kRescaleThreshold
-// (`rescale_ok`: a PV product of this item has run), running max and sum.
-template <int NC>
-FA_DEV void softmax_tile(uint32_t s_base, uint32_t o_base, int col0, uint32_t bits, bool diag,
-                         int r, float c, bool rescale_ok, float &m_run, float &l_run) {
+// Softmax of one 128-column S tile of head t for the row r of this thread:
+// mask (the 4-bit block mask `bits`, causal on the diagonal tile), row max,
+// P = 2^(s*c - m) written as bf16 pairs into the first 64 columns of S_t (the
+// A operand of the PV product), O rescaled when the running max grew by more
+// than kRescaleThreshold (`rescale_ok`: a PV product of this item has run),
+// running max and sum.
+FA_DEV void softmax_tile(uint32_t s_base, uint32_t o_base, uint32_t bits, bool diag, int r,
+                         float c, bool rescale_ok, float &m_run, float &l_run) {
+  constexpr int NC = BN;
   float s[NC];
   {
     uint32_t raw[NC];
-    if constexpr (NC == BN) {
-      tmem_ld128_wait(s_base, raw);
-    } else {
-      tmem_ld64_wait(s_base + static_cast<uint32_t>(col0), raw);
-    }
+    tmem_ld128_wait(s_base, raw);
 #pragma unroll
     for (int i = 0; i < NC; ++i) s[i] = __uint_as_float(raw[i]);
   }
@@ -998,7 +962,7 @@ FA_DEV void softmax_tile(uint32_t s_base, uint32_t o_base, int col0, uint32_t bi
     const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
-      const bool keep = ((rb >> ((col0 + i) >> 6)) & 1u) && (!diag || col0 + i <= r);
+      const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
       s[i] = keep ? s[i] : -INFINITY;
     }
   }
@@ -1039,7 +1003,7 @@ FA_DEV void softmax_tile(uint32_t s_base, uint32_t o_base, int col0, uint32_t bi
       acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
       pk[i] = pack_bf16x2(p0, p1);
     }
-    tmem_st32(s_base + static_cast<uint32_t>(col0 / 2 + q2 * 32), pk);
+    tmem_st32(s_base + q2 * 32, pk);
   }
   // S_t(j) ready implies PV_t(j-1) is done (MMAs complete in order), so
   // O_t may be rescaled here before P_t(j) is released.
@@ -1110,12 +1074,7 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
         break;
       }
       tc_fence_after_sync();
-      const int half = im.sparse ? half_of(bits) : 0;
-      if (half == 0)
-        softmax_tile<BN>(s_base, o_base, 0, bits, n == im.qt, r, c, j > 0, m_run, l_run);
-      else
-        softmax_tile<BN / 2>(s_base, o_base, half == 2 ? BN / 2 : 0, bits, n == im.qt, r, c,
-                             j > 0, m_run, l_run);
+      softmax_tile(s_base, o_base, bits, n == im.qt, r, c, j > 0, m_run, l_run);
       tmem_st_wait();
       tc_fence_before_sync();
       mbar_arrive_a(sh.bar(Smem::P_FULL0 + t));
@@ -1124,11 +1083,23 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
     }
     if (!ok) break;
 
-    // Epilogue: O / l -> bf16, one row per thread; then hand O back.
+    // Epilogue: read all of O_t at once and hand its TMEM columns back (the
+    // next item's first PV may start while this one stores), then O / l ->
+    // bf16, one row per thread.
     const bool have_o =
         j > 0 && warp_wait(sh.bar(Smem::O_DONE0 + t), static_cast<uint32_t>(done_items) & 1u, sh, p);
     if (j > 0 && !have_o) break;
     tc_fence_after_sync();
+    uint32_t o[HD];
+    if (have_o) {
+      tmem_ld128_wait(o_base, o);
+      tc_fence_before_sync();
+      mbar_arrive_a(sh.bar(Smem::O_FREE0 + t));
+      ++done_items;
+    } else {
+#pragma unroll
+      for (int i = 0; i < HD; ++i) o[i] = 0u;
+    }
     const int tok = im.qt * BM + r;
     const bool aborted = ld_shared_s32(sh.abort_flag()) != 0;
     const bool store = (tok < im.L) && !aborted;
@@ -1144,14 +1115,6 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int q4 = 0; q4 < HD / 32; ++q4) {
-      uint32_t o[32];
-      if (have_o) {
-        tmem_ld32(o_base + q4 * 32, o);
-        tmem_ld_wait(o);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
-      }
       if (tma) {
         const uint32_t box = sh.stg(4 * t + wq, q4 & 1);
         if (lane == 0) bulk_wait_read1();    // the store that last used this box has read it
@@ -1159,14 +1122,15 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
         const uint32_t row = box + 64u * static_cast<uint32_t>(lane);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const uint32_t w0 = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
-                                          __uint_as_float(o[8 * v + 1]) * inv_l);
-          const uint32_t w1 = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
-                                          __uint_as_float(o[8 * v + 3]) * inv_l);
-          const uint32_t w2 = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
-                                          __uint_as_float(o[8 * v + 5]) * inv_l);
-          const uint32_t w3 = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
-                                          __uint_as_float(o[8 * v + 7]) * inv_l);
+          const uint32_t *ov = o + 32 * q4 + 8 * v;
+          const uint32_t w0 = pack_bf16x2(__uint_as_float(ov[0]) * inv_l,
+                                          __uint_as_float(ov[1]) * inv_l);
+          const uint32_t w1 = pack_bf16x2(__uint_as_float(ov[2]) * inv_l,
+                                          __uint_as_float(ov[3]) * inv_l);
+          const uint32_t w2 = pack_bf16x2(__uint_as_float(ov[4]) * inv_l,
+                                          __uint_as_float(ov[5]) * inv_l);
+          const uint32_t w3 = pack_bf16x2(__uint_as_float(ov[6]) * inv_l,
+                                          __uint_as_float(ov[7]) * inv_l);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + 16u * v), "r"(w0),
                        "r"(w1), "r"(w2), "r"(w3)
                        : "memory");
@@ -1176,14 +1140,12 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
         if (lane == 0 && im.qt * BM + 32 * wq < im.L)   // rows past the end are clipped
           tma_store_4d_commit(tmO, box, q4 * 32, h, im.tma_tok0 + im.qt * BM + 32 * wq, im.tma_b);
       } else if (store) {
+        uint32_t oc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) oc[i] = o[32 * q4 + i];
         uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
-        prefill::store_row_chunk(dst, o, inv_l, p.mix_r, im.b);
+        prefill::store_row_chunk(dst, oc, inv_l, p.mix_r, im.b);
       }
-    }
-    if (have_o) {
-      tc_fence_before_sync();
-      mbar_arrive_a(sh.bar(Smem::O_FREE0 + t));
-      ++done_items;
     }
     if (store && p.lse) {
       const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
