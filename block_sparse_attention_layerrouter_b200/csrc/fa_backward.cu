@@ -200,6 +200,7 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
                          int total, int &kv_n, int &li) {
   kv_n = 0;       // K/V loads issued
   li = 0;         // stage loads issued (continues across items)
+  if (c_skip_loads) return;      // testing mode: no loads, every wait runs out
   bool ok = true;
   for (int k = 0; ok; ++k) {
     const int w = item_index(k, total);
@@ -1011,7 +1012,11 @@ int run_main(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
                                              static_cast<long long>(pl.nkt) * (pl.nkt - 1));
   const long long acc_bytes = static_cast<long long>(a.B) * a.Hq * pl.Sp * HD * 4;
   const bool balanced = static_cast<long long>(pl.nqb) * sms <= full_blocks;
-  p.cq_full = (balanced && acc_bytes <= (256ll << 20)) ? pl.nqb : cq;
+#ifndef FA_BWD_WHOLE_TILE_ACC_MB
+#define FA_BWD_WHOLE_TILE_ACC_MB 256
+#endif
+  p.cq_full = (balanced && acc_bytes <= (static_cast<long long>(FA_BWD_WHOLE_TILE_ACC_MB) << 20))
+                  ? pl.nqb : cq;
   p.cq_sparse = cq;
   const bool any_sparse = sparse && (a.mode_dev != nullptr || a.mode_default == FA_MODE_SPARSE);
   const int cq_min = any_sparse ? (p.cq_full < cq ? p.cq_full : cq) : p.cq_full;
@@ -1059,7 +1064,7 @@ size_t backward_workspace_bytes(int B, int S, int Hq, int Hkv) {
   return make_plan(B, S, Hq, Hkv, nullptr).bytes;
 }
 
-int set_wait_limit_backward(uint64_t ns) { return set_wait_limit_local(ns); }
+int set_wait_limit_backward(uint64_t ns, int skip_loads) { return set_wait_limit_local(ns, skip_loads); }
 
 int launch_backward(const BackwardLaunch &a, cudaStream_t stream) {
   const Plan pl = make_plan(a.B, a.S, a.Hq, a.Hkv, a.workspace);

@@ -24,17 +24,21 @@ namespace fa {
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
 
 // The bound the kernels use, in constant memory so that a test can change
-// it (fa_debug_set_wait_limit_ns) and make a wait run out on purpose.  Each
-// translation unit that includes this header holds its own copy;
-// set_wait_limit_local() sets the copy of the unit it is called from, on the
-// current device.  0 is the testing mode: a wait whose phase is not complete
-// at its first (non-blocking) test gives up at once.  (With a positive bound
-// a wait can still outlast it: mbarrier.try_wait may suspend the thread until
-// the phase completes, and the bound is checked between tries.)
+// it (fa_debug_set_wait_limit_ns) and make a wait run out on purpose.  It is
+// read only on a wait's slow path (after mbarrier.try_wait, which may suspend
+// the thread until the phase completes, came back empty).  Testing mode
+// (c_skip_loads): the roles that issue TMA loads issue none, so every wait on
+// a load runs out after the bound and the kernel gives up; each role reads the
+// flag once, so the pipelines' code is otherwise unchanged.  Each translation
+// unit that includes this header holds its own copies; set_wait_limit_local()
+// sets those of the unit it is called from, on the current device.
 static __constant__ uint64_t c_wait_limit_ns = kWaitTimeoutNs;
+static __constant__ int c_skip_loads = 0;
 
-static inline int set_wait_limit_local(uint64_t ns) {
-  return cudaMemcpyToSymbol(c_wait_limit_ns, &ns, sizeof(ns)) == cudaSuccess ? 0 : -1;
+static inline int set_wait_limit_local(uint64_t ns, int skip_loads) {
+  if (cudaMemcpyToSymbol(c_wait_limit_ns, &ns, sizeof(ns)) != cudaSuccess) return -1;
+  return cudaMemcpyToSymbol(c_skip_loads, &skip_loads, sizeof(skip_loads)) == cudaSuccess ? 0
+                                                                                          : -1;
 }
 
 FA_DEV uint32_t smem_u32(const void *p) {
@@ -82,27 +86,9 @@ FA_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-FA_DEV bool mbar_test_wait_a(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait until the phase of parity `parity` of `bar` has completed.  Returns
 // false (and sets *abort) if the CTA is aborting or the wait ran out.
 FA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *status) {
-  if (c_wait_limit_ns == 0) {   // testing mode: give up unless complete already
-    if (mbar_test_wait_a(smem_u32(bar), parity)) return true;
-    *abort = 1;
-    report(status, FA_DEV_TIMEOUT);
-    return false;
-  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -148,12 +134,6 @@ FA_DEV void st_shared_s32(uint32_t addr, int v) {
 }
 // Bounded wait; `abort_flag` is the shared address of the CTA's abort word.
 FA_DEV bool mbar_wait_a(uint32_t bar, uint32_t parity, uint32_t abort_flag, int32_t *status) {
-  if (c_wait_limit_ns == 0) {   // testing mode: give up unless complete already
-    if (mbar_test_wait_a(bar, parity)) return true;
-    st_shared_s32(abort_flag, 1);
-    report(status, FA_DEV_TIMEOUT);
-    return false;
-  }
   if (mbar_try_wait_a(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {

@@ -287,7 +287,9 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     }
     issued = i + 1;
   };
-  if (tid == 0) {
+  // Testing mode: no loads, every wait runs out.
+  const bool skip_loads = c_skip_loads != 0;
+  if (tid == 0 && !skip_loads) {
     for (int i = 0; i < NSTAGE && i < ntiles; ++i) issue(i);
   }
 
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     // Past this barrier every thread is done with tile i-1 (its PV came before
     // these scores), so its stage takes tile i-1+NSTAGE.
     if (__syncthreads_or(!ok)) break;
-    if (tid == 0 && i >= 1 && i - 1 + NSTAGE < ntiles) issue(i - 1 + NSTAGE);
+    if (tid == 0 && !skip_loads && i >= 1 && i - 1 + NSTAGE < ntiles) issue(i - 1 + NSTAGE);
 
     // ---- rare: move the reference to the running max, rescale, redo P
     if (reref[i & 1]) {
@@ -617,7 +619,7 @@ int decode_num_splits(int B, int Hkv, int Lmax) {
   return decode_splits_for_tiles(B, Hkv, (Lmax + decode::KT - 1) / decode::KT);
 }
 
-int set_wait_limit_decode(uint64_t ns) { return set_wait_limit_local(ns); }
+int set_wait_limit_decode(uint64_t ns, int skip_loads) { return set_wait_limit_local(ns, skip_loads); }
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lmax) {
   const size_t ns = static_cast<size_t>(decode_num_splits(B, Hkv, Lmax));

@@ -171,11 +171,12 @@ int launch_soft_backward(const SoftBackwardLaunch &a, cudaStream_t stream);
 // Counts one kernel launch (the total is fa_kernel_launches()).
 void note_launch();
 
-// Bound of the kernels' waits (ns) in each kernel file's constant memory,
-// on the current device; 0 on success.
-int set_wait_limit_prefill(uint64_t ns);
-int set_wait_limit_decode(uint64_t ns);
-int set_wait_limit_backward(uint64_t ns);
+// Bound of the kernels' waits (ns) and the testing flag that makes the
+// load-issuing roles issue nothing, in each kernel file's constant memory, on
+// the current device; 0 on success.
+int set_wait_limit_prefill(uint64_t ns, int skip_loads);
+int set_wait_limit_decode(uint64_t ns, int skip_loads);
+int set_wait_limit_backward(uint64_t ns, int skip_loads);
 
 long long index_nnz(int nrows, int sb, int wb);
 int launch_index(int nrows, int sb, int wb, int32_t *row_ptr, int32_t *col_idx,

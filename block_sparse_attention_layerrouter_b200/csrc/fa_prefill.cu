@@ -207,10 +207,12 @@ FA_DEV Shared carve(uint8_t *raw) {
 }
 
 // ------------------------------------------------------------- producer ---
-// Returns the number of ring loads issued (the abort path drains them).
+// Returns the number of ring loads issued (the abort path drains them and
+// the Q load), or -1 if it issued nothing at all.
 FA_DEV int run_producer(const Shared &sh, const CUtensorMap *tmQ, const CUtensorMap *tmK,
                         const CUtensorMap *tmV, const Params &p, int qt, int b, int h,
                         int kvh, bool sparse) {
+  if (c_skip_loads) return -1;   // testing mode: no loads, every wait runs out
   mbar_arrive_expect_tx(sh.q_full, TILE_BYTES);
   tma_load_4d(sh.q, tmQ, sh.q_full, 0, h, qt * BM, b);
   tma_load_4d(sh.q + HALF_BYTES, tmQ, sh.q_full, 64, h, qt * BM, b);
@@ -512,7 +514,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // producer waits (bounded) for its last loads to land and the MMA thread
   // for its MMAs to finish before TMEM is freed and the CTA exits.
   const bool aborted = *sh.abort != 0;
-  if (aborted && warp == 0 && lane == 0) {
+  if (aborted && warp == 0 && lane == 0 && loads >= 0) {
     mbar_wait_drain(sh.q_full, 0, kDrainNs);
     for (int x = (loads > NSLOT ? loads - NSLOT : 0); x < loads; ++x)
       mbar_wait_drain(&sh.full[x % NSLOT], static_cast<uint32_t>(x / NSLOT) & 1u, kDrainNs);
@@ -764,6 +766,7 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
                          int &nq) {
   li = 0;           // ring loads issued (continues across items)
   nq = 0;           // Q loads issued
+  if (c_skip_loads) return;      // testing mode: no loads, every wait runs out
   int ig = 0;       // tile entries handed to the MMA and softmax warps
   bool ok = true;
   for (int k = 0; ok; ++k) {
@@ -1287,7 +1290,7 @@ __global__ void __launch_bounds__(1024) varlen_items_kernel(const int32_t *cu, i
 }  // namespace prefill2
 
 // ----------------------------------------------------------------- host ---
-int set_wait_limit_prefill(uint64_t ns) { return set_wait_limit_local(ns); }
+int set_wait_limit_prefill(uint64_t ns, int skip_loads) { return set_wait_limit_local(ns, skip_loads); }
 
 size_t varlen_workspace_bytes(int B, int total_tokens) {
   const size_t max_items = static_cast<size_t>(total_tokens) / prefill2::BM + B + 1;

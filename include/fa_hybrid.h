@@ -81,14 +81,15 @@ FA_API const char *fa_status_string(int status);
 FA_API int fa_version(void);
 
 /* Testing aid: sets the bound of every wait inside this library's kernels
- * (default 2 s) on the current device.  Each wait in a kernel is bounded; a
- * wait that runs out makes the kernel give up (FA_DEV_TIMEOUT in dev_status,
- * the outputs of that call invalid; a decode head whose split gave up reads
- * NaN), let its copies and MMAs in flight finish and return, leaving the
- * device usable.  A short bound (0 works) makes that happen on purpose, so a
- * test can check the path; put the default back afterwards.  Synchronous (a
- * copy to device constant memory): not during stream capture or while this
- * library's kernels run.  Returns FA_OK or FA_ERR_CUDA. */
+ * (default 2e9 ns) on the current device.  Each wait in a kernel is bounded;
+ * a wait that runs out makes the kernel give up (FA_DEV_TIMEOUT in
+ * dev_status, the outputs of that call invalid; a decode head whose split
+ * gave up reads NaN), let its copies and MMAs in flight finish and return,
+ * leaving the device usable.  ns = 0 is the testing mode that makes this
+ * happen on purpose: the kernels issue no TMA loads, so every wait on a load
+ * runs out, after a bound of 1 ms.  Put the default back afterwards.
+ * Synchronous (a copy to device constant memory): not during stream capture
+ * or while this library's kernels run.  Returns FA_OK or FA_ERR_CUDA. */
 FA_API int fa_debug_set_wait_limit_ns(unsigned long long ns);
 
 /* Number of kernels this library has enqueued in this process so far, on

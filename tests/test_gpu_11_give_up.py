@@ -1,9 +1,10 @@
-"""GPU: the give-up path of the kernels' bounded waits.  With the bound set
-to zero (fa_debug_set_wait_limit_ns), a wait that is not over at once runs
-out: the kernel reports FA_DEV_TIMEOUT in the status word, lets its copies
-and MMAs in flight finish, frees its tensor memory and returns.  The call
-then ends normally, and the next call with the default bound on the same
-stream gives the oracle's result: the device stayed usable."""
+"""GPU: the give-up path of the kernels' bounded waits.  In the testing mode
+of fa_debug_set_wait_limit_ns(0) the kernels issue no TMA loads, so their
+waits on loads run out (after 1 ms): the kernel reports FA_DEV_TIMEOUT in the
+status word, lets what it has in flight finish, frees its tensor memory and
+returns.  The call then ends normally, and the next call with the default
+bound on the same stream gives the oracle's result: the device stayed
+usable."""
 import contextlib
 import math
 

@@ -80,9 +80,9 @@ def test_noalloc_matches_decode_and_the_oracle_on_two_calls_in_a_row():
 
 @pytest.mark.gpu
 def test_noalloc_never_returns_an_earlier_calls_result_after_a_give_up():
-    """A good call fills the scratch; then a call on other inputs whose waits
-    are bounded by zero gives up: its heads read NaN or this call's own
-    result, never the earlier call's."""
+    """A good call fills the scratch; then a call on other inputs in the
+    testing mode of the bounded waits gives up: its heads read NaN or this
+    call's own result, never the earlier call's."""
     build.build()
     B, Lmax, Hq, Hkv = 2, 4096, 8, 2
     a = _case(B, Lmax, Hq, Hkv, [4096, 4000], capi.FA_MODE_FULL, 1024, 73)
