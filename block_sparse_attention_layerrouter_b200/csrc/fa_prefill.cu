@@ -945,68 +945,119 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
 }
 
 
-// Softmax of one 128-column S tile of head t for the row r of this thread:
-// mask (the 4-bit block mask `bits`, causal on the diagonal tile), row max,
-// P = 2^(s*c - m) written as bf16 pairs into the first 64 columns of S_t (the
-// A operand of the PV product), O rescaled when the running max grew by more
-// than kRescaleThreshold (`rescale_ok`: a PV product of this item has run),
-// running max and sum.
-FA_DEV void softmax_tile(uint32_t s_base, uint32_t o_base, uint32_t bits, bool diag, int r,
-                         float c, bool rescale_ok, float &m_run, float &l_run) {
-  constexpr int NC = BN;
-  float s[NC];
-  {
-    uint32_t raw[NC];
-    tmem_ld128_wait(s_base, raw);
-#pragma unroll
-    for (int i = 0; i < NC; ++i) s[i] = __uint_as_float(raw[i]);
-  }
-  if (diag || bits != 0xFu) {
-    const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
-#pragma unroll
-    for (int i = 0; i < NC; ++i) {
-      const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
-      s[i] = keep ? s[i] : -INFINITY;
-    }
-  }
-  // Row max: 3-input max over pairs, 8 independent chains.
+// Row max of the 128 scores: 3-input max over pairs, 8 independent chains.
+FA_DEV float row_max(const float (&s)[BN]) {
   float mx8[8];
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmaxf(s[2 * kk], s[2 * kk + 1]);
 #pragma unroll
-  for (int i = 16; i < NC; i += 16)
+  for (int i = 16; i < BN; i += 16)
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmax3(mx8[kk], s[i + 2 * kk], s[i + 2 * kk + 1]);
-  const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                         fmaxf(mx8[6], mx8[7]));
-  const float m_new = fmaxf(m_run, mx * c);
-  const bool need = m_new > m_run + kRescaleThreshold;
-  const float m_next = need ? m_new : m_run;
-  const float m_use = (m_next == -INFINITY) ? 0.f : m_next;
-  // p = 2^(s*c - m), two lanes per instruction (the argument and the
-  // sums); ex2.approx, or the FMA-pipe polynomial for kPolyPer8 keys of 8.
+  return fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+               fmaxf(mx8[6], mx8[7]));
+}
+
+#ifndef FA_LAZY_MAX
+#define FA_LAZY_MAX 1
+#endif
+constexpr bool kLazyMax = FA_LAZY_MAX != 0;
+// Largest row sum of one tile's p = 2^(s*c - m) accepted without taking the
+// tile's max: p stays far inside the bf16 / fp32 range (2^127).
+constexpr float kLazySumLimit = 4294967296.0f;   // 2^32
+
+// The 128 scores of this thread's row of S_t, masked: the 4-bit block mask
+// `bits` (sparse tiles) and causality on the diagonal tile.
+FA_DEV void load_scores(uint32_t s_base, uint32_t bits, bool diag, int r, float (&s)[BN]) {
+  {
+    uint32_t raw[BN];
+    tmem_ld128_wait(s_base, raw);
+#pragma unroll
+    for (int i = 0; i < BN; ++i) s[i] = __uint_as_float(raw[i]);
+  }
+  if (diag || bits != 0xFu) {
+    const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
+#pragma unroll
+    for (int i = 0; i < BN; ++i) {
+      const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
+      s[i] = keep ? s[i] : -INFINITY;
+    }
+  }
+}
+
+// p = 2^(s*c - m) for the 128 scores, packed as bf16 pairs into pk; returns
+// the row sum.  Two lanes per instruction (the argument and the sums);
+// ex2.approx, or the FMA-pipe polynomial for kPolyPer8 keys of 8.
+FA_DEV float row_exp2(const float (&s)[BN], float c, float m, uint32_t (&pk)[BN / 2]) {
+  const float m_use = (m == -INFINITY) ? 0.f : m;
   const uint64_t c2 = f2_make(c, c), negm2 = f2_make(-m_use, -m_use);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-  for (int q2 = 0; q2 < NC / 64; ++q2) {
-    uint32_t pk[32];
+  for (int i = 0; i < BN / 2; ++i) {
+    const int k0 = 2 * i;
+    const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
+    float p0, p1;
+    if ((k0 & 7) >= 8 - kPolyPer8) {
+      ex2_poly2(x, p0, p1);
+    } else {
+      float x0, x1;
+      f2_split(x, x0, x1);
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
+    pk[i] = pack_bf16x2(p0, p1);
+  }
+  float a0, a1;
+  f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+  return a0 + a1;
+}
+
+// Softmax of one 128-column S tile of head t for the row r of this thread:
+// P = 2^(s*c - m) written as bf16 pairs into the first 64 columns of S_t (the
+// A operand of the PV product), O rescaled when the reference max moved
+// (`rescale_ok`: a PV product of this item has run), running max and sum.
+// The reference m: lazily (the default) the running max of the earlier
+// tiles, with no max over this tile; the row sum tells when some score rose
+// so far above it that p left the safe range (sum > 2^32, or not finite) --
+// then the warp reads S again (P is not stored yet), takes the tile's max
+// and redoes the exponentials.  An item's first tile takes its max first.
+// Eagerly: the tile's max, moved into m only when it passes m by more than
+// kRescaleThreshold.
+FA_DEV void softmax_tile(uint32_t s_base, uint32_t o_base, uint32_t bits, bool diag, int r,
+                         float c, bool rescale_ok, float &m_run, float &l_run) {
+  float m_ref = m_run, m_new = m_run;
+  bool need = false;
+  uint32_t pk[BN / 2];
+  float l_tile;
+  {
+    float s[BN];
+    load_scores(s_base, bits, diag, r, s);
+    const bool lazy = kLazyMax && !__any_sync(0xffffffffu, m_run == -INFINITY);
+    if (!lazy) {
+      m_new = fmaxf(m_run, row_max(s) * c);
+      need = m_new > m_run + kRescaleThreshold;
+      m_ref = need ? m_new : m_run;
+    }
+    l_tile = row_exp2(s, c, m_ref, pk);
+  }
+  if (kLazyMax && __any_sync(0xffffffffu, !(l_tile <= kLazySumLimit))) {
+    float s[BN];
+    load_scores(s_base, bits, diag, r, s);
+    m_new = fmaxf(m_run, row_max(s) * c);
+    need = m_new > m_run;
+    m_ref = need ? m_new : m_run;
+    l_tile = row_exp2(s, c, m_ref, pk);
+  }
+  {
+    uint32_t lo[32], hi[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const int k0 = q2 * 64 + 2 * i;
-      const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
-      float p0, p1;
-      if ((k0 & 7) >= 8 - kPolyPer8) {
-        ex2_poly2(x, p0, p1);
-      } else {
-        float x0, x1;
-        f2_split(x, x0, x1);
-        p0 = ex2(x0);
-        p1 = ex2(x1);
-      }
-      acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
-      pk[i] = pack_bf16x2(p0, p1);
+      lo[i] = pk[i];
+      hi[i] = pk[32 + i];
     }
-    tmem_st32(s_base + q2 * 32, pk);
+    tmem_st32(s_base, lo);
+    tmem_st32(s_base + 32, hi);
   }
   // S_t(j) ready implies PV_t(j-1) is done (MMAs complete in order), so
   // O_t may be rescaled here before P_t(j) is released.
@@ -1023,12 +1074,8 @@ FA_DEV void softmax_tile(uint32_t s_base, uint32_t o_base, uint32_t bits, bool d
     }
   }
   if (need) l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
-  m_run = m_next;
-  {
-    float a0, a1;
-    f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
-    l_run += a0 + a1;
-  }
+  m_run = m_ref;
+  l_run += l_tile;
 }
 
 FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CUtensorMap *tmO,
