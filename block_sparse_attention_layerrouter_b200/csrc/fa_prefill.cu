@@ -547,11 +547,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // runs.  MMAs complete in issue order, so "S_t(j) ready" (a commit after
 // QK_t(j)) also means PV_t(j-1) has finished: the softmax may rescale O_t
 // and overwrite S_t with P_t without any further wait.
-// exp2 runs on the special-function unit (ex2.approx); a polynomial on the
-// FMA pipe can take a share of the keys (kPolyPer8 of every 8, in pairs) to
-// unload it, but with this schedule moving a quarter of the keys there
-// measured no faster on full layers and 5 % slower on sparse ones, so the
-// default share is 0.
+// exp2 runs on the special-function unit (ex2.approx) for most keys; a
+// polynomial on the FMA pipe takes a share (kPolyPer8 of every 8, in pairs):
+// a quarter of the keys by default, which shortens the softmax of a tile
+// (the special-function unit alone needs 8 cycles per warp instruction, 1024
+// per 128-key row); half the keys there is slower again (the polynomial's
+// own instructions then fill the issue slots).
 // =====================================================================
 namespace prefill2 {
 
@@ -599,7 +600,7 @@ constexpr uint64_t kDrainNs = 200000000ull;
 // max relative error 1.0e-4, below bf16 rounding of P), and n added to the
 // exponent field.  Inputs below -127 give 0.
 #ifndef FA_POLY_PER_8
-#define FA_POLY_PER_8 0
+#define FA_POLY_PER_8 2
 #endif
 // Key pairs (k, k+1), k even, with (k mod 8) >= 8 - kPolyPer8 take the
 // polynomial (so kPolyPer8 counts in steps of 2); the rest use ex2.approx.
@@ -827,6 +828,17 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
   }
 }
 
+// True on one lane of the warp (elect.sync).
+FA_DEV bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+               : "=r"(e)::"memory");
+  return e != 0;
+}
+
+// Each product's eight MMAs are issued back to back by one elected lane
+// (one election per product rather than per MMA; the issue rate of this
+// warp is on the critical path of every tile).
 FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   constexpr uint32_t kIdescQK = idesc_bf16_f32(BM, BN, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, true);
@@ -866,11 +878,14 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   auto qk = [&](int t, int slot) {
     const uint64_t qd = t ? q_desc1 : q_desc0;
     const uint64_t kd = k_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
+    if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
-      const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-      mma_bf16_ss_w(tmem + 256u * t, qd + off, kd + off, kIdescQK, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+        mma_bf16_ss(tmem + 256u * t, qd + off, kd + off, kIdescQK, kk > 0 ? 1u : 0u);
+      }
     }
+    __syncwarp();
     tc_commit_w(sh.bar(Smem::S_FULL0 + t));
   };
   auto pv = [&](int t, bool first, int slot) -> bool {
@@ -881,12 +896,15 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       return false;
     tc_fence_after_sync();
     const uint64_t vd = v_desc_base + static_cast<uint64_t>(slot * (TILE_BYTES >> 4));
+    if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
-      mma_bf16_ts_w(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
+      for (int kk = 0; kk < BN / 16; ++kk) {
+        mma_bf16_ts(tmem + 256u * t + 128u, tmem + 256u * t + kk * 8,
                     vd + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
                     (!first || kk > 0) ? 1u : 0u);
+      }
     }
+    __syncwarp();
     return true;
   };
 
@@ -913,8 +931,9 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     tc_commit_w(sh.bar(Smem::EMPTY0 + k_slot));
     if (!has_next) tc_commit_w(sh.bar(Smem::Q_EMPTY));     // the last QK of this item is issued
     for (int j = 0;; ++j) {
+      // V of tile j and K of tile j+1 (the producer is tiles ahead) are taken
+      // before the PV waits for P_0, so PV_0(j) and QK_0(j+1) go out back to back.
       if (!(ok = take(v_slot))) break;
-      if (!(ok = pv(0, j == 0, v_slot))) break;
       if (has_next) {
         if (im.sparse) {                      // tile j+1: is it the last?
           const int e = take_info(ok);
@@ -924,6 +943,9 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
           has_next2 = j + 1 < im.qt;
         }
         if (!(ok = take(k_slot))) break;
+      }
+      if (!(ok = pv(0, j == 0, v_slot))) break;
+      if (has_next) {
         qk(0, k_slot);
       } else {
         tc_commit_w(sh.bar(Smem::O_DONE0));
@@ -1127,7 +1149,8 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
       softmax_tile(s_base, o_base, bits, n == im.qt, r, c, j > 0, m_run, l_run);
       tmem_st_wait();
       tc_fence_before_sync();
-      mbar_arrive_a(sh.bar(Smem::P_FULL0 + t));
+      __syncwarp();     // one arrive per warp, after all its lanes' P stores
+      if ((threadIdx.x & 31) == 0) mbar_arrive_a(sh.bar(Smem::P_FULL0 + t));
       ++j;
       ++js;
     }
@@ -1224,7 +1247,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int t = 0; t < NQ; ++t) {
       mbar_init_a(sh.bar(Smem::S_FULL0 + t), 1);
-      mbar_init_a(sh.bar(Smem::P_FULL0 + t), 128);
+      mbar_init_a(sh.bar(Smem::P_FULL0 + t), 4);     // one arrive per softmax warp
       mbar_init_a(sh.bar(Smem::O_DONE0 + t), 1);
       mbar_init_a(sh.bar(Smem::O_FREE0 + t), 128);
     }
