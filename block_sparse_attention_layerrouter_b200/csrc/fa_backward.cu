@@ -245,6 +245,8 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
 }
 
 // ------------------------------------------------------------------ MMA
+// The warp runs warp-wide; each product's MMAs are issued back to back by
+// one elected lane (one election per product, not per MMA).
 FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   constexpr uint32_t kIdS = idesc_bf16_f32_ab(BK, BQ, false, false);   // S^T, dP^T
   constexpr uint32_t kIdKV = idesc_bf16_f32_ab(BK, HD, false, true);   // dV, dK
@@ -272,25 +274,30 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       return false;
     tc_fence_after_sync();
     const uint64_t so = static_cast<uint64_t>((s * STAGE_BYTES) >> 4);
+    if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
-      const uint64_t ok_ = static_cast<uint64_t>(((kk >> 2) * KV_HALF + (kk & 3) * 32) >> 4);
-      const uint64_t oq = static_cast<uint64_t>(((kk >> 2) * QT_HALF + (kk & 3) * 32) >> 4);
-      mma_bf16_ss_w(tmem + 64u * u, k_kmaj + ok_, q_kmaj + so + oq, kIdS, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint64_t ok_ = static_cast<uint64_t>(((kk >> 2) * KV_HALF + (kk & 3) * 32) >> 4);
+        const uint64_t oq = static_cast<uint64_t>(((kk >> 2) * QT_HALF + (kk & 3) * 32) >> 4);
+        mma_bf16_ss(tmem + 64u * u, k_kmaj + ok_, q_kmaj + so + oq, kIdS, kk > 0 ? 1u : 0u);
+      }
     }
+    __syncwarp();
     tc_commit_w(sh.bar(Smem::S_FULL0 + u));
     // dP^T_u is where dQ^T of step nf-2 lives until its readout is done.
     if (nf >= 2 &&
         !warp_wait(sh.bar(Smem::DQ_FREE0 + u), static_cast<uint32_t>((nf >> 1) - 1) & 1u, sh, p))
       return false;
     tc_fence_after_sync();
+    if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
-      const uint64_t ok_ = static_cast<uint64_t>(((kk >> 2) * KV_HALF + (kk & 3) * 32) >> 4);
-      const uint64_t oq = static_cast<uint64_t>(((kk >> 2) * QT_HALF + (kk & 3) * 32) >> 4);
-      mma_bf16_ss_w(tmem + 128u + 64u * u, v_kmaj + ok_, o_kmaj + so + oq, kIdS,
-                    kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint64_t ok_ = static_cast<uint64_t>(((kk >> 2) * KV_HALF + (kk & 3) * 32) >> 4);
+        const uint64_t oq = static_cast<uint64_t>(((kk >> 2) * QT_HALF + (kk & 3) * 32) >> 4);
+        mma_bf16_ss(tmem + 128u + 64u * u, v_kmaj + ok_, o_kmaj + so + oq, kIdS, kk > 0 ? 1u : 0u);
+      }
     }
+    __syncwarp();
     tc_commit_w(sh.bar(Smem::DP_FULL0 + u));
     ++nf;
     return true;
@@ -305,23 +312,30 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     tc_fence_after_sync();
     const uint64_t so = static_cast<uint64_t>((s * STAGE_BYTES) >> 4);
     const uint64_t du = static_cast<uint64_t>((u * DS_BYTES) >> 4);
+    if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < BQ / 16; ++kk) {   // dV += P^T dO
-      mma_bf16_ts_w(t_dv, tmem + 64u * u + kk * 8, o_mn + so + static_cast<uint64_t>((kk * 2048) >> 4),
-                    kIdKV, (first && kk == 0) ? 0u : 1u);
-    }
+      for (int kk = 0; kk < BQ / 16; ++kk) {   // dV += P^T dO
+        mma_bf16_ts(t_dv, tmem + 64u * u + kk * 8,
+                    o_mn + so + static_cast<uint64_t>((kk * 2048) >> 4), kIdKV,
+                    (first && kk == 0) ? 0u : 1u);
+      }
 #pragma unroll
-    for (int kk = 0; kk < BQ / 16; ++kk) {   // dK += dS^T Q (dS^T from TMEM)
-      mma_bf16_ts_w(t_dk, tmem + 128u + 64u * u + kk * 8,
+      for (int kk = 0; kk < BQ / 16; ++kk) {   // dK += dS^T Q (dS^T from TMEM)
+        mma_bf16_ts(t_dk, tmem + 128u + 64u * u + kk * 8,
                     q_mn + so + static_cast<uint64_t>((kk * 2048) >> 4), kIdKV,
                     (first && kk == 0) ? 0u : 1u);
+      }
     }
+    __syncwarp();
     tc_commit_w(sh.bar(Smem::ST_EMPTY0 + s));
+    if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < BK / 16; ++kk) {   // dQ^T = K^T dS^T
-      mma_bf16_ss_w(tmem + 128u + 64u * u, k_mn + static_cast<uint64_t>((kk * 2048) >> 4),
+      for (int kk = 0; kk < BK / 16; ++kk) {   // dQ^T = K^T dS^T
+        mma_bf16_ss(tmem + 128u + 64u * u, k_mn + static_cast<uint64_t>((kk * 2048) >> 4),
                     ds_mn + du + static_cast<uint64_t>((kk * 2048) >> 4), kIdQ, kk > 0 ? 1u : 0u);
+      }
     }
+    __syncwarp();
     tc_commit_w(sh.bar(Smem::DQ_FULL0 + u));
     if (last) {
       tc_commit_w(sh.bar(Smem::ACC_FULL));

@@ -251,6 +251,15 @@ FA_DEV void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint3
       : "memory");
 }
 
+// True on one lane of the warp (elect.sync); a warp that issues several
+// MMAs in a row elects once and lets that lane issue them all.
+FA_DEV bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+               : "=r"(e)::"memory");
+  return e != 0;
+}
+
 // ---- warp-wide forms: every lane of the warp executes the call with the
 // same (warp-uniform) operands and exactly one elected lane issues the
 // operation, so the surrounding loop stays on the uniform datapath.

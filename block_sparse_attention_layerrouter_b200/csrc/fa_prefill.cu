@@ -828,14 +828,6 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
   }
 }
 
-// True on one lane of the warp (elect.sync).
-FA_DEV bool elect_one() {
-  uint32_t e;
-  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
-               : "=r"(e)::"memory");
-  return e != 0;
-}
-
 // Each product's eight MMAs are issued back to back by one elected lane
 // (one election per product rather than per MMA; the issue rate of this
 // warp is on the critical path of every tile).
