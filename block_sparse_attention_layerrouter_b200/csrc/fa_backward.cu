@@ -466,10 +466,13 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
         const float4 L = ld_shared_f4(lse_s + 16u * j4);
         const float l4[4] = {L.x, L.y, L.z, L.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < 4; e += 2) {
           const int j = 4 * j4 + e;
-          const bool keep = any && (j + rel >= 0);
-          pv[j] = keep ? ex2(fmaf(pv[j], c, -l4[e])) : 0.0f;
+          float x0, x1;     // two keys per packed fp32x2 instruction
+          f2_split(f2_fma(f2_make(pv[j], pv[j + 1]), f2_make(c, c), f2_make(-l4[e], -l4[e + 1])),
+                   x0, x1);
+          pv[j] = (any && (j + rel >= 0)) ? ex2(x0) : 0.0f;
+          pv[j + 1] = (any && (j + 1 + rel >= 0)) ? ex2(x1) : 0.0f;
         }
       }
       {
@@ -499,9 +502,11 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
           const float4 Dv = ld_shared_f4(d_s + 16u * (8 * hlf + j4));
           const float d4[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < 4; e += 2) {
             const int j = 4 * j4 + e;
-            ds[j] = pv[32 * hlf + j] * (__uint_as_float(a[j]) - d4[e]);
+            const uint64_t t2 = f2_add(f2_make(__uint_as_float(a[j]), __uint_as_float(a[j + 1])),
+                                       f2_make(-d4[e], -d4[e + 1]));
+            f2_split(f2_mul(f2_make(pv[32 * hlf + j], pv[32 * hlf + j + 1]), t2), ds[j], ds[j + 1]);
           }
         }
         uint32_t pk[16];
@@ -523,7 +528,8 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before_sync();
-      mbar_arrive_a(sh.bar(Smem::EW_DONE0 + u));
+      __syncwarp();     // one arrive per warp, after all its lanes' stores
+      if ((threadIdx.x & 31) == 0) mbar_arrive_a(sh.bar(Smem::EW_DONE0 + u));
     }
     if (!ok) break;
     // Epilogue: dV and scale * dK of this key row.
@@ -589,7 +595,8 @@ FA_DEV void run_dq(const Smem &sh, uint32_t tmem, const CUtensorMap *tmA, const 
       tmem_ld_wait(a);
       tmem_ld_wait(b);
       tc_fence_before_sync();
-      mbar_arrive_a(sh.bar(Smem::DQ_FREE0 + u));
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive_a(sh.bar(Smem::DQ_FREE0 + u));
       bulk_wait_read0();          // the previous reduce has read the staging box
       __syncwarp();
 #pragma unroll
@@ -627,9 +634,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int u = 0; u < 2; ++u) {
       mbar_init_a(sh.bar(Smem::S_FULL0 + u), 1);
       mbar_init_a(sh.bar(Smem::DP_FULL0 + u), 1);
-      mbar_init_a(sh.bar(Smem::EW_DONE0 + u), 128);
+      mbar_init_a(sh.bar(Smem::EW_DONE0 + u), 4);     // one arrive per warp
       mbar_init_a(sh.bar(Smem::DQ_FULL0 + u), 1);
-      mbar_init_a(sh.bar(Smem::DQ_FREE0 + u), 128);
+      mbar_init_a(sh.bar(Smem::DQ_FREE0 + u), 4);     // one arrive per warp
     }
     mbar_init_a(sh.bar(Smem::ACC_FULL), 1);
     mbar_init_a(sh.bar(Smem::ACC_FREE), 128);
