@@ -14,7 +14,9 @@
 //   csc_*_kernel   for the sparse path: per 128-key tile, the 64-query
 //                  blocks whose CSR rows keep one of its two key blocks.
 //   bwd_kernel     persistent, one CTA per SM; a work item is one 128-key
-//                  tile of one (batch, KV head).  It walks the 64-query
+//                  tile of one (batch, KV head) (or a chunk of its query
+//                  blocks), claimed from a global counter heaviest first, so
+//                  CTAs that drew long items take fewer.  It walks the 64-query
 //                  blocks that attend the tile, for all G query heads of the
 //                  group, with five tcgen05 MMAs per step:
 //                    S^T  = K Q^T      (M=128 keys, N=64 queries, K=D)
@@ -67,7 +69,8 @@ struct Smem {
     KV_FULL = 0, KV_EMPTY = 1, ST_FULL0 = 2, ST_EMPTY0 = ST_FULL0 + NST,
     S_FULL0 = ST_EMPTY0 + NST, DP_FULL0 = S_FULL0 + 2, EW_DONE0 = DP_FULL0 + 2,
     DQ_FULL0 = EW_DONE0 + 2, DQ_FREE0 = DQ_FULL0 + 2, ACC_FULL = DQ_FREE0 + 2,
-    ACC_FREE = ACC_FULL + 1, DRAIN = ACC_FREE + 1, NBARS = DRAIN + 1
+    ACC_FREE = ACC_FULL + 1, DRAIN = ACC_FREE + 1, ITEM_FULL0 = DRAIN + 1,
+    ITEM_EMPTY0 = ITEM_FULL0 + 4, NBARS = ITEM_EMPTY0 + 4
   };
   FA_DEV uint32_t k() const { return base + kK; }
   FA_DEV uint32_t v() const { return base + kV; }
@@ -80,8 +83,13 @@ struct Smem {
   FA_DEV uint32_t bar(uint32_t i) const { return base + kBars + 8u * i; }
   FA_DEV uint32_t tmem_slot() const { return base + kBars + 8u * NBARS; }
   FA_DEV uint32_t abort_flag() const { return tmem_slot() + 4u; }
+  // Work-item ring (NITEM entries) the producer fills for the other roles.
+  FA_DEV uint32_t item(int slot) const {
+    return tmem_slot() + 16u + 4u * static_cast<uint32_t>(slot);
+  }
 };
-constexpr int SMEM_BYTES = 1024 + Smem::kBars + 8 * Smem::NBARS + 16;
+constexpr int NITEM = 4;
+constexpr int SMEM_BYTES = 1024 + Smem::kBars + 8 * Smem::NBARS + 16 + 4 * NITEM;
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 
 struct Params {
@@ -99,6 +107,8 @@ struct Params {
   int32_t *status;
   int B, S, Sp, Hq, Hkv, G, nqb, nkt;
   int cq_full, cq_sparse, cmax;      // query blocks per chunk (per mode), chunks per tile
+  int *item_counter;                 // next unclaimed work item (zeroed before the launch)
+  int order;                         // item numbering: kOrderChunk / kOrderTile / kOrderChunkDesc
   float scale, scale_log2;
 };
 
@@ -133,6 +143,19 @@ struct Item {
   int kt, b, kvh, nq, ct0, q0, nq_total;
   bool sparse, split;
 };
+// Work items are claimed in numbering order from a global counter, so each
+// CTA takes the next one when it is done (the heaviest items should come
+// first).  Numberings:
+//  * kOrderChunk: one chunk index across all tiles, then the next -- the full
+//    path: chunk 0 holds the last query blocks, which every tile attends (the
+//    heaviest), and the CTAs running together reduce into the same dQ rows.
+//  * kOrderTile: all chunks of a tile, then the next tile -- the sparse path
+//    when the dQ accumulator is small: the sink tiles' chunks (every query
+//    block attends them) come first.
+//  * kOrderChunkDesc: chunk-major from the last chunk down -- the sparse path
+//    with a large accumulator: the sink tiles' later chunks first, and the
+//    CTAs still share query rows.
+constexpr int kOrderChunk = 0, kOrderTile = 1, kOrderChunkDesc = 2;
 FA_DEV int tile_nq(const Params &p, int kt, bool sparse, int &ct0) {
   if (sparse) {
     ct0 = p.ct_ptr[kt];
@@ -148,10 +171,19 @@ FA_DEV bool batch_sparse(const Params &p, int b) {
 FA_DEV Item item_of(const Params &p, int w) {
   Item it;
   const int bh = p.B * p.Hkv, per_c = p.nkt * bh;
-  const int c = w / per_c;
-  int rem = w % per_c;
-  it.kt = rem / bh;
-  rem %= bh;
+  int c, rem;
+  if (p.order == kOrderTile) {    // all chunks of a tile, then the next tile
+    it.kt = w / (p.cmax * bh);
+    rem = w % (p.cmax * bh);
+    c = rem / bh;
+    rem %= bh;
+  } else {                        // one chunk index across all tiles, then the next
+    c = w / per_c;
+    rem = w % per_c;
+    it.kt = rem / bh;
+    rem %= bh;
+    if (p.order == kOrderChunkDesc) c = p.cmax - 1 - c;
+  }
   it.b = rem / p.Hkv;
   it.kvh = rem % p.Hkv;
   it.sparse = batch_sparse(p, it.b);
@@ -178,11 +210,6 @@ FA_DEV void q_block(const Params &p, const Item &it, int qi, int &qb, uint32_t &
     bits = 3u;
   }
 }
-FA_DEV int item_index(int k, int total) {
-  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-  const int w = k * G + ((k & 1) ? (G - 1 - c) : c);
-  return w < total ? w : -1;
-}
 FA_DEV float out_factor(const Params &p, int b) {
   if (!p.gscale) return 1.0f;
   return p.gscale_complement ? 1.0f - p.gscale[b] : p.gscale[b];
@@ -191,6 +218,18 @@ FA_DEV float out_factor(const Params &p, int b) {
 FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const Smem &sh, const Params &p) {
   const bool done = mbar_wait_a(bar, parity, sh.abort_flag(), p.status);
   return __all_sync(0xffffffffu, done);
+}
+
+// The k-th work item of this CTA from the producer's ring (-1: no more), or
+// -2 after an abort.  One arrive per warp frees the entry.
+FA_DEV int next_item(const Smem &sh, const Params &p, int k) {
+  const int slot = k & (NITEM - 1);
+  if (!warp_wait(sh.bar(Smem::ITEM_FULL0 + slot), static_cast<uint32_t>(k / NITEM) & 1u, sh, p))
+    return -2;
+  const int w = ld_shared_s32(sh.item(slot));
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_a(sh.bar(Smem::ITEM_EMPTY0 + slot));
+  return w;
 }
 
 // ------------------------------------------------------------- producer
@@ -203,7 +242,30 @@ FA_DEV void run_producer(const Smem &sh, const CUtensorMap *tmQ, const CUtensorM
   if (c_skip_loads) return;      // testing mode: no loads, every wait runs out
   bool ok = true;
   for (int k = 0; ok; ++k) {
-    const int w = item_index(k, total);
+    // Claim the next item that has work (or zero rows to write) from the
+    // global counter and publish it to the other roles through the ring.
+    int w = 0;
+    if ((threadIdx.x & 31) == 0) {
+      while (true) {
+        w = atomicAdd(p.item_counter, 1);
+        if (w >= total) {
+          w = -1;
+          break;
+        }
+        const Item t = item_of(p, w);
+        if (t.nq > 0 || (t.nq_total == 0 && t.q0 == 0)) break;   // else an empty chunk
+      }
+    }
+    w = __shfl_sync(0xffffffffu, w, 0);
+    {
+      const int slot = k & (NITEM - 1);
+      if (k >= NITEM && !warp_wait(sh.bar(Smem::ITEM_EMPTY0 + slot),
+                                   static_cast<uint32_t>(k / NITEM - 1) & 1u, sh, p))
+        break;
+      if ((threadIdx.x & 31) == 0) st_shared_s32(sh.item(slot), w);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive_a(sh.bar(Smem::ITEM_FULL0 + slot));
+    }
     if (w < 0) break;
     const Item it = item_of(p, w);
     const int n_it = it.nq * p.G;
@@ -346,7 +408,11 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   };
 
   for (int k = 0; ok; ++k) {
-    const int w = item_index(k, total);
+    const int w = next_item(sh, p, k);
+    if (w == -2) {
+      ok = false;
+      break;
+    }
     if (w < 0) break;
     const Item it = item_of(p, w);
     const int n_it = it.nq * p.G;
@@ -415,7 +481,7 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
   int n = 0, acc_n = 0;
   bool ok = true;
   for (int k = 0; ok; ++k) {
-    const int w = item_index(k, total);
+    const int w = next_item(sh, p, k);
     if (w < 0) break;
     const Item it = item_of(p, w);
     const int n_it = it.nq * p.G;
@@ -573,7 +639,7 @@ FA_DEV void run_dq(const Smem &sh, uint32_t tmem, const CUtensorMap *tmA, const 
   int n = 0;
   bool ok = true;
   for (int k = 0; ok; ++k) {
-    const int w = item_index(k, total);
+    const int w = next_item(sh, p, k);
     if (w < 0) break;
     const Item it = item_of(p, w);
     const int n_it = it.nq * p.G;
@@ -641,6 +707,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init_a(sh.bar(Smem::ACC_FULL), 1);
     mbar_init_a(sh.bar(Smem::ACC_FREE), 128);
     mbar_init_a(sh.bar(Smem::DRAIN), 1);
+    for (int i = 0; i < NITEM; ++i) {
+      mbar_init_a(sh.bar(Smem::ITEM_FULL0 + i), 1);
+      mbar_init_a(sh.bar(Smem::ITEM_EMPTY0 + i), 9);   // MMA warp, 4 EW and 4 dQ warps
+    }
     st_shared_s32(sh.abort_flag(), 0);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -917,7 +987,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 struct Plan {
   int nqb, nkt, Sp;
   float *acc, *dvec, *lse2, *dkv_acc;
-  int32_t *ct_ptr, *ct_q;
+  int32_t *ct_ptr, *ct_q, *counter;
   size_t bytes;
 };
 Plan make_plan(int B, int S, int Hq, int Hkv, void *workspace) {
@@ -940,6 +1010,7 @@ Plan make_plan(int B, int S, int Hq, int Hkv, void *workspace) {
       take(static_cast<size_t>(pl.nkt) * static_cast<size_t>(pl.nqb) * 4));
   pl.dkv_acc = reinterpret_cast<float *>(
       take(2 * static_cast<size_t>(B) * Hkv * pl.nkt * backward::BK * backward::HD * 4));
+  pl.counter = reinterpret_cast<int32_t *>(take(4));
   pl.bytes = off;
   return pl;
 }
@@ -1038,11 +1109,18 @@ int run_main(const BackwardLaunch &a, const Plan &pl, cudaStream_t stream) {
 #endif
   p.cq_full = (balanced && acc_bytes <= (static_cast<long long>(FA_BWD_WHOLE_TILE_ACC_MB) << 20))
                   ? pl.nqb : cq;
-  p.cq_sparse = cq;
+  // Sparse: at least 64 query blocks per chunk, so a window tile (which at
+  // most W/64 + 2 blocks attend) is seldom cut; only the sink tiles are.
+  p.cq_sparse = cq > 64 ? cq : 64;
   const bool any_sparse = sparse && (a.mode_dev != nullptr || a.mode_default == FA_MODE_SPARSE);
-  const int cq_min = any_sparse ? (p.cq_full < cq ? p.cq_full : cq) : p.cq_full;
+  const int cq_min =
+      any_sparse ? (p.cq_full < p.cq_sparse ? p.cq_full : p.cq_sparse) : p.cq_full;
   p.cmax = (pl.nqb + cq_min - 1) / cq_min;
   p.dkv_acc = pl.dkv_acc;
+  p.item_counter = pl.counter;
+  p.order = !any_sparse ? kOrderChunk
+                        : (acc_bytes <= (256ll << 20) ? kOrderTile : kOrderChunkDesc);
+  if (cudaMemsetAsync(pl.counter, 0, sizeof(int32_t), stream) != cudaSuccess) return FA_ERR_CUDA;
   const long long total = static_cast<long long>(p.cmax) * pl.nkt * a.B * a.Hkv;
   if (total <= 0 || total > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   const long long n4 = 2ll * a.B * a.Hkv * pl.nkt * BK * HD / 4;
