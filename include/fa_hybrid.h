@@ -190,7 +190,10 @@ FA_API int fa_attn_decode(const void *q, const void *kcache, const void *vcache,
  *   offending rows are reported as FA_DEV_BAD_INDEX).
  *   workspace >= fa_attn_backward_workspace_size(B, S, Hq, Hkv, D) bytes,
  *   16-byte aligned device memory: an fp32 dQ accumulator [B, S, Hq, D], the
- *   row terms D and the LSE in base 2, and the transposed block pattern.
+ *   row terms D and the LSE in base 2, the transposed block pattern, fp32
+ *   dK/dV partial sums of tiles cut into chunks, and the work-item counter
+ *   (reset on the stream by each call, so calls that share one workspace
+ *   must be ordered on one stream).
  * D must be 128.  Returns FA_OK or an fa_status; enqueues only. */
 FA_API size_t fa_attn_backward_workspace_size(int B, int S, int Hq, int Hkv, int D);
 FA_API int fa_attn_prefill_backward(const void *q, const void *k, const void *v,
