@@ -24,6 +24,7 @@ FA_MODE_FULL = 0
 FA_MODE_SPARSE = 1
 FA_DEV_TIMEOUT = 1
 FA_DEV_BAD_INDEX = 2
+FA_DEV_DEBUG_BOUNDS = 4
 
 
 class FaError(RuntimeError):
@@ -109,6 +110,17 @@ def lib():
             f.argtypes = args
         _lib = l
     return _lib
+
+
+def use_library(path: str) -> str:
+    """Load the library at `path` from now on (e.g. the debug build,
+    libfa_hybrid_debug.so, whose kernels bounds-check their output stores);
+    returns the path in use before."""
+    global _lib, LIB_PATH
+    old = LIB_PATH
+    LIB_PATH = path
+    _lib = None
+    return old
 
 
 def status_string(status: int) -> str:

@@ -601,7 +601,16 @@ FA_DEV void run_ew(const Smem &sh, uint32_t tmem, const Params &p, int total) {
     // Epilogue: dV and scale * dK of this key row.
     if (!warp_wait(sh.bar(Smem::ACC_FULL), static_cast<uint32_t>(acc_n) & 1u, sh, p)) break;
     tc_fence_after_sync();
-    const bool store = key < p.S && !ld_shared_s32(sh.abort_flag());
+    bool store = key < p.S && !ld_shared_s32(sh.abort_flag());
+    // Debug builds: the gradient row and, for a split tile, its fp32 partial row.
+    if (store)
+      store = it.split
+                  ? in_bounds(p.status, static_cast<long long>(((static_cast<size_t>(it.b) * p.Hkv +
+                                                                 it.kvh) * p.nkt * BK + key) * HD),
+                              static_cast<long long>(p.B) * p.Hkv * p.nkt * BK * HD)
+                  : in_bounds(p.status,
+                              ((static_cast<long long>(it.b) * p.S + key) * p.Hkv + it.kvh) * HD,
+                              static_cast<long long>(p.B) * p.S * p.Hkv * HD);
     const size_t acc_row = ((static_cast<size_t>(it.b) * p.Hkv + it.kvh) * p.nkt * BK + key) * HD;
     const size_t acc_half = static_cast<size_t>(p.B) * p.Hkv * p.nkt * BK * HD;
     {

@@ -55,6 +55,20 @@ FA_DEV void report(int32_t *status, int32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
+// Debug builds (-DFA_DEBUG=1, libfa_hybrid_debug.so) check the flattened
+// element index of each direct global store of an output against the
+// tensor's element count -- computed from the shape, apart from the index
+// arithmetic it checks -- and report bit 4 (FA_DEV_DEBUG_BOUNDS) instead of
+// storing.  Release builds compile the check away.
+#ifndef FA_DEBUG
+#define FA_DEBUG 0
+#endif
+FA_DEV bool in_bounds(int32_t *status, long long idx, long long count) {
+  if (!FA_DEBUG || (idx >= 0 && idx < count)) return true;
+  report(status, 4);
+  return false;
+}
+
 // ----------------------------------------------------------------- mbarrier
 FA_DEV void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)

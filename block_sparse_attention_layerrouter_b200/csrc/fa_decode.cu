@@ -490,8 +490,11 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     // held before.
     if (tid < G) {
       const size_t r0 = (static_cast<size_t>(b) * p.Hq + kvh * G + tid) * p.nsplit + split;
-      p.ml_part[r0 * 2] = __int_as_float(0x7fc00000);
-      p.ml_part[r0 * 2 + 1] = __int_as_float(0x7fc00000);
+      if (in_bounds(p.status, static_cast<long long>(r0) * 2 + 1,
+                    static_cast<long long>(p.B) * p.Hq * p.nsplit * 2)) {
+        p.ml_part[r0 * 2] = __int_as_float(0x7fc00000);
+        p.ml_part[r0 * 2 + 1] = __int_as_float(0x7fc00000);
+      }
     }
     __syncthreads();
     return;
@@ -522,15 +525,21 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     float sum = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) sum += red[(s * G + g) * HD + dd];
-    p.o_part[(row0 + static_cast<size_t>(g) * p.nsplit) * HD + dd] = sum * vs;
+    const size_t oi = (row0 + static_cast<size_t>(g) * p.nsplit) * HD + dd;
+    if (in_bounds(p.status, static_cast<long long>(oi),
+                  static_cast<long long>(p.B) * p.Hq * p.nsplit * HD))
+      p.o_part[oi] = sum * vs;
   }
   if (tid < G) {
     float l = 0.f;
 #pragma unroll
     for (int w = 0; w < NT / 32; ++w) l += lsum_sm[w * G + tid];
-    float *ml = p.ml_part + (row0 + static_cast<size_t>(tid) * p.nsplit) * 2;
-    ml[0] = mref_sm[tid];
-    ml[1] = l;
+    const size_t mi = (row0 + static_cast<size_t>(tid) * p.nsplit) * 2;
+    if (in_bounds(p.status, static_cast<long long>(mi) + 1,
+                  static_cast<long long>(p.B) * p.Hq * p.nsplit * 2)) {
+      p.ml_part[mi] = mref_sm[tid];
+      p.ml_part[mi + 1] = l;
+    }
   }
 }
 

@@ -443,12 +443,15 @@ FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[i] = 0u;
     }
-    if (store) {
+    if (store && in_bounds(p.status, ((static_cast<long long>(b) * p.S + t) * p.Hq + h) * HD + q4 * 32,
+                           static_cast<long long>(p.B) * p.S * p.Hq * HD)) {
       uint4 *dst = reinterpret_cast<uint4 *>(orow + q4 * 32);
       store_row_chunk(dst, o, inv_l, p.mix_r, b);
     }
   }
-  if (store && p.lse) {
+  if (store && p.lse &&
+      in_bounds(p.status, (static_cast<long long>(b) * p.Hq + h) * p.S + t,
+                static_cast<long long>(p.B) * p.Hq * p.S)) {
     const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + t] = lse;
   }
@@ -1166,6 +1169,9 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
       for (int i = 0; i < HD; ++i) o[i] = 0u;
     }
     const int tok = im.qt * BM + r;
+    // Token rows of O (and LSE entries per head): the packed tensor's, or B * S.
+    const long long rows_total =
+        p.cu_seqlens ? static_cast<long long>(p.total_tokens) : static_cast<long long>(p.B) * p.S;
     const bool aborted = ld_shared_s32(sh.abort_flag()) != 0;
     const bool store = (tok < im.L) && !aborted;
     const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
@@ -1204,7 +1210,9 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
         __syncwarp();
         if (lane == 0 && im.qt * BM + 32 * wq < im.L)   // rows past the end are clipped
           tma_store_4d_commit(tmO, box, q4 * 32, h, im.tma_tok0 + im.qt * BM + 32 * wq, im.tma_b);
-      } else if (store) {
+      } else if (store && in_bounds(p.status,
+                                    ((static_cast<long long>(im.row0) + tok) * p.Hq + h) * HD + q4 * 32,
+                                    rows_total * p.Hq * HD)) {
         uint32_t oc[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) oc[i] = o[32 * q4 + i];
@@ -1212,7 +1220,9 @@ FA_DEV void run_softmax(const Smem &sh, uint32_t tmem, const Params &p, const CU
         prefill::store_row_chunk(dst, oc, inv_l, p.mix_r, im.b);
       }
     }
-    if (store && p.lse) {
+    if (store && p.lse &&
+        in_bounds(p.status, im.lse0 + static_cast<long long>(h) * im.lse_hs + tok,
+                  rows_total * p.Hq)) {
       const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       p.lse[im.lse0 + static_cast<long long>(h) * im.lse_hs + tok] = lse;
     }
@@ -1345,7 +1355,7 @@ __global__ void __launch_bounds__(1024) varlen_items_kernel(const int32_t *cu, i
     int pos = 0;
     for (int b = 0; b < B; ++b) pos += max(0, nq[b] - v - 1);
     for (int b = 0; b < B; ++b)
-      if (nq[b] > v) items[pos++] = (v << 12) | b;
+      if (nq[b] > v && in_bounds(status, pos, max_items)) items[pos++] = (v << 12) | b;
   }
 }
 

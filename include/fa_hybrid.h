@@ -58,6 +58,9 @@ typedef enum {
 #define FA_DEV_TIMEOUT   1     /* a bounded wait ran out; outputs invalid */
 #define FA_DEV_BAD_INDEX 2     /* a block index outside [0, query block] or
                                   out of order was skipped */
+#define FA_DEV_DEBUG_BOUNDS 4  /* debug builds only (libfa_hybrid_debug.so):
+                                  a store's index fell outside its tensor
+                                  and the store was skipped */
 
 typedef enum { FA_MODE_FULL = 0, FA_MODE_SPARSE = 1 } fa_mode;
 
