@@ -676,11 +676,11 @@ FA_DEV Smem carve(uint8_t *raw) {
 //    CTAs running together cover every KV head.
 //  * KV-head-major bands (long sequences): a band is band_q query tiles; its
 //    items are ordered by KV stream (batch, KV head), then query tile, then
-//    head pair, so the CTAs running together (band_q x pairs-per-KV-head =
-//    one CTA per SM) all stream the K/V tiles of the same KV head and each
-//    tile is read from HBM about once per band rather than once per CTA
-//    that drifted out of L2 reach.  Lengths inside a band differ by at most
-//    band_q tiles.
+//    head pair, so the CTAs running together all stream the K/V tiles of the
+//    same KV head, and so do the rounds after them until the band's items of
+//    that head run out: the head's K/V stays in L2 instead of being read
+//    from HBM again by CTAs that drifted out of L2 reach.  The launcher
+//    makes the whole sequence one band.
 struct Item {
   int qt, b, h0, kvh;
   bool sparse;
@@ -1447,15 +1447,18 @@ int launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
 #endif
     const long long cap = FA_PREFILL_PERSISTENT ? sms : grid;
     const int ctas = static_cast<int>(grid < cap ? grid : cap);
-    // KV-head-major bands when the sequence is long enough for several bands
-    // of one CTA per SM (the K/V of one head then no longer fits the L2
-    // share the query-tile-major order leaves it).
+    // KV-head-major order when the sequence holds at least four rounds of
+    // one CTA per SM per KV head (the K/V of one head then no longer fits the
+    // L2 share the query-tile-major order leaves it): one band of the whole
+    // sequence, so every round streams one KV head after another.  At 256K
+    // this read ~200 GB from HBM per FULL launch, against ~480 GB with bands
+    // of one round (74 query tiles) and ~900 GB query-tile-major.
 #ifndef FA_BAND_ORDER
 #define FA_BAND_ORDER 1
 #endif
     const int ppk = G / 2;
     const int band = ctas / ppk;
-    p.band_q = (FA_BAND_ORDER && !varlen && band >= 1 && p.n_qtiles >= 4 * band) ? band : 0;
+    p.band_q = (FA_BAND_ORDER && !varlen && band >= 1 && p.n_qtiles >= 4 * band) ? p.n_qtiles : 0;
     prefill2::prefill2_kernel<<<ctas, prefill2::NUM_THREADS, prefill2::SMEM_BYTES, stream>>>(
         tmQ, tmK, tmV, tmO, p, static_cast<int>(grid));
     note_launch();

@@ -143,8 +143,8 @@ def test_backward_split_tiles_write_only_their_gradients(mode):
 @pytest.mark.parametrize("mode", ["full", "sparse"])
 def test_prefill_long_sequence_item_order_covers_every_row(mode):
     """S = 40000 with 4 query heads per KV head: long enough for the
-    KV-head-major item order (bands of 74 query tiles and a partial last
-    band; the last tile ragged).  Every output row must be written exactly
+    KV-head-major item order (the whole sequence one band, so each KV
+    head's items run one after another; the last tile ragged).  Every output row must be written exactly
     where it belongs: all rows finite inside the fences, sampled rows equal
     to the oracle's."""
     B, S, Hq, Hkv = 2, 40000, 8, 2
