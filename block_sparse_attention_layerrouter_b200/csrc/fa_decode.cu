@@ -1,4 +1,5 @@
-// fa_decode.cu -- single-token decode attention over a bf16 KV cache, sm_100a.
+// fa_decode.cu -- single-token decode attention over a bf16 or FP8 KV cache,
+// sm_100a.
 //
 // o = softmax(scale * q K^T) V for the query at position L-1 of each sequence.
 // FULL attends keys 0..L-1; SPARSE attends the sink blocks and the local
@@ -8,26 +9,36 @@
 //
 // Grid (split, kv head, batch).  A CTA owns one KV head (all G query heads
 // of its group share each K/V tile) and a contiguous share of the sequence's
-// 64-key tiles.  Thread 0 streams the tiles with 4-D TMA loads (128-byte
-// swizzle; bf16: 2 boxes of 64 keys x 64 dims per K or V tile, 3 stages;
-// fp8: 1 box of 64 keys x 128 dims, 6 stages) into a ring; all threads
-// compute from shared memory:
-//   QK^T   thread = (key, 1/PARTS of the head dim), dot products for the G
-//          heads, reduced across the PARTS lanes by a butterfly that leaves
-//          each head's score on one lane, which also forms its probability
-//          2^(s - m) against a per-head reference max m (log2 units);
-//   PV     thread = (8 output dims, one of 16 key streams), G accumulators.
-// The reference only moves, for the whole CTA, on a tile holding a score more
-// than 16 above it (always the first): then the accumulators and row sums
-// are rescaled and the tile's probabilities redone.  One block barrier per
-// tile otherwise.  Each CTA writes its partial (reference, sum, unnormalised
-// output) per head; the combine kernel merges the splits by log-sum-exp.
+// 64-key blocks.  Thread 0 streams them with 4-D TMA loads (128-byte swizzle;
+// bf16: 2 boxes of 64 keys x 64 dims per K or V tile, one block per stage;
+// FP8: 1 box of 64 keys x 128 dims, two blocks per stage) into a 3-stage
+// ring; one block barrier per stage releases it.  The dot products run on the
+// tensor cores (warp-level mma.sync: the query group is a handful of rows,
+// far below the 64-row minimum of a tcgen05 product; the kernel stays bound
+// by HBM and the MMAs only replace CUDA-core FMAs and conversions).  Each of
+// the 8 warps takes its own keys of every stage:
+//   S    = Q K^T     m16n8k16: A = the G query heads (rows G..15 zero), held
+//                    in registers for the whole split; B = K rows by
+//                    ldmatrix (FP8: codes widened to f16, one cvt per pair).
+//   O^T += V^T P^T   bf16: m16n8k8, A = V by ldmatrix.trans; FP8: m16n8k16,
+//                    A = byte-paired words of two keys, one cvt per pair.
+//                    B = P, straight from the S accumulators (their lane
+//                    layout is the B fragment's).
+// Each warp keeps per head a reference max (log2 units) that moves only for
+// a score more than kRefSlack above it (then it rescales its accumulators),
+// the row sum of its rounded P and its O^T (128 dims x the heads); after the
+// last tile the warps merge by log-sum-exp in shared memory and the CTA
+// writes its partial (reference, sum, unnormalised output) per head; the
+// combine kernel merges the splits.
 //
 // Paged cache: with a block table, tile n of sequence b is page
 // block_table[b][n] of a pool [num_pages, 64, Hkv, 128] (one page = one
 // 64-token block, so the sparse mode skips whole pages).  FP8 cache: E4M3
-// codes with one dequantisation scale per KV head for K and for V; the K
-// scale is folded into the query, the V scale into the partial outputs.
+// codes with one dequantisation scale per KV head for K and for V; the
+// products are in f16 (E4M3 codes are exact in f16; the query is scaled by a
+// power of two per head so that its largest element lies in [2^14, 2^15)),
+// the K scale and that power are folded into the score scale, the V scale
+// into the partial outputs.
 #include "fa_common.cuh"
 #include "fa_internal.h"
 
@@ -96,31 +107,6 @@ struct TileList {
   FA_DEV int block(int pos) const { return pos < a ? pos : lo + (pos - a); }
 };
 
-template <int G>
-struct Cfg {
-  static constexpr int PARTS = (G <= 4) ? 8 : 16;       // threads per key in QK^T
-  static constexpr int DPT = HD / PARTS;                 // dims per thread
-  static constexpr int KPP = NT / PARTS;                 // keys per pass
-  static constexpr int MIN_BLOCKS = (G <= 4) ? 2 : 1;
-};
-
-FA_DEV void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-
-// Eight bf16 (one 16-byte chunk) -> four packed fp32 pairs (element 2i in
-// the low lane of pair i).
-FA_DEV void bf16x8_to_f2(const uint4 &v, uint64_t (&f)[4]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) f[i] = f2_make(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
-}
-
 // Byte offset of the 16-byte chunk holding dims [8*chunk16, 8*chunk16+8) of
 // `key` inside one K or V tile written by TMA with the 128-byte swizzle.
 FA_DEV uint32_t tile_offset(int key, int chunk16) {
@@ -129,38 +115,10 @@ FA_DEV uint32_t tile_offset(int key, int chunk16) {
   return static_cast<uint32_t>(box * BOX_BYTES + key * 128 + phys * 16);
 }
 
-// The same for an FP8 tile (one 128-byte row per key): byte offset of the
-// 8 codes of dims [8*g8, 8*g8+8).
-FA_DEV uint32_t tile_offset_fp8(int key, int g8) {
-  const int phys = (g8 >> 1) ^ (key & 7);
-  return static_cast<uint32_t>(key * 128 + phys * 16 + (g8 & 1) * 8);
-}
-
-// Eight E4M3 codes (8 bytes) -> four packed fp32 pairs, exact.
-FA_DEV void fp8x8_to_f2(const uint2 &v, uint64_t (&f)[4]) {
-  const uint32_t w[2] = {v.x, v.y};
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
-          static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * j)) & 0xffffu), __NV_E4M3);
-      const float2 fl = __half22float2(*reinterpret_cast<const __half2 *>(&h));
-      f[2 * i + j] = f2_make(fl.x, fl.y);
-    }
-  }
-}
-
-// K or V of eight dims of one key (0 .. TK-1) from a stage's K or V part, as
-// four fp32 pairs.
-template <bool FP8>
-FA_DEV void load8(const uint8_t *tile, int key, int g8, uint64_t (&f)[4]) {
-  if constexpr (FP8) {
-    const uint8_t *blk = tile + (key >> 6) * KvT<true>::BLK;
-    fp8x8_to_f2(*reinterpret_cast<const uint2 *>(blk + tile_offset_fp8(key & 63, g8)), f);
-  } else {
-    bf16x8_to_f2(*reinterpret_cast<const uint4 *>(tile + tile_offset(key, g8)), f);
-  }
+// Byte offset of byte `byte` (0..127) of `key`'s row inside one FP8 block
+// (one 128-byte row per key, 16-byte units swizzled like the bf16 boxes).
+FA_DEV uint32_t fp8_offset(int key, int byte) {
+  return static_cast<uint32_t>(key * 128 + (((byte >> 4) ^ (key & 7)) << 4) + (byte & 15));
 }
 
 // Page id of block `blk` of sequence b; an id outside the pool is reported
@@ -175,58 +133,100 @@ __device__ __noinline__ int page_of(const int32_t *block_table, int max_pages, i
   return pg;
 }
 
+// A warp's reference moves only for a score more than this above it (log2
+// units): p <= 2^8 stays inside the f16 range of the FP8 path's P.
+constexpr float kRefSlack = 8.0f;
+
+FA_DEV void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+FA_DEV void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+FA_DEV uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+// d += A B, m16n8k16, fp32 accumulators; A rows 8..15 (a1, a3) are zero.
+template <bool F16>
+FA_DEV void mma_k16_top(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  if constexpr (F16)
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+  else
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+FA_DEV void mma_k16_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                        uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+FA_DEV void mma_k8_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+// Four E4M3 codes (bytes 0..3 of x) -> two f16x2: lo = (byte 0, byte 1),
+// hi = (byte 2, byte 3), the lower byte in the lower half.  Exact.
+FA_DEV void e4m3x4_to_f16x2(uint32_t x, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+FA_DEV uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
 // Shared memory of one decode CTA (offsets from a 1024-byte aligned base):
-// K/V ring | stage barriers | abort and re-reference flags | P pairs
-// (double-buffered [2][TK][G], each probability stored twice so a packed
-// FMA reads it as one 64-bit operand) | raw scores of a re-referenced tile
-// [G][TK] | per-head reference max and rescale factor, per-warp row sums |
-// page ids.
-template <int G, bool FP8>
+// K/V ring (after the last tile: the warps' partials) | stage barriers |
+// abort flag | page ids.
+template <bool FP8>
 struct Lay {
-  static constexpr int TK = KvT<FP8>::TK;
   static constexpr int FULL = RING_BYTES;
   static constexpr int FLAGS = FULL + 8 * MAX_STAGES;
-  static constexpr int P2 = FLAGS + 16;
-  static constexpr int SRAW = P2 + 2 * TK * G * 8;
-  static constexpr int REF = SRAW + TK * G * 4;
-  static constexpr int PAGES = REF + (8 + 8 + 8 * 8) * 4;
+  static constexpr int PAGES = FLAGS + 16;
   static constexpr int BYTES = 1024 + PAGES + PAGE_CACHE * 4;
 };
 
-// A tile is scored against a fixed per-head reference max; only a score
-// more than kRefSlack (log2 units) above it, or the first tile, makes the
-// whole CTA move the reference (the rare path).  p <= 2^kRefSlack keeps
-// every fp32 sum far from overflow.
-constexpr float kRefSlack = 16.0f;
-
 template <int G, bool FP8, bool PAGED>
-__global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
+__global__ void __launch_bounds__(NT, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const Params p) {
-  using C = Cfg<G>;
+  static_assert(G >= 1 && G <= 8, "query heads per KV head");
   using T = KvT<FP8>;
-  using Y = Lay<G, FP8>;
-  constexpr int NSTAGE = T::NST, STAGE_BYTES = T::STAGE, TK = T::TK, NB = T::NB;
-  constexpr int PASSES = TK / C::KPP;
+  using Y = Lay<FP8>;
+  constexpr int NSTAGE = T::NST, STAGE_BYTES = T::STAGE, NB = T::NB;
+  constexpr int NW = NT / 32;
+  constexpr int KW = T::TK / NW;       // keys per warp per iteration: 8 (bf16), 16 (FP8)
+  constexpr int NT8 = KW / 8;          // n8 score tiles per warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *stages = base;
   uint64_t *full = reinterpret_cast<uint64_t *>(base + Y::FULL);
   volatile int *abort = reinterpret_cast<volatile int *>(base + Y::FLAGS);
-  // reref[i & 1]: some score of tile i passed its reference.  One flag per
-  // tile parity: a thread may already be scoring tile i+1 (and raising its
-  // flag) while another still reads tile i's.
-  volatile int *reref = abort + 1;
-  uint64_t *p2_sm = reinterpret_cast<uint64_t *>(base + Y::P2);
-  float *sraw_sm = reinterpret_cast<float *>(base + Y::SRAW);
-  float *mref_sm = reinterpret_cast<float *>(base + Y::REF);   // [8]
-  float *alpha_sm = mref_sm + 8;                                // [8]
-  float *lsum_sm = alpha_sm + 8;                                // [8 warps][G]
-  int *page_sm = reinterpret_cast<int *>(base + Y::PAGES);     // [PAGE_CACHE]
+  int *page_sm = reinterpret_cast<int *>(base + Y::PAGES);
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;   // mma fragment row / column pair
   const int L_raw = p.seqlens[b];
   const int L = max(1, min(L_raw, p.Lmax));   // out-of-range lengths are clamped
   if (L != L_raw && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(p.status, FA_DEV_BAD_INDEX);
@@ -242,12 +242,8 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
   if (tid == 0) {
     for (int i = 0; i < NSTAGE; ++i) mbar_init(&full[i], 1);
     *abort = 0;
-    reref[0] = 0;
-    reref[1] = 0;
     fence_mbar_init();
   }
-  if (tid < 8) mref_sm[tid] = -INFINITY;
-  // Page ids of this CTA's tiles (paged cache), read once by all threads.
   if constexpr (PAGED) {
     for (int i = tid; i < nblocks && i < PAGE_CACHE; i += NT)
       page_sm[i] = page_of(p.block_table, p.max_pages, p.num_pages, p.status, b,
@@ -255,12 +251,12 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
   }
   __syncthreads();
 
-  int issued = 0;            // tiles whose copies thread 0 has started
-  auto issue = [&](int i) {  // iteration i of this CTA into stage i % NSTAGE
+  int issued = 0;
+  auto issue = [&](int i) {
     const int st = i % NSTAGE;
     uint8_t *dst = stages + st * STAGE_BYTES;
     mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
-    if constexpr (FP8) {     // paged: NB pages; a missing last one reads zeros
+    if constexpr (FP8) {
 #pragma unroll
       for (int h = 0; h < NB; ++h) {
         const int j = NB * i + h;
@@ -287,196 +283,184 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     }
     issued = i + 1;
   };
-  // Testing mode: no loads, every wait runs out.
   const bool skip_loads = c_skip_loads != 0;
   if (tid == 0 && !skip_loads) {
     for (int i = 0; i < NSTAGE && i < ntiles; ++i) issue(i);
   }
 
-  // QK^T: the PARTS threads of a key each hold G partial dot products.  Slot
-  // j of this thread accumulates query head j ^ hsel, where bit s of `part`
-  // contributes G >> (s+1) to hsel: then a butterfly that at each step keeps
-  // the lower half of the slots and sends the upper half sums every head with
-  // G - 1 shuffles and no selects, leaving head hsel's total in slot 0.
-  const int part = tid % C::PARTS;
-  int hsel = 0;
+  // ---- query fragments (row g = head g of the group; rows >= G are zero)
+  // k-step s: qa[s][0] = dims (2t, 2t+1), qa[s][1] = dims (2t+8, 2t+9) of
+  // dims 16s.. (bf16); FP8: dims (4t, 4t+1) and (4t+2, 4t+3) of 16s.., the
+  // order in which ldmatrix hands out a 16-byte row of codes.
+  const bool hv = g < G;
+  const __nv_bfloat16 *qrow = p.q + (static_cast<size_t>(b) * p.Hq + kvh * G + (hv ? g : 0)) * HD;
+  uint32_t qa[8][2];
+  float sc = p.scale_log2;
+  if constexpr (!FP8) {
 #pragma unroll
-  for (int s = 0; (G >> (s + 1)) > 0; ++s)
-    if ((part >> s) & 1) hsel |= G >> (s + 1);
-  const bool writer = part < G;   // one thread per (key, head) scores it
-  // Chunk (8 dims) of the head dim for step c8 of this thread's QK^T.  bf16:
-  // chunk c8*PARTS + part, so the 8 lanes of a key that share a shared-memory
-  // phase read 8 different swizzled slots of one box (no bank conflicts).
-  // FP8: the thread's chunks are adjacent (a conflict-free order measured
-  // slower there: it costs registers).
-  auto chunk_of = [&](int c8) {
-    return FP8 ? part * (C::DPT / 8) + c8 : c8 * C::PARTS + part;
-  };
-  // Query slice of this thread, pre-scaled by scale*log2(e) (and by the K
-  // dequantisation scale of this KV head).
-  float qscale = p.scale_log2;
-  if constexpr (FP8) qscale *= p.k_scale[kvh];
-  uint64_t qr[G][C::DPT / 2];   // packed pairs of dims
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const __nv_bfloat16 *qrow =
-        p.q + (static_cast<size_t>(b) * p.Hq + kvh * G + (g ^ hsel)) * HD;
-#pragma unroll
-    for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
-      float f[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + chunk_of(c8) * 8), f);
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        qr[g][c8 * 4 + e] = f2_make(f[2 * e] * qscale, f[2 * e + 1] * qscale);
+    for (int s = 0; s < 8; ++s) {
+      qa[s][0] = hv ? *reinterpret_cast<const uint32_t *>(qrow + 16 * s + 2 * t) : 0u;
+      qa[s][1] = hv ? *reinterpret_cast<const uint32_t *>(qrow + 16 * s + 8 + 2 * t) : 0u;
     }
+  } else {
+    float qf[8][4];
+    float mx = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint2 w = hv ? *reinterpret_cast<const uint2 *>(qrow + 16 * s + 4 * t) : make_uint2(0, 0);
+      qf[s][0] = __uint_as_float(w.x << 16);
+      qf[s][1] = __uint_as_float(w.x & 0xffff0000u);
+      qf[s][2] = __uint_as_float(w.y << 16);
+      qf[s][3] = __uint_as_float(w.y & 0xffff0000u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(qf[s][e]));
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    int ex = 0;
+    if (mx > 0.f) frexpf(mx, &ex);            // mx < 2^ex
+    const int sh = mx > 0.f ? 15 - ex : 0;    // max |q| * 2^sh in [2^14, 2^15)
+    const float pw = ldexpf(1.0f, sh);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      qa[s][0] = pack_f16x2(qf[s][0] * pw, qf[s][1] * pw);
+      qa[s][1] = pack_f16x2(qf[s][2] * pw, qf[s][3] * pw);
+    }
+    sc = p.scale_log2 * p.k_scale[kvh] * ldexpf(1.0f, -sh);
   }
-  const int dc = tid & 15;     // PV: output dims [8*dc, 8*dc+8)
-  const int ks = tid >> 4;     // PV: key stream
-  uint64_t acc[G][4];           // packed pairs of output dims
+
+  float o[8][4];               // O^T: m-tile M (16 dims) x heads (2t, 2t+1)
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+  for (int M = 0; M < 8; ++M)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[g][e] = 0ull;
-  float mref = -INFINITY;       // writer: reference max of head hsel (log2 units)
-  float l_part = 0.f;           // writer: its share of head hsel's row sum
+    for (int e = 0; e < 4; ++e) o[M][e] = 0.f;
+  float m_ref = -INFINITY;     // reference max of head g in this warp (log2 units)
+  float l_sum = 0.f;           // this lane's share of head g's row sum
+
+  // This warp's keys inside an iteration: block wb, keys kb .. kb+KW-1.
+  const int wb = FP8 ? (warp >> 2) : 0;
+  const int kb = FP8 ? 16 * (warp & 3) : 8 * warp;
 
   for (int i = 0; i < ntiles; ++i) {
     const int st = i % NSTAGE;
-    // Every thread runs the scores even if its wait failed (the shuffles need
-    // the whole warp; the reads stay inside shared memory); the barrier after
-    // them agrees on leaving.
     const bool ok = mbar_wait(&full[st], static_cast<uint32_t>(i / NSTAGE) & 1u, abort, p.status);
-    const uint8_t *sK = stages + st * STAGE_BYTES;
-    const uint8_t *sV = sK + T::KBYTES;
-    uint64_t *p2b = p2_sm + (i & 1) * TK * G;
-    // Token position of key 0 of each block of this iteration (a missing
-    // block: past every length, so its keys are masked).
-    int key_base[NB];
-#pragma unroll
-    for (int h = 0; h < NB; ++h)
-      key_base[h] = (NB * i + h < nblocks) ? tl.block(pos0 + NB * i + h) * KT : INT_MAX / 2;
+    const uint32_t sK = smem_u32(stages + st * STAGE_BYTES) + wb * T::BLK;
+    const uint32_t sV = sK + T::KBYTES;
+    const int blk_i = NB * i + wb;
+    const int key0 = (blk_i < nblocks) ? tl.block(pos0 + blk_i) * KT + kb : INT_MAX / 2;
 
-    // ---- scores and probabilities against the reference
-    float s_keep[PASSES];
-    float l_tile = 0.f;           // writer: this tile's share, added once the reference holds
-    bool over = false;
+    // ---- S = Q K^T for this warp's keys
+    float s[NT8][4];
 #pragma unroll
-    for (int pass = 0; pass < PASSES; ++pass) {
-      const int key = pass * C::KPP + tid / C::PARTS;
-      uint64_t d2[G];
+    for (int j = 0; j < NT8; ++j)
 #pragma unroll
-      for (int g = 0; g < G; ++g) d2[g] = 0ull;
+      for (int e = 0; e < 4; ++e) s[j][e] = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < C::DPT / 8; ++c8) {
-        uint64_t k2[4];
-        load8<FP8>(sK, key, chunk_of(c8), k2);
+    for (int j = 0; j < NT8; ++j) {
+      const int key = kb + 8 * j + (lane & 7);
+      if constexpr (!FP8) {
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) d2[g] = f2_fma(qr[g][c8 * 4 + e], k2[e], d2[g]);
-      }
-      float d[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float lo, hi;
-        f2_split(d2[g], lo, hi);
-        d[g] = lo + hi;
-      }
-#pragma unroll
-      for (int half = G / 2; half >= 1; half >>= 1)
-#pragma unroll
-        for (int j = 0; j < half; ++j)
-          d[j] += __shfl_xor_sync(0xffffffffu, d[j + half], G / (2 * half));
-#pragma unroll
-      for (int off = G; off < C::PARTS; off <<= 1)
-        d[0] += __shfl_xor_sync(0xffffffffu, d[0], off);
-      const bool valid = key_base[key / KT] + (key % KT) < L;
-      const float s = valid ? d[0] : -INFINITY;
-      s_keep[pass] = s;
-      if (writer) {
-        const bool up = s > mref + kRefSlack;
-        over |= up;
-        const float pj = (up || s == -INFINITY) ? 0.f : ex2(s - mref);
-        l_tile += pj;
-        p2b[key * G + hsel] = f2_make(pj, pj);
-      }
-    }
-    if (over) reref[i & 1] = 1;
-    // Past this barrier every thread is done with tile i-1 (its PV came before
-    // these scores), so its stage takes tile i-1+NSTAGE.
-    if (__syncthreads_or(!ok)) break;
-    if (tid == 0 && !skip_loads && i >= 1 && i - 1 + NSTAGE < ntiles) issue(i - 1 + NSTAGE);
-
-    // ---- rare: move the reference to the running max, rescale, redo P
-    if (reref[i & 1]) {
-      if (writer) {
-#pragma unroll
-        for (int pass = 0; pass < PASSES; ++pass)
-          sraw_sm[hsel * TK + pass * C::KPP + tid / C::PARTS] = s_keep[pass];
-      }
-      __syncthreads();
-      if (tid == 0) reref[i & 1] = 0;   // every thread read it before this barrier; the
-                                        // next write to it comes after the next tile's barrier
-      if (warp < G) {
-        float mt = -INFINITY;
-#pragma unroll
-        for (int j = lane; j < TK; j += 32) mt = fmaxf(mt, sraw_sm[warp * TK + j]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-        if (lane == 0) {
-          const float mo = mref_sm[warp];
-          const float mn = fmaxf(mo, mt);
-          alpha_sm[warp] = (mo == -INFINITY) ? 0.f : ex2(mo - mn);
-          mref_sm[warp] = mn;
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[4];
+          ldsm_x4(sK + tile_offset(key, 4 * c + (lane >> 3)), r);
+          mma_k16_top<false>(s[j], qa[2 * c][0], qa[2 * c][1], r[0], r[1]);
+          mma_k16_top<false>(s[j], qa[2 * c + 1][0], qa[2 * c + 1][1], r[2], r[3]);
         }
-      }
-      __syncthreads();
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const uint64_t a2 = f2_make(alpha_sm[g], alpha_sm[g]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[g][e] = f2_mul(acc[g][e], a2);
-      }
-      if (writer) {
-        l_part *= alpha_sm[hsel];
-        mref = mref_sm[hsel];
-#pragma unroll
-        for (int pass = 0; pass < PASSES; ++pass) {
-          const float s = s_keep[pass];
-          const float pj = (s == -INFINITY) ? 0.f : ex2(s - mref);
-          l_part += pj;
-          p2b[(pass * C::KPP + tid / C::PARTS) * G + hsel] = f2_make(pj, pj);
-        }
-      }
-      __syncthreads();
-    } else {
-      l_part += l_tile;
-    }
-
-    // ---- O += P V (P of the G heads of a key: G packed pairs, 16-byte loads)
-#pragma unroll
-    for (int kk = 0; kk < TK / 16; ++kk) {
-      const int key = ks + 16 * kk;
-      uint64_t v2[4];
-      load8<FP8>(sV, key, dc, v2);
-      if constexpr (G == 1) {
-        const uint64_t pg = p2b[key];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[0][e] = f2_fma(pg, v2[e], acc[0][e]);
       } else {
 #pragma unroll
-        for (int g2 = 0; g2 < G / 2; ++g2) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(p2b + key * G + 2 * g2);
-          const uint64_t pa = (static_cast<uint64_t>(w.y) << 32) | w.x;
-          const uint64_t pb = (static_cast<uint64_t>(w.w) << 32) | w.z;
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[4];
+          const int chunk = 4 * c + (lane >> 3);
+          ldsm_x4(sK + fp8_offset(key, 16 * chunk), r);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            acc[2 * g2][e] = f2_fma(pa, v2[e], acc[2 * g2][e]);
-            acc[2 * g2 + 1][e] = f2_fma(pb, v2[e], acc[2 * g2 + 1][e]);
+          for (int x = 0; x < 4; ++x) {
+            uint32_t b0, b1;
+            e4m3x4_to_f16x2(r[x], b0, b1);
+            mma_k16_top<true>(s[j], qa[4 * c + x][0], qa[4 * c + x][1], b0, b1);
           }
         }
       }
     }
+
+    // ---- scores (log2 units), reference, probabilities
+    float sv[NT8][2];
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NT8; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool valid = key0 + 8 * j + 2 * t + e < L;
+        sv[j][e] = valid ? s[j][e] * sc : -INFINITY;
+        tmax = fmaxf(tmax, sv[j][e]);
+      }
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+    const bool up = tmax > m_ref + kRefSlack;
+    if (__any_sync(0xffffffffu, up)) {   // rare: move this warp's references
+      const float alpha = up ? ((m_ref == -INFINITY) ? 0.f : ex2(m_ref - tmax)) : 1.f;
+      if (up) m_ref = tmax;
+      l_sum *= alpha;
+      // This lane's O^T columns are heads 2t and 2t+1, whose factors sit in
+      // lanes 8t and 8t+4.
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * t);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);
+#pragma unroll
+      for (int M = 0; M < 8; ++M) {
+        o[M][0] *= a0;
+        o[M][1] *= a1;
+        o[M][2] *= a0;
+        o[M][3] *= a1;
+      }
+    }
+    uint32_t pb[NT8];
+#pragma unroll
+    for (int j = 0; j < NT8; ++j) {
+      const float p0 = (sv[j][0] == -INFINITY) ? 0.f : ex2(sv[j][0] - m_ref);
+      const float p1 = (sv[j][1] == -INFINITY) ? 0.f : ex2(sv[j][1] - m_ref);
+      if constexpr (FP8) {   // f16 keeps 11 bits: the sum of the unrounded p differs by ~2^-12
+        pb[j] = pack_f16x2(p0, p1);
+        l_sum += p0 + p1;
+      } else {
+        pb[j] = pack_bf16x2(p0, p1);
+        l_sum += __uint_as_float(pb[j] << 16) + __uint_as_float(pb[j] & 0xffff0000u);
+      }
+    }
+
+    // ---- O^T += V^T P^T
+    if constexpr (!FP8) {
+      const int key = kb + (lane & 7);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[4];
+        ldsm_x4_t(sV + tile_offset(key, 4 * c + (lane >> 3)), r);
+        mma_k8_bf16(o[2 * c], r[0], r[1], pb[0]);       // dims 32c + (0..15)
+        mma_k8_bf16(o[2 * c + 1], r[2], r[3], pb[0]);   // dims 32c + (16..31)
+      }
+    } else {
+      // Lane (g, t): keys kb + {2t, 2t+1, 2t+8, 2t+9}, dims 32q + 4g + (0..3).
+      // m-tile 2q+m: row g = dim 32q + 4g + 2m, row g+8 = dim 32q + 4g + 2m + 1.
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int key = kb + 2 * t + (kk & 1) + 8 * (kk >> 1);
+          w[kk] = lds32(sV + fp8_offset(key, 32 * q + 4 * g));
+        }
+        // (key 2t, key 2t+1) byte pairs of dims +0 / +1 (lo) and +2 / +3 (hi).
+        uint32_t a[2][4];
+        e4m3x4_to_f16x2(__byte_perm(w[0], w[1], 0x5140), a[0][0], a[0][1]);
+        e4m3x4_to_f16x2(__byte_perm(w[2], w[3], 0x5140), a[0][2], a[0][3]);
+        e4m3x4_to_f16x2(__byte_perm(w[0], w[1], 0x7362), a[1][0], a[1][1]);
+        e4m3x4_to_f16x2(__byte_perm(w[2], w[3], 0x7362), a[1][2], a[1][3]);
+        mma_k16_f16(o[2 * q], a[0][0], a[0][1], a[0][2], a[0][3], pb[0], pb[1]);
+        mma_k16_f16(o[2 * q + 1], a[1][0], a[1][1], a[1][2], a[1][3], pb[0], pb[1]);
+      }
+    }
+    // Past this barrier every warp is done with this stage: it takes tile
+    // i + NSTAGE.
+    if (__syncthreads_or(!ok)) break;
+    if (tid == 0 && !skip_loads && i + NSTAGE < ntiles) issue(i + NSTAGE);
   }
   __syncthreads();   // every thread is done with the stages (reused below)
 
@@ -485,9 +469,6 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
       for (int x = (issued > NSTAGE ? issued - NSTAGE : 0); x < issued; ++x)
         mbar_wait_drain(&full[x % NSTAGE], static_cast<uint32_t>(x / NSTAGE) & 1u, 200000000ull);
     }
-    // Mark this split's partials as missing (NaN reference): the combine then
-    // writes NaN for these heads instead of merging whatever the workspace
-    // held before.
     if (tid < G) {
       const size_t r0 = (static_cast<size_t>(b) * p.Hq + kvh * G + tid) * p.nsplit + split;
       if (in_bounds(p.status, static_cast<long long>(r0) * 2 + 1,
@@ -500,46 +481,61 @@ __global__ void __launch_bounds__(NT, Cfg<G>::MIN_BLOCKS)
     return;
   }
 
-  // ---- row sums: the writers of a head share `part`; one total per warp
+  // ---- merge the warps: per head, M = max of the warps' references
+  l_sum += __shfl_xor_sync(0xffffffffu, l_sum, 1);
+  l_sum += __shfl_xor_sync(0xffffffffu, l_sum, 2);
+  float *red_o = reinterpret_cast<float *>(stages);   // [NW][G][HD]
+  float *red_m = red_o + NW * G * HD;                  // [NW][G]
+  float *red_l = red_m + NW * G;                       // [NW][G]
+  float *red_w = red_l + NW * G;                       // [NW][G] merge weights
+  float *red_M = red_w + NW * G;                       // [G]
+  if (t == 0 && hv) {
+    red_m[warp * G + g] = m_ref;
+    red_l[warp * G + g] = l_sum;
+  }
 #pragma unroll
-  for (int off = C::PARTS; off < 32; off <<= 1) l_part += __shfl_xor_sync(0xffffffffu, l_part, off);
-  if (lane < G) lsum_sm[warp * G + hsel] = l_part;   // lane < G: part = lane, a writer
-
-  // ---- reduce the 16 key streams through shared memory (stage buffers free)
-  float *red = reinterpret_cast<float *>(stages);   // [16][G][HD]
-  float vs = 1.0f;
-  if constexpr (FP8) vs = p.v_scale[kvh];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
+  for (int M = 0; M < 8; ++M)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      float lo, hi;
-      f2_split(acc[g][e], lo, hi);
-      red[(ks * G + g) * HD + dc * 8 + 2 * e] = lo;
-      red[(ks * G + g) * HD + dc * 8 + 2 * e + 1] = hi;
+      const int h = 2 * t + (e & 1);
+      const int d = FP8 ? 32 * (M >> 1) + 4 * g + 2 * (M & 1) + (e >> 1)
+                        : 16 * M + g + 8 * (e >> 1);
+      if (h < G) red_o[(warp * G + h) * HD + d] = o[M][e];
     }
   __syncthreads();
+  if (tid < G) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) mx = fmaxf(mx, red_m[w * G + tid]);
+    float l = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float mw = red_m[w * G + tid];
+      const float wt = (mw == -INFINITY) ? 0.f : ex2(mw - mx);
+      red_w[w * G + tid] = wt;
+      l = fmaf(wt, red_l[w * G + tid], l);
+    }
+    red_M[tid] = mx;
+    const size_t mi = ((static_cast<size_t>(b) * p.Hq + kvh * G + tid) * p.nsplit + split) * 2;
+    if (in_bounds(p.status, static_cast<long long>(mi) + 1,
+                  static_cast<long long>(p.B) * p.Hq * p.nsplit * 2)) {
+      p.ml_part[mi] = mx;
+      p.ml_part[mi + 1] = l;
+    }
+  }
+  __syncthreads();
+  float vs = 1.0f;
+  if constexpr (FP8) vs = p.v_scale[kvh];
   const size_t row0 = (static_cast<size_t>(b) * p.Hq + kvh * G) * p.nsplit + split;
   for (int idx = tid; idx < G * HD; idx += NT) {
-    const int g = idx / HD, dd = idx % HD;
+    const int h = idx / HD, d = idx % HD;
     float sum = 0.f;
 #pragma unroll
-    for (int s = 0; s < 16; ++s) sum += red[(s * G + g) * HD + dd];
-    const size_t oi = (row0 + static_cast<size_t>(g) * p.nsplit) * HD + dd;
+    for (int w = 0; w < NW; ++w) sum = fmaf(red_w[w * G + h], red_o[(w * G + h) * HD + d], sum);
+    const size_t oi = (row0 + static_cast<size_t>(h) * p.nsplit) * HD + d;
     if (in_bounds(p.status, static_cast<long long>(oi),
                   static_cast<long long>(p.B) * p.Hq * p.nsplit * HD))
       p.o_part[oi] = sum * vs;
-  }
-  if (tid < G) {
-    float l = 0.f;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) l += lsum_sm[w * G + tid];
-    const size_t mi = (row0 + static_cast<size_t>(tid) * p.nsplit) * 2;
-    if (in_bounds(p.status, static_cast<long long>(mi) + 1,
-                  static_cast<long long>(p.B) * p.Hq * p.nsplit * 2)) {
-      p.ml_part[mi] = mref_sm[tid];
-      p.ml_part[mi + 1] = l;
-    }
   }
 }
 
@@ -685,18 +681,18 @@ int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
   // FP8 caches are always paged (a contiguous cache is the identity table).
   if (a.fp8 && !paged) return FA_ERR_UNSUPPORTED;
   switch (G * 4 + (a.fp8 ? 2 : 0) + (paged ? 1 : 0)) {
-    case 4: kern = decode_kernel<1, false, false>, smem = Lay<1, false>::BYTES; break;
-    case 8: kern = decode_kernel<2, false, false>, smem = Lay<2, false>::BYTES; break;
-    case 16: kern = decode_kernel<4, false, false>, smem = Lay<4, false>::BYTES; break;
-    case 32: kern = decode_kernel<8, false, false>, smem = Lay<8, false>::BYTES; break;
-    case 5: kern = decode_kernel<1, false, true>, smem = Lay<1, false>::BYTES; break;
-    case 9: kern = decode_kernel<2, false, true>, smem = Lay<2, false>::BYTES; break;
-    case 17: kern = decode_kernel<4, false, true>, smem = Lay<4, false>::BYTES; break;
-    case 33: kern = decode_kernel<8, false, true>, smem = Lay<8, false>::BYTES; break;
-    case 7: kern = decode_kernel<1, true, true>, smem = Lay<1, true>::BYTES; break;
-    case 11: kern = decode_kernel<2, true, true>, smem = Lay<2, true>::BYTES; break;
-    case 19: kern = decode_kernel<4, true, true>, smem = Lay<4, true>::BYTES; break;
-    case 35: kern = decode_kernel<8, true, true>, smem = Lay<8, true>::BYTES; break;
+    case 4: kern = decode_kernel<1, false, false>, smem = Lay<false>::BYTES; break;
+    case 8: kern = decode_kernel<2, false, false>, smem = Lay<false>::BYTES; break;
+    case 16: kern = decode_kernel<4, false, false>, smem = Lay<false>::BYTES; break;
+    case 32: kern = decode_kernel<8, false, false>, smem = Lay<false>::BYTES; break;
+    case 5: kern = decode_kernel<1, false, true>, smem = Lay<false>::BYTES; break;
+    case 9: kern = decode_kernel<2, false, true>, smem = Lay<false>::BYTES; break;
+    case 17: kern = decode_kernel<4, false, true>, smem = Lay<false>::BYTES; break;
+    case 33: kern = decode_kernel<8, false, true>, smem = Lay<false>::BYTES; break;
+    case 7: kern = decode_kernel<1, true, true>, smem = Lay<true>::BYTES; break;
+    case 11: kern = decode_kernel<2, true, true>, smem = Lay<true>::BYTES; break;
+    case 19: kern = decode_kernel<4, true, true>, smem = Lay<true>::BYTES; break;
+    case 35: kern = decode_kernel<8, true, true>, smem = Lay<true>::BYTES; break;
     default: return FA_ERR_UNSUPPORTED;
   }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
