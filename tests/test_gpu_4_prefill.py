@@ -144,18 +144,22 @@ def test_deterministic():
 
 @pytest.mark.parametrize("Hq,Hkv", [(4, 2), (3, 3)])
 @pytest.mark.parametrize("mode", ["full", "sparse"])
-def test_prefill_scores_that_grow_across_tiles(Hq, Hkv, mode):
-    """Keys past token 256 are scaled by 16 (exact in bf16), so their scores
-    lie up to ~60 (log2) above everything the first tiles saw: p = 2^(s - m)
-    against the running maximum would leave the safe range (a tile's row sum
-    far above 2^32), so the kernel must take the tile's own maximum and redo
-    the tile.  The result must still be the oracle's."""
+@pytest.mark.parametrize("start", [256, 320])
+def test_prefill_scores_that_grow_across_tiles(Hq, Hkv, mode, start):
+    """Keys from token `start` on are scaled by 16 (exact in bf16), so their
+    scores lie up to ~60 (log2) above everything the first tiles saw: p =
+    2^(s - m) against the running maximum would leave the safe range (a
+    row sum far above 2^32), so the kernel must move the reference to the
+    tile's own maximum.  start = 256: the growth begins with a 128-key tile;
+    start = 320: in the middle of one (the tile's first half still sits near
+    the old reference, its second half far above it).  The result must still
+    be the oracle's."""
     S = 768
     q, k, v = inputs.qkv(1, S, Hq, Hkv, 128, seed=1201)
-    k[:, 256:] = (k[:, 256:].float() * 16.0).to(torch.bfloat16)
+    k[:, start:] = (k[:, start:].float() * 16.0).to(torch.bfloat16)
     # The test only means something if the scores really outgrow the first tiles' maximum.
-    sc = torch.einsum("bthd,bshd->bhts", q.float()[:, 256:, :1], k.float()[:, :, :1]) / 128 ** 0.5
-    assert float(sc[..., 256:].max() - sc[..., :128].max()) * 1.4427 > 40
+    sc = torch.einsum("bthd,bshd->bhts", q.float()[:, start:, :1], k.float()[:, :, :1]) / 128 ** 0.5
+    assert float(sc[..., start:].max() - sc[..., :128].max()) * 1.4427 > 40
     o, lse = _run(q, k, v, mode, window=256)
     ref, ref_lse = _oracle(q, k, v, mode, window=256)
     assert_close_attention(to_f64(o), ref, "growing scores %s" % mode)

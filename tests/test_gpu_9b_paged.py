@@ -178,3 +178,66 @@ def test_fp8_paged_decode_full_size(mode):
                                       sink=wl.sink, window=wl.window)
         got = to_f64(o[b, kvh * G:(kvh + 1) * G])
         assert_close_attention(got, ref[0], "fp8 full size b%d mode %d" % (b, mode))
+
+
+def _fp8_case(B, Hq, Hkv, seqlens, mode, seed, q_scale=None, pull=()):
+    """An FP8 paged decode against the oracle on the dequantised cache.
+    q_scale [Hq]: per-head factors on the query (bf16 after scaling); pull:
+    (b, lo, hi, head, factor) -- keys lo..hi-1 of sequence b get factor x that
+    query head added before quantisation (scores far above the rest)."""
+    max_pages = (max(seqlens) + 63) // 64
+    kp, vp, bt = _pool(B, max_pages, Hkv, seed=seed)
+    q = inputs.randn_bf16((B, Hq, 128), seed + 1)
+    if q_scale is not None:
+        q = (q.float() * torch.tensor(q_scale, dtype=torch.float32)[None, :, None]).to(torch.bfloat16)
+    G = Hq // Hkv
+    kf = kp.float()
+    for b, lo, hi, head, factor in pull:
+        t = np.arange(lo, hi)
+        pages = torch.from_numpy(bt[b, t // 64].astype(np.int64))
+        slots = torch.from_numpy(t % 64)
+        kf[pages, slots, head // G] += factor * q[b, head].float()
+    kp = kf.to(torch.bfloat16)
+    ks, vs = _fp8_scales(Hkv, seed + 2)
+    kc, vc = _quantize_pool(inputs.bits(kp), ks), _quantize_pool(inputs.bits(vp), vs)
+    c = capi.cfg(64, 64, 256)
+    status = zero_status()
+    lse = torch.empty(B, Hq, device="cuda")
+    sl = np.array(seqlens, np.int32)
+    o = capi.attn_decode_paged(q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(bt).cuda(),
+                               torch.from_numpy(sl).cuda(), capi.FA_KV_FP8_E4M3,
+                               torch.from_numpy(ks).cuda(), torch.from_numpy(vs).cuda(),
+                               mode=mode, c=c, lse=lse, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kval = oracle.e4m3_decode(kc.numpy()) * ks[None, None, :, None]
+    vval = oracle.e4m3_decode(vc.numpy()) * vs[None, None, :, None]
+    kg = oracle.paged_gather(kval, bt, sl)
+    vg = oracle.paged_gather(vval, bt, sl)
+    ref, ref_lse = oracle.decode_values(oracle.bf16_bits_to_f64(inputs.bits(q)), kg, vg, sl,
+                                        SCALE, mode=mode, sink=64, window=256)
+    what = "fp8 G=%d mode=%d" % (G, mode)
+    assert_close_attention(to_f64(o), ref, what)
+    np.testing.assert_allclose(to_f64(lse), ref_lse, atol=LSE_ABS_TOL, err_msg=what)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (8, 1)])
+def test_fp8_decode_group_widths_and_query_ranges(mode, Hq, Hkv):
+    """G = 1, 2, 8 with FP8 caches: the f16 products scale each query head by
+    a power of two of its own; heads here span 1e-3 .. 300 in magnitude and
+    one is zero (its output is the mean of V)."""
+    q_scale = [1e-3, 0.05, 1.0, 300.0, 0.0, 7.0, 1.0 / 3.0, 40.0]
+    _fp8_case(3, Hq, Hkv, [1000, 321, 64], mode, 741, q_scale=q_scale)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_fp8_decode_rising_score_plateaus(mode):
+    """FP8 cache: runs of keys pulled towards one query head so that their
+    scores jump about 26 and then 45 (log2) above the rest in the middle of a
+    split; every warp that meets them moves its reference and rescales.  The
+    pulled values saturate E4M3 in places; both sides read the same codes."""
+    L = 3000
+    pull = [(0, 700, L, 1, 1.6), (0, 2050, L, 1, 1.2), (1, 140, L - 74, 6, 1.6),
+            (1, 5, 6, 6, 2.0)]
+    _fp8_case(2, 8, 2, [L, L - 74], mode, 751, pull=pull)
