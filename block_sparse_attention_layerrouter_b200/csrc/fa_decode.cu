@@ -197,7 +197,6 @@ FA_DEV uint32_t pack_f16x2(float lo, float hi) {
 // Shared memory of one decode CTA (offsets from a 1024-byte aligned base):
 // K/V ring (after the last tile: the warps' partials) | stage barriers |
 // abort flag | page ids.
-template <bool FP8>
 struct Lay {
   static constexpr int FULL = RING_BYTES;
   static constexpr int FLAGS = FULL + 8 * MAX_STAGES;
@@ -211,7 +210,7 @@ __global__ void __launch_bounds__(NT, 2)
                   const Params p) {
   static_assert(G >= 1 && G <= 8, "query heads per KV head");
   using T = KvT<FP8>;
-  using Y = Lay<FP8>;
+  using Y = Lay;
   constexpr int NSTAGE = T::NST, STAGE_BYTES = T::STAGE, NB = T::NB;
   constexpr int NW = NT / 32;
   constexpr int KW = T::TK / NW;       // keys per warp per iteration: 8 (bf16), 16 (FP8)
@@ -319,7 +318,10 @@ __global__ void __launch_bounds__(NT, 2)
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     int ex = 0;
     if (mx > 0.f) frexpf(mx, &ex);            // mx < 2^ex
-    const int sh = mx > 0.f ? 15 - ex : 0;    // max |q| * 2^sh in [2^14, 2^15)
+    // max |q| * 2^sh in [2^14, 2^15), with 2^sh at most 2^64 so that it stays
+    // finite in fp32: the cap only acts on heads whose largest |q| is below
+    // 2^-49, whose scores are below 2^-40 in magnitude either way.
+    const int sh = mx > 0.f ? min(15 - ex, 64) : 0;
     const float pw = ldexpf(1.0f, sh);
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
@@ -681,18 +683,18 @@ int launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
   // FP8 caches are always paged (a contiguous cache is the identity table).
   if (a.fp8 && !paged) return FA_ERR_UNSUPPORTED;
   switch (G * 4 + (a.fp8 ? 2 : 0) + (paged ? 1 : 0)) {
-    case 4: kern = decode_kernel<1, false, false>, smem = Lay<false>::BYTES; break;
-    case 8: kern = decode_kernel<2, false, false>, smem = Lay<false>::BYTES; break;
-    case 16: kern = decode_kernel<4, false, false>, smem = Lay<false>::BYTES; break;
-    case 32: kern = decode_kernel<8, false, false>, smem = Lay<false>::BYTES; break;
-    case 5: kern = decode_kernel<1, false, true>, smem = Lay<false>::BYTES; break;
-    case 9: kern = decode_kernel<2, false, true>, smem = Lay<false>::BYTES; break;
-    case 17: kern = decode_kernel<4, false, true>, smem = Lay<false>::BYTES; break;
-    case 33: kern = decode_kernel<8, false, true>, smem = Lay<false>::BYTES; break;
-    case 7: kern = decode_kernel<1, true, true>, smem = Lay<true>::BYTES; break;
-    case 11: kern = decode_kernel<2, true, true>, smem = Lay<true>::BYTES; break;
-    case 19: kern = decode_kernel<4, true, true>, smem = Lay<true>::BYTES; break;
-    case 35: kern = decode_kernel<8, true, true>, smem = Lay<true>::BYTES; break;
+    case 4: kern = decode_kernel<1, false, false>, smem = Lay::BYTES; break;
+    case 8: kern = decode_kernel<2, false, false>, smem = Lay::BYTES; break;
+    case 16: kern = decode_kernel<4, false, false>, smem = Lay::BYTES; break;
+    case 32: kern = decode_kernel<8, false, false>, smem = Lay::BYTES; break;
+    case 5: kern = decode_kernel<1, false, true>, smem = Lay::BYTES; break;
+    case 9: kern = decode_kernel<2, false, true>, smem = Lay::BYTES; break;
+    case 17: kern = decode_kernel<4, false, true>, smem = Lay::BYTES; break;
+    case 33: kern = decode_kernel<8, false, true>, smem = Lay::BYTES; break;
+    case 7: kern = decode_kernel<1, true, true>, smem = Lay::BYTES; break;
+    case 11: kern = decode_kernel<2, true, true>, smem = Lay::BYTES; break;
+    case 19: kern = decode_kernel<4, true, true>, smem = Lay::BYTES; break;
+    case 35: kern = decode_kernel<8, true, true>, smem = Lay::BYTES; break;
     default: return FA_ERR_UNSUPPORTED;
   }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=

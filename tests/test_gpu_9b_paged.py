@@ -225,9 +225,10 @@ def _fp8_case(B, Hq, Hkv, seqlens, mode, seed, q_scale=None, pull=()):
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (8, 1)])
 def test_fp8_decode_group_widths_and_query_ranges(mode, Hq, Hkv):
     """G = 1, 2, 8 with FP8 caches: the f16 products scale each query head by
-    a power of two of its own; heads here span 1e-3 .. 300 in magnitude and
-    one is zero (its output is the mean of V)."""
-    q_scale = [1e-3, 0.05, 1.0, 300.0, 0.0, 7.0, 1.0 / 3.0, 40.0]
+    a power of two of its own; heads here span 1e-36 .. 300 in magnitude
+    (1e-36: the scaling is capped so that it stays finite, and the head's
+    scores are ~0 either way) and one is zero (its output is the mean of V)."""
+    q_scale = [1e-3, 1e-36, 1.0, 300.0, 0.0, 7.0, 1.0 / 3.0, 40.0]
     _fp8_case(3, Hq, Hkv, [1000, 321, 64], mode, 741, q_scale=q_scale)
 
 
