@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -190,15 +191,24 @@ def measured_peaks():
 HOST_MARK = "// ----------------------------------------------------------------- host ---"
 
 
+def _code_tokens(text):
+    """Source text without // and /* */ comments, whitespace collapsed: what
+    the compiler sees, so that editing a comment keeps the hash."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def prefill_device_sha():
     """Hash of the prefill kernels' device code: fa_prefill.cu up to its host
-    section, plus the shared device helpers (fa_common.cuh).  A DRAM traffic
-    record taken with ncu is only reported while this hash is unchanged."""
+    section, plus the shared device helpers (fa_common.cuh), comments and
+    whitespace left out.  A DRAM traffic record taken with ncu is only
+    reported while this hash is unchanged."""
     h = hashlib.sha256()
-    src = open(os.path.join(CSRC, "fa_prefill.cu"), "rb").read()
-    cut = src.find(HOST_MARK.encode())
-    h.update(src[:cut] if cut >= 0 else src)
-    h.update(open(os.path.join(CSRC, "fa_common.cuh"), "rb").read())
+    src = open(os.path.join(CSRC, "fa_prefill.cu")).read()
+    cut = src.find(HOST_MARK)
+    h.update(_code_tokens(src[:cut] if cut >= 0 else src).encode())
+    h.update(_code_tokens(open(os.path.join(CSRC, "fa_common.cuh")).read()).encode())
     return h.hexdigest()[:16]
 
 

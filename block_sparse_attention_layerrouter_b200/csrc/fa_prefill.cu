@@ -14,10 +14,13 @@
 //   warp 1      MMA issuer (one thread) and TMEM owner: S_j = Q K_j^T into one
 //               of two TMEM score buffers, O += P_j V_j with P read from TMEM.
 //   warps 4-7   softmax warpgroup, one thread per query row: reads S_j from
-//               TMEM, masks, updates the running max/sum, writes P_j (bf16) to
-//               TMEM, rescales O in TMEM only when the running max grew by
-//               more than 2^8 (exact: the final division uses the same max),
-//               and finally normalises O and stores it.
+//               TMEM, masks, forms P_j = 2^(s*c - m) (bf16) against a lazy
+//               reference m -- the running max of the earlier tiles, moved
+//               (with O rescaled in TMEM) only on a tile whose row sum leaves
+//               the safe range, and on the first tile -- writes P_j to TMEM,
+//               and finally normalises O and stores it (exact: the final
+//               division uses the same reference as the sum).
+// (prefill2_kernel below: the persistent two-head version of the same.)
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
 // All operands are bf16; accumulation and softmax are fp32.
 #include "fa_common.cuh"
@@ -26,6 +29,104 @@
 #include <math.h>
 
 namespace fa {
+
+// ------------------------------------------------ softmax arithmetic ---
+// Shared by both prefill kernels: exponentials in log2 units against a
+// reference max, two lanes per instruction.
+
+// 2^x on the FMA pipe: round-to-nearest range reduction with the 1.5*2^23
+// shifter (x = n + f, f in [-1/2, 1/2]), a degree-3 polynomial for 2^f
+// (coefficients fitted here by minimax linear programming on [-1/2, 1/2];
+// max relative error 1.0e-4, below bf16 rounding of P), and n added to the
+// exponent field.  Inputs below -127 give 0.
+#ifndef FA_POLY_PER_8
+#define FA_POLY_PER_8 2
+#endif
+// Key pairs (k, k+1), k even, with (k mod 8) >= 8 - kPolyPer8 take the
+// polynomial (so kPolyPer8 counts in steps of 2); the rest use ex2.approx.
+constexpr int kPolyPer8 = FA_POLY_PER_8;
+constexpr float kExp2C1 = 0.693282962f;
+constexpr float kExp2C2 = 0.242210999f;
+constexpr float kExp2C3 = 0.0550087839f;
+FA_DEV float ex2_poly(float x) {
+  x = fmaxf(x, -127.0f);
+  const float t = x + 12582912.0f;          // 1.5 * 2^23: low mantissa bits = round(x)
+  const float n = t - 12582912.0f;
+  const float f = x - n;
+  float p = fmaf(kExp2C3, f, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+// The same for two lanes at once with the packed fp32x2 instructions.
+FA_DEV void ex2_poly2(uint64_t x2, float &r0, float &r1) {
+  float a, b;
+  f2_split(x2, a, b);
+  const uint64_t x = f2_make(fmaxf(a, -127.0f), fmaxf(b, -127.0f));
+  const uint64_t t = f2_add(x, f2_make(12582912.0f, 12582912.0f));
+  const uint64_t n = f2_add(t, f2_make(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(n, f2_make(-1.0f, -1.0f), x);
+  uint64_t p = f2_fma(f2_make(kExp2C3, kExp2C3), f, f2_make(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_make(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_make(1.0f, 1.0f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// Row max of N scores: 3-input max over pairs, 8 independent chains.
+template <int N>
+FA_DEV float row_max(const float (&s)[N]) {
+  float mx8[8];
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmaxf(s[2 * kk], s[2 * kk + 1]);
+#pragma unroll
+  for (int i = 16; i < N; i += 16)
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmax3(mx8[kk], s[i + 2 * kk], s[i + 2 * kk + 1]);
+  return fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+               fmaxf(mx8[6], mx8[7]));
+}
+
+#ifndef FA_LAZY_MAX
+#define FA_LAZY_MAX 1
+#endif
+constexpr bool kLazyMax = FA_LAZY_MAX != 0;
+// Largest row sum of one tile's p = 2^(s*c - m) accepted without taking the
+// tile's max: p stays far inside the bf16 / fp32 range (2^127).
+constexpr float kLazySumLimit = 4294967296.0f;   // 2^32
+
+// p = 2^(s*c - m) for N scores, packed as bf16 pairs into pk; returns the
+// row sum.  Two lanes per instruction (the argument and the sums);
+// ex2.approx, or the FMA-pipe polynomial for kPolyPer8 keys of 8.
+template <int N>
+FA_DEV float row_exp2(const float (&s)[N], float c, float m, uint32_t (&pk)[N / 2]) {
+  const float m_use = (m == -INFINITY) ? 0.f : m;
+  const uint64_t c2 = f2_make(c, c), negm2 = f2_make(-m_use, -m_use);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const int k0 = 2 * i;
+    const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
+    float p0, p1;
+    if ((k0 & 7) >= 8 - kPolyPer8) {
+      ex2_poly2(x, p0, p1);
+    } else {
+      float x0, x1;
+      f2_split(x, x0, x1);
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
+    pk[i] = pack_bf16x2(p0, p1);
+  }
+  float a0, a1;
+  f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+  return a0 + a1;
+}
+
 namespace prefill {
 
 constexpr int BM = 128;                       // query rows per CTA (MMA M)
@@ -320,6 +421,27 @@ FA_DEV bool warp_wait(uint64_t *bar, uint32_t parity, const Shared &sh, const Pa
   return __all_sync(0xffffffffu, done);
 }
 
+// The 128 scores of this thread's row of an S buffer, masked: the 4-bit
+// block mask `bits` (sparse tiles) and causality on the diagonal tile.
+FA_DEV void load_tile_scores(uint32_t sa, uint32_t bits, bool diag, int r, float (&s)[BN]) {
+#pragma unroll
+  for (int q4 = 0; q4 < BN / 32; ++q4) {
+    uint32_t raw[32];
+    tmem_ld32(sa + q4 * 32, raw);
+    tmem_ld_wait(raw);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(raw[i]);
+  }
+  if (diag || bits != 0xFu) {
+    const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
+#pragma unroll
+    for (int i = 0; i < BN; ++i) {
+      const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
+      s[i] = keep ? s[i] : -INFINITY;
+    }
+  }
+}
+
 FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt, int b, int h,
                         bool sparse) {
   const int r = threadIdx.x - 128;                  // row within the tile
@@ -339,40 +461,39 @@ FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt
       break;
     }
     tc_fence_after_sync();
-    float s[BN];
-    {
-      const uint32_t sa = lane_base + ((j & 1) ? TM_S1 : TM_S0);
-#pragma unroll
-      for (int q4 = 0; q4 < BN / 32; ++q4) {
-        uint32_t raw[32];
-        tmem_ld32(sa + q4 * 32, raw);
-        tmem_ld_wait(raw);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(raw[i]);
-      }
-    }
+    // Lazy reference max (as in the two-tile kernel): the running max of the
+    // earlier tiles, no max over this tile; a row sum past kLazySumLimit (or
+    // not finite) means some score rose far above it -- then the warp reads
+    // S again, takes the tile's max and redoes the exponentials.  The first
+    // tile takes its max first.
+    const uint32_t sa = lane_base + ((j & 1) ? TM_S1 : TM_S0);
     const bool diag = (n == qt);
-    if (diag || bits != 0xFu) {
-      const uint32_t rb = (bits >> ((r >> 6) * 2)) & 3u;
-#pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        const bool keep = ((rb >> (i >> 6)) & 1u) && (!diag || i <= r);
-        s[i] = keep ? s[i] : -INFINITY;
+    float m_ref = m_run, m_new = m_run;
+    bool need = false;
+    uint32_t pk[BN / 2];
+    float l_tile;
+    {
+      float s[BN];
+      load_tile_scores(sa, bits, diag, r, s);
+      const bool lazy = kLazyMax && !__any_sync(0xffffffffu, m_run == -INFINITY);
+      if (!lazy) {
+        m_new = fmaxf(m_run, row_max(s) * c);
+        need = m_new > m_run + kRescaleThreshold;
+        m_ref = need ? m_new : m_run;
       }
+      l_tile = row_exp2(s, c, m_ref, pk);
     }
-    float mx8[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) mx8[k] = s[k];
-#pragma unroll
-    for (int i = 8; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
-    float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-    const float m_tile = mx * c;
-    const float m_new = fmaxf(m_run, m_tile);
-    const bool need = m_new > m_run + kRescaleThreshold;
+    if (kLazyMax && __any_sync(0xffffffffu, !(l_tile <= kLazySumLimit))) {
+      float s[BN];
+      load_tile_scores(sa, bits, diag, r, s);
+      m_new = fmaxf(m_run, row_max(s) * c);
+      need = m_new > m_run;
+      m_ref = need ? m_new : m_run;
+      l_tile = row_exp2(s, c, m_ref, pk);
+    }
     if (j > 0 && __any_sync(0xffffffffu, need)) {
-      // O holds sum_{k<j} exp2(s*c - m_run) V; bring it to the new max.  The
-      // previous PV must have landed first.
+      // O holds sum_{k<j} exp2(s*c - m_run) V; bring it to the new reference.
+      // The previous PV must have landed first.
       if (!warp_wait(&sh.pv_done[(j - 1) & 1], static_cast<uint32_t>((j - 1) >> 1) & 1u, sh, p)) {
         ok = false;
         break;
@@ -390,18 +511,9 @@ FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt
       }
       tmem_st_wait();
     }
-    if (need) {
-      l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
-      m_run = m_new;
-    }
-    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-    float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < BN; ++i) {
-      s[i] = ex2(fmaf(s[i], c, -m_use));
-      sum4[i & 3] += s[i];
-    }
-    l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+    if (need) l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2(m_run - m_new);
+    m_run = m_ref;
+    l_run += l_tile;
     // P buffer j&1 was last read by PV(j-2).
     if (j >= 2 && !warp_wait(&sh.pv_done[j & 1], static_cast<uint32_t>((j - 2) >> 1) & 1u, sh, p)) {
       ok = false;
@@ -410,13 +522,14 @@ FA_DEV void run_softmax(const Shared &sh, uint32_t tmem, const Params &p, int qt
     tc_fence_after_sync();
     {
       const uint32_t pa = lane_base + ((j & 1) ? TM_P1 : TM_P0);
+      uint32_t lo[32], hi[32];
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[q2 * 64 + 2 * i], s[q2 * 64 + 2 * i + 1]);
-        tmem_st32(pa + q2 * 32, pk);
+      for (int i = 0; i < 32; ++i) {
+        lo[i] = pk[i];
+        hi[i] = pk[32 + i];
       }
+      tmem_st32(pa, lo);
+      tmem_st32(pa + 32, hi);
       tmem_st_wait();
     }
     tc_fence_before_sync();
@@ -596,48 +709,6 @@ static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint64_t kDrainNs = 200000000ull;
-
-// 2^x on the FMA pipe: round-to-nearest range reduction with the 1.5*2^23
-// shifter (x = n + f, f in [-1/2, 1/2]), a degree-3 polynomial for 2^f
-// (coefficients fitted here by minimax linear programming on [-1/2, 1/2];
-// max relative error 1.0e-4, below bf16 rounding of P), and n added to the
-// exponent field.  Inputs below -127 give 0.
-#ifndef FA_POLY_PER_8
-#define FA_POLY_PER_8 2
-#endif
-// Key pairs (k, k+1), k even, with (k mod 8) >= 8 - kPolyPer8 take the
-// polynomial (so kPolyPer8 counts in steps of 2); the rest use ex2.approx.
-constexpr int kPolyPer8 = FA_POLY_PER_8;
-constexpr float kExp2C1 = 0.693282962f;
-constexpr float kExp2C2 = 0.242210999f;
-constexpr float kExp2C3 = 0.0550087839f;
-FA_DEV float ex2_poly(float x) {
-  x = fmaxf(x, -127.0f);
-  const float t = x + 12582912.0f;          // 1.5 * 2^23: low mantissa bits = round(x)
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(kExp2C3, f, kExp2C2);
-  p = fmaf(p, f, kExp2C1);
-  p = fmaf(p, f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-// The same for two lanes at once with the packed fp32x2 instructions.
-FA_DEV void ex2_poly2(uint64_t x2, float &r0, float &r1) {
-  float a, b;
-  f2_split(x2, a, b);
-  const uint64_t x = f2_make(fmaxf(a, -127.0f), fmaxf(b, -127.0f));
-  const uint64_t t = f2_add(x, f2_make(12582912.0f, 12582912.0f));
-  const uint64_t n = f2_add(t, f2_make(-12582912.0f, -12582912.0f));
-  const uint64_t f = f2_fma(n, f2_make(-1.0f, -1.0f), x);
-  uint64_t p = f2_fma(f2_make(kExp2C3, kExp2C3), f, f2_make(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_make(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_make(1.0f, 1.0f));
-  float p0, p1, t0, t1;
-  f2_split(p, p0, p1);
-  f2_split(t, t0, t1);
-  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
 
 // Shared-memory layout, as offsets from one 1024-byte aligned base:
 // Q tiles | K/V ring | epilogue staging | mbarriers | TMEM address | abort word.
@@ -962,27 +1033,6 @@ FA_DEV void run_mma(const Smem &sh, uint32_t tmem, const Params &p, int total) {
 }
 
 
-// Row max of the 128 scores: 3-input max over pairs, 8 independent chains.
-FA_DEV float row_max(const float (&s)[BN]) {
-  float mx8[8];
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmaxf(s[2 * kk], s[2 * kk + 1]);
-#pragma unroll
-  for (int i = 16; i < BN; i += 16)
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) mx8[kk] = fmax3(mx8[kk], s[i + 2 * kk], s[i + 2 * kk + 1]);
-  return fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-               fmaxf(mx8[6], mx8[7]));
-}
-
-#ifndef FA_LAZY_MAX
-#define FA_LAZY_MAX 1
-#endif
-constexpr bool kLazyMax = FA_LAZY_MAX != 0;
-// Largest row sum of one tile's p = 2^(s*c - m) accepted without taking the
-// tile's max: p stays far inside the bf16 / fp32 range (2^127).
-constexpr float kLazySumLimit = 4294967296.0f;   // 2^32
-
 // The 128 scores of this thread's row of S_t, masked: the 4-bit block mask
 // `bits` (sparse tiles) and causality on the diagonal tile.
 FA_DEV void load_scores(uint32_t s_base, uint32_t bits, bool diag, int r, float (&s)[BN]) {
@@ -1000,34 +1050,6 @@ FA_DEV void load_scores(uint32_t s_base, uint32_t bits, bool diag, int r, float 
       s[i] = keep ? s[i] : -INFINITY;
     }
   }
-}
-
-// p = 2^(s*c - m) for the 128 scores, packed as bf16 pairs into pk; returns
-// the row sum.  Two lanes per instruction (the argument and the sums);
-// ex2.approx, or the FMA-pipe polynomial for kPolyPer8 keys of 8.
-FA_DEV float row_exp2(const float (&s)[BN], float c, float m, uint32_t (&pk)[BN / 2]) {
-  const float m_use = (m == -INFINITY) ? 0.f : m;
-  const uint64_t c2 = f2_make(c, c), negm2 = f2_make(-m_use, -m_use);
-  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-  for (int i = 0; i < BN / 2; ++i) {
-    const int k0 = 2 * i;
-    const uint64_t x = f2_fma(f2_make(s[k0], s[k0 + 1]), c2, negm2);
-    float p0, p1;
-    if ((k0 & 7) >= 8 - kPolyPer8) {
-      ex2_poly2(x, p0, p1);
-    } else {
-      float x0, x1;
-      f2_split(x, x0, x1);
-      p0 = ex2(x0);
-      p1 = ex2(x1);
-    }
-    acc[i & 3] = f2_add(acc[i & 3], f2_make(p0, p1));
-    pk[i] = pack_bf16x2(p0, p1);
-  }
-  float a0, a1;
-  f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
-  return a0 + a1;
 }
 
 // Softmax of one 128-column S tile of head t for the row r of this thread:

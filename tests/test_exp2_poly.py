@@ -1,5 +1,5 @@
 """The FMA-pipe exp2 the prefill kernel can use for a share of the softmax
-(a compile-time share, 0 by default):
+(a compile-time share: a quarter of the keys by default):
 range reduction x = n + f with the 1.5*2^23 shifter, a degree-3 polynomial
 for 2^f on [-1/2, 1/2], n added to the exponent field.  The constants are
 read from the kernel source and the routine is replayed in fp32 numpy, op
